@@ -1,0 +1,226 @@
+"""NumPy float64 oracle: the plain definition of forward Differential Attention V2.
+
+TEST INFRASTRUCTURE ONLY (see the package docstring): never imported by the product path.
+
+Sources (page title, then section / equation):
+  [L16]  "Differential Attention (V2)" lesson (AI Engineering from Scratch, phase 10, 16):
+         "The differential concept" -- A1 = softmax(Q1 K1^T / sqrt(d)),
+         A2 = softmax(Q2 K2^T / sqrt(d)), DiffAttn = (A1 - lambda * A2) V;
+         the lambda re-parameterisation lambda = exp(lq1.lk1) - exp(lq2.lk2) + lambda_init;
+         "Build it", Step 1 (numerically stable softmax: subtract the row max, exponentiate,
+         divide by the sum) and Step 3 (two softmax branches, subtract, multiply by V);
+         "Exercises" 4 (lambda = 0 is the pure first softmax) and 5 (GQA + V2 cache size).
+  [L07]  "Attention variants: sliding window, sparse, differential" lesson (phase 7, 15):
+         "Build it", Step 1 (causal mask: 0 where j <= i, -inf otherwise) and Step 4
+         (diff_attention: causal softmax per branch, then (A1 - lam*A2) @ V).
+  [HF]   "Differential Transformer V2 soll KI-Training stabiler machen" (summary of the
+         Hugging Face blog), section "Gemeinsamer KV-Cache statt Spezialkernel": two adjacent
+         query heads inside one GQA group share K and V; section "Weniger Ausreisser und
+         Gradientenspitzen": lambda is projected per token and per head and bounded by a
+         sigmoid.
+
+Readings of points the pages leave open (each also listed in the design notes):
+  * head 2p of a pair is branch 1 (A1, +), head 2p+1 is branch 2 (A2, -lambda);
+  * the KV head of pair p is g = (2p) // (Hq / Hkv);
+  * lambda is one value per token and per output head (= pair): [B, S, Hq/2] for prefill,
+    [B, Hq/2] for decode; it arrives already bounded (the model applies the sigmoid);
+  * the score scale is 1/sqrt(D) for both branches (the toy's `scale` read as sqrt(d));
+  * causal means key j is visible from query i when j <= i, with Sq == Sk;
+  * decode attends to keys [0, seqlen_b), the new token's key already appended.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+__all__ = [
+    "stable_softmax",
+    "causal_mask",
+    "pair_layout",
+    "diff_attention_block",
+    "prefill",
+    "prefill_rows",
+    "decode",
+    "lambda_v1",
+    "branch_weights",
+    "snr",
+]
+
+
+def stable_softmax(x: np.ndarray) -> np.ndarray:
+    """Row softmax along the last axis, the two-pass stable form of [L16] Step 1.
+
+    m = max(row); e = exp(x - m); return e / sum(e). Entries equal to -inf (masked keys)
+    get weight exactly 0. A row must hold at least one finite entry.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    m = np.max(x, axis=-1, keepdims=True)
+    e = np.exp(x - m)
+    return e / np.sum(e, axis=-1, keepdims=True)
+
+
+def causal_mask(n_q: int, n_k: int, q_offset: int = 0) -> np.ndarray:
+    """Additive causal mask of [L07] Step 1: 0.0 where key j <= query i, else -inf.
+
+    Query rows are numbered q_offset .. q_offset + n_q - 1 (a row block of a longer
+    sequence); keys are numbered 0 .. n_k - 1.
+    """
+    i = np.arange(q_offset, q_offset + n_q)[:, None]
+    j = np.arange(n_k)[None, :]
+    return np.where(j <= i, 0.0, -np.inf)
+
+
+def pair_layout(Hq: int, Hkv: int):
+    """V2 head pairing of [HF] (shared KV cache section) and [L16] "V1 vs V2".
+
+    Returns a list of (p, h1, h2, g): pair p, its branch-1 head h1 = 2p, its branch-2 head
+    h2 = 2p+1, and the KV head g both heads read. Both heads of a pair must sit in the same
+    GQA group, which holds when Hq is a multiple of 2*Hkv.
+    """
+    if Hq % 2 != 0 or Hkv <= 0 or Hq % (2 * Hkv) != 0:
+        raise ValueError(f"need Hq even and a multiple of 2*Hkv (Hq={Hq}, Hkv={Hkv})")
+    G = Hq // Hkv
+    out = []
+    for p in range(Hq // 2):
+        h1, h2 = 2 * p, 2 * p + 1
+        g = h1 // G
+        assert h2 // G == g
+        out.append((p, h1, h2, g))
+    return out
+
+
+def diff_attention_block(q1, q2, k, v, lam, mask):
+    """DiffAttn for one pair over a block of query rows: [L16] eq. DiffAttn, [L07] Step 4.
+
+    q1, q2: [n, D] the two heads of the pair; k, v: [m, D] their shared K/V head;
+    lam: [n] one lambda per query row; mask: [n, m] additive (0 or -inf).
+    Returns [n, D] = (softmax(q1 k^T / sqrt(D) + mask) - lam * softmax(q2 k^T / sqrt(D) + mask)) v.
+    """
+    D = q1.shape[-1]
+    inv_sqrt_d = 1.0 / math.sqrt(D)
+    a1 = stable_softmax(q1 @ k.T * inv_sqrt_d + mask)
+    a2 = stable_softmax(q2 @ k.T * inv_sqrt_d + mask)
+    w = a1 - lam[:, None] * a2
+    return w @ v
+
+
+def _f64(t) -> np.ndarray:
+    """Exact upcast of a torch tensor or array (bf16/fp32 values) to float64."""
+    if hasattr(t, "detach"):
+        import torch  # local: only for the dtype conversion of inputs
+
+        return t.detach().to(torch.float64).cpu().numpy()
+    return np.asarray(t, dtype=np.float64)
+
+
+def prefill(q, k, v, lam, causal: bool = True, row_block: int = 512) -> np.ndarray:
+    """Forward prefill over the whole batch: out[B, S, Hq/2, D] in float64.
+
+    q [B,S,Hq,D], k/v [B,S,Hkv,D], lam [B,S,Hq/2]. For every batch b and pair p the rows are
+    processed in blocks of `row_block` (a memory bound only: every row is computed exactly
+    as the definition states, over all its visible keys).
+    """
+    q, k, v, lam = _f64(q), _f64(k), _f64(v), _f64(lam)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    out = np.zeros((B, S, Hq // 2, D), dtype=np.float64)
+    for b in range(B):
+        for p, h1, h2, g in pair_layout(Hq, Hkv):
+            kk, vv = k[b, :, g], v[b, :, g]
+            for r0 in range(0, S, row_block):
+                r1 = min(S, r0 + row_block)
+                n_k = r1 if causal else S
+                mask = causal_mask(r1 - r0, n_k, r0) if causal else np.zeros((r1 - r0, S))
+                out[b, r0:r1, p] = diff_attention_block(
+                    q[b, r0:r1, h1], q[b, r0:r1, h2], kk[:n_k], vv[:n_k], lam[b, r0:r1, p], mask)
+    return out
+
+
+def prefill_rows(q, k, v, lam, rows, causal: bool = True) -> np.ndarray:
+    """Selected output rows of a prefill: rows is a list of (b, i, p); returns [len(rows), D].
+
+    Each row is the definition applied to query i of pair p in batch b over keys j <= i
+    (causal) or all keys. Used for sampled checks of full-size outputs.
+    """
+    Hq = q.shape[2]
+    Hkv = k.shape[2]
+    layout = {p: (h1, h2, g) for p, h1, h2, g in pair_layout(Hq, Hkv)}
+    S = q.shape[1]
+    res = []
+    for b, i, p in rows:
+        h1, h2, g = layout[p]
+        n_k = i + 1 if causal else S
+        q1 = _f64(q[b, i, h1])[None, :]
+        q2 = _f64(q[b, i, h2])[None, :]
+        kk = _f64(k[b, :n_k, g])
+        vv = _f64(v[b, :n_k, g])
+        lm = np.array([float(lam[b, i, p])], dtype=np.float64)
+        res.append(diff_attention_block(q1, q2, kk, vv, lm, np.zeros((1, n_k)))[0])
+    return np.stack(res) if res else np.zeros((0, q.shape[3]))
+
+
+def decode(q, kcache, vcache, seqlens, lam) -> np.ndarray:
+    """One decode step: out[B, Hq/2, D] in float64.
+
+    q [B,Hq,D] is the new token's query; the caches [B,Smax,Hkv,D] already hold its key and
+    value, and sequence b attends to keys [0, seqlens[b]). lam [B,Hq/2]. A sequence with
+    seqlens[b] == 0 has no visible key; its output is defined as 0.
+    """
+    B, Hq, D = q.shape
+    Hkv = kcache.shape[2]
+    out = np.zeros((B, Hq // 2, D), dtype=np.float64)
+    for b in range(B):
+        n = int(seqlens[b])
+        if n <= 0:
+            continue
+        for g in range(Hkv):
+            kk = _f64(kcache[b, :n, g])
+            vv = _f64(vcache[b, :n, g])
+            for p, h1, h2, gg in pair_layout(Hq, Hkv):
+                if gg != g:
+                    continue
+                q1 = _f64(q[b, h1])[None, :]
+                q2 = _f64(q[b, h2])[None, :]
+                lm = np.array([float(lam[b, p])], dtype=np.float64)
+                out[b, p] = diff_attention_block(q1, q2, kk, vv, lm, np.zeros((1, n)))[0]
+    return out
+
+
+def lambda_v1(lq1, lk1, lq2, lk2, lambda_init: float = 0.8) -> np.ndarray:
+    """V1 lambda re-parameterisation of [L16] "The differential concept":
+    lambda = exp(lq1 . lk1) - exp(lq2 . lk2) + lambda_init, one scalar per pair.
+
+    Inputs are [n_pairs, d] (one set of four vectors per pair); returns [n_pairs] float64.
+    The value may be negative or above 1 ([L16] key-terms table, "lambda").
+    """
+    a, b, c, e = (_f64(x) for x in (lq1, lk1, lq2, lk2))
+    return np.exp(np.sum(a * b, axis=-1)) - np.exp(np.sum(c * e, axis=-1)) + float(lambda_init)
+
+
+def branch_weights(q1, q2, k, lam, n_visible=None):
+    """Attention weights of one query row: (a1, a2, a1 - lam * a2) over its visible keys.
+
+    q1, q2: [D]; k: [m, D]. Keys n_visible.. are masked out (weight 0). Follows [L16]
+    Step 3 (`diff_weights`).
+    """
+    q1, q2, k = _f64(q1), _f64(q2), _f64(k)
+    m = k.shape[0] if n_visible is None else int(n_visible)
+    D = q1.shape[-1]
+    s1 = k[:m] @ q1 / math.sqrt(D)
+    s2 = k[:m] @ q2 / math.sqrt(D)
+    a1 = stable_softmax(s1)
+    a2 = stable_softmax(s2)
+    return a1, a2, a1 - float(lam) * a2
+
+
+def snr(weights, signal_index: int) -> float:
+    """Signal-to-noise ratio of one weight row ([L16] key-terms table, "Signal-to-noise
+    ratio"): weight on the signal position over the average weight on the unrelated positions.
+
+    Differential weights can be negative ([L16] Step 3 note), so the average over unrelated
+    positions is taken of the absolute weights.
+    """
+    w = np.asarray(weights, dtype=np.float64)
+    others = np.delete(w, signal_index)
+    return float(w[signal_index] / np.mean(np.abs(others)))

@@ -1,0 +1,310 @@
+"""Pins for the float64 oracle: checks against what the pages and the mathematics fix.
+
+Every pin compares the oracle with something other than itself: a library routine
+(torch scaled_dot_product_attention, scipy softmax), a closed form, an invariant, the
+worked example printed on the pages, or the independent stdlib brute force. The
+mutation tests in test_oracle_mutations.py plant plausible mistakes in the oracle and
+check that these pins catch each one.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import brute
+from oracle import diffattn_f64 as ora
+import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand_prefill(B=2, S=37, Hq=8, Hkv=2, D=16, seed=0, lam_range=(-0.5, 1.5)):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, S, Hq, D))
+    k = rng.standard_normal((B, S, Hkv, D))
+    v = rng.standard_normal((B, S, Hkv, D))
+    lam = rng.uniform(*lam_range, size=(B, S, Hq // 2))
+    return q, k, v, lam
+
+
+def _sdpa_head(q, k, v, h, g, causal=True):
+    """Ordinary softmax attention of query head h over KV head g (torch, float64, CPU)."""
+    qt = torch.from_numpy(q[:, :, h, :]).permute(0, 1, 2)[:, None]  # [B,1,S,D]
+    kt = torch.from_numpy(k[:, :, g, :])[:, None]
+    vt = torch.from_numpy(v[:, :, g, :])[:, None]
+    o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=causal)
+    return o[:, 0].numpy()
+
+
+# ----------------------------------------------------------------------------- pins
+# Each pin_* returns True when the oracle satisfies it; the tests assert them and the
+# mutation tests check that a planted mistake makes at least one of them False.
+
+def pin_softmax_library(seed=0):
+    from scipy.special import softmax as sp_softmax
+
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((7, 33)) * 30.0
+    ok = np.allclose(ora.stable_softmax(x), sp_softmax(x, axis=-1), rtol=1e-13, atol=1e-300)
+    xm = x.copy()
+    xm[:, 5:] = -np.inf
+    ok &= np.allclose(ora.stable_softmax(xm)[:, :5], sp_softmax(x[:, :5], axis=-1), rtol=1e-13)
+    ok &= bool(np.all(ora.stable_softmax(xm)[:, 5:] == 0.0))
+    # shift invariance holds for logits far outside exp's range too
+    ok &= np.allclose(ora.stable_softmax(x + 900.0), sp_softmax(x, axis=-1), rtol=1e-12)
+    return bool(ok)
+
+
+def pin_lambda0_is_softmax_attention(causal=True):
+    """lambda = 0 leaves the pure first softmax ("Differential Attention (V2)" lesson,
+    Exercise 4): pair p must equal ordinary attention of head 2p over its GQA KV head."""
+    q, k, v, lam = _rand_prefill(seed=1)
+    lam[:] = 0.0
+    out = ora.prefill(q, k, v, lam, causal=causal, row_block=16)
+    Hq, Hkv = q.shape[2], k.shape[2]
+    G = Hq // Hkv
+    ok = True
+    for p in range(Hq // 2):
+        ref = _sdpa_head(q, k, v, 2 * p, (2 * p) // G, causal=causal)
+        ok &= np.allclose(out[:, :, p], ref, rtol=1e-11, atol=1e-12)
+    return bool(ok)
+
+
+def pin_second_branch_is_odd_head(causal=True):
+    """O(0) - O(1) = A2 V: the subtracted branch is head 2p+1 over the same KV head."""
+    q, k, v, lam = _rand_prefill(seed=2)
+    o0 = ora.prefill(q, k, v, np.zeros_like(lam), causal=causal)
+    o1 = ora.prefill(q, k, v, np.ones_like(lam), causal=causal)
+    Hq, Hkv = q.shape[2], k.shape[2]
+    G = Hq // Hkv
+    ok = True
+    for p in range(Hq // 2):
+        ref = _sdpa_head(q, k, v, 2 * p + 1, (2 * p + 1) // G, causal=causal)
+        ok &= np.allclose(o0[:, :, p] - o1[:, :, p], ref, rtol=1e-10, atol=1e-11)
+    return bool(ok)
+
+
+def pin_equal_queries_lambda1_zero():
+    """Q1 = Q2 with lambda = 1 gives exactly zero (both branches computed identically)."""
+    q, k, v, lam = _rand_prefill(seed=3)
+    q[:, :, 1::2] = q[:, :, 0::2]
+    out = ora.prefill(q, k, v, np.ones_like(lam))
+    return bool(np.all(out == 0.0))
+
+
+def pin_rows_sum_to_one_minus_lambda():
+    """With V == 1 every output element is the row sum of A1 - lam*A2, which is 1 - lam."""
+    q, k, v, lam = _rand_prefill(seed=4)
+    v[:] = 1.0
+    out = ora.prefill(q, k, v, lam)
+    return bool(np.allclose(out, (1.0 - lam)[..., None], rtol=0, atol=1e-12))
+
+
+def pin_causal_row0():
+    """Causal row 0 sees only key 0, so out[b,0,p] = (1 - lam) * v[b,0,g]."""
+    q, k, v, lam = _rand_prefill(seed=5)
+    out = ora.prefill(q, k, v, lam)
+    Hq, Hkv = q.shape[2], k.shape[2]
+    G = Hq // Hkv
+    ok = True
+    for p in range(Hq // 2):
+        g = (2 * p) // G
+        ok &= np.allclose(out[:, 0, p], (1.0 - lam[:, 0, p])[:, None] * v[:, 0, g], atol=1e-13)
+    return bool(ok)
+
+
+def pin_linear_in_lambda():
+    """O(lam) = O(0) - lam * (O(0) - O(1)) for three lambda values."""
+    q, k, v, lam = _rand_prefill(seed=6)
+    o0 = ora.prefill(q, k, v, np.zeros_like(lam))
+    o1 = ora.prefill(q, k, v, np.ones_like(lam))
+    ok = True
+    for c in (-0.7, 0.37, 2.5):
+        oc = ora.prefill(q, k, v, np.full_like(lam, c))
+        ok &= np.allclose(oc, o0 - c * (o0 - o1), atol=1e-11)
+    return bool(ok)
+
+
+def pin_brute_force_prefill(causal=True):
+    q, k, v, lam = _rand_prefill(B=2, S=9, Hq=8, Hkv=2, D=5, seed=7)
+    ref = np.array(brute.prefill(q.tolist(), k.tolist(), v.tolist(), lam.tolist(), causal=causal))
+    out = ora.prefill(q, k, v, lam, causal=causal, row_block=4)
+    return bool(np.allclose(out, ref, rtol=0, atol=1e-12))
+
+
+def pin_brute_force_decode():
+    rng = np.random.default_rng(8)
+    B, Smax, Hq, Hkv, D = 3, 11, 8, 2, 6
+    q = rng.standard_normal((B, Hq, D))
+    kc = rng.standard_normal((B, Smax, Hkv, D))
+    vc = rng.standard_normal((B, Smax, Hkv, D))
+    seqlens = np.array([11, 1, 0])
+    lam = rng.uniform(-1, 2, size=(B, Hq // 2))
+    ref = np.array(brute.decode(q.tolist(), kc.tolist(), vc.tolist(), seqlens.tolist(), lam.tolist()))
+    out = ora.decode(q, kc, vc, seqlens, lam)
+    return bool(np.allclose(out, ref, rtol=0, atol=1e-12))
+
+
+def pin_decode_is_last_prefill_row():
+    """A decode step over n cached keys equals row n-1 of a causal prefill of length n."""
+    rng = np.random.default_rng(9)
+    B, S, Hq, Hkv, D = 2, 21, 8, 2, 8
+    q, k, v, lam = _rand_prefill(B=B, S=S, Hq=Hq, Hkv=Hkv, D=D, seed=9)
+    seqlens = np.array([S, 13])
+    qd = np.stack([q[0, S - 1], q[1, 12]])
+    lamd = np.stack([lam[0, S - 1], lam[1, 12]])
+    dec = ora.decode(qd, k, v, seqlens, lamd)
+    full = ora.prefill(q, k, v, lam)
+    ok = np.allclose(dec[0], full[0, S - 1], atol=1e-13)
+    ok &= np.allclose(dec[1], ora.prefill(q[1:, :13], k[1:, :13], v[1:, :13], lam[1:, :13])[0, 12],
+                      atol=1e-13)
+    del rng
+    return bool(ok)
+
+
+def pin_prefill_rows_match_full():
+    q, k, v, lam = _rand_prefill(seed=10)
+    full = ora.prefill(q, k, v, lam)
+    rows = [(0, 0, 0), (1, 36, 3), (0, 17, 2), (1, 5, 1)]
+    sel = ora.prefill_rows(q, k, v, lam, rows)
+    return bool(all(np.allclose(sel[n], full[b, i, p], atol=1e-13) for n, (b, i, p) in enumerate(rows)))
+
+
+def pin_lambda_v1_closed_form():
+    """lambda = exp(lq1.lk1) - exp(lq2.lk2) + lambda_init with dot products ln2 and 0 -> 1.8,
+    and 0 and ln3 -> -1.2 (lambda may be negative)."""
+    d = 4
+    a = np.zeros((2, d)); b = np.zeros((2, d)); c = np.zeros((2, d)); e = np.zeros((2, d))
+    a[0, 0], b[0, 0] = math.log(2.0), 1.0          # pair 0: a.b = ln 2, c.e = 0
+    c[1, 1], e[1, 1] = math.log(3.0) / 2.0, 2.0    # pair 1: a.b = 0,    c.e = ln 3
+    lam = ora.lambda_v1(a, b, c, e, 0.8)
+    ok = abs(lam[0] - 1.8) < 1e-14 and abs(lam[1] - (-1.2)) < 1e-14
+    rng = np.random.default_rng(11)
+    vec = [rng.standard_normal((5, 7)) * 0.3 for _ in range(4)]
+    ok &= np.allclose(ora.lambda_v1(*vec, 0.8), brute.lambda_v1(*(x.tolist() for x in vec), 0.8),
+                      atol=1e-14)
+    return bool(ok)
+
+
+def pin_noise_mass_golden():
+    """The 128k worked example of the lesson's "The problem" section (golden fixture)."""
+    with open(os.path.join(GOLDEN, "noise_mass_128k.json")) as f:
+        gold = json.load(f)
+    n = gold["context_tokens"]
+    w = gold["per_token_weight"]
+    # one matching token with logit x and n-1 unrelated tokens with logit 0 such that each
+    # unrelated token gets weight w: 1/(e^x + n - 1) = w
+    x = math.log(1.0 / w - (n - 1))
+    row = np.zeros(n)
+    row[0] = x
+    a = ora.stable_softmax(row)
+    mass = float(np.sum(a[1:]))
+    ok = abs(a[1] - w) < 1e-18 and abs(mass - gold["noise_mass"]) < 1e-12
+    ok &= round(100 * mass) == gold["noise_mass_rounded_percent"]
+    return bool(ok)
+
+
+def pin_uniform_logits():
+    """N equal logits give every token weight exactly-ish 1/N (the O(1/N) noise floor)."""
+    ok = True
+    for n in (1, 7, 4096):
+        a = ora.stable_softmax(np.full(n, 3.25))
+        ok &= np.allclose(a, 1.0 / n, rtol=1e-14)
+    return bool(ok)
+
+
+def pin_weights_rows_sum():
+    rng = np.random.default_rng(12)
+    k = rng.standard_normal((50, 16))
+    ok = True
+    for lam in (-0.3, 0.0, 0.8, 1.0):
+        a1, a2, w = ora.branch_weights(rng.standard_normal(16), rng.standard_normal(16), k, lam, 31)
+        ok &= abs(a1.sum() - 1) < 1e-14 and abs(a2.sum() - 1) < 1e-14
+        ok &= abs(w.sum() - (1 - lam)) < 1e-13 and len(w) == 31
+    return bool(ok)
+
+
+ALL_PINS = {
+    "softmax_library": pin_softmax_library,
+    "lambda0_is_softmax_attention": pin_lambda0_is_softmax_attention,
+    "lambda0_noncausal": lambda: pin_lambda0_is_softmax_attention(causal=False),
+    "second_branch_is_odd_head": pin_second_branch_is_odd_head,
+    "equal_queries_lambda1_zero": pin_equal_queries_lambda1_zero,
+    "rows_sum_to_one_minus_lambda": pin_rows_sum_to_one_minus_lambda,
+    "causal_row0": pin_causal_row0,
+    "linear_in_lambda": pin_linear_in_lambda,
+    "brute_force_prefill": pin_brute_force_prefill,
+    "brute_force_prefill_noncausal": lambda: pin_brute_force_prefill(causal=False),
+    "brute_force_decode": pin_brute_force_decode,
+    "decode_is_last_prefill_row": pin_decode_is_last_prefill_row,
+    "prefill_rows_match_full": pin_prefill_rows_match_full,
+    "lambda_v1_closed_form": pin_lambda_v1_closed_form,
+    "noise_mass_golden": pin_noise_mass_golden,
+    "uniform_logits": pin_uniform_logits,
+    "weights_rows_sum": pin_weights_rows_sum,
+}
+
+
+@pytest.mark.parametrize("name", sorted(ALL_PINS))
+def test_pin(name):
+    assert ALL_PINS[name]()
+
+
+# ------------------------------------------------------------ the noise-cancellation toy
+
+def _planted_c1():
+    case = workloads.CONFIGS["c1_tiny_fp32_prefill"]
+    inp = workloads.make_prefill(case)
+    row, sig = workloads.plant_signal_row(inp)
+    return inp, row, sig
+
+
+def test_planted_row_noise_cancels():
+    """"Differential Attention (V2)" lesson, Step 4: with a shared noise floor the difference
+    map has a higher signal-to-noise ratio than the first softmax alone, for lambda in
+    [0.5, 1]."""
+    inp, row, sig = _planted_c1()
+    q, k = inp["q"], inp["k"]
+    for lam in (0.5, 0.75, 0.9, 1.0):
+        a1, _, w = ora.branch_weights(q[0, row, 0], q[0, row, 1], k[0, :, 0], lam, row + 1)
+        assert ora.snr(w, sig) > ora.snr(a1, sig)
+    # lambda = 0 leaves the first softmax unchanged
+    a1, _, w = ora.branch_weights(q[0, row, 0], q[0, row, 1], k[0, :, 0], 0.0, row + 1)
+    assert np.array_equal(a1, w)
+
+
+def test_planted_toy_length_1024_reports_ratio(capsys):
+    """The lesson's length-1024 toy: report the SNR ratio diff/standard (the pages claim
+    3x-10x qualitatively; this is reported, and only a ratio > 1 is asserted)."""
+    case = workloads.PrefillCase(B=1, S=1024, Hq=2, Hkv=1, D=64, dtype="f32", seed=2024)
+    inp = workloads.make_prefill(case)
+    row, sig = workloads.plant_signal_row(inp, signal_key=300)
+    q, k = inp["q"], inp["k"]
+    a1, _, w = ora.branch_weights(q[0, row, 0], q[0, row, 1], k[0, :, 0], 0.9, row + 1)
+    ratio = ora.snr(w, sig) / ora.snr(a1, sig)
+    with capsys.disabled():
+        print(f"\n[toy] length-1024 SNR diff/standard at lambda=0.9: {ratio:.2f}x")
+    assert ratio > 1.0
+
+
+def test_v2_kv_cache_matches_gqa_baseline():
+    """Exercise 5 of the lesson: with 8 KV heads and 32 query heads the V2 cache is the
+    same size as a baseline GQA cache -- it depends on Hkv, never on Hq."""
+    a = workloads.make_decode(workloads.DecodeCase(B=2, Smax=16, Hq=32, Hkv=8, D=8,
+                                                   len_lo=16, len_hi=16, seed=1))
+    b = workloads.make_decode(workloads.DecodeCase(B=2, Smax=16, Hq=16, Hkv=8, D=8,
+                                                   len_lo=16, len_hi=16, seed=1))
+    nbytes = lambda t: t.numel() * t.element_size()
+    assert nbytes(a["kcache"]) + nbytes(a["vcache"]) == 2 * 16 * 8 * 8 * 2 * 2
+    assert nbytes(a["kcache"]) == nbytes(b["kcache"])
+
+
+def test_pair_layout_rejects_straddling_pairs():
+    with pytest.raises(ValueError):
+        ora.pair_layout(6, 2)  # G = 3: pair (2,3) would straddle KV heads 0 and 1
+    with pytest.raises(ValueError):
+        ora.pair_layout(5, 1)
+    assert ora.pair_layout(64, 8)[5] == (5, 10, 11, 1)

@@ -1,0 +1,136 @@
+"""Planted mistakes in the oracle (on the CPU) must each fail at least one pin.
+
+Each mutant replaces one oracle function with a plausibly wrong version -- a dropped
+term, a wrong sign, a swapped head, a wrong GQA index, an off-by-one mask -- and the test
+checks that the pin suite of test_oracle.py notices. This shows the pins constrain every
+part of the definition rather than only re-reading it.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import diffattn_f64 as ora
+from tests.test_oracle import ALL_PINS
+
+
+def _block_plus_sign(q1, q2, k, v, lam, mask):
+    D = q1.shape[-1]
+    a1 = ora.stable_softmax(q1 @ k.T / math.sqrt(D) + mask)
+    a2 = ora.stable_softmax(q2 @ k.T / math.sqrt(D) + mask)
+    return (a1 + lam[:, None] * a2) @ v
+
+
+def _block_no_scale(q1, q2, k, v, lam, mask):
+    a1 = ora.stable_softmax(q1 @ k.T + mask)
+    a2 = ora.stable_softmax(q2 @ k.T + mask)
+    return (a1 - lam[:, None] * a2) @ v
+
+
+def _block_scale_d(q1, q2, k, v, lam, mask):
+    D = q1.shape[-1]
+    a1 = ora.stable_softmax(q1 @ k.T / D + mask)
+    a2 = ora.stable_softmax(q2 @ k.T / D + mask)
+    return (a1 - lam[:, None] * a2) @ v
+
+
+def _block_lambda_on_first(q1, q2, k, v, lam, mask):
+    D = q1.shape[-1]
+    a1 = ora.stable_softmax(q1 @ k.T / math.sqrt(D) + mask)
+    a2 = ora.stable_softmax(q2 @ k.T / math.sqrt(D) + mask)
+    return (lam[:, None] * a1 - a2) @ v
+
+
+def _block_shared_query(q1, q2, k, v, lam, mask):
+    D = q1.shape[-1]
+    a1 = ora.stable_softmax(q1 @ k.T / math.sqrt(D) + mask)
+    return ((1.0 - lam[:, None]) * a1) @ v
+
+
+def _block_softmax_wrong_axis(q1, q2, k, v, lam, mask):
+    D = q1.shape[-1]
+    s1 = q1 @ k.T / math.sqrt(D) + mask
+    s2 = q2 @ k.T / math.sqrt(D) + mask
+    a1 = np.nan_to_num(np.exp(s1) / np.sum(np.exp(s1), axis=0, keepdims=True))
+    a2 = np.nan_to_num(np.exp(s2) / np.sum(np.exp(s2), axis=0, keepdims=True))
+    return (a1 - lam[:, None] * a2) @ v
+
+
+def _layout_swapped(Hq, Hkv):
+    G = Hq // Hkv
+    return [(p, 2 * p + 1, 2 * p, (2 * p) // G) for p in range(Hq // 2)]
+
+
+def _layout_wrong_group(Hq, Hkv):
+    return [(p, 2 * p, 2 * p + 1, p % Hkv) for p in range(Hq // 2)]
+
+
+def _layout_split_heads(Hq, Hkv):
+    # pairs (p, p + Hq/2) instead of adjacent heads
+    G = Hq // Hkv
+    return [(p, p, p + Hq // 2, p // G) for p in range(Hq // 2)]
+
+
+def _mask_off_by_one(n_q, n_k, q_offset=0):
+    # lets each query see one future key
+    i = np.arange(q_offset, q_offset + n_q)[:, None]
+    j = np.arange(n_k)[None, :]
+    return np.where(j <= i + 1, 0.0, -np.inf)
+
+
+def _mask_transposed(n_q, n_k, q_offset=0):
+    i = np.arange(q_offset, q_offset + n_q)[:, None]
+    j = np.arange(n_k)[None, :]
+    return np.where(j >= i, 0.0, -np.inf)
+
+
+def _softmax_no_max(x):
+    x = np.asarray(x, dtype=np.float64)
+    e = np.exp(x)
+    return e / np.sum(e, axis=-1, keepdims=True)
+
+
+def _softmax_off(x):
+    x = np.asarray(x, dtype=np.float64)
+    m = np.max(x, axis=-1, keepdims=True)
+    e = np.exp(x - m)
+    return e / (np.sum(e, axis=-1, keepdims=True) + 1e-6)
+
+
+def _lambda_v1_plus(lq1, lk1, lq2, lk2, lambda_init=0.8):
+    a, b, c, e = (np.asarray(x, dtype=np.float64) for x in (lq1, lk1, lq2, lk2))
+    return np.exp(np.sum(a * b, -1)) + np.exp(np.sum(c * e, -1)) + lambda_init
+
+
+MUTANTS = {
+    "plus_sign": ("diff_attention_block", _block_plus_sign),
+    "no_scale": ("diff_attention_block", _block_no_scale),
+    "scale_by_d": ("diff_attention_block", _block_scale_d),
+    "lambda_on_first_branch": ("diff_attention_block", _block_lambda_on_first),
+    "second_branch_dropped": ("diff_attention_block", _block_shared_query),
+    "softmax_wrong_axis": ("diff_attention_block", _block_softmax_wrong_axis),
+    "heads_swapped": ("pair_layout", _layout_swapped),
+    "wrong_gqa_group": ("pair_layout", _layout_wrong_group),
+    "non_adjacent_pairs": ("pair_layout", _layout_split_heads),
+    "mask_off_by_one": ("causal_mask", _mask_off_by_one),
+    "mask_transposed": ("causal_mask", _mask_transposed),
+    "softmax_unstable": ("stable_softmax", _softmax_no_max),
+    "softmax_epsilon": ("stable_softmax", _softmax_off),
+    "lambda_v1_plus": ("lambda_v1", _lambda_v1_plus),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, monkeypatch):
+    attr, fn = MUTANTS[name]
+    monkeypatch.setattr(ora, attr, fn)
+    failed = []
+    with np.errstate(all="ignore"):
+        for pin_name, pin in ALL_PINS.items():
+            try:
+                ok = pin()
+            except Exception:  # a crash counts as a caught mutant
+                ok = False
+            if not ok:
+                failed.append(pin_name)
+    assert failed, f"mutant {name} passed every pin"
