@@ -1,0 +1,463 @@
+"""Benchmark of the forward Differential Attention V2 hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step is one pass of the whole hot path over one batch of synthetic input:
+  * prefill: causal bf16 DiffAttn V2 over B=4 x S=4096, Hq=64 (32 pairs), Hkv=8, D=128
+    (one tcgen05 kernel launch), then
+  * decode: one bf16 decode step for 64 sequences with lengths uniform in [1024, 8192]
+    over an [64, 8192, 8, 128] KV cache (split kernel + combine kernel).
+`value` is the prefill throughput in TFLOP/s (algorithmic FLOPs = 4*D*Hq*B*S(S+1)/2 over
+the prefill kernel's CUDA-event time inside the timed steps); the decode throughput in
+GB/s (every visible K/V row once, plus q, lambda and out) is reported beside it.
+Inputs are resident in HBM before the timed region and are larger than L2 (q alone is
+268 MB and the decode streams 1.2 GB per step), so no extra L2 flush is done.
+
+--impl reference times the float64 CPU oracle (the test oracle, as it stands) on a bounded
+sample of the same workload on the host cores; with N > 1 only rank 0 runs it.
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs the same per-GPU workload on its
+own seeded inputs (weak scaling: (b, KV-head) units are independent, so there is no
+data-path collective); the timed region is bracketed by a barrier and a synchronize and
+the time is the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "DiffAttnV2 fwd: prefill TFLOP/s (% bf16 peak); decode GB/s (% HBM)"
+PREFILL_CFG = "c2_bf16_prefill"
+DECODE_CFG = "c4_bf16_decode"
+
+# Measured roofline denominators of this machine's B200s (measured copy bandwidth and
+# cuBLAS bf16 GEMM); used when the peaks file is absent.
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic per launch from an ncu capture, keyed by the kernel source it was taken on;
+# reported as null once the source differs from the one captured.
+NCU_TRAFFIC = {
+    "prefill": {"bytes": None, "source_sha": None},
+    "decode": {"bytes": None, "source_sha": None},
+}
+
+
+def _src_sha(name):
+    p = os.path.join(ROOT, "differential_attention_v2_b200", "csrc", name)
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.strip()]
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, r[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------- distributed
+def _dist_init(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        return rank, world, local, dist
+    if n_gpus != 1:
+        print(f"warning: --gpus {n_gpus} without torchrun; running one process", file=sys.stderr)
+    return 0, 1, 0, None
+
+
+def _barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+def _max_over_ranks(x, dist):
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# -------------------------------------------------------------------------- our arm
+def _inputs(rank):
+    pc = workloads.CONFIGS[PREFILL_CFG]
+    dc = workloads.CONFIGS[DECODE_CFG]
+    pc = workloads.PrefillCase(**{**pc.__dict__, "seed": pc.seed + 100 * rank})
+    dc = workloads.DecodeCase(**{**dc.__dict__, "seed": dc.seed + 100 * rank})
+    return pc, workloads.make_prefill(pc), dc, workloads.make_decode(dc)
+
+
+def run_ours(args, rank, world, local, dist):
+    import differential_attention_v2_b200 as da
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    pc, pin, dc, din = _inputs(rank)
+    stream = torch.cuda.current_stream(dev)
+
+    # device-resident inputs and outputs
+    q, k, v, lam = (pin[x].to(dev) for x in ("q", "k", "v", "lam"))
+    out = torch.empty(pc.B, pc.S, pc.Hq // 2, pc.D, dtype=torch.bfloat16, device=dev)
+    dq, kc, vc, sl, dl = (din[x].to(dev) for x in ("q", "kcache", "vcache", "seqlens", "lam"))
+    dout = torch.empty(dc.B, dc.Hq // 2, dc.D, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(da.decode_workspace_size(dc.B, dc.Smax, dc.Hq, dc.Hkv, dc.D), dtype=torch.uint8, device=dev)
+
+    flops = workloads.prefill_flops(pc.B, pc.S, pc.Hq, pc.D, causal=True)
+    dbytes = workloads.decode_bytes(din["seqlens"].tolist(), dc.Hkv, dc.D, dc.Hq)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        da.prefill(q, k, v, lam, out=out, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        da.decode(dq, kc, vc, sl, dl, out=dout, workspace=ws, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    if da.device_error(stream) != 0:
+        raise RuntimeError("kernel reported a device-side error during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local) if rank == 0 else None
+    if clocks:
+        clocks.start()
+    _barrier(dist)
+    torch.cuda.synchronize(dev)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    _barrier(dist)
+    total_ms = t_start.elapsed_time(t_end)
+    pre_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    dec_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+    total_ms = _max_over_ranks(total_ms, dist)
+    pre_ms = _max_over_ranks(pre_ms, dist)
+    dec_ms = _max_over_ranks(dec_ms, dist)
+    err = da.device_error(stream)
+
+    # ------------------------------------------------ end to end through host buffers
+    h = {x: pin[x].pin_memory() for x in ("q", "k", "v", "lam")}
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hd = {x: din[x].pin_memory() for x in ("q", "seqlens", "lam")}
+    hd_out = torch.empty(dout.shape, dtype=dout.dtype).pin_memory()
+    e2e_steps = max(3, min(args.steps, 50))
+
+    def e2e_step():
+        for name, dst in (("q", q), ("k", k), ("v", v), ("lam", lam)):
+            dst.copy_(h[name], non_blocking=True)
+        da.prefill(q, k, v, lam, out=out, stream=stream)
+        h_out.copy_(out, non_blocking=True)
+        for name, dst in (("q", dq), ("seqlens", sl), ("lam", dl)):
+            dst.copy_(hd[name], non_blocking=True)
+        da.decode(dq, kc, vc, sl, dl, out=dout, workspace=ws, stream=stream)
+        hd_out.copy_(dout, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    _barrier(dist)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    _barrier(dist)
+    e2e_ms = _max_over_ranks(e0.elapsed_time(e1), dist)
+    clk = clocks.stop() if clocks else None
+    err |= da.device_error(stream)
+    if err:
+        raise RuntimeError(f"kernel reported device error {err}")
+
+    h2d = sum(t.numel() * t.element_size() for t in h.values()) + sum(t.numel() * t.element_size() for t in hd.values())
+    d2h = h_out.numel() * h_out.element_size() + hd_out.numel() * hd_out.element_size()
+
+    if rank != 0:
+        return None
+    peaks, peak_src = _peaks()
+    K = args.steps
+    pre_launch_ms = pre_ms / K
+    dec_launch_ms = dec_ms / K
+    tflops = flops / (pre_launch_ms * 1e-3) / 1e12
+    gbs = dbytes / (dec_launch_ms * 1e-3) / 1e9
+    value = world * flops * K / (pre_ms * 1e-3) / 1e12  # whole job: every rank's prefill FLOPs
+    dec_value = world * dbytes * K / (dec_ms * 1e-3) / 1e9
+    peak_t = peaks["bf16_tflops"]
+    tr = NCU_TRAFFIC["prefill"]
+    traffic = tr["bytes"] if tr["source_sha"] == _src_sha("prefill_sm100.cu") else None
+    trd = NCU_TRAFFIC["decode"]
+    traffic_d = trd["bytes"] if trd["source_sha"] == _src_sha("decode_sm100.cu") else None
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": max(args.warmup, 3),
+        "ms_per_step": round(total_ms / K, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic: seeded N(0,1) q/k/v rounded to bf16, lambda = sigmoid(N(0,1)) fp32, "
+                "decode lengths uniform in [1024, 8192]",
+        "config": {
+            "workload": "prefill B=4 S=4096 Hq=64 Hkv=8 D=128 causal bf16 + decode B=64 Smax=8192 "
+                        "len U[1024,8192] Hq=64 Hkv=8 D=128 bf16",
+            "prefill": {"B": pc.B, "S": pc.S, "Hq": pc.Hq, "Hkv": pc.Hkv, "D": pc.D, "causal": True,
+                        "flops_per_step": flops},
+            "decode": {"B": dc.B, "Smax": dc.Smax, "Hq": dc.Hq, "Hkv": dc.Hkv, "D": dc.D,
+                       "sum_seqlens": int(din["seqlens"].sum()), "bytes_per_step": dbytes},
+            "parallelism": f"replicas x{world} (independent per-GPU batches)",
+            "l2": "no flush: inputs larger than L2 (q 268 MB; decode streams 1.2 GB per step)",
+        },
+        "decode": {
+            "value": round(dec_value, 1), "unit": "GB/s", "us_per_step": round(1000 * dec_launch_ms, 2),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": traffic_d,
+                         "peak_source": f"{peak_src} hbm_gbs"},
+        },
+        "roofline": {
+            "bound": "tensor", "achieved": round(tflops, 2), "peak": peak_t, "unit": "TFLOP/s",
+            "frac": round(tflops / peak_t, 4), "traffic": traffic,
+            "kernel": "diffattn_prefill_sm100", "flops_per_launch": flops,
+            "launch_ms": round(pre_launch_ms, 4), "peak_source": f"{peak_src} bf16_tflops (burst)",
+        },
+        "e2e": {
+            "value": round(world * flops * e2e_steps / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+            "ms_per_step": round(e2e_ms / e2e_steps, 3),
+            "note": "prefill FLOPs over a step that copies q/k/v/lambda and the decode q/seqlens/lambda "
+                    "from pinned host memory, runs both kernels through the C ABI and copies both "
+                    "outputs back",
+        },
+        "gpu_launches": 3 * K,
+        "clocks": clk,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
+    else:
+        line["cpu_baseline"] = None
+    return line
+
+
+# ------------------------------------------------------------- the oracle on the host
+def _oracle_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _prefill_units(inp, case, n_units, seed):
+    """Time the oracle on n_units random (b, pair, 128-row tile) units of the prefill."""
+    from oracle import diffattn_f64 as ora
+    import numpy as np
+
+    rng = np.random.default_rng(seed)
+    n_tiles = case.S // 128
+    layout = ora.pair_layout(case.Hq, case.Hkv)
+    flops = 0
+    t0 = time.perf_counter()
+    for _ in range(n_units):
+        b = int(rng.integers(case.B))
+        p = int(rng.integers(case.Hq // 2))
+        t = int(rng.integers(n_tiles))
+        _, h1, h2, g = layout[p]
+        r0, r1 = 128 * t, 128 * t + 128
+        kk = inp["k"][b, :r1, g].double().numpy()
+        vv = inp["v"][b, :r1, g].double().numpy()
+        q1 = inp["q"][b, r0:r1, h1].double().numpy()
+        q2 = inp["q"][b, r0:r1, h2].double().numpy()
+        lm = inp["lam"][b, r0:r1, p].double().numpy()
+        ora.diff_attention_block(q1, q2, kk, vv, lm, ora.causal_mask(128, r1, r0))
+        flops += 4 * case.D * 2 * sum(r + 1 for r in range(r0, r1))  # both heads of the pair
+    return flops, time.perf_counter() - t0
+
+
+def _decode_seqs(inp, case, n_seqs, seed):
+    from oracle import diffattn_f64 as ora
+    import numpy as np
+
+    rng = np.random.default_rng(seed)
+    byts = 0
+    t0 = time.perf_counter()
+    for _ in range(n_seqs):
+        b = int(rng.integers(case.B))
+        n = int(inp["seqlens"][b])
+        sl = inp["seqlens"][b:b + 1]
+        ora.decode(inp["q"][b:b + 1], inp["kcache"][b:b + 1], inp["vcache"][b:b + 1], sl, inp["lam"][b:b + 1])
+        byts += n * case.Hkv * case.D * 2 * 2
+    return byts, time.perf_counter() - t0
+
+
+def cpu_baseline(seconds=15.0, inputs=None):
+    """The float64 oracle on a bounded sample of the same workload, timed on the host."""
+    pc = workloads.CONFIGS[PREFILL_CFG]
+    dc = workloads.CONFIGS[DECODE_CFG]
+    if inputs is None:
+        inputs = (workloads.make_prefill(pc), workloads.make_decode(dc))
+    pin, din = inputs
+    # calibrate with 4 units, then size the sample to about `seconds` of CPU work
+    f, t = _prefill_units(pin, pc, 4, seed=1)
+    n = max(4, int(0.8 * seconds / max(t / 4, 1e-6)))
+    f, t = _prefill_units(pin, pc, n, seed=2)
+    b, td = _decode_seqs(din, dc, 2, seed=3)
+    return {"value": round(f / t / 1e12, 6), "unit": "TFLOP/s", "cores": _oracle_threads(), "kind": "oracle",
+            "sample": f"{n} random (batch, pair, 128-row tile) units of the B=4 S=4096 prefill "
+                      f"({t:.1f} s); decode: 2 full sequences of the B=64 decode ({td:.1f} s)",
+            "decode_gbs": round(b / td / 1e9, 4)}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: each step a bounded sample of the same workload."""
+    pc = workloads.CONFIGS[PREFILL_CFG]
+    dc = workloads.CONFIGS[DECODE_CFG]
+    pin, din = workloads.make_prefill(pc), workloads.make_decode(dc)
+    units = args.ref_units
+    for i in range(args.warmup):
+        _prefill_units(pin, pc, max(1, units // 4), seed=100 + i)
+    flops, secs = 0, 0.0
+    dbytes, dsecs = 0, 0.0
+    for i in range(args.steps):
+        f, t = _prefill_units(pin, pc, units, seed=1000 + i)
+        flops += f
+        secs += t
+        b, td = _decode_seqs(din, dc, 1, seed=2000 + i)
+        dbytes += b
+        dsecs += td
+    value = flops / secs / 1e12
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1000 * (secs + dsecs) / args.steps, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic: the same seeded inputs as the GPU arm",
+        "config": {"workload": "prefill B=4 S=4096 Hq=64 Hkv=8 D=128 causal + decode B=64 Smax=8192 len "
+                               "U[1024,8192]; each step a bounded sample", "units_per_step": units},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": _oracle_threads(), "kind": "oracle",
+                         "sample": f"{units} random (batch, pair, 128-row tile) prefill units and one full decode "
+                                   f"sequence per step"},
+        "decode": {"value": round(dbytes / dsecs / 1e9, 4), "unit": "GB/s"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-units", type=int, default=24, help="prefill units per reference step")
+    args = ap.parse_args(argv)
+
+    if args.impl == "reference":
+        if int(os.environ.get("RANK", "0")) != 0:
+            return 0
+        print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    rank, world, local, dist = _dist_init(args.gpus)
+    try:
+        line = run_ours(args, rank, world, local, dist)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,189 @@
+"""ctypes binding of libdiffattn_v2.so: the same entry points as include/diffattn_v2.h.
+
+Argument marshalling only: every step of the operator runs in the CUDA library. The
+wrappers take torch CUDA tensors, check dtype/shape/contiguity, pass data pointers and the
+current (or given) stream, and raise on a non-OK status. Output tensors and the decode
+workspace are allocated with torch when the caller does not pass them.
+
+There is no CPU fallback: if the library is missing, importing fails with an error that
+says how to build it.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdiffattn_v2.so")
+
+OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_DEVICE = 0, -1, -2, -3, -4
+
+_vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+
+_SIGNATURES = {
+    "diffattn_v2_version": (_i, []),
+    "diffattn_v2_status_string": (ctypes.c_char_p, [_i]),
+    "diffattn_v2_prefill": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
+    "diffattn_v2_prefill_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
+    "diffattn_v2_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
+    "diffattn_v2_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "diffattn_v2_decode_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
+    "diffattn_v2_lambda_v1": (_i, [_vp, _vp, _vp, _vp, _f, _i, _i, _i, _vp, _vp]),
+    "diffattn_v2_device_error": (_i, [ctypes.POINTER(_i), _vp]),
+}
+EXPORTED = tuple(_SIGNATURES)
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing; build it with `python -m differential_attention_v2_b200.build` "
+            "(nvcc, sm_100a). There is no fallback implementation.")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in _SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+LIB = _load()
+
+
+class DiffAttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {LIB.diffattn_v2_status_string(status).decode()} ({status})")
+
+
+def _check(status: int, what: str):
+    if status != OK:
+        raise DiffAttnError(status, what)
+
+
+def _stream(stream, device):
+    if stream is None:
+        return torch.cuda.current_stream(device).cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _need(t, name, dtype, ndim):
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name}: expected {ndim} dimensions, got shape {tuple(t.shape)}")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+
+
+def version() -> int:
+    return LIB.diffattn_v2_version()
+
+
+def prefill(q, k, v, lam, out=None, causal=True, stream=None):
+    """bf16 prefill: q [B,S,Hq,D], k/v [B,S,Hkv,D], lam fp32 [B,S,Hq/2] -> out bf16 [B,S,Hq/2,D]."""
+    for t, n, nd in ((q, "q", 4), (k, "k", 4), (v, "v", 4)):
+        _need(t, n, torch.bfloat16, nd)
+    _need(lam, "lam", torch.float32, 3)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if out is None:
+        out = torch.empty((B, S, Hq // 2, D), dtype=torch.bfloat16, device=q.device)
+    _need(out, "out", torch.bfloat16, 4)
+    st = LIB.diffattn_v2_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(out), B, S, Hq, Hkv, D,
+                                 1 if causal else 0, _stream(stream, q.device))
+    _check(st, "diffattn_v2_prefill")
+    return out
+
+
+def prefill_f32(q, k, v, lam, out=None, causal=True, stream=None):
+    """fp32 prefill on CUDA cores; same layout as prefill with fp32 tensors."""
+    for t, n, nd in ((q, "q", 4), (k, "k", 4), (v, "v", 4), (lam, "lam", 3)):
+        _need(t, n, torch.float32, nd)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if out is None:
+        out = torch.empty((B, S, Hq // 2, D), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32, 4)
+    st = LIB.diffattn_v2_prefill_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(out), B, S, Hq, Hkv, D,
+                                     1 if causal else 0, _stream(stream, q.device))
+    _check(st, "diffattn_v2_prefill_f32")
+    return out
+
+
+def decode_workspace_size(B, Smax, Hq, Hkv, D) -> int:
+    return int(LIB.diffattn_v2_decode_workspace_size(B, Smax, Hq, Hkv, D))
+
+
+def decode(q, kcache, vcache, seqlens, lam, out=None, workspace=None, stream=None):
+    """bf16 decode step: q [B,Hq,D], caches [B,Smax,Hkv,D], seqlens int32 [B], lam fp32 [B,Hq/2]."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(kcache, "kcache", torch.bfloat16, 4)
+    _need(vcache, "vcache", torch.bfloat16, 4)
+    _need(seqlens, "seqlens", torch.int32, 1)
+    _need(lam, "lam", torch.float32, 2)
+    B, Hq, D = q.shape
+    Smax, Hkv = kcache.shape[1], kcache.shape[2]
+    if out is None:
+        out = torch.empty((B, Hq // 2, D), dtype=torch.bfloat16, device=q.device)
+    _need(out, "out", torch.bfloat16, 3)
+    need = decode_workspace_size(B, Smax, Hq, Hkv, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    st = LIB.diffattn_v2_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(lam), _ptr(out), B, Smax,
+                                Hq, Hkv, D, _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                _stream(stream, q.device))
+    _check(st, "diffattn_v2_decode")
+    return out
+
+
+def decode_f32(q, kcache, vcache, seqlens, lam, out=None, stream=None):
+    """fp32 decode step on CUDA cores; same layout as decode with fp32 tensors."""
+    _need(q, "q", torch.float32, 3)
+    _need(kcache, "kcache", torch.float32, 4)
+    _need(vcache, "vcache", torch.float32, 4)
+    _need(seqlens, "seqlens", torch.int32, 1)
+    _need(lam, "lam", torch.float32, 2)
+    B, Hq, D = q.shape
+    Smax, Hkv = kcache.shape[1], kcache.shape[2]
+    if out is None:
+        out = torch.empty((B, Hq // 2, D), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32, 3)
+    st = LIB.diffattn_v2_decode_f32(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(lam), _ptr(out), B,
+                                    Smax, Hq, Hkv, D, _stream(stream, q.device))
+    _check(st, "diffattn_v2_decode_f32")
+    return out
+
+
+def lambda_v1(lq1, lk1, lq2, lk2, lambda_init=0.8, rows=1, out=None, stream=None):
+    """V1 lambda per pair, broadcast to `rows` rows: out fp32 [rows, n_pairs]."""
+    for t, n in ((lq1, "lq1"), (lk1, "lk1"), (lq2, "lq2"), (lk2, "lk2")):
+        _need(t, n, torch.float32, 2)
+    n_pairs, d = lq1.shape
+    if out is None:
+        out = torch.empty((rows, n_pairs), dtype=torch.float32, device=lq1.device)
+    if out.dtype != torch.float32 or not out.is_contiguous() or out.numel() != rows * n_pairs:
+        raise ValueError("out must be a contiguous fp32 tensor with rows*n_pairs elements")
+    st = LIB.diffattn_v2_lambda_v1(_ptr(lq1), _ptr(lk1), _ptr(lq2), _ptr(lk2), float(lambda_init), n_pairs, d, rows,
+                                   _ptr(out), _stream(stream, lq1.device))
+    _check(st, "diffattn_v2_lambda_v1")
+    return out
+
+
+def device_error(stream=None, device=None) -> int:
+    """Synchronise the stream and return (and clear) the kernels' device error word."""
+    code = ctypes.c_int(0)
+    st = LIB.diffattn_v2_device_error(ctypes.byref(code), _stream(stream, device))
+    if st == ERR_CUDA:
+        raise DiffAttnError(st, "diffattn_v2_device_error")
+    return code.value

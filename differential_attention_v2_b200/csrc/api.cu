@@ -1,0 +1,227 @@
+// api.cu -- the C ABI of include/diffattn_v2.h: argument checks, TMA descriptor encoding,
+// split planning and kernel dispatch. No allocation, no state beyond a per-device cache of
+// the device error word's address.
+
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "../../include/diffattn_v2.h"
+#include "internal.h"
+
+namespace {
+
+// Device error word that kernels set (atomicCAS from 0) when a bounded wait expires.
+__device__ int g_device_error = 0;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int* g_err_ptr[kMaxDevices] = {};
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int status_of(cudaError_t e) { return e == cudaSuccess ? DA2_OK : DA2_ERR_CUDA; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Address of the device error word on the current device.
+cudaError_t device_error_ptr(int** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_err_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_device_error);
+    if (e != cudaSuccess) return e;
+    g_err_ptr[dev] = static_cast<int*>(p);
+  }
+  *out = g_err_ptr[dev];
+  return cudaSuccess;
+}
+
+cudaError_t get_encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_encode) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (e != cudaSuccess) return e;
+    if (q != cudaDriverEntryPointSuccess || !p) return cudaErrorNotSupported;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  *fn = g_encode;
+  return cudaSuccess;
+}
+
+// 4-D bf16 tensor map over a [d3, d2, d1, d0] row-major array (d0 = D innermost), box
+// {box0, 1, box2, 1}, 128-byte swizzle, out-of-range elements read as zero.
+cudaError_t encode_bshd(CUtensorMap* map, const void* base, uint64_t D, uint64_t H, uint64_t S, uint64_t B,
+                        uint32_t box0, uint32_t box2) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  cudaError_t e = get_encoder(&enc);
+  if (e != cudaSuccess) return e;
+  const cuuint64_t dims[4] = {D, H, S, B};
+  const cuuint64_t strides[3] = {D * 2, H * D * 2, S * H * D * 2};  // bytes, dims 1..3
+  const cuuint32_t box[4] = {box0, 1, box2, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// Shape checks shared by prefill and decode: sizes positive, Hq even, pairs inside groups.
+bool heads_ok(int Hq, int Hkv) { return Hq > 0 && Hkv > 0 && (Hq % 2) == 0 && (Hq % (2 * Hkv)) == 0; }
+
+}  // namespace
+
+namespace da2 {
+
+void decode_split_plan(int B, int Smax, int Hkv, int* split_len, int* nsplit) {
+  // Aim for about 8 waves of 2 CTAs per SM over the (b, g) units, with splits that are a
+  // multiple of the 64-token stage and between 512 and 4096 tokens long.
+  const long long units = static_cast<long long>(B) * Hkv;
+  const long long target_ctas = 148LL * 2 * 8;
+  long long L = (static_cast<long long>(Smax) * units + target_ctas - 1) / target_ctas;
+  L = ((L + 63) / 64) * 64;
+  if (L < 512) L = 512;
+  if (L > 4096) L = 4096;
+  *split_len = static_cast<int>(L);
+  *nsplit = static_cast<int>((Smax + L - 1) / L);
+}
+
+}  // namespace da2
+
+extern "C" {
+
+int diffattn_v2_version(void) { return 100; }
+
+const char* diffattn_v2_status_string(int status) {
+  switch (status) {
+    case DA2_OK: return "ok";
+    case DA2_ERR_INVALID: return "invalid argument";
+    case DA2_ERR_UNSUPPORTED: return "unsupported configuration";
+    case DA2_ERR_CUDA: return "CUDA runtime error";
+    case DA2_ERR_DEVICE: return "kernel reported a device-side error";
+    default: return "unknown status";
+  }
+}
+
+int diffattn_v2_prefill(const void* q, const void* k, const void* v, const float* lambda, void* out, int B, int S,
+                        int Hq, int Hkv, int D, int causal, da2_stream_t stream) {
+  if (B < 0 || S < 0 || D <= 0 || !heads_ok(Hq, Hkv)) return DA2_ERR_INVALID;
+  if (causal != 0 && causal != 1) return DA2_ERR_INVALID;
+  if (B == 0 || S == 0) return DA2_OK;
+  if (!q || !k || !v || !lambda || !out) return DA2_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(lambda) || !aligned16(out))
+    return DA2_ERR_INVALID;
+  if (D != 128) return DA2_ERR_UNSUPPORTED;
+  if ((S + 127) / 128 > 65535) return DA2_ERR_UNSUPPORTED;
+  int* err = nullptr;
+  cudaError_t e = device_error_ptr(&err);
+  if (e != cudaSuccess) return DA2_ERR_CUDA;
+  CUtensorMap tq, tk, tv;
+  if (encode_bshd(&tq, q, D, Hq, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  if (encode_bshd(&tk, k, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  if (encode_bshd(&tv, v, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  e = da2::launch_prefill(tq, tk, tv, lambda, static_cast<__nv_bfloat16*>(out), err, B, S, Hq, Hkv, causal,
+                          reinterpret_cast<cudaStream_t>(stream));
+  return status_of(e);
+}
+
+int diffattn_v2_prefill_f32(const float* q, const float* k, const float* v, const float* lambda, float* out, int B,
+                            int S, int Hq, int Hkv, int D, int causal, da2_stream_t stream) {
+  if (B < 0 || S < 0 || D <= 0 || !heads_ok(Hq, Hkv)) return DA2_ERR_INVALID;
+  if (causal != 0 && causal != 1) return DA2_ERR_INVALID;
+  if (B == 0 || S == 0) return DA2_OK;
+  if (!q || !k || !v || !lambda || !out) return DA2_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(lambda) || !aligned16(out))
+    return DA2_ERR_INVALID;
+  if (D != 64 && D != 128) return DA2_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * (Hq / 2) > 65535) return DA2_ERR_UNSUPPORTED;
+  return status_of(da2::launch_prefill_f32(q, k, v, lambda, out, B, S, Hq, Hkv, D, causal,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t diffattn_v2_decode_workspace_size(int B, int Smax, int Hq, int Hkv, int D) {
+  if (B <= 0 || Smax <= 0 || D <= 0 || !heads_ok(Hq, Hkv)) return 0;
+  int split_len = 0, nsplit = 0;
+  da2::decode_split_plan(B, Smax, Hkv, &split_len, &nsplit);
+  const size_t rows = static_cast<size_t>(B) * Hq * nsplit;
+  return rows * static_cast<size_t>(D) * sizeof(float) + rows * 2 * sizeof(float);
+}
+
+int diffattn_v2_decode(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens,
+                       const float* lambda, void* out, int B, int Smax, int Hq, int Hkv, int D, void* workspace,
+                       size_t workspace_bytes, da2_stream_t stream) {
+  if (B < 0 || Smax <= 0 || D <= 0 || !heads_ok(Hq, Hkv)) return DA2_ERR_INVALID;
+  if (B == 0) return DA2_OK;
+  if (!q || !kcache || !vcache || !seqlens || !lambda || !out || !workspace) return DA2_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(seqlens) || !aligned16(lambda) ||
+      !aligned16(out) || !aligned16(workspace))
+    return DA2_ERR_INVALID;
+  if (workspace_bytes < diffattn_v2_decode_workspace_size(B, Smax, Hq, Hkv, D)) return DA2_ERR_INVALID;
+  const int group = Hq / Hkv;
+  if (D != 128 || !(group == 2 || group == 4 || group == 8 || group == 16)) return DA2_ERR_UNSUPPORTED;
+  if (B > 65535 || Hkv > 65535) return DA2_ERR_UNSUPPORTED;
+  int* err = nullptr;
+  cudaError_t e = device_error_ptr(&err);
+  if (e != cudaSuccess) return DA2_ERR_CUDA;
+  int split_len = 0, nsplit = 0;
+  da2::decode_split_plan(B, Smax, Hkv, &split_len, &nsplit);
+  CUtensorMap tk, tv;
+  if (encode_bshd(&tk, kcache, D, Hkv, Smax, B, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
+  if (encode_bshd(&tv, vcache, D, Hkv, Smax, B, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
+  float* ws_o = static_cast<float*>(workspace);
+  float* ws_ml = ws_o + static_cast<size_t>(B) * Hq * nsplit * D;
+  e = da2::launch_decode(tk, tv, static_cast<const __nv_bfloat16*>(q), seqlens, lambda,
+                         static_cast<__nv_bfloat16*>(out), ws_o, ws_ml, err, B, Smax, Hq, Hkv, nsplit, split_len,
+                         reinterpret_cast<cudaStream_t>(stream));
+  return status_of(e);
+}
+
+int diffattn_v2_decode_f32(const float* q, const float* kcache, const float* vcache, const int32_t* seqlens,
+                           const float* lambda, float* out, int B, int Smax, int Hq, int Hkv, int D,
+                           da2_stream_t stream) {
+  if (B < 0 || Smax <= 0 || D <= 0 || !heads_ok(Hq, Hkv)) return DA2_ERR_INVALID;
+  if (B == 0) return DA2_OK;
+  if (!q || !kcache || !vcache || !seqlens || !lambda || !out) return DA2_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(seqlens) || !aligned16(lambda) ||
+      !aligned16(out))
+    return DA2_ERR_INVALID;
+  if (D != 64 && D != 128) return DA2_ERR_UNSUPPORTED;
+  return status_of(da2::launch_decode_f32(q, kcache, vcache, seqlens, lambda, out, B, Smax, Hq, Hkv, D,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int diffattn_v2_lambda_v1(const float* lq1, const float* lk1, const float* lq2, const float* lk2, float lambda_init,
+                          int n_pairs, int d, int rows, float* lambda_out, da2_stream_t stream) {
+  if (n_pairs <= 0 || d <= 0 || rows < 0) return DA2_ERR_INVALID;
+  if (rows == 0) return DA2_OK;
+  if (!lq1 || !lk1 || !lq2 || !lk2 || !lambda_out) return DA2_ERR_INVALID;
+  if (!aligned16(lq1) || !aligned16(lk1) || !aligned16(lq2) || !aligned16(lk2) || !aligned16(lambda_out))
+    return DA2_ERR_INVALID;
+  return status_of(da2::launch_lambda_v1(lq1, lk1, lq2, lk2, lambda_init, n_pairs, d, rows, lambda_out,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int diffattn_v2_device_error(int* code, da2_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return DA2_ERR_CUDA;
+  int* err = nullptr;
+  e = device_error_ptr(&err);
+  if (e != cudaSuccess) return DA2_ERR_CUDA;
+  int h = 0;
+  e = cudaMemcpy(&h, err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return DA2_ERR_CUDA;
+  if (h != 0) {
+    const int zero = 0;
+    e = cudaMemcpy(err, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return DA2_ERR_CUDA;
+  }
+  if (code) *code = h;
+  return h ? DA2_ERR_DEVICE : DA2_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,39 @@
+// internal.h -- host-side launchers shared between the C ABI (api.cu) and the kernel files.
+// Not installed; the public interface is include/diffattn_v2.h.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace da2 {
+
+// bf16 prefill on tcgen05 (D = 128). Tensor maps: Q over [B,S,Hq,D], K/V over [B,S,Hkv,D],
+// boxes of 64 (d) x 1 (head) x 128 (rows) x 1, 128-byte swizzle.
+cudaError_t launch_prefill(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                           const float* lambda, __nv_bfloat16* out, int* err, int B, int S, int Hq, int Hkv,
+                           int causal, cudaStream_t stream);
+
+// bf16 decode (D = 128): split kernel + combine. Tensor maps over the caches [B,Smax,Hkv,D],
+// boxes of 64 (d) x 1 x 64 (tokens) x 1, 128-byte swizzle.
+cudaError_t launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const __nv_bfloat16* q,
+                          const int32_t* seqlens, const float* lambda, __nv_bfloat16* out, float* ws_o,
+                          float* ws_ml, int* err, int B, int Smax, int Hq, int Hkv, int nsplit,
+                          int split_len, cudaStream_t stream);
+
+// Tokens per split and number of splits of the bf16 decode for these sizes.
+void decode_split_plan(int B, int Smax, int Hkv, int* split_len, int* nsplit);
+
+// fp32 CUDA-core paths (D in {64, 128}).
+cudaError_t launch_prefill_f32(const float* q, const float* k, const float* v, const float* lambda, float* out,
+                               int B, int S, int Hq, int Hkv, int D, int causal, cudaStream_t stream);
+cudaError_t launch_decode_f32(const float* q, const float* kc, const float* vc, const int32_t* seqlens,
+                              const float* lambda, float* out, int B, int Smax, int Hq, int Hkv, int D,
+                              cudaStream_t stream);
+
+// V1 lambda, broadcast to `rows` rows.
+cudaError_t launch_lambda_v1(const float* lq1, const float* lk1, const float* lq2, const float* lk2,
+                             float lambda_init, int n_pairs, int d, int rows, float* out, cudaStream_t stream);
+
+}  // namespace da2

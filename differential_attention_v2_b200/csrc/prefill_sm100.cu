@@ -1,0 +1,385 @@
+// prefill_sm100.cu -- bf16 DiffAttn V2 prefill on the 5th-generation tensor cores (sm_100a).
+//
+// Operator ("Differential Attention (V2)" lesson, "The differential concept"; causal mask of
+// the "Attention variants" lesson, Step 1; V2 pairing of "Differential Transformer V2 soll
+// KI-Training stabiler machen", shared-KV section):
+//   out[b,i,p] = softmax(q[b,i,2p] K_g^T/sqrt(D)) V_g - lambda[b,i,p] softmax(q[b,i,2p+1] K_g^T/sqrt(D)) V_g
+//
+// One CTA computes a 128-row query tile of one pair (both heads) of one batch element.
+// Each 128x128 K and V tile of the shared KV head is brought into shared memory by TMA
+// ONCE and feeds both heads. The four GEMM blocks per KV tile run on tcgen05 with fp32
+// accumulators in tensor memory:
+//
+//   TMEM columns   [  0,128) S1 = Q1 K^T   (P1, bf16, is written over its first 64 columns)
+//                  [128,256) S2 = Q2 K^T   (P2 likewise)
+//                  [256,384) O1 += P1 V
+//                  [384,512) O2 += P2 V
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax of branch 1 (head 2p): thread r owns query row r of the tile
+//   warps 4-7  softmax of branch 2 (head 2p+1)
+//   warp 8     TMA producer (Q once, then K/V tiles through a 2-stage ring)
+//   warp 9     tcgen05 MMA issuer; also allocates and frees tensor memory
+//
+// Issue order on the tensor core for KV tile j: S1_j, PV2_{j-1}, S2_j, PV1_j. Softmax of
+// branch 1 on S1_j overlaps PV2_{j-1} and S2_j; softmax of branch 2 on S2_j overlaps PV1_j
+// and S1_{j+1}. tcgen05.mma instructions from one thread execute in issue order, so S_b(j+1)
+// overwrites the P_b(j) columns only after PV_b(j) has read them.
+//
+// Online softmax per branch in the log2 domain: x = s * log2(e)/sqrt(D), P = 2^(x - m).
+// The running max m is raised only when a row's max exceeds it by more than 8 (a factor of
+// 256); then O and l are rescaled by 2^(m_old - m_new). O/l is the same for any such m, so
+// this is exact up to rounding while skipping most rescales. The epilogue forms
+// O1/l1 - lambda O2/l2 in fp32 and rounds once to bf16.
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace da2 {
+namespace prefill {
+
+constexpr int BM = 128;  // query rows per CTA
+constexpr int BN = 128;  // keys per KV tile
+constexpr int HD = 128;  // head dim
+constexpr int kThreads = 320;
+constexpr int kStages = 2;
+
+constexpr uint32_t kChunkBytes = 128 * 64 * 2;     // 128 rows x 64 bf16 (one swizzle-128B half)
+constexpr uint32_t kTileBytes = 2 * kChunkBytes;   // 128 rows x 128 bf16
+
+constexpr uint32_t kOffQ = 0;                                 // Q1, Q2
+constexpr uint32_t kOffK = kOffQ + 2 * kTileBytes;            // K stages
+constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;      // V stages
+constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;    // mbarriers
+constexpr uint32_t kOffMisc = kOffBar + 256;                  // tmem slot, abort flag
+constexpr uint32_t kOffL = kOffMisc + 64;                     // 2 x 128 fp32 row sums
+constexpr uint32_t kSmemUsed = kOffL + 2 * BM * 4;
+constexpr uint32_t kSmemBytes = kSmemUsed + 1024;             // slack for 1024-B alignment
+
+// mbarrier slots (8 bytes each)
+enum Bar : int {
+  kQFull = 0,
+  kKFull = 1,    // +stage
+  kKEmpty = 3,   // +stage
+  kVFull = 5,    // +stage
+  kVEmpty = 7,   // +stage
+  kSFull = 9,    // +branch
+  kPFull = 11,   // +branch
+  kOFull = 13,
+  kDrain = 14,
+  kNumBars = 15
+};
+
+constexpr uint32_t kTmS1 = 0, kTmS2 = 128, kTmO1 = 256, kTmO2 = 384;
+
+struct Params {
+  const float* lambda;    // [B,S,Hq/2]
+  __nv_bfloat16* out;     // [B,S,Hq/2,D]
+  int* err;               // device error word
+  int B, S, Hq, Hkv, causal;
+  int n_row_tiles;
+  float scale_log2;       // log2(e)/sqrt(D)
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sbase + kOffBar + 8u * static_cast<uint32_t>(i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);
+  float* l_xchg = reinterpret_cast<float*>(smem + kOffL);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // heaviest row tiles first: blockIdx.y runs slowest in the launch order
+  const int tile = p.n_row_tiles - 1 - static_cast<int>(blockIdx.y);
+  const int n_pairs = p.Hq >> 1;
+  const int b = static_cast<int>(blockIdx.x) / n_pairs;
+  const int pair = static_cast<int>(blockIdx.x) % n_pairs;
+  const int group = p.Hq / p.Hkv;
+  const int g = (2 * pair) / group;
+  const int m0 = tile * BM;
+  const int n_kv_total = (p.S + BN - 1) / BN;
+  const int n_kv = p.causal ? min(tile + 1, n_kv_total) : n_kv_total;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kNumBars; ++i) {
+      uint32_t count = 1;
+      if (i == kPFull || i == kPFull + 1) count = 128;  // every softmax thread of the branch
+      mbar_init(bar(i), count);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar(kQFull), 2 * kTileBytes);
+      for (int h = 0; h < 2; ++h)
+        for (int c = 0; c < 2; ++c)
+          tma_load_4d(sbase + kOffQ + h * kTileBytes + c * kChunkBytes, &tmQ, bar(kQFull), c * 64,
+                      2 * pair + h, m0, b);
+      int k_issued = 0, v_issued = 0;
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (!mbar_wait(bar(kKEmpty + s), ph ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(kKFull + s), kTileBytes);
+        for (int c = 0; c < 2; ++c)
+          tma_load_4d(sbase + kOffK + s * kTileBytes + c * kChunkBytes, &tmK, bar(kKFull + s), c * 64, g,
+                      j * BN, b);
+        k_issued = j + 1;
+        if (!mbar_wait(bar(kVEmpty + s), ph ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(kVFull + s), kTileBytes);
+        for (int c = 0; c < 2; ++c)
+          tma_load_4d(sbase + kOffV + s * kTileBytes + c * kChunkBytes, &tmV, bar(kVFull + s), c * 64, g,
+                      j * BN, b);
+        v_issued = j + 1;
+      }
+      if (*abort_flag) {
+        // let copies still in flight land before the CTA's shared memory is released
+        volatile int no_abort = 0;
+        mbar_wait(bar(kQFull), 0, &no_abort);
+        for (int j = max(0, k_issued - kStages); j < k_issued; ++j)
+          mbar_wait(bar(kKFull + (j & 1)), (j >> 1) & 1, &no_abort);
+        for (int j = max(0, v_issued - kStages); j < v_issued; ++j)
+          mbar_wait(bar(kVFull + (j & 1)), (j >> 1) & 1, &no_abort);
+      }
+    }
+  } else if (warp == 9) {
+    // -------------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, HD, true);
+      auto desc_q = [&](int h, int kk) {
+        return sdesc_sw128(sbase + kOffQ + h * kTileBytes + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024);
+      };
+      auto desc_k = [&](int s, int kk) {
+        return sdesc_sw128(sbase + kOffK + s * kTileBytes + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024);
+      };
+      // V tile: keys x d with d contiguous (MN-major B operand); 16 keys per K-step.
+      auto desc_v = [&](int s, int kk) {
+        return sdesc_sw128(sbase + kOffV + s * kTileBytes + kk * 2048, kChunkBytes, 1024);
+      };
+      bool ok = mbar_wait(bar(kQFull), 0, abort_flag);
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const int s = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (!(ok = mbar_wait(bar(kKFull + s), ph, abort_flag))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk)
+          mma_bf16_ss(tmem + kTmS1, desc_q(0, kk), desc_k(s, kk), idesc_qk, kk > 0 ? 1u : 0u);
+        tc_commit(bar(kSFull + 0));
+        if (j > 0) {
+          const int sp = (j - 1) & 1;
+          if (!(ok = mbar_wait(bar(kPFull + 1), (j - 1) & 1, abort_flag))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            mma_bf16_ts(tmem + kTmO2, tmem + kTmS2 + kk * 8, desc_v(sp, kk), idesc_pv,
+                        (j - 1 > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(bar(kVEmpty + sp));
+        }
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk)
+          mma_bf16_ss(tmem + kTmS2, desc_q(1, kk), desc_k(s, kk), idesc_qk, kk > 0 ? 1u : 0u);
+        tc_commit(bar(kSFull + 1));
+        tc_commit(bar(kKEmpty + s));
+        if (!(ok = mbar_wait(bar(kVFull + s), ph, abort_flag))) break;
+        if (!(ok = mbar_wait(bar(kPFull + 0), j & 1, abort_flag))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_bf16_ts(tmem + kTmO1, tmem + kTmS1 + kk * 8, desc_v(s, kk), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+      }
+      if (ok) {
+        const int jl = n_kv - 1;
+        const int sl = jl & 1;
+        if (mbar_wait(bar(kPFull + 1), jl & 1, abort_flag)) {
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            mma_bf16_ts(tmem + kTmO2, tmem + kTmS2 + kk * 8, desc_v(sl, kk), idesc_pv, (jl > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(bar(kOFull));
+        }
+      }
+      // every MMA of this CTA must be complete before tensor memory is freed
+      tc_commit(bar(kDrain));
+      volatile int no_abort = 0;
+      mbar_wait(bar(kDrain), 0, &no_abort);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int br = warp >> 2;               // branch 0 (head 2p) or 1 (head 2p+1)
+    const int r = threadIdx.x & 127;        // row of the tile == TMEM lane
+    const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t s_col = br ? kTmS2 : kTmS1;
+    const uint32_t o_col = br ? kTmO2 : kTmO1;
+    const int qi = m0 + r;                  // global query index of this row
+    float m_run = -INFINITY;
+    float l_run = 0.f;
+    bool ok = true;
+
+    for (int j = 0; j < n_kv; ++j) {
+      if (!(ok = mbar_wait(bar(kSFull + br), j & 1, abort_flag))) break;
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(trow + s_col + 32 * c, sr[c]);
+      tmem_ld_wait(sr[0]);
+      reg_fence(sr[1]);
+      reg_fence(sr[2]);
+      reg_fence(sr[3]);
+
+      const bool need_mask = (p.causal && j == tile) || ((j + 1) * BN > p.S);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          float x = __uint_as_float(sr[c][e]) * p.scale_log2;
+          if (need_mask) {
+            const int key = j * BN + 32 * c + e;
+            if ((p.causal && key > qi) || key >= p.S) x = -INFINITY;
+          }
+          sr[c][e] = __float_as_uint(x);
+          mx = fmaxf(mx, x);
+        }
+      }
+      // raise the running max only when the tile's max exceeds it by more than 2^8
+      const bool rescale = mx > m_run + 8.f;
+      float alpha = 1.f;
+      if (rescale) {
+        alpha = fast_exp2(m_run - mx);  // 0 on the first tile
+        l_run *= alpha;
+        m_run = mx;
+      }
+      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+      float lsum = 0.f;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = 2 * half + cc;
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float p0 = fast_exp2(__uint_as_float(sr[c][e]) - m_use);
+            const float p1 = fast_exp2(__uint_as_float(sr[c][e + 1]) - m_use);
+            lsum += p0 + p1;
+            pk[cc * 16 + (e >> 1)] = pack_bf16x2(p0, p1);
+          }
+        }
+        // P for keys 64*half .. 64*half+63 -> columns 32*half .. 32*half+31 (bf16 pairs)
+        tmem_st_32x32b_x32(trow + s_col + 32 * half, pk);
+      }
+      l_run += lsum;
+      if (rescale && j > 0) {
+        // O_b holds the sum up to tile j-1, complete: S_b(j) was committed after PV_b(j-1),
+        // and PV_b(j) is issued only after this thread arrives on P_full below
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld_32x32b_x32(trow + o_col + 32 * c, o);
+          tmem_ld_wait(o);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st_32x32b_x32(trow + o_col + 32 * c, o);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(kPFull + br));
+    }
+
+    if (ok) ok = mbar_wait(bar(kOFull), 0, abort_flag);
+    l_xchg[br * BM + r] = l_run;
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    if (ok && !*abort_flag) {
+      tc_fence_after();
+      const float inv1 = 1.f / l_xchg[r];
+      const float inv2 = 1.f / l_xchg[BM + r];
+      const bool row_valid = qi < p.S;
+      const size_t row_off = (static_cast<size_t>(b) * p.S + (row_valid ? qi : 0)) * n_pairs + pair;
+      const float lam = row_valid ? __ldg(p.lambda + row_off) : 0.f;
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
+        const uint32_t col = 64 * br + 32 * cc;
+        uint32_t o1[32], o2[32];
+        tmem_ld_32x32b_x32(trow + kTmO1 + col, o1);
+        tmem_ld_32x32b_x32(trow + kTmO2 + col, o2);
+        tmem_ld_wait(o1);
+        reg_fence(o2);
+        uint32_t packed[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          // each branch normalised with its own rounding, then one fused subtract: equal
+          // branches (Q1 == Q2, lambda == 1) cancel exactly
+          const float y0 = __fmaf_rn(-lam, __fmul_rn(__uint_as_float(o2[e]), inv2), __fmul_rn(__uint_as_float(o1[e]), inv1));
+          const float y1 = __fmaf_rn(-lam, __fmul_rn(__uint_as_float(o2[e + 1]), inv2),
+                                     __fmul_rn(__uint_as_float(o1[e + 1]), inv1));
+          packed[e >> 1] = pack_bf16x2(y0, y1);
+        }
+        if (row_valid) {
+          uint4* dst = reinterpret_cast<uint4*>(p.out + row_off * HD + col);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) atomicCAS(p.err, 0, kErrPrefillWait);
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace prefill
+
+cudaError_t launch_prefill(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                           const float* lambda, __nv_bfloat16* out, int* err, int B, int S, int Hq, int Hkv,
+                           int causal, cudaStream_t stream) {
+  using namespace prefill;
+  Params p;
+  p.lambda = lambda;
+  p.out = out;
+  p.err = err;
+  p.B = B;
+  p.S = S;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.causal = causal;
+  p.n_row_tiles = (S + BM - 1) / BM;
+  p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HD));
+  cudaError_t e = cudaFuncSetAttribute(diffattn_prefill_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid(B * (Hq / 2), p.n_row_tiles);
+  diffattn_prefill_sm100<<<grid, kThreads, kSmemBytes, stream>>>(tmQ, tmK, tmV, p);
+  return cudaGetLastError();
+}
+
+}  // namespace da2

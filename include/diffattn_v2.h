@@ -1,0 +1,168 @@
+/*
+ * diffattn_v2.h -- C ABI of the forward Differential Attention V2 operator for NVIDIA B200
+ * (sm_100a).
+ *
+ * What the operator computes. For every batch element b, every query row i and every pair
+ * p of adjacent query heads (h1 = 2p, h2 = 2p+1), which share one key/value head
+ * g = 2p / (Hq/Hkv) of the grouped-query layout:
+ *
+ *     A1 = softmax(q[b,i,h1] . K_g^T / sqrt(D))      A2 = softmax(q[b,i,h2] . K_g^T / sqrt(D))
+ *     out[b,i,p] = (A1 - lambda[b,i,p] * A2) . V_g
+ *
+ * over the keys visible from row i (causal: j <= i; decode: j < seqlens[b]).
+ * Sources: "Differential Attention (V2)" lesson (AI Engineering from Scratch), section
+ * "The differential concept" (equations for A1, A2 and DiffAttn); "Attention variants"
+ * lesson, "Build it", Steps 1 and 4 (causal mask, causal diff_attention); "Differential
+ * Transformer V2 soll KI-Training stabiler machen", sections "Gemeinsamer KV-Cache statt
+ * Spezialkernel" (adjacent heads of one GQA group share K/V) and "Weniger Ausreisser und
+ * Gradientenspitzen" (a sigmoid-bounded lambda per token and per head).
+ *
+ * Conventions shared by every entry point:
+ *   - Layout "BSHD": row-major, contiguous, the head dimension D innermost.
+ *       prefill  q [B,S,Hq,D]   k, v [B,S,Hkv,D]   lambda fp32 [B,S,Hq/2]   out [B,S,Hq/2,D]
+ *       decode   q [B,Hq,D]     kcache, vcache [B,Smax,Hkv,D]   seqlens int32 [B]
+ *                lambda fp32 [B,Hq/2]   out [B,Hq/2,D]
+ *   - Pairing contract: Hq is even and a multiple of 2*Hkv, so both heads of a pair sit in
+ *     the same KV group. Head 2p is the first (+) branch, head 2p+1 the subtracted one.
+ *   - Every pointer is a DEVICE pointer (or managed memory) unless stated otherwise. The
+ *     caller owns every buffer and the stream; the library never allocates, frees or keeps
+ *     a pointer after the call returns.
+ *   - Calls are asynchronous on `stream` (NULL = the legacy default stream) and reentrant:
+ *     the library holds no per-call state. A return of DA2_OK means the work was enqueued.
+ *   - Argument checks happen on the host before anything is launched; a failed check
+ *     returns an error and launches nothing. Null pointers, sizes <= 0 (except the B == 0
+ *     or S == 0 no-op), an odd Hq, Hq % (2*Hkv) != 0, pointers not 16-byte aligned and a
+ *     too-small workspace give DA2_ERR_INVALID. Valid shapes the kernels do not implement
+ *     give DA2_ERR_UNSUPPORTED. A failed CUDA call gives DA2_ERR_CUDA.
+ *   - Kernels never trap. Every wait inside a kernel is bounded; on expiry the kernel
+ *     records an error word on the device and returns. diffattn_v2_device_error() reads
+ *     and clears it.
+ *   - The score scale is 1/sqrt(D) for both branches. lambda may be any finite fp32
+ *     value (the V2 sigmoid-bounded value in (0,1), or a V1 value that may be negative or
+ *     above 1).
+ */
+#ifndef DIFFATTN_V2_H_
+#define DIFFATTN_V2_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__) || defined(__clang__)
+#define DA2_API __attribute__((visibility("default")))
+#else
+#define DA2_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Opaque CUDA stream handle; identical to cudaStream_t / CUstream. */
+typedef struct CUstream_st* da2_stream_t;
+
+/* Status codes returned by every entry point. */
+enum {
+  DA2_OK = 0,
+  DA2_ERR_INVALID = -1,     /* an argument failed a host-side check; nothing launched   */
+  DA2_ERR_UNSUPPORTED = -2, /* valid arguments this build does not implement            */
+  DA2_ERR_CUDA = -3,        /* a CUDA runtime call failed (launch, attribute, symbol)   */
+  DA2_ERR_DEVICE = -4       /* a kernel recorded an internal error (bounded wait expired) */
+};
+
+/* Library version: 100 * major + minor. */
+DA2_API int diffattn_v2_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+DA2_API const char* diffattn_v2_status_string(int status);
+
+/*
+ * Causal (or full) prefill, bf16 in / bf16 out, fp32 accumulation and softmax.
+ * Source: "The differential concept" (DiffAttn = (A1 - lambda A2) V) with the causal
+ * mask of the attention-variants lesson, Step 1, and the V2 head pairing above.
+ *   q      bf16 [B,S,Hq,D]        k, v  bf16 [B,S,Hkv,D]
+ *   lambda fp32 [B,S,Hq/2]        out   bf16 [B,S,Hq/2,D] (fully overwritten)
+ *   causal 1: key j visible from query i iff j <= i (Sq == Sk == S); 0: all S keys visible.
+ * Supported: D == 128. Other D give DA2_ERR_UNSUPPORTED. Each (b, p) output row is
+ * O1/l1 - lambda*O2/l2 formed in fp32 and rounded once to bf16 (round to nearest even).
+ * Kernel: tcgen05 tensor-core MMAs with TMEM accumulators, TMA-staged K/V tiles loaded
+ * once per pair, two online softmaxes. B == 0 or S == 0 is a no-op returning DA2_OK.
+ */
+DA2_API int diffattn_v2_prefill(const void* q, const void* k, const void* v, const float* lambda,
+                        void* out, int B, int S, int Hq, int Hkv, int D, int causal,
+                        da2_stream_t stream);
+
+/*
+ * The same operator in fp32 end to end (CUDA-core arithmetic, no tensor cores), for
+ * callers that need results within ~1e-5 of exact. q, k, v, out are fp32 with the prefill
+ * layout above. Supported: D in {64, 128}. Same argument checks and semantics.
+ */
+DA2_API int diffattn_v2_prefill_f32(const float* q, const float* k, const float* v,
+                            const float* lambda, float* out, int B, int S, int Hq, int Hkv,
+                            int D, int causal, da2_stream_t stream);
+
+/*
+ * Workspace (bytes) that diffattn_v2_decode needs for these sizes: the per-split partial
+ * results (running max, running sum and unnormalised output of each head), fp32. Returns 0
+ * for invalid sizes. The workspace holds no state between calls.
+ */
+DA2_API size_t diffattn_v2_decode_workspace_size(int B, int Smax, int Hq, int Hkv, int D);
+
+/*
+ * One decode step, bf16 in / bf16 out: the new token of each sequence attends to its
+ * cached keys [0, seqlens[b]) (the new key and value are already appended by the caller).
+ * Source: "Differential Attention (V2)" lesson, "V1 vs V2" (the KV cache is read once per
+ * step for both branches; arithmetic intensity doubles) and the DiffAttn equation.
+ *   q        bf16 [B,Hq,D]            kcache, vcache bf16 [B,Smax,Hkv,D]
+ *   seqlens  int32 [B] (device), each clamped on the device to [0, Smax]
+ *   lambda   fp32 [B,Hq/2]            out bf16 [B,Hq/2,D] (fully overwritten)
+ *   workspace device buffer of at least diffattn_v2_decode_workspace_size() bytes,
+ *            16-byte aligned, owned by the caller; calls that share one workspace must not
+ *            overlap on the GPU.
+ * A sequence with seqlens[b] == 0 gets an all-zero output. Supported: D == 128 and a GQA
+ * group size Hq/Hkv in {2, 4, 8, 16}. Kernels: a split-KV streaming kernel (TMA-staged
+ * K/V, every visible K/V row read once for all query heads of the group) and a combine
+ * kernel merging the per-split (max, sum, output) partials of both branches. The grid is
+ * sized from Smax on the host, so the call needs no host synchronisation.
+ */
+DA2_API int diffattn_v2_decode(const void* q, const void* kcache, const void* vcache,
+                       const int32_t* seqlens, const float* lambda, void* out, int B, int Smax,
+                       int Hq, int Hkv, int D, void* workspace, size_t workspace_bytes,
+                       da2_stream_t stream);
+
+/*
+ * The decode step in fp32 end to end (CUDA cores), same layout with fp32 q, caches and
+ * out, no workspace. Supported: D in {64, 128}.
+ */
+DA2_API int diffattn_v2_decode_f32(const float* q, const float* kcache, const float* vcache,
+                           const int32_t* seqlens, const float* lambda, float* out, int B,
+                           int Smax, int Hq, int Hkv, int D, da2_stream_t stream);
+
+/*
+ * V1-style lambda: lambda_p = exp(lq1_p . lk1_p) - exp(lq2_p . lk2_p) + lambda_init, one
+ * value per pair, written to `rows` consecutive rows of n_pairs values each
+ * (lambda_out[r*n_pairs + p], fp32), so the result can feed the decode ([B,Hq/2], rows=B)
+ * or prefill ([B,S,Hq/2], rows=B*S) lambda argument directly.
+ * Source: "Differential Attention (V2)" lesson, "The differential concept" (the lambda
+ * re-parameterisation; lambda_init a small positive number such as 0.8; the value can be
+ * negative).
+ *   lq1, lk1, lq2, lk2  fp32 [n_pairs, d] (device)     lambda_out fp32 [rows, n_pairs]
+ * Computed in fp32 with the accurate expf. Requires n_pairs > 0, d > 0, rows >= 0.
+ */
+DA2_API int diffattn_v2_lambda_v1(const float* lq1, const float* lk1, const float* lq2,
+                          const float* lk2, float lambda_init, int n_pairs, int d, int rows,
+                          float* lambda_out, da2_stream_t stream);
+
+/*
+ * Synchronise `stream`, then read and clear the device error word that kernels set when a
+ * bounded wait expires. *code receives 0 when no kernel reported an error, else the code
+ * of the first error recorded (1 = pipeline wait expired in prefill, 2 = in decode).
+ * Returns DA2_ERR_DEVICE when *code != 0, DA2_OK when it is 0, DA2_ERR_CUDA on a CUDA
+ * failure. `code` is a HOST pointer and may be NULL.
+ */
+DA2_API int diffattn_v2_device_error(int* code, da2_stream_t stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* DIFFATTN_V2_H_ */

@@ -141,22 +141,29 @@ def prefill_rows(q, k, v, lam, rows, causal: bool = True) -> np.ndarray:
     """Selected output rows of a prefill: rows is a list of (b, i, p); returns [len(rows), D].
 
     Each row is the definition applied to query i of pair p in batch b over keys j <= i
-    (causal) or all keys. Used for sampled checks of full-size outputs.
+    (causal) or all keys. Used for sampled checks of full-size outputs. The K/V slice of a
+    (b, g) is upcast once and shared by the rows that read it.
     """
     Hq = q.shape[2]
     Hkv = k.shape[2]
     layout = {p: (h1, h2, g) for p, h1, h2, g in pair_layout(Hq, Hkv)}
     S = q.shape[1]
-    res = []
-    for b, i, p in rows:
-        h1, h2, g = layout[p]
-        n_k = i + 1 if causal else S
-        q1 = _f64(q[b, i, h1])[None, :]
-        q2 = _f64(q[b, i, h2])[None, :]
-        kk = _f64(k[b, :n_k, g])
-        vv = _f64(v[b, :n_k, g])
-        lm = np.array([float(lam[b, i, p])], dtype=np.float64)
-        res.append(diff_attention_block(q1, q2, kk, vv, lm, np.zeros((1, n_k)))[0])
+    res = [None] * len(rows)
+    by_slice = {}
+    for n, (b, i, p) in enumerate(rows):
+        by_slice.setdefault((b, layout[p][2]), []).append(n)
+    for (b, g), idx in by_slice.items():
+        n_max = max(rows[n][1] for n in idx) + 1 if causal else S
+        kk = _f64(k[b, :n_max, g])
+        vv = _f64(v[b, :n_max, g])
+        for n in idx:
+            _, i, p = rows[n]
+            h1, h2, _ = layout[p]
+            n_k = i + 1 if causal else S
+            q1 = _f64(q[b, i, h1])[None, :]
+            q2 = _f64(q[b, i, h2])[None, :]
+            lm = np.array([float(lam[b, i, p])], dtype=np.float64)
+            res[n] = diff_attention_block(q1, q2, kk[:n_k], vv[:n_k], lm, np.zeros((1, n_k)))[0]
     return np.stack(res) if res else np.zeros((0, q.shape[3]))
 
 

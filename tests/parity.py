@@ -1,0 +1,51 @@
+"""Helpers for the GPU parity tests: tolerances and comparisons against the oracle."""
+import numpy as np
+import torch
+
+# Tolerances of the operator's contract: fp32 paths max-abs 1e-5; bf16 paths max-abs 2e-2
+# and relative Frobenius 5e-3 (output rounded once to bf16 from an fp32 epilogue, P rounded
+# to bf16 for the PV product).
+F32_MAX_ABS = 1e-5
+BF16_MAX_ABS = 2e-2
+BF16_REL_FRO = 5e-3
+
+
+def to64(t):
+    return t.detach().to(torch.float64).cpu().numpy()
+
+
+def bf16_close(got, ref, what=""):
+    got = to64(got) if hasattr(got, "detach") else np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    err = np.abs(got - ref)
+    max_abs = float(err.max()) if err.size else 0.0
+    den = float(np.linalg.norm(ref))
+    rel = float(np.linalg.norm(got - ref) / den) if den > 0 else float(np.linalg.norm(got))
+    assert max_abs <= BF16_MAX_ABS, f"{what}: max-abs {max_abs:.3e} > {BF16_MAX_ABS}"
+    assert rel <= BF16_REL_FRO, f"{what}: rel-Frobenius {rel:.3e} > {BF16_REL_FRO}"
+    return max_abs, rel
+
+
+def f32_close(got, ref, what=""):
+    got = to64(got) if hasattr(got, "detach") else np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    err = float(np.abs(got - ref).max()) if got.size else 0.0
+    assert err <= F32_MAX_ABS, f"{what}: max-abs {err:.3e} > {F32_MAX_ABS}"
+    return err
+
+
+def sample_rows(B, S, n_pairs, n=1024, seed=0, tile=128):
+    """Seeded stratified sample of (b, i, p): tile boundaries, first and last rows, every pair."""
+    rng = np.random.default_rng(seed)
+    special = sorted({0, 1, tile - 1, tile, tile + 1, 2 * tile - 1, S // 2, S - 2, S - 1} & set(range(S)))
+    rows = []
+    for b in range(B):
+        for p in range(n_pairs):
+            for i in special:
+                rows.append((b, i, p))
+    while len(rows) < n + len(special) * B * n_pairs:
+        rows.append((int(rng.integers(B)), int(rng.integers(S)), int(rng.integers(n_pairs))))
+    return rows

@@ -1,0 +1,119 @@
+"""The C-ABI library without a GPU: it loads, exports every declared entry point, and its
+host-side argument checks reject bad input before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "diffattn_v2.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"DA2_API\s+[\w\s\*]+?\b(diffattn_v2_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from differential_attention_v2_b200.build import build
+
+    build()
+    import differential_attention_v2_b200 as da
+
+    return da.LIB
+
+
+def test_header_declares_entry_points():
+    names = _declared()
+    assert "diffattn_v2_prefill" in names and "diffattn_v2_decode" in names
+    assert len(names) >= 9
+
+
+def test_library_exports_every_declared_symbol(lib):
+    import differential_attention_v2_b200 as da
+
+    for name in _declared():
+        assert hasattr(lib, name), name
+        assert name in da.EXPORTED, f"binding lacks {name}"
+
+
+def test_version_and_status_strings(lib):
+    assert lib.diffattn_v2_version() == 100
+    for code in (0, -1, -2, -3, -4, 7):
+        assert lib.diffattn_v2_status_string(code)
+
+
+# Fake, never dereferenced, 16-byte aligned device addresses: every call below must be
+# rejected (or be a no-op) by the host-side checks, before any CUDA call.
+P = 1 << 20
+Q = P + 4096
+K = P + 8192
+V = P + 12288
+L = P + 16384
+O = P + 20480
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((Q, K, V, L, O, 2, 256, 7, 1, 128, 1), -1),        # odd Hq
+    ((Q, K, V, L, O, 2, 256, 6, 2, 128, 1), -1),        # a pair would straddle KV heads
+    ((Q, K, V, L, O, 2, 256, 8, 0, 128, 1), -1),        # Hkv = 0
+    ((Q, K, V, L, O, -1, 256, 8, 2, 128, 1), -1),       # negative B
+    ((Q, K, V, L, O, 2, 256, 8, 2, 0, 1), -1),          # D = 0
+    ((None, K, V, L, O, 2, 256, 8, 2, 128, 1), -1),     # null q
+    ((Q, K, V, None, O, 2, 256, 8, 2, 128, 1), -1),     # null lambda
+    ((Q + 2, K, V, L, O, 2, 256, 8, 2, 128, 1), -1),    # misaligned q
+    ((Q, K, V, L, O, 2, 256, 8, 2, 128, 2), -1),        # causal flag not 0/1
+    ((Q, K, V, L, O, 2, 256, 8, 2, 64, 1), -2),         # bf16 path implements D = 128 only
+    ((Q, K, V, L, O, 0, 256, 8, 2, 128, 1), 0),         # B = 0: no-op
+    ((Q, K, V, L, O, 2, 0, 8, 2, 128, 1), 0),           # S = 0: no-op
+    ((None, None, None, None, None, 0, 0, 8, 2, 128, 1), 0),
+])
+def test_prefill_host_checks(lib, args, expect):
+    assert lib.diffattn_v2_prefill(*args, None) == expect
+
+
+def test_prefill_f32_host_checks(lib):
+    assert lib.diffattn_v2_prefill_f32(Q, K, V, L, O, 1, 16, 4, 1, 96, 1, None) == -2
+    assert lib.diffattn_v2_prefill_f32(Q, K, V, L, O, 1, 16, 4, 3, 64, 1, None) == -1
+    assert lib.diffattn_v2_prefill_f32(None, K, V, L, O, 1, 16, 4, 1, 64, 1, None) == -1
+
+
+def test_decode_workspace_size(lib):
+    import differential_attention_v2_b200 as da
+
+    assert da.decode_workspace_size(0, 8192, 64, 8, 128) == 0
+    assert da.decode_workspace_size(4, 8192, 6, 2, 128) == 0
+    ws = da.decode_workspace_size(64, 8192, 64, 8, 128)
+    assert ws > 0 and ws % 16 == 0
+    # fp32 (m, l, O[D]) per (b, head, split): a multiple of B*Hq*(D+2)*4
+    assert ws % (64 * 64 * 130 * 4) == 0
+    # grows with Smax (more splits), never with nothing
+    assert da.decode_workspace_size(64, 65536, 64, 8, 128) >= ws
+
+
+def test_decode_host_checks(lib):
+    ws = lib.diffattn_v2_decode_workspace_size(2, 1024, 16, 2, 128)
+    S = P + 24576
+    W = P + 65536
+    args = (Q, K, V, S, L, O, 2, 1024, 16, 2, 128, W, ws, None)
+    bad_ws = args[:12] + (ws - 16,) + args[13:]
+    assert lib.diffattn_v2_decode(*bad_ws) == -1                       # workspace too small
+    no_ws = args[:11] + (None,) + args[12:]
+    assert lib.diffattn_v2_decode(*no_ws) == -1                        # null workspace
+    odd = (Q, K, V, S, L, O, 2, 1024, 10, 1, 128, W, ws, None)
+    assert lib.diffattn_v2_decode(*odd) == -2                          # group size 10
+    d64 = (Q, K, V, S, L, O, 2, 1024, 16, 2, 64, W, 1 << 30, None)
+    assert lib.diffattn_v2_decode(*d64) == -2
+    b0 = (None, None, None, None, None, None, 0, 1024, 16, 2, 128, None, 0, None)
+    assert lib.diffattn_v2_decode(*b0) == 0
+    assert lib.diffattn_v2_decode(Q, K, V, S, L, O, 2, 0, 16, 2, 128, W, ws, None) == -1
+    assert lib.diffattn_v2_decode_f32(Q, K, V, S, L, O, 2, 1024, 16, 3, 64, None) == -1
+
+
+def test_lambda_v1_host_checks(lib):
+    assert lib.diffattn_v2_lambda_v1(Q, K, V, L, 0.8, 0, 128, 1, O, None) == -1
+    assert lib.diffattn_v2_lambda_v1(Q, K, V, L, 0.8, 4, 0, 1, O, None) == -1
+    assert lib.diffattn_v2_lambda_v1(Q, K, V, L, 0.8, 4, 128, 0, O, None) == 0
+    assert lib.diffattn_v2_lambda_v1(None, K, V, L, 0.8, 4, 128, 1, O, None) == -1

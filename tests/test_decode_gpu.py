@@ -1,0 +1,115 @@
+"""GPU parity of the decode and lambda entry points against the float64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from oracle import diffattn_f64 as ora
+from tests.parity import bf16_close, f32_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def da():
+    import differential_attention_v2_b200 as m
+
+    assert torch.cuda.is_available()
+    return m
+
+
+def _decode_case(B, Smax, Hq, Hkv, lens, seed, dtype="bf16"):
+    inp = workloads.make_decode(workloads.DecodeCase(B=B, Smax=Smax, Hq=Hq, Hkv=Hkv, D=128, len_lo=1,
+                                                     len_hi=Smax, dtype=dtype, seed=seed))
+    inp["seqlens"] = torch.tensor(lens, dtype=torch.int32)
+    return inp
+
+
+def _run(da, inp):
+    out = da.decode(inp["q"].cuda(), inp["kcache"].cuda(), inp["vcache"].cuda(), inp["seqlens"].cuda(),
+                    inp["lam"].cuda())
+    assert da.device_error() == 0
+    return out
+
+
+@pytest.mark.parametrize("B,Smax,Hq,Hkv,lens", [
+    (3, 300, 16, 2, [300, 1, 0]),            # full, single key, empty sequence
+    (4, 1000, 64, 8, [1000, 999, 64, 65]),    # group of 8, stage boundaries
+    (2, 700, 8, 4, [700, 129]),               # group of 2
+    (2, 700, 16, 4, [511, 700]),              # group of 4
+    (2, 900, 32, 2, [900, 333]),              # group of 16 (two head tiles)
+    (1, 5000, 8, 1, [5000]),                  # several splits
+])
+def test_decode_bf16_matches_oracle(da, B, Smax, Hq, Hkv, lens):
+    inp = _decode_case(B, Smax, Hq, Hkv, lens, seed=B * Smax + Hq)
+    out = _run(da, inp)
+    ref = ora.decode(inp["q"], inp["kcache"], inp["vcache"], inp["seqlens"], inp["lam"])
+    bf16_close(out, ref, f"decode B={B} Smax={Smax} Hq={Hq} Hkv={Hkv}")
+    for b, n in enumerate(lens):
+        if n == 0:
+            assert torch.count_nonzero(out[b]).item() == 0
+
+
+def test_decode_matches_last_prefill_row(da):
+    """One decode step over n cached keys equals row n-1 of a prefill of length n."""
+    case = workloads.PrefillCase(B=1, S=333, Hq=16, Hkv=2, D=128, seed=21)
+    inp = workloads.make_prefill(case)
+    pre = da.prefill(inp["q"].cuda(), inp["k"].cuda(), inp["v"].cuda(), inp["lam"].cuda()).cpu()
+    dec = da.decode(inp["q"][:, -1].contiguous().cuda(), inp["k"].cuda(), inp["v"].cuda(),
+                    torch.tensor([333], dtype=torch.int32, device="cuda"), inp["lam"][:, -1].contiguous().cuda()).cpu()
+    ref = ora.prefill_rows(inp["q"], inp["k"], inp["v"], inp["lam"], [(0, 332, p) for p in range(8)])
+    bf16_close(dec[0], ref, "decode row")
+    bf16_close(pre[0, -1], ref, "prefill row")
+
+
+def test_decode_c4_full_size(da):
+    """The 64-sequence decode workload (lengths uniform in [1024, 8192]) in full."""
+    inp = workloads.make_decode(workloads.CONFIGS["c4_bf16_decode"])
+    out = _run(da, inp)
+    ref = ora.decode(inp["q"], inp["kcache"], inp["vcache"], inp["seqlens"], inp["lam"])
+    bf16_close(out, ref, "c4")
+
+
+def test_decode_c5_needle_with_v1_lambda(da):
+    """The 128k needle workload with the V1 lambda computed on the GPU, in full."""
+    case = workloads.CONFIGS["c5_needle_decode"]
+    inp = workloads.make_decode(case)
+    B, n_pairs = case.B, case.Hq // 2
+    lam = da.lambda_v1(inp["lq1"].cuda(), inp["lk1"].cuda(), inp["lq2"].cuda(), inp["lk2"].cuda(),
+                       inp["lambda_init"], rows=B)
+    lam_ref = ora.lambda_v1(inp["lq1"], inp["lk1"], inp["lq2"], inp["lk2"], inp["lambda_init"])
+    np.testing.assert_allclose(lam.cpu().double().numpy(), np.broadcast_to(lam_ref, (B, n_pairs)), rtol=2e-6, atol=2e-6)
+    inp["lam"] = lam.cpu()
+    out = _run(da, inp)
+    ref = ora.decode(inp["q"], inp["kcache"], inp["vcache"], inp["seqlens"], inp["lam"])
+    bf16_close(out, ref, "c5 needle")
+
+
+def test_lambda_v1_matches_oracle(da):
+    g = torch.Generator().manual_seed(4)
+    vec = [torch.randn(32, 128, generator=g) * 0.3 for _ in range(4)]
+    for init in (0.8, 0.0, -0.2):
+        got = da.lambda_v1(*(x.cuda() for x in vec), lambda_init=init, rows=5)
+        ref = ora.lambda_v1(*vec, init)
+        np.testing.assert_allclose(got.cpu().double().numpy(), np.broadcast_to(ref, (5, 32)), rtol=1e-5, atol=1e-6)
+
+
+@pytest.mark.parametrize("lens,D", [([300, 1, 0], 128), ([77, 200], 64)])
+def test_decode_f32_matches_oracle(da, lens, D):
+    B, Smax, Hq, Hkv = len(lens), max(lens), 8, 2
+    inp = workloads.make_decode(workloads.DecodeCase(B=B, Smax=Smax, Hq=Hq, Hkv=Hkv, D=D, len_lo=1, len_hi=Smax,
+                                                     dtype="f32", seed=D))
+    inp["seqlens"] = torch.tensor(lens, dtype=torch.int32)
+    out = da.decode_f32(inp["q"].cuda(), inp["kcache"].cuda(), inp["vcache"].cuda(), inp["seqlens"].cuda(),
+                        inp["lam"].cuda())
+    ref = ora.decode(inp["q"], inp["kcache"], inp["vcache"], inp["seqlens"], inp["lam"])
+    f32_close(out, ref, "fp32 decode")
+
+
+def test_decode_equal_heads_cancel_exactly(da):
+    """Q1 = Q2 with lambda = 1 cancels exactly in the decode path too."""
+    inp = _decode_case(3, 700, 16, 2, [700, 5, 380], seed=31)
+    inp["q"][:, 1::2] = inp["q"][:, 0::2]
+    inp["lam"].fill_(1.0)
+    out = _run(da, inp)
+    assert torch.count_nonzero(out).item() == 0
