@@ -160,12 +160,12 @@ def _max_over_ranks(x, dist):
 
 
 # -------------------------------------------------------------------------- our arm
-def _inputs(rank):
+def _inputs(rank, do_pre=True, do_dec=True):
     pc = workloads.CONFIGS[PREFILL_CFG]
     dc = workloads.CONFIGS[DECODE_CFG]
     pc = workloads.PrefillCase(**{**pc.__dict__, "seed": pc.seed + 100 * rank})
     dc = workloads.DecodeCase(**{**dc.__dict__, "seed": dc.seed + 100 * rank})
-    return pc, workloads.make_prefill(pc), dc, workloads.make_decode(dc)
+    return (pc, workloads.make_prefill(pc) if do_pre else None, dc, workloads.make_decode(dc) if do_dec else None)
 
 
 def run_ours(args, rank, world, local, dist):
@@ -173,26 +173,33 @@ def run_ours(args, rank, world, local, dist):
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    pc, pin, dc, din = _inputs(rank)
+    do_pre = args.only in (None, "prefill")
+    do_dec = args.only in (None, "decode")
+    pc, pin, dc, din = _inputs(rank, do_pre, do_dec)
     stream = torch.cuda.current_stream(dev)
 
     # device-resident inputs and outputs
-    q, k, v, lam = (pin[x].to(dev) for x in ("q", "k", "v", "lam"))
-    out = torch.empty(pc.B, pc.S, pc.Hq // 2, pc.D, dtype=torch.bfloat16, device=dev)
-    dq, kc, vc, sl, dl = (din[x].to(dev) for x in ("q", "kcache", "vcache", "seqlens", "lam"))
-    dout = torch.empty(dc.B, dc.Hq // 2, dc.D, dtype=torch.bfloat16, device=dev)
-    ws = torch.empty(da.decode_workspace_size(dc.B, dc.Smax, dc.Hq, dc.Hkv, dc.D), dtype=torch.uint8, device=dev)
+    if do_pre:
+        q, k, v, lam = (pin[x].to(dev) for x in ("q", "k", "v", "lam"))
+        out = torch.empty(pc.B, pc.S, pc.Hq // 2, pc.D, dtype=torch.bfloat16, device=dev)
+    if do_dec:
+        dq, kc, vc, sl, dl = (din[x].to(dev) for x in ("q", "kcache", "vcache", "seqlens", "lam"))
+        dout = torch.empty(dc.B, dc.Hq // 2, dc.D, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(da.decode_workspace_size(dc.B, dc.Smax, dc.Hq, dc.Hkv, dc.D), dtype=torch.uint8,
+                         device=dev)
 
-    flops = workloads.prefill_flops(pc.B, pc.S, pc.Hq, pc.D, causal=True)
-    dbytes = workloads.decode_bytes(din["seqlens"].tolist(), dc.Hkv, dc.D, dc.Hq)
+    flops = workloads.prefill_flops(pc.B, pc.S, pc.Hq, pc.D, causal=True) if do_pre else 0
+    dbytes = workloads.decode_bytes(din["seqlens"].tolist(), dc.Hkv, dc.D, dc.Hq) if do_dec else 0
 
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        da.prefill(q, k, v, lam, out=out, stream=stream)
+        if do_pre:
+            da.prefill(q, k, v, lam, out=out, stream=stream)
         if ev is not None:
             ev[1].record(stream)
-        da.decode(dq, kc, vc, sl, dl, out=dout, workspace=ws, stream=stream)
+        if do_dec:
+            da.decode(dq, kc, vc, sl, dl, out=dout, workspace=ws, stream=stream)
         if ev is not None:
             ev[2].record(stream)
 
@@ -224,21 +231,23 @@ def run_ours(args, rank, world, local, dist):
     err = da.device_error(stream)
 
     # ------------------------------------------------ end to end through host buffers
-    h = {x: pin[x].pin_memory() for x in ("q", "k", "v", "lam")}
-    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    hd = {x: din[x].pin_memory() for x in ("q", "seqlens", "lam")}
-    hd_out = torch.empty(dout.shape, dtype=dout.dtype).pin_memory()
+    h = {x: pin[x].pin_memory() for x in ("q", "k", "v", "lam")} if do_pre else {}
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory() if do_pre else torch.empty(0)
+    hd = {x: din[x].pin_memory() for x in ("q", "seqlens", "lam")} if do_dec else {}
+    hd_out = torch.empty(dout.shape, dtype=dout.dtype).pin_memory() if do_dec else torch.empty(0)
     e2e_steps = max(3, min(args.steps, 50))
 
     def e2e_step():
-        for name, dst in (("q", q), ("k", k), ("v", v), ("lam", lam)):
-            dst.copy_(h[name], non_blocking=True)
-        da.prefill(q, k, v, lam, out=out, stream=stream)
-        h_out.copy_(out, non_blocking=True)
-        for name, dst in (("q", dq), ("seqlens", sl), ("lam", dl)):
-            dst.copy_(hd[name], non_blocking=True)
-        da.decode(dq, kc, vc, sl, dl, out=dout, workspace=ws, stream=stream)
-        hd_out.copy_(dout, non_blocking=True)
+        if do_pre:
+            for name, dst in (("q", q), ("k", k), ("v", v), ("lam", lam)):
+                dst.copy_(h[name], non_blocking=True)
+            da.prefill(q, k, v, lam, out=out, stream=stream)
+            h_out.copy_(out, non_blocking=True)
+        if do_dec:
+            for name, dst in (("q", dq), ("seqlens", sl), ("lam", dl)):
+                dst.copy_(hd[name], non_blocking=True)
+            da.decode(dq, kc, vc, sl, dl, out=dout, workspace=ws, stream=stream)
+            hd_out.copy_(dout, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize(dev)
@@ -266,10 +275,10 @@ def run_ours(args, rank, world, local, dist):
     K = args.steps
     pre_launch_ms = pre_ms / K
     dec_launch_ms = dec_ms / K
-    tflops = flops / (pre_launch_ms * 1e-3) / 1e12
-    gbs = dbytes / (dec_launch_ms * 1e-3) / 1e9
-    value = world * flops * K / (pre_ms * 1e-3) / 1e12  # whole job: every rank's prefill FLOPs
-    dec_value = world * dbytes * K / (dec_ms * 1e-3) / 1e9
+    tflops = flops / (pre_launch_ms * 1e-3) / 1e12 if do_pre else 0.0
+    gbs = dbytes / (dec_launch_ms * 1e-3) / 1e9 if do_dec else 0.0
+    value = world * flops * K / (pre_ms * 1e-3) / 1e12 if do_pre else 0.0  # whole job: every rank's FLOPs
+    dec_value = world * dbytes * K / (dec_ms * 1e-3) / 1e9 if do_dec else 0.0
     peak_t = peaks["bf16_tflops"]
     tr = NCU_TRAFFIC["prefill"]
     traffic = tr["bytes"] if tr["source_sha"] == _src_sha("prefill_sm100.cu") else None
@@ -295,7 +304,7 @@ def run_ours(args, rank, world, local, dist):
             "prefill": {"B": pc.B, "S": pc.S, "Hq": pc.Hq, "Hkv": pc.Hkv, "D": pc.D, "causal": True,
                         "flops_per_step": flops},
             "decode": {"B": dc.B, "Smax": dc.Smax, "Hq": dc.Hq, "Hkv": dc.Hkv, "D": dc.D,
-                       "sum_seqlens": int(din["seqlens"].sum()), "bytes_per_step": dbytes},
+                       "sum_seqlens": int(din["seqlens"].sum()) if do_dec else None, "bytes_per_step": dbytes},
             "parallelism": f"replicas x{world} (independent per-GPU batches)",
             "l2": "no flush: inputs larger than L2 (q 268 MB; decode streams 1.2 GB per step)",
         },
@@ -312,17 +321,20 @@ def run_ours(args, rank, world, local, dist):
             "launch_ms": round(pre_launch_ms, 4), "peak_source": f"{peak_src} bf16_tflops (burst)",
         },
         "e2e": {
-            "value": round(world * flops * e2e_steps / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "value": round(world * flops * e2e_steps / (e2e_ms * 1e-3) / 1e12, 3) if do_pre else None,
+            "unit": "TFLOP/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
             "ms_per_step": round(e2e_ms / e2e_steps, 3),
             "note": "prefill FLOPs over a step that copies q/k/v/lambda and the decode q/seqlens/lambda "
                     "from pinned host memory, runs both kernels through the C ABI and copies both "
                     "outputs back",
         },
-        "gpu_launches": 3 * K,
+        "gpu_launches": (int(do_pre) + 2 * int(do_dec)) * K,
         "clocks": clk,
     }
-    if world == 1 and not args.no_cpu_baseline:
+    if args.only:
+        line["only"] = args.only
+    if world == 1 and not args.no_cpu_baseline and do_pre and do_dec:
         line["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
     else:
         line["cpu_baseline"] = None
@@ -398,34 +410,39 @@ def cpu_baseline(seconds=15.0, inputs=None):
 
 
 def run_reference(args):
-    """The oracle as the reference arm: each step a bounded sample of the same workload."""
+    """The oracle as the reference arm: each step a bounded sample of the same workload,
+    sized so that the whole run stays within a few minutes of host time."""
     pc = workloads.CONFIGS[PREFILL_CFG]
     dc = workloads.CONFIGS[DECODE_CFG]
     pin, din = workloads.make_prefill(pc), workloads.make_decode(dc)
-    units = args.ref_units
+    f, t = _prefill_units(pin, pc, 2, seed=99)
+    per_unit = t / 2
+    budget = min(3.0, max(0.05, args.ref_seconds / max(1, args.steps + args.warmup)))
+    units = max(1, int(0.8 * budget / per_unit))
     for i in range(args.warmup):
-        _prefill_units(pin, pc, max(1, units // 4), seed=100 + i)
+        _prefill_units(pin, pc, units, seed=100 + i)
     flops, secs = 0, 0.0
     dbytes, dsecs = 0, 0.0
     for i in range(args.steps):
         f, t = _prefill_units(pin, pc, units, seed=1000 + i)
         flops += f
         secs += t
-        b, td = _decode_seqs(din, dc, 1, seed=2000 + i)
-        dbytes += b
-        dsecs += td
+        if i % max(1, args.steps // 8) == 0:
+            b, td = _decode_seqs(din, dc, 1, seed=2000 + i)
+            dbytes += b
+            dsecs += td
     value = flops / secs / 1e12
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": 1,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1000 * (secs + dsecs) / args.steps, 2),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1000 * secs / args.steps, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic: the same seeded inputs as the GPU arm",
         "config": {"workload": "prefill B=4 S=4096 Hq=64 Hkv=8 D=128 causal + decode B=64 Smax=8192 len "
-                               "U[1024,8192]; each step a bounded sample", "units_per_step": units},
+                               "U[1024,8192]; each step a bounded sample", "prefill_units_per_step": units},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": _oracle_threads(), "kind": "oracle",
-                         "sample": f"{units} random (batch, pair, 128-row tile) prefill units and one full decode "
-                                   f"sequence per step"},
-        "decode": {"value": round(dbytes / dsecs / 1e9, 4), "unit": "GB/s"},
+                         "sample": f"{units} random (batch, pair, 128-row tile) prefill units per step; "
+                                   f"decode: one full sequence on every {max(1, args.steps // 8)}-th step"},
+        "decode": {"value": round(dbytes / dsecs / 1e9, 4) if dsecs else None, "unit": "GB/s"},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
@@ -439,7 +456,10 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ref-units", type=int, default=24, help="prefill units per reference step")
+    ap.add_argument("--ref-seconds", type=float, default=120.0,
+                    help="host-time budget of the whole reference run (warm-up and timed steps)")
+    ap.add_argument("--only", choices=("prefill", "decode"), default=None,
+                    help="run one half of the step (for profiling a single kernel on less device memory)")
     args = ap.parse_args(argv)
 
     if args.impl == "reference":
