@@ -8,7 +8,7 @@ use raises ImportError (there is no fallback implementation).
 import importlib
 
 _BINDING_NAMES = (
-    "prefill", "prefill_f32", "decode", "decode_f32", "decode_workspace_size", "lambda_v1",
+    "prefill", "prefill_f32", "decode", "decode_f32", "decode_workspace_size", "lambda_v1", "decode_noalloc",
     "device_error", "version", "DiffAttnError", "EXPORTED", "LIB_PATH", "LIB",
 )
 __all__ = list(_BINDING_NAMES)

@@ -32,6 +32,7 @@ _SIGNATURES = {
     "diffattn_v2_decode_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
     "diffattn_v2_lambda_v1": (_i, [_vp, _vp, _vp, _vp, _f, _i, _i, _i, _vp, _vp]),
     "diffattn_v2_device_error": (_i, [ctypes.POINTER(_i), _vp]),
+    "diffattn_v2_decode_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
 }
 EXPORTED = tuple(_SIGNATURES)
 
@@ -187,3 +188,26 @@ def device_error(stream=None, device=None) -> int:
     if st == ERR_CUDA:
         raise DiffAttnError(st, "diffattn_v2_device_error")
     return code.value
+
+
+def decode_noalloc(q, kcache, vcache, seqlens, lam, out=None, stream=None):
+    """bf16 decode step whose partials live in the library's fixed 16 MiB device array.
+
+    For callers that cannot allocate device memory (a KV-cache pool or caching allocator
+    that owns nearly all HBM, plugin interfaces without a workspace). The library allocates
+    nothing; calls that overlap on the GPU share the array and race, so serialise them.
+    Sizes needing more than 16 MiB of partials raise (DA2_ERR_UNSUPPORTED)."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(kcache, "kcache", torch.bfloat16, 4)
+    _need(vcache, "vcache", torch.bfloat16, 4)
+    _need(seqlens, "seqlens", torch.int32, 1)
+    _need(lam, "lam", torch.float32, 2)
+    B, Hq, D = q.shape
+    Smax, Hkv = kcache.shape[1], kcache.shape[2]
+    if out is None:
+        out = torch.empty((B, Hq // 2, D), dtype=torch.bfloat16, device=q.device)
+    _need(out, "out", torch.bfloat16, 3)
+    st = LIB.diffattn_v2_decode_noalloc(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(lam), _ptr(out),
+                                        B, Smax, Hq, Hkv, D, _stream(stream, q.device))
+    _check(st, "diffattn_v2_decode_noalloc")
+    return out

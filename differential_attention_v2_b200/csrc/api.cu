@@ -91,6 +91,14 @@ void decode_split_plan(int B, int Smax, int Hkv, int* split_len, int* nsplit) {
   *nsplit = static_cast<int>((Smax + L - 1) / L);
 }
 
+// Accessors for other translation units of the library.
+cudaError_t device_error_word(int** out) { return device_error_ptr(out); }
+
+cudaError_t encode_bshd_bf16(CUtensorMap* map, const void* base, uint64_t D, uint64_t H, uint64_t S, uint64_t B,
+                             uint32_t box0, uint32_t box2) {
+  return encode_bshd(map, base, D, H, S, B, box0, box2);
+}
+
 }  // namespace da2
 
 extern "C" {

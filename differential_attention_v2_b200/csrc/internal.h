@@ -36,4 +36,11 @@ cudaError_t launch_decode_f32(const float* q, const float* kc, const float* vc, 
 cudaError_t launch_lambda_v1(const float* lq1, const float* lk1, const float* lq2, const float* lk2,
                              float lambda_init, int n_pairs, int d, int rows, float* out, cudaStream_t stream);
 
+// Address of the device error word on the current device.
+cudaError_t device_error_word(int** out);
+
+// 4-D bf16 tensor map over a row-major [B,S,H,D] array, box {box0, 1, box2, 1}, 128-byte swizzle.
+cudaError_t encode_bshd_bf16(CUtensorMap* map, const void* base, uint64_t D, uint64_t H, uint64_t S, uint64_t B,
+                             uint32_t box0, uint32_t box2);
+
 }  // namespace da2

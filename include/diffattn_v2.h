@@ -153,6 +153,32 @@ DA2_API int diffattn_v2_lambda_v1(const float* lq1, const float* lk1, const floa
                           float* lambda_out, da2_stream_t stream);
 
 /*
+ * The bf16 decode step of diffattn_v2_decode (same arguments, layout, semantics and kernels)
+ * without a workspace argument, for callers that cannot allocate device memory: serving
+ * engines that give nearly all HBM to a KV-cache pool or caching allocator up front, plugin
+ * interfaces that hand over only input and output buffers, and loops that must not take
+ * the device-wide synchronisation an allocation may imply. The pages describe no such entry
+ * point; it has no counterpart there.
+ *   - The per-split partials live in a fixed 16 MiB device array inside the library
+ *     (16777216 bytes). Every GPU that loads the library holds that array until the process
+ *     exits. The call allocates nothing: no cudaMalloc, no cudaFree, no allocating library
+ *     routine.
+ *   - Sizes whose partials need more than the array, i.e. whenever
+ *     diffattn_v2_decode_workspace_size(B, Smax, Hq, Hkv, D) > 16777216, are refused with
+ *     DA2_ERR_UNSUPPORTED before anything is launched.
+ *   - The first call on a device (with that device current) looks up the array's device
+ *     address once (cudaGetSymbolAddress) and caches it; make that first call before any
+ *     stream capture.
+ *   - All calls on a device share the one array, and it keeps the last call's contents
+ *     (nothing in it needs to start at zero). Calls that overlap on the GPU -- on different
+ *     streams, or from different host threads without ordering -- race on it and give wrong
+ *     results: serialise them.
+ */
+DA2_API int diffattn_v2_decode_noalloc(const void* q, const void* kcache, const void* vcache,
+                                       const int32_t* seqlens, const float* lambda, void* out, int B,
+                                       int Smax, int Hq, int Hkv, int D, da2_stream_t stream);
+
+/*
  * Synchronise `stream`, then read and clear the device error word that kernels set when a
  * bounded wait expires. *code receives 0 when no kernel reported an error, else the code
  * of the first error recorded (1 = pipeline wait expired in prefill, 2 = in decode).
