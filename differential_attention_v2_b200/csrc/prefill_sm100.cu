@@ -81,6 +81,66 @@ struct Params {
   float scale_log2;       // log2(e)/sqrt(D)
 };
 
+// Set scores of keys past column `lim` of this row to -inf.
+__device__ __forceinline__ void mask_row(uint32_t (&sr)[4][32], int lim) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+      if (32 * c + e > lim) sr[c][e] = __float_as_uint(-INFINITY);
+}
+
+// Max of the 128 raw scores of a row: 3-input max, four independent chains.
+__device__ __forceinline__ float row_max(const uint32_t (&sr)[4][32]) {
+  float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+#pragma unroll
+    for (int e = 0; e < 32; e += 8) {
+      m0 = fmax3(m0, __uint_as_float(sr[c][e + 0]), __uint_as_float(sr[c][e + 1]));
+      m1 = fmax3(m1, __uint_as_float(sr[c][e + 2]), __uint_as_float(sr[c][e + 3]));
+      m2 = fmax3(m2, __uint_as_float(sr[c][e + 4]), __uint_as_float(sr[c][e + 5]));
+      m3 = fmax3(m3, __uint_as_float(sr[c][e + 6]), __uint_as_float(sr[c][e + 7]));
+    }
+  return fmax3(m0, m1, fmaxf(m2, m3));
+}
+
+// P = 2^(s*scale - m) for the 128 scores of the row, packed to bf16 pairs and stored over
+// the first 64 TMEM columns of the row's S tile (keys 2c, 2c+1 -> column c). Returns the
+// fp32 row sum of P. The exponent argument of two keys is one packed FMA.
+__device__ __forceinline__ float exp_pack_store(const uint32_t (&sr)[4][32], float scale, float m_use,
+                                                uint32_t taddr) {
+  const uint64_t scale2 = f2_pack(scale, scale);
+  const uint64_t negm2 = f2_pack(-m_use, -m_use);
+  uint64_t sum_a = f2_pack(0.f, 0.f), sum_b = f2_pack(0.f, 0.f);
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      const int c = 2 * half + cc;
+#pragma unroll
+      for (int e = 0; e < 32; e += 2) {
+        const uint64_t arg = f2_fma(f2_pack(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])), scale2, negm2);
+        float a0, a1;
+        f2_unpack(arg, a0, a1);
+        const float p0 = fast_exp2(a0);
+        const float p1 = fast_exp2(a1);
+        if ((e >> 1) & 1)
+          sum_b = f2_add(sum_b, f2_pack(p0, p1));
+        else
+          sum_a = f2_add(sum_a, f2_pack(p0, p1));
+        pk[cc * 16 + (e >> 1)] = pack_bf16x2(p0, p1);
+      }
+    }
+    tmem_st_32x32b_x32(taddr + 32 * half, pk);
+  }
+  float s0, s1, s2, s3;
+  f2_unpack(sum_a, s0, s1);
+  f2_unpack(sum_b, s2, s3);
+  return (s0 + s1) + (s2 + s3);
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const Params p) {
@@ -250,21 +310,14 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       reg_fence(sr[2]);
       reg_fence(sr[3]);
 
-      const bool need_mask = (p.causal && j == tile) || ((j + 1) * BN > p.S);
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          float x = __uint_as_float(sr[c][e]) * p.scale_log2;
-          if (need_mask) {
-            const int key = j * BN + 32 * c + e;
-            if ((p.causal && key > qi) || key >= p.S) x = -INFINITY;
-          }
-          sr[c][e] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
-        }
-      }
+      // Keys visible to this row in this tile are columns 0..lim; only the diagonal tile of
+      // a causal launch and a ragged last key tile have lim < 127.
+      int lim = BN - 1;
+      if (p.causal && j == tile) lim = r;
+      lim = min(lim, p.S - 1 - j * BN);
+      if (lim < BN - 1) mask_row(sr, lim);
+      const float mx = row_max(sr) * p.scale_log2;
+
       // raise the running max only when the tile's max exceeds it by more than 2^8
       const bool rescale = mx > m_run + 8.f;
       float alpha = 1.f;
@@ -274,25 +327,7 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         m_run = mx;
       }
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      float lsum = 0.f;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int c = 2 * half + cc;
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float p0 = fast_exp2(__uint_as_float(sr[c][e]) - m_use);
-            const float p1 = fast_exp2(__uint_as_float(sr[c][e + 1]) - m_use);
-            lsum += p0 + p1;
-            pk[cc * 16 + (e >> 1)] = pack_bf16x2(p0, p1);
-          }
-        }
-        // P for keys 64*half .. 64*half+63 -> columns 32*half .. 32*half+31 (bf16 pairs)
-        tmem_st_32x32b_x32(trow + s_col + 32 * half, pk);
-      }
-      l_run += lsum;
+      l_run += exp_pack_store(sr, p.scale_log2, m_use, trow + s_col);
       if (rescale && j > 0) {
         // O_b holds the sum up to tile j-1, complete: S_b(j) was committed after PV_b(j-1),
         // and PV_b(j) is issued only after this thread arrives on P_full below
