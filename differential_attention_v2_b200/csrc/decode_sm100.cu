@@ -156,7 +156,8 @@ diffattn_decode_split(const __grid_constant__ CUtensorMap tmK, const __grid_cons
     for (int i = 0; i < n_stages; ++i) {
       const int s = i % kStages;
       const uint32_t ph = (i / kStages) & 1;
-      if (!mbar_wait(full(s), ph, abort_flag)) break;
+      // the warp leaves together: the loop body is made of warp-collective instructions
+      if (!__all_sync(0xffffffffu, mbar_wait(full(s), ph, abort_flag))) break;
       const uint32_t kb = sbase + s * kStageBytes;
       const uint32_t vb = kb + 2 * kHalfBytes;
 

@@ -64,10 +64,10 @@ enum Bar : int {
   kVFull = 5,    // +stage
   kVEmpty = 7,   // +stage
   kSFull = 9,    // +branch
-  kPFull = 11,   // +branch
-  kOFull = 13,
-  kDrain = 14,
-  kNumBars = 15
+  kPFull = 11,   // +2*branch+half: P of keys 64*half .. 64*half+63 is in TMEM
+  kOFull = 15,
+  kDrain = 16,
+  kNumBars = 17
 };
 
 constexpr uint32_t kTmS1 = 0, kTmS2 = 128, kTmO1 = 256, kTmO2 = 384;
@@ -105,36 +105,66 @@ __device__ __forceinline__ float row_max(const uint32_t (&sr)[4][32]) {
   return fmax3(m0, m1, fmaxf(m2, m3));
 }
 
-// P = 2^(s*scale - m) for the 128 scores of the row, packed to bf16 pairs and stored over
-// the first 64 TMEM columns of the row's S tile (keys 2c, 2c+1 -> column c). Returns the
-// fp32 row sum of P. The exponent argument of two keys is one packed FMA.
-__device__ __forceinline__ float exp_pack_store(const uint32_t (&sr)[4][32], float scale, float m_use,
+// 2^x of two values on the FMA pipe (no MUFU): x = n + f with n = rint(x) and f in
+// [-1/2, 1/2]; 2^f by a cubic fitted for minimax relative error on [-1/2, 1/2] (Remez
+// exchange, max relative error 7.5e-5, well under bf16's 2^-9); 2^n is added to the
+// exponent field. x is clamped to -126 so the exponent never underflows past zero.
+// Adding 1.5 * 2^23 rounds x to an integer held in the low mantissa bits of t, so
+// bits(t) << 23 == n << 23 (mod 2^32).
+constexpr float kExpShift = 12582912.0f;  // 1.5 * 2^23
+constexpr float kExpC0 = 0.99992806f, kExpC1 = 0.69326097f, kExpC2 = 0.24261113f, kExpC3 = 0.05517167f;
+
+__device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float& y0, float& y1) {
+  const uint64_t x = f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t t = f2_add(x, f2_pack(kExpShift, kExpShift));
+  const uint64_t n = f2_add(t, f2_pack(-kExpShift, -kExpShift));
+  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), x);
+  uint64_t q = f2_fma(f2_pack(kExpC3, kExpC3), f, f2_pack(kExpC2, kExpC2));
+  q = f2_fma(q, f, f2_pack(kExpC1, kExpC1));
+  q = f2_fma(q, f, f2_pack(kExpC0, kExpC0));
+  float q0, q1, t0, t1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(t, t0, t1);
+  y0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
+// Pairs of keys whose exponentials go to the FMA pipe instead of the MUFU: one pair in four.
+__host__ __device__ constexpr bool exp_on_fma(int pair) { return (pair & 3) == 3; }
+
+// P = 2^(s*scale - m) for keys 64*half .. 64*half+63 of the row, packed to bf16 pairs and
+// stored over TMEM columns 32*half .. 32*half+31 of the row's S tile (keys 2c, 2c+1 ->
+// column c). Returns the fp32 sum of these P. The exponent argument of two keys is one
+// packed FMA; with kEmulate, one pair in four is exponentiated on the FMA pipe.
+template <bool kEmulate>
+__device__ __forceinline__ float exp_pack_store(const uint32_t (&sr)[4][32], int half, float scale, float m_use,
                                                 uint32_t taddr) {
   const uint64_t scale2 = f2_pack(scale, scale);
   const uint64_t negm2 = f2_pack(-m_use, -m_use);
   uint64_t sum_a = f2_pack(0.f, 0.f), sum_b = f2_pack(0.f, 0.f);
+  uint32_t pk[32];
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    uint32_t pk[32];
+  for (int cc = 0; cc < 2; ++cc) {
+    const int c = 2 * half + cc;
 #pragma unroll
-    for (int cc = 0; cc < 2; ++cc) {
-      const int c = 2 * half + cc;
-#pragma unroll
-      for (int e = 0; e < 32; e += 2) {
-        const uint64_t arg = f2_fma(f2_pack(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])), scale2, negm2);
-        float a0, a1;
-        f2_unpack(arg, a0, a1);
-        const float p0 = fast_exp2(a0);
-        const float p1 = fast_exp2(a1);
-        if ((e >> 1) & 1)
-          sum_b = f2_add(sum_b, f2_pack(p0, p1));
-        else
-          sum_a = f2_add(sum_a, f2_pack(p0, p1));
-        pk[cc * 16 + (e >> 1)] = pack_bf16x2(p0, p1);
+    for (int e = 0; e < 32; e += 2) {
+      const uint64_t arg = f2_fma(f2_pack(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])), scale2, negm2);
+      float a0, a1, p0, p1;
+      f2_unpack(arg, a0, a1);
+      if (kEmulate && exp_on_fma(e >> 1)) {
+        exp2_poly_x2(a0, a1, p0, p1);
+      } else {
+        p0 = fast_exp2(a0);
+        p1 = fast_exp2(a1);
       }
+      if ((e >> 1) & 1)
+        sum_b = f2_add(sum_b, f2_pack(p0, p1));
+      else
+        sum_a = f2_add(sum_a, f2_pack(p0, p1));
+      pk[cc * 16 + (e >> 1)] = pack_bf16x2(p0, p1);
     }
-    tmem_st_32x32b_x32(taddr + 32 * half, pk);
   }
+  tmem_st_32x32b_x32(taddr + 32 * half, pk);
   float s0, s1, s2, s3;
   f2_unpack(sum_a, s0, s1);
   f2_unpack(sum_b, s2, s3);
@@ -169,7 +199,7 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i) {
       uint32_t count = 1;
-      if (i == kPFull || i == kPFull + 1) count = 128;  // every softmax thread of the branch
+      if (i >= kPFull && i < kPFull + 4) count = 128;  // every softmax thread of the branch
       mbar_init(bar(i), count);
     }
     *abort_flag = 0;
@@ -239,6 +269,19 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       auto desc_v = [&](int s, int kk) {
         return sdesc_sw128(sbase + kOffV + s * kTileBytes + kk * 2048, kChunkBytes, 1024);
       };
+      // O_b (+)= P_b V for KV tile j: the first 64 keys as soon as that half of P is in TMEM,
+      // the other 64 when the second half is
+      auto issue_pv = [&](uint32_t o_tmem, uint32_t p_tmem, int stage, int j, uint32_t half0, uint32_t half1) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (!mbar_wait(h ? half1 : half0, j & 1, abort_flag)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
+            mma_bf16_ts(o_tmem, p_tmem + kk * 8, desc_v(stage, kk), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        return true;
+      };
       bool ok = mbar_wait(bar(kQFull), 0, abort_flag);
       for (int j = 0; ok && j < n_kv; ++j) {
         const int s = j & 1;
@@ -251,12 +294,7 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         tc_commit(bar(kSFull + 0));
         if (j > 0) {
           const int sp = (j - 1) & 1;
-          if (!(ok = mbar_wait(bar(kPFull + 1), (j - 1) & 1, abort_flag))) break;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk)
-            mma_bf16_ts(tmem + kTmO2, tmem + kTmS2 + kk * 8, desc_v(sp, kk), idesc_pv,
-                        (j - 1 > 0 || kk > 0) ? 1u : 0u);
+          if (!(ok = issue_pv(tmem + kTmO2, tmem + kTmS2, sp, j - 1, bar(kPFull + 2), bar(kPFull + 3)))) break;
           tc_commit(bar(kVEmpty + sp));
         }
 #pragma unroll
@@ -265,22 +303,12 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         tc_commit(bar(kSFull + 1));
         tc_commit(bar(kKEmpty + s));
         if (!(ok = mbar_wait(bar(kVFull + s), ph, abort_flag))) break;
-        if (!(ok = mbar_wait(bar(kPFull + 0), j & 1, abort_flag))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_bf16_ts(tmem + kTmO1, tmem + kTmS1 + kk * 8, desc_v(s, kk), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        if (!(ok = issue_pv(tmem + kTmO1, tmem + kTmS1, s, j, bar(kPFull + 0), bar(kPFull + 1)))) break;
       }
       if (ok) {
         const int jl = n_kv - 1;
         const int sl = jl & 1;
-        if (mbar_wait(bar(kPFull + 1), jl & 1, abort_flag)) {
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk)
-            mma_bf16_ts(tmem + kTmO2, tmem + kTmS2 + kk * 8, desc_v(sl, kk), idesc_pv, (jl > 0 || kk > 0) ? 1u : 0u);
-          tc_commit(bar(kOFull));
-        }
+        if (issue_pv(tmem + kTmO2, tmem + kTmS2, sl, jl, bar(kPFull + 2), bar(kPFull + 3))) tc_commit(bar(kOFull));
       }
       // every MMA of this CTA must be complete before tensor memory is freed
       tc_commit(bar(kDrain));
@@ -300,7 +328,8 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     bool ok = true;
 
     for (int j = 0; j < n_kv; ++j) {
-      if (!(ok = mbar_wait(bar(kSFull + br), j & 1, abort_flag))) break;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(kSFull + br), j & 1, abort_flag));
+      if (!ok) break;
       tc_fence_after();
       uint32_t sr[4][32];
 #pragma unroll
@@ -312,10 +341,15 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 
       // Keys visible to this row in this tile are columns 0..lim; only the diagonal tile of
       // a causal launch and a ragged last key tile have lim < 127.
-      int lim = BN - 1;
-      if (p.causal && j == tile) lim = r;
-      lim = min(lim, p.S - 1 - j * BN);
-      if (lim < BN - 1) mask_row(sr, lim);
+      // tile_masked is uniform over the CTA: every branch below that holds a warp-collective
+      // tcgen05 instruction must be taken by all 32 lanes together
+      const bool tile_masked = (p.causal && j == tile) || ((j + 1) * BN > p.S);
+      if (tile_masked) {
+        int lim = BN - 1;
+        if (p.causal && j == tile) lim = r;
+        lim = min(lim, p.S - 1 - j * BN);
+        mask_row(sr, lim);
+      }
       const float mx = row_max(sr) * p.scale_log2;
 
       // raise the running max only when the tile's max exceeds it by more than 2^8
@@ -326,30 +360,38 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         l_run *= alpha;
         m_run = mx;
       }
-      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      l_run += exp_pack_store(sr, p.scale_log2, m_use, trow + s_col);
-      if (rescale && j > 0) {
+      // the warp rescales its 32 rows together (alpha = 1 for rows that keep their max)
+      if (__any_sync(0xffffffffu, rescale) && j > 0) {
         // O_b holds the sum up to tile j-1, complete: S_b(j) was committed after PV_b(j-1),
-        // and PV_b(j) is issued only after this thread arrives on P_full below
+        // and PV_b(j) is issued only after this thread arrives on the P barriers below
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          tmem_ld_32x32b_x32(trow + o_col + 32 * c, o);
-          tmem_ld_wait(o);
+        for (int c = 0; c < 8; ++c) {
+          uint32_t o[16];
+          tmem_ld_32x32b_x16(trow + o_col + 16 * c, o);
+          tmem_ld_wait16(o);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st_32x32b_x32(trow + o_col + 32 * c, o);
+          for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st_32x32b_x16(trow + o_col + 16 * c, o);
         }
       }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bar(kPFull + br));
+      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+      float lsum = 0.f;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        // masked tiles take every exponential on the MUFU so masked keys stay exactly 0
+        lsum += tile_masked ? exp_pack_store<false>(sr, half, p.scale_log2, m_use, trow + s_col)
+                            : exp_pack_store<true>(sr, half, p.scale_log2, m_use, trow + s_col);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(kPFull + 2 * br + half));
+      }
+      l_run += lsum;
     }
 
     if (ok) ok = mbar_wait(bar(kOFull), 0, abort_flag);
     l_xchg[br * BM + r] = l_run;
     asm volatile("bar.sync 1, 256;" ::: "memory");
-    if (ok && !*abort_flag) {
+    if (__all_sync(0xffffffffu, ok && !*abort_flag)) {
       tc_fence_after();
       const float inv1 = 1.f / l_xchg[r];
       const float inv2 = 1.f / l_xchg[BM + r];
@@ -388,6 +430,7 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag) atomicCAS(p.err, 0, kErrPrefillWait);
   if (warp == 9) {
+    __syncwarp();  // lane 0 ran the MMA loop alone; dealloc is warp-collective
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
