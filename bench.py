@@ -146,6 +146,28 @@ def _dist_init(n_gpus):
     return 0, 1, 0, None
 
 
+def head_shard(Hq, Hkv, world, rank):
+    """KV heads and query heads of `rank` when the heads are split over `world` GPUs.
+
+    Returns (kv0, kv1, q0, q1): KV heads [kv0, kv1) and their query heads [q0, q1). Whole
+    GQA groups move together, so every pair of adjacent query heads keeps its K/V head and
+    the ranks never exchange data: each computes out[..., q0/2:q1/2, :] on its own.
+    """
+    if Hkv % world:
+        raise ValueError(f"Hkv={Hkv} KV heads do not split evenly over {world} ranks")
+    group = Hq // Hkv
+    per = Hkv // world
+    kv0, kv1 = rank * per, (rank + 1) * per
+    return kv0, kv1, kv0 * group, kv1 * group
+
+
+def shard_prefill_inputs(inp, Hq, Hkv, world, rank):
+    """Contiguous per-rank slices (q, k, v, lambda) of a head-sharded prefill."""
+    kv0, kv1, q0, q1 = head_shard(Hq, Hkv, world, rank)
+    return {"q": inp["q"][:, :, q0:q1].contiguous(), "k": inp["k"][:, :, kv0:kv1].contiguous(),
+            "v": inp["v"][:, :, kv0:kv1].contiguous(), "lam": inp["lam"][:, :, q0 // 2:q1 // 2].contiguous()}
+
+
 def _barrier(dist):
     if dist is not None:
         dist.barrier()
@@ -154,18 +176,34 @@ def _barrier(dist):
 def _max_over_ranks(x, dist):
     if dist is None:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
 # -------------------------------------------------------------------------- our arm
-def _inputs(rank, do_pre=True, do_dec=True):
+def _inputs(rank, do_pre=True, do_dec=True, world=1, strong=False):
+    """Per-rank inputs. Weak scaling: every rank its own seeded batch of the full size.
+    Strong scaling: one seeded problem, each rank its head shard (a whole number of GQA
+    groups), so the ranks together compute exactly the single-GPU workload."""
     pc = workloads.CONFIGS[PREFILL_CFG]
     dc = workloads.CONFIGS[DECODE_CFG]
-    pc = workloads.PrefillCase(**{**pc.__dict__, "seed": pc.seed + 100 * rank})
-    dc = workloads.DecodeCase(**{**dc.__dict__, "seed": dc.seed + 100 * rank})
-    return (pc, workloads.make_prefill(pc) if do_pre else None, dc, workloads.make_decode(dc) if do_dec else None)
+    if not strong:
+        pc = workloads.PrefillCase(**{**pc.__dict__, "seed": pc.seed + 100 * rank})
+        dc = workloads.DecodeCase(**{**dc.__dict__, "seed": dc.seed + 100 * rank})
+    pin = workloads.make_prefill(pc) if do_pre else None
+    din = workloads.make_decode(dc) if do_dec else None
+    if strong and world > 1:
+        kv0, kv1, q0, q1 = head_shard(pc.Hq, pc.Hkv, world, rank)
+        if pin is not None:
+            pin = shard_prefill_inputs(pin, pc.Hq, pc.Hkv, world, rank)
+        if din is not None:
+            din = {**din, "q": din["q"][:, q0:q1].contiguous(), "kcache": din["kcache"][:, :, kv0:kv1].contiguous(),
+                   "vcache": din["vcache"][:, :, kv0:kv1].contiguous(), "lam": din["lam"][:, q0 // 2:q1 // 2].contiguous()}
+        pc = workloads.PrefillCase(**{**pc.__dict__, "Hq": q1 - q0, "Hkv": kv1 - kv0})
+        dc = workloads.DecodeCase(**{**dc.__dict__, "Hq": q1 - q0, "Hkv": kv1 - kv0})
+    return pc, pin, dc, din
 
 
 def run_ours(args, rank, world, local, dist):
@@ -175,7 +213,8 @@ def run_ours(args, rank, world, local, dist):
     torch.cuda.set_device(dev)
     do_pre = args.only in (None, "prefill")
     do_dec = args.only in (None, "decode")
-    pc, pin, dc, din = _inputs(rank, do_pre, do_dec)
+    strong = args.scaling == "strong"
+    pc, pin, dc, din = _inputs(rank, do_pre, do_dec, world, strong)
     stream = torch.cuda.current_stream(dev)
 
     # device-resident inputs and outputs
@@ -277,7 +316,8 @@ def run_ours(args, rank, world, local, dist):
     dec_launch_ms = dec_ms / K
     tflops = flops / (pre_launch_ms * 1e-3) / 1e12 if do_pre else 0.0
     gbs = dbytes / (dec_launch_ms * 1e-3) / 1e9 if do_dec else 0.0
-    value = world * flops * K / (pre_ms * 1e-3) / 1e12 if do_pre else 0.0  # whole job: every rank's FLOPs
+    # whole job: every rank's work over the slowest rank's time (each rank's share is equal)
+    value = world * flops * K / (pre_ms * 1e-3) / 1e12 if do_pre else 0.0
     dec_value = world * dbytes * K / (dec_ms * 1e-3) / 1e9 if do_dec else 0.0
     peak_t = peaks["bf16_tflops"]
     tr = NCU_TRAFFIC["prefill"]
@@ -293,7 +333,7 @@ def run_ours(args, rank, world, local, dist):
         "warmup": max(args.warmup, 3),
         "ms_per_step": round(total_ms / K, 4),
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": args.scaling,
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic: seeded N(0,1) q/k/v rounded to bf16, lambda = sigmoid(N(0,1)) fp32, "
@@ -305,7 +345,8 @@ def run_ours(args, rank, world, local, dist):
                         "flops_per_step": flops},
             "decode": {"B": dc.B, "Smax": dc.Smax, "Hq": dc.Hq, "Hkv": dc.Hkv, "D": dc.D,
                        "sum_seqlens": int(din["seqlens"].sum()) if do_dec else None, "bytes_per_step": dbytes},
-            "parallelism": f"replicas x{world} (independent per-GPU batches)",
+            "parallelism": (f"head-parallel x{world} (whole GQA groups per rank, no data exchange)" if strong
+                            else f"replicas x{world} (independent per-GPU batches)"),
             "l2": "no flush: inputs larger than L2 (q 268 MB; decode streams 1.2 GB per step)",
         },
         "decode": {
@@ -458,6 +499,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=120.0,
                     help="host-time budget of the whole reference run (warm-up and timed steps)")
+    ap.add_argument("--scaling", choices=("weak", "strong"), default="weak",
+                    help="weak: each GPU runs the full per-GPU workload; strong: the heads of one workload "
+                         "are split over the GPUs")
     ap.add_argument("--only", choices=("prefill", "decode"), default=None,
                     help="run one half of the step (for profiling a single kernel on less device memory)")
     args = ap.parse_args(argv)

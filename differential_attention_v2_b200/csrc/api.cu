@@ -6,7 +6,7 @@
 
 #include <mutex>
 
-#include "../../include/diffattn_v2.h"
+#include "diffattn_v2.h"
 #include "internal.h"
 
 namespace {

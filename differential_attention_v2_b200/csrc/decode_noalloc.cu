@@ -18,7 +18,7 @@
 
 #include <cudaTypedefs.h>
 
-#include "../../include/diffattn_v2.h"
+#include "diffattn_v2.h"
 #include "internal.h"
 
 namespace {

@@ -129,8 +129,17 @@ __device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float& y0, floa
   y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
-// Pairs of keys whose exponentials go to the FMA pipe instead of the MUFU: one pair in four.
-__host__ __device__ constexpr bool exp_on_fma(int pair) { return (pair & 3) == 3; }
+// Pairs of keys whose exponentials go to the FMA pipe instead of the MUFU: one pair in
+// kExpFmaEvery (0: none). Measured on B200 (B=4 x 4k and 1 x 32k causal): none is fastest.
+// The kernel runs at the 1 kW power cap, where the extra FMA-pipe work lowers the SM clock
+// by more than the MUFU time it saves.
+#ifndef DA2_EXP_FMA_EVERY
+#define DA2_EXP_FMA_EVERY 0
+#endif
+constexpr int kExpFmaEvery = DA2_EXP_FMA_EVERY;
+__host__ __device__ constexpr bool exp_on_fma(int pair) {
+  return kExpFmaEvery > 0 && (pair % (kExpFmaEvery > 0 ? kExpFmaEvery : 1)) == (kExpFmaEvery - 1);
+}
 
 // P = 2^(s*scale - m) for keys 64*half .. 64*half+63 of the row, packed to bf16 pairs and
 // stored over TMEM columns 32*half .. 32*half+31 of the row's S tile (keys 2c, 2c+1 ->
