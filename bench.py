@@ -52,8 +52,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic per launch from an ncu capture, keyed by the kernel source it was taken on;
 # reported as null once the source differs from the one captured.
 NCU_TRAFFIC = {
-    "prefill": {"bytes": None, "source_sha": None},
-    "decode": {"bytes": None, "source_sha": None},
+    # dram__bytes_read.sum + dram__bytes_write.sum of one launch (B=4 x 4k causal prefill)
+    "prefill": {"bytes": 766537216, "source_sha": "cc174fd0353f516e"},
+    # split (1.228e9 + 9.13e6) + combine (6.62e6) of one B=64 decode step
+    "decode": {"bytes": 1243700000, "source_sha": "bbed945a81dc3b45"},
 }
 
 

@@ -27,9 +27,12 @@ _SIGNATURES = {
     "diffattn_v2_status_string": (ctypes.c_char_p, [_i]),
     "diffattn_v2_prefill": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
     "diffattn_v2_prefill_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
+    "diffattn_v2_prefill_window": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
+    "diffattn_v2_prefill_varlen": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]),
     "diffattn_v2_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "diffattn_v2_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "diffattn_v2_decode_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
+    "diffattn_v2_decode_paged": (_i, [_vp] * 7 + [_i] * 7 + [_vp, _sz, _vp]),
     "diffattn_v2_lambda_v1": (_i, [_vp, _vp, _vp, _vp, _f, _i, _i, _i, _vp, _vp]),
     "diffattn_v2_device_error": (_i, [ctypes.POINTER(_i), _vp]),
     "diffattn_v2_decode_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
@@ -107,6 +110,41 @@ def prefill(q, k, v, lam, out=None, causal=True, stream=None):
     return out
 
 
+def prefill_window(q, k, v, lam, window, out=None, stream=None):
+    """bf16 causal prefill where query i sees only keys i-window+1 .. i."""
+    for t, n, nd in ((q, "q", 4), (k, "k", 4), (v, "v", 4)):
+        _need(t, n, torch.bfloat16, nd)
+    _need(lam, "lam", torch.float32, 3)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if out is None:
+        out = torch.empty((B, S, Hq // 2, D), dtype=torch.bfloat16, device=q.device)
+    _need(out, "out", torch.bfloat16, 4)
+    st = LIB.diffattn_v2_prefill_window(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(out), B, S, Hq, Hkv, D,
+                                        int(window), _stream(stream, q.device))
+    _check(st, "diffattn_v2_prefill_window")
+    return out
+
+
+def prefill_varlen(q, k, v, lam, cu_seqlens, max_seqlen, out=None, causal=True, stream=None):
+    """bf16 prefill of packed sequences: q [T,Hq,D], k/v [T,Hkv,D], lam fp32 [T,Hq/2],
+    cu_seqlens int32 [B+1] on the device; max_seqlen >= the longest sequence."""
+    for t, n, nd in ((q, "q", 3), (k, "k", 3), (v, "v", 3)):
+        _need(t, n, torch.bfloat16, nd)
+    _need(lam, "lam", torch.float32, 2)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    T, Hq, D = q.shape
+    Hkv = k.shape[1]
+    B = cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty((T, Hq // 2, D), dtype=torch.bfloat16, device=q.device)
+    _need(out, "out", torch.bfloat16, 3)
+    st = LIB.diffattn_v2_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(out), _ptr(cu_seqlens), B,
+                                        int(max_seqlen), T, Hq, Hkv, D, 1 if causal else 0, _stream(stream, q.device))
+    _check(st, "diffattn_v2_prefill_varlen")
+    return out
+
+
 def prefill_f32(q, k, v, lam, out=None, causal=True, stream=None):
     """fp32 prefill on CUDA cores; same layout as prefill with fp32 tensors."""
     for t, n, nd in ((q, "q", 4), (k, "k", 4), (v, "v", 4), (lam, "lam", 3)):
@@ -145,6 +183,31 @@ def decode(q, kcache, vcache, seqlens, lam, out=None, workspace=None, stream=Non
                                 Hq, Hkv, D, _ptr(workspace), workspace.numel() * workspace.element_size(),
                                 _stream(stream, q.device))
     _check(st, "diffattn_v2_decode")
+    return out
+
+
+def decode_paged(q, kpages, vpages, block_table, seqlens, lam, out=None, workspace=None, stream=None):
+    """bf16 decode over a paged cache: kpages/vpages [num_pages, page_size, Hkv, D],
+    block_table int32 [B, max_pages], seqlens int32 [B], lam fp32 [B, Hq/2]."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(kpages, "kpages", torch.bfloat16, 4)
+    _need(vpages, "vpages", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seqlens, "seqlens", torch.int32, 1)
+    _need(lam, "lam", torch.float32, 2)
+    B, Hq, D = q.shape
+    num_pages, page_size, Hkv = kpages.shape[0], kpages.shape[1], kpages.shape[2]
+    max_pages = block_table.shape[1]
+    if out is None:
+        out = torch.empty((B, Hq // 2, D), dtype=torch.bfloat16, device=q.device)
+    _need(out, "out", torch.bfloat16, 3)
+    need = decode_workspace_size(B, max_pages * page_size, Hq, Hkv, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    st = LIB.diffattn_v2_decode_paged(_ptr(q), _ptr(kpages), _ptr(vpages), _ptr(block_table), _ptr(seqlens), _ptr(lam),
+                                      _ptr(out), B, max_pages, page_size, num_pages, Hq, Hkv, D, _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), _stream(stream, q.device))
+    _check(st, "diffattn_v2_decode_paged")
     return out
 
 

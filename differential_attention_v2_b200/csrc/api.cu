@@ -133,8 +133,54 @@ int diffattn_v2_prefill(const void* q, const void* k, const void* v, const float
   if (encode_bshd(&tq, q, D, Hq, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tk, k, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tv, v, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
-  e = da2::launch_prefill(tq, tk, tv, lambda, static_cast<__nv_bfloat16*>(out), err, B, S, Hq, Hkv, causal,
-                          reinterpret_cast<cudaStream_t>(stream));
+  e = da2::launch_prefill(tq, tk, tv, lambda, static_cast<__nv_bfloat16*>(out), err, B, S, Hq, Hkv, causal, 0,
+                          nullptr, reinterpret_cast<cudaStream_t>(stream));
+  return status_of(e);
+}
+
+int diffattn_v2_prefill_window(const void* q, const void* k, const void* v, const float* lambda, void* out, int B,
+                               int S, int Hq, int Hkv, int D, int window, da2_stream_t stream) {
+  if (B < 0 || S < 0 || D <= 0 || !heads_ok(Hq, Hkv) || window < 1) return DA2_ERR_INVALID;
+  if (B == 0 || S == 0) return DA2_OK;
+  if (!q || !k || !v || !lambda || !out) return DA2_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(lambda) || !aligned16(out))
+    return DA2_ERR_INVALID;
+  if (D != 128) return DA2_ERR_UNSUPPORTED;
+  if ((S + 127) / 128 > 65535) return DA2_ERR_UNSUPPORTED;
+  int* err = nullptr;
+  cudaError_t e = device_error_ptr(&err);
+  if (e != cudaSuccess) return DA2_ERR_CUDA;
+  CUtensorMap tq, tk, tv;
+  if (encode_bshd(&tq, q, D, Hq, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  if (encode_bshd(&tk, k, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  if (encode_bshd(&tv, v, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  // a window of S or more keys is the plain causal mask
+  e = da2::launch_prefill(tq, tk, tv, lambda, static_cast<__nv_bfloat16*>(out), err, B, S, Hq, Hkv, 1,
+                          window >= S ? 0 : window, nullptr, reinterpret_cast<cudaStream_t>(stream));
+  return status_of(e);
+}
+
+int diffattn_v2_prefill_varlen(const void* q, const void* k, const void* v, const float* lambda, void* out,
+                               const int32_t* cu_seqlens, int B, int max_seqlen, int total_tokens, int Hq, int Hkv,
+                               int D, int causal, da2_stream_t stream) {
+  if (B < 0 || max_seqlen < 0 || total_tokens < 0 || D <= 0 || !heads_ok(Hq, Hkv)) return DA2_ERR_INVALID;
+  if (causal != 0 && causal != 1) return DA2_ERR_INVALID;
+  if (B == 0 || max_seqlen == 0 || total_tokens == 0) return DA2_OK;
+  if (!q || !k || !v || !lambda || !out || !cu_seqlens) return DA2_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(lambda) || !aligned16(out) ||
+      !aligned16(cu_seqlens))
+    return DA2_ERR_INVALID;
+  if (D != 128) return DA2_ERR_UNSUPPORTED;
+  if ((max_seqlen + 127) / 128 > 65535) return DA2_ERR_UNSUPPORTED;
+  int* err = nullptr;
+  cudaError_t e = device_error_ptr(&err);
+  if (e != cudaSuccess) return DA2_ERR_CUDA;
+  CUtensorMap tq, tk, tv;  // the packed tokens as one batch of total_tokens rows
+  if (encode_bshd(&tq, q, D, Hq, total_tokens, 1, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  if (encode_bshd(&tk, k, D, Hkv, total_tokens, 1, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  if (encode_bshd(&tv, v, D, Hkv, total_tokens, 1, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  e = da2::launch_prefill(tq, tk, tv, lambda, static_cast<__nv_bfloat16*>(out), err, B, max_seqlen, Hq, Hkv, causal,
+                          0, cu_seqlens, reinterpret_cast<cudaStream_t>(stream));
   return status_of(e);
 }
 
@@ -185,7 +231,43 @@ int diffattn_v2_decode(const void* q, const void* kcache, const void* vcache, co
   float* ws_ml = ws_o + static_cast<size_t>(B) * Hq * nsplit * D;
   e = da2::launch_decode(tk, tv, static_cast<const __nv_bfloat16*>(q), seqlens, lambda,
                          static_cast<__nv_bfloat16*>(out), ws_o, ws_ml, err, B, Smax, Hq, Hkv, nsplit, split_len,
-                         reinterpret_cast<cudaStream_t>(stream));
+                         nullptr, 0, 0, reinterpret_cast<cudaStream_t>(stream));
+  return status_of(e);
+}
+
+int diffattn_v2_decode_paged(const void* q, const void* kpages, const void* vpages, const int32_t* block_table,
+                             const int32_t* seqlens, const float* lambda, void* out, int B, int max_pages,
+                             int page_size, int num_pages, int Hq, int Hkv, int D, void* workspace,
+                             size_t workspace_bytes, da2_stream_t stream) {
+  if (B < 0 || max_pages <= 0 || num_pages <= 0 || D <= 0 || !heads_ok(Hq, Hkv)) return DA2_ERR_INVALID;
+  if (page_size < 8 || page_size > 4096 || (page_size & (page_size - 1)) != 0) return DA2_ERR_INVALID;
+  if (static_cast<long long>(max_pages) * page_size > (1LL << 30)) return DA2_ERR_INVALID;
+  if (B == 0) return DA2_OK;
+  if (!q || !kpages || !vpages || !block_table || !seqlens || !lambda || !out || !workspace) return DA2_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(kpages) || !aligned16(vpages) || !aligned16(block_table) || !aligned16(seqlens) ||
+      !aligned16(lambda) || !aligned16(out) || !aligned16(workspace))
+    return DA2_ERR_INVALID;
+  const int Smax = max_pages * page_size;
+  if (workspace_bytes < diffattn_v2_decode_workspace_size(B, Smax, Hq, Hkv, D)) return DA2_ERR_INVALID;
+  const int group = Hq / Hkv;
+  if (D != 128 || !(group == 2 || group == 4 || group == 8 || group == 16)) return DA2_ERR_UNSUPPORTED;
+  if (B > 65535 || Hkv > 65535) return DA2_ERR_UNSUPPORTED;
+  int* err = nullptr;
+  cudaError_t e = device_error_ptr(&err);
+  if (e != cudaSuccess) return DA2_ERR_CUDA;
+  int split_len = 0, nsplit = 0;
+  da2::decode_split_plan(B, Smax, Hkv, &split_len, &nsplit);
+  int page_shift = 0;
+  while ((1 << page_shift) < page_size) ++page_shift;
+  const uint32_t box = static_cast<uint32_t>(page_size < 64 ? page_size : 64);
+  CUtensorMap tk, tv;  // pages as a [num_pages, page_size] batch of rows
+  if (encode_bshd(&tk, kpages, D, Hkv, page_size, num_pages, 64, box) != cudaSuccess) return DA2_ERR_CUDA;
+  if (encode_bshd(&tv, vpages, D, Hkv, page_size, num_pages, 64, box) != cudaSuccess) return DA2_ERR_CUDA;
+  float* ws_o = static_cast<float*>(workspace);
+  float* ws_ml = ws_o + static_cast<size_t>(B) * Hq * nsplit * D;
+  e = da2::launch_decode(tk, tv, static_cast<const __nv_bfloat16*>(q), seqlens, lambda,
+                         static_cast<__nv_bfloat16*>(out), ws_o, ws_ml, err, B, Smax, Hq, Hkv, nsplit, split_len,
+                         block_table, max_pages, page_shift, reinterpret_cast<cudaStream_t>(stream));
   return status_of(e);
 }
 

@@ -44,7 +44,9 @@ constexpr uint32_t kHalfBytes = kTok * 64 * 2;        // 64 tokens x 64 d bf16 =
 constexpr uint32_t kStageBytes = 4 * kHalfBytes;      // K lo/hi + V lo/hi = 32 KB
 constexpr uint32_t kOffBar = kStages * kStageBytes;
 constexpr uint32_t kOffMisc = kOffBar + 8 * 2 * kStages;
-constexpr uint32_t kSmemUsed = kOffMisc + 16;
+constexpr uint32_t kOffPages = kOffMisc + 16;                // page indices of a paged split
+constexpr int kMaxSplitPages = 512;                           // split_len (<= 4096) / page_size (>= 8)
+constexpr uint32_t kSmemUsed = kOffPages + 4 * kMaxSplitPages;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;
 
 struct Params {
@@ -55,6 +57,10 @@ struct Params {
   int* err;
   int B, Smax, Hq, Hkv, nsplit, split_len;
   float scale_log2;
+  // paged caches [num_pages, page_size, Hkv, D]: logical token t of sequence b is row
+  // t % page_size of page block_table[b * max_pages + t / page_size]; null = [B, Smax] caches
+  const int32_t* block_table;
+  int max_pages, page_shift, box_tok;  // page_size = 1 << page_shift; tokens per TMA box
 };
 
 // NT = number of 8-head column tiles per group (1 for group size <= 8, 2 for 16).
@@ -94,6 +100,16 @@ diffattn_decode_split(const __grid_constant__ CUtensorMap tmK, const __grid_cons
 
   if (warp == kConsumerWarps) {
     // --------------------------------------------------------------------- producer
+    int* pages = reinterpret_cast<int*>(smem + kOffPages);
+    const int page_size = 1 << p.page_shift;
+    const int first_page = t0 >> p.page_shift;
+    if (p.block_table) {
+      // the split's page indices, read once: logical pages first_page .. (t1-1) / page_size
+      const int n_pages = ((t1 - 1) >> p.page_shift) - first_page + 1;
+      for (int i = lane; i < n_pages; i += 32)
+        pages[i] = __ldg(p.block_table + static_cast<size_t>(b) * p.max_pages + first_page + i);
+      __syncwarp();
+    }
     if (lane == 0) {
       int issued = 0;
       for (int i = 0; i < n_stages; ++i) {
@@ -103,10 +119,26 @@ diffattn_decode_split(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         const uint32_t dst = sbase + s * kStageBytes;
         const int tok = t0 + i * kTok;
         mbar_arrive_expect_tx(full(s), kStageBytes);
-        tma_load_4d(dst + 0 * kHalfBytes, &tmK, full(s), 0, g, tok, b);
-        tma_load_4d(dst + 1 * kHalfBytes, &tmK, full(s), 64, g, tok, b);
-        tma_load_4d(dst + 2 * kHalfBytes, &tmV, full(s), 0, g, tok, b);
-        tma_load_4d(dst + 3 * kHalfBytes, &tmV, full(s), 64, g, tok, b);
+        if (!p.block_table) {
+          tma_load_4d(dst + 0 * kHalfBytes, &tmK, full(s), 0, g, tok, b);
+          tma_load_4d(dst + 1 * kHalfBytes, &tmK, full(s), 64, g, tok, b);
+          tma_load_4d(dst + 2 * kHalfBytes, &tmV, full(s), 0, g, tok, b);
+          tma_load_4d(dst + 3 * kHalfBytes, &tmV, full(s), 64, g, tok, b);
+        } else {
+          // one box per page (or per 64 tokens of a larger page); a box's rows land at the
+          // same smem rows a single 64-token box would fill, so the swizzle is unchanged.
+          // Tokens past the sequence read page -1: out of range, filled with zeros.
+          for (int sb = 0; sb < kTok; sb += p.box_tok) {
+            const int tk = tok + sb;
+            const int page = tk < t1 ? pages[(tk >> p.page_shift) - first_page] : -1;
+            const int row = tk & (page_size - 1);
+            const uint32_t o = static_cast<uint32_t>(sb) * 128u;
+            tma_load_4d(dst + 0 * kHalfBytes + o, &tmK, full(s), 0, g, row, page);
+            tma_load_4d(dst + 1 * kHalfBytes + o, &tmK, full(s), 64, g, row, page);
+            tma_load_4d(dst + 2 * kHalfBytes + o, &tmV, full(s), 0, g, row, page);
+            tma_load_4d(dst + 3 * kHalfBytes + o, &tmV, full(s), 64, g, row, page);
+          }
+        }
         issued = i + 1;
       }
       if (*abort_flag) {
@@ -345,7 +377,8 @@ diffattn_decode_combine(const float* __restrict__ ws_o, const float* __restrict_
 cudaError_t launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const __nv_bfloat16* q,
                           const int32_t* seqlens, const float* lambda, __nv_bfloat16* out, float* ws_o,
                           float* ws_ml, int* err, int B, int Smax, int Hq, int Hkv, int nsplit,
-                          int split_len, cudaStream_t stream) {
+                          int split_len, const int32_t* block_table, int max_pages, int page_shift,
+                          cudaStream_t stream) {
   using namespace decode;
   Params p;
   p.q = q;
@@ -360,6 +393,10 @@ cudaError_t launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const 
   p.nsplit = nsplit;
   p.split_len = split_len;
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HD));
+  p.block_table = block_table;
+  p.max_pages = max_pages;
+  p.page_shift = page_shift;
+  p.box_tok = block_table ? min(1 << page_shift, kTok) : kTok;
   const int group = Hq / Hkv;
   dim3 grid(nsplit, Hkv, B);
   cudaError_t e;

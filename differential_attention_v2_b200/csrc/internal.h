@@ -9,18 +9,23 @@
 
 namespace da2 {
 
-// bf16 prefill on tcgen05 (D = 128). Tensor maps: Q over [B,S,Hq,D], K/V over [B,S,Hkv,D],
+// bf16 prefill on tcgen05 (D = 128); window > 0 (causal only) limits query i to keys
+// i-window+1 .. i. With cu_seqlens (device, B+1 entries) the tensors hold B packed sequences
+// as one [1,T] batch and S is the longest sequence. Tensor maps: Q over [B,S,Hq,D], K/V over [B,S,Hkv,D],
 // boxes of 64 (d) x 1 (head) x 128 (rows) x 1, 128-byte swizzle.
 cudaError_t launch_prefill(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                            const float* lambda, __nv_bfloat16* out, int* err, int B, int S, int Hq, int Hkv,
-                           int causal, cudaStream_t stream);
+                           int causal, int window, const int* cu_seqlens, cudaStream_t stream);
 
 // bf16 decode (D = 128): split kernel + combine. Tensor maps over the caches [B,Smax,Hkv,D],
-// boxes of 64 (d) x 1 x 64 (tokens) x 1, 128-byte swizzle.
+// boxes of 64 (d) x 1 x 64 (tokens) x 1, 128-byte swizzle. With block_table the maps cover
+// pages [num_pages, 1 << page_shift, Hkv, D] with boxes of min(page_size, 64) tokens and
+// Smax = max_pages << page_shift.
 cudaError_t launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const __nv_bfloat16* q,
                           const int32_t* seqlens, const float* lambda, __nv_bfloat16* out, float* ws_o,
                           float* ws_ml, int* err, int B, int Smax, int Hq, int Hkv, int nsplit,
-                          int split_len, cudaStream_t stream);
+                          int split_len, const int32_t* block_table, int max_pages, int page_shift,
+                          cudaStream_t stream);
 
 // Tokens per split and number of splits of the bf16 decode for these sizes.
 void decode_split_plan(int B, int Smax, int Hkv, int* split_len, int* nsplit);

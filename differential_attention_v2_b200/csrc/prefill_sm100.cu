@@ -77,17 +77,19 @@ struct Params {
   __nv_bfloat16* out;     // [B,S,Hq/2,D]
   int* err;               // device error word
   int B, S, Hq, Hkv, causal;
+  int window;             // causal sliding window (keys i-window+1 .. i); 0 = none
+  const int* cu_seqlens;  // packed sequences: sequence b is tokens cu[b] .. cu[b+1]-1; null = [B,S]
   int n_row_tiles;
   float scale_log2;       // log2(e)/sqrt(D)
 };
 
-// Set scores of keys past column `lim` of this row to -inf.
-__device__ __forceinline__ void mask_row(uint32_t (&sr)[4][32], int lim) {
+// Set scores of keys outside columns lo..hi of this row to -inf.
+__device__ __forceinline__ void mask_row(uint32_t (&sr)[4][32], int lo, int hi) {
 #pragma unroll
   for (int c = 0; c < 4; ++c)
 #pragma unroll
     for (int e = 0; e < 32; ++e)
-      if (32 * c + e > lim) sr[c][e] = __float_as_uint(-INFINITY);
+      if (32 * c + e > hi || 32 * c + e < lo) sr[c][e] = __float_as_uint(-INFINITY);
 }
 
 // Max of the 128 raw scores of a row: 3-input max, four independent chains.
@@ -180,6 +182,9 @@ __device__ __forceinline__ float exp_pack_store(const uint32_t (&sr)[4][32], int
   return (s0 + s1) + (s2 + s3);
 }
 
+// kVarlen: packed sequences (p.cu_seqlens); kWindow: causal sliding window (p.window). The
+// plain [B,S] prefill is the <false, false> instance and carries neither.
+template <bool kVarlen, bool kWindow>
 __global__ void __launch_bounds__(kThreads, 1)
 diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const Params p) {
@@ -202,8 +207,22 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   const int group = p.Hq / p.Hkv;
   const int g = (2 * pair) / group;
   const int m0 = tile * BM;
-  const int n_kv_total = (p.S + BN - 1) / BN;
-  const int n_kv = p.causal ? min(tile + 1, n_kv_total) : n_kv_total;
+  // Sequence extent: a [B,S] batch, or packed sequences whose tensors are one [1,T] batch;
+  // tok0 is the sequence's first row in the tensor maps, row_base its first output row.
+  int S = p.S, tok0 = 0, tb = b;
+  if (kVarlen) {
+    tok0 = __ldg(p.cu_seqlens + b);
+    S = __ldg(p.cu_seqlens + b + 1) - tok0;
+    tb = 0;
+  }
+  if (m0 >= S) return;  // uniform over the CTA: this row tile lies past the sequence's end
+  const size_t row_base = kVarlen ? static_cast<size_t>(tok0) : static_cast<size_t>(b) * p.S;
+  const int n_kv_total = (S + BN - 1) / BN;
+  const int j_last = p.causal ? min(tile, n_kv_total - 1) : n_kv_total - 1;
+  // with a sliding window the first KV tile holds key m0 - window + 1 (or key 0)
+  const int win_lo = m0 - p.window + 1;
+  const int j_first = (kWindow && win_lo > 0) ? win_lo / BN : 0;
+  const int n_kv = j_last - j_first + 1;  // KV tiles this CTA visits: j = j_first + it
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i) {
@@ -235,23 +254,24 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       for (int h = 0; h < 2; ++h)
         for (int c = 0; c < 2; ++c)
           tma_load_4d(sbase + kOffQ + h * kTileBytes + c * kChunkBytes, &tmQ, bar(kQFull), c * 64,
-                      2 * pair + h, m0, b);
+                      2 * pair + h, tok0 + m0, tb);
       int k_issued = 0, v_issued = 0;
-      for (int j = 0; j < n_kv; ++j) {
-        const int s = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
+      for (int it = 0; it < n_kv; ++it) {
+        const int j = j_first + it;
+        const int s = it & 1;
+        const uint32_t ph = (it >> 1) & 1;
         if (!mbar_wait(bar(kKEmpty + s), ph ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(bar(kKFull + s), kTileBytes);
         for (int c = 0; c < 2; ++c)
           tma_load_4d(sbase + kOffK + s * kTileBytes + c * kChunkBytes, &tmK, bar(kKFull + s), c * 64, g,
-                      j * BN, b);
-        k_issued = j + 1;
+                      tok0 + j * BN, tb);
+        k_issued = it + 1;
         if (!mbar_wait(bar(kVEmpty + s), ph ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(bar(kVFull + s), kTileBytes);
         for (int c = 0; c < 2; ++c)
           tma_load_4d(sbase + kOffV + s * kTileBytes + c * kChunkBytes, &tmV, bar(kVFull + s), c * 64, g,
-                      j * BN, b);
-        v_issued = j + 1;
+                      tok0 + j * BN, tb);
+        v_issued = it + 1;
       }
       if (*abort_flag) {
         // let copies still in flight land before the CTA's shared memory is released
@@ -292,6 +312,8 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         return true;
       };
       bool ok = mbar_wait(bar(kQFull), 0, abort_flag);
+      // j counts the KV tiles this CTA visits (stage, parity, first-accumulate); the MMAs never
+      // need the tile's key position
       for (int j = 0; ok && j < n_kv; ++j) {
         const int s = j & 1;
         const uint32_t ph = (j >> 1) & 1;
@@ -336,8 +358,9 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     float l_run = 0.f;
     bool ok = true;
 
-    for (int j = 0; j < n_kv; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(kSFull + br), j & 1, abort_flag));
+    for (int it = 0; it < n_kv; ++it) {
+      const int j = j_first + it;  // KV tile index (key position); it drives the barriers
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(kSFull + br), it & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
       uint32_t sr[4][32];
@@ -352,12 +375,15 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       // a causal launch and a ragged last key tile have lim < 127.
       // tile_masked is uniform over the CTA: every branch below that holds a warp-collective
       // tcgen05 instruction must be taken by all 32 lanes together
-      const bool tile_masked = (p.causal && j == tile) || ((j + 1) * BN > p.S);
+      // some row of the tile has keys of this KV tile below its window
+      const bool win_edge = kWindow && j * BN < m0 + BM - p.window;
+      const bool tile_masked = (p.causal && j == tile) || ((j + 1) * BN > S) || win_edge;
       if (tile_masked) {
-        int lim = BN - 1;
-        if (p.causal && j == tile) lim = r;
-        lim = min(lim, p.S - 1 - j * BN);
-        mask_row(sr, lim);
+        int hi = BN - 1;
+        if (p.causal && j == tile) hi = r;
+        hi = min(hi, S - 1 - j * BN);
+        const int lo = kWindow ? qi - p.window + 1 - j * BN : 0;
+        mask_row(sr, lo, hi);
       }
       const float mx = row_max(sr) * p.scale_log2;
 
@@ -370,8 +396,9 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         m_run = mx;
       }
       // the warp rescales its 32 rows together (alpha = 1 for rows that keep their max)
-      if (__any_sync(0xffffffffu, rescale) && j > 0) {
-        // O_b holds the sum up to tile j-1, complete: S_b(j) was committed after PV_b(j-1),
+      if (__any_sync(0xffffffffu, rescale) && it > 0) {
+        // O_b holds the sum up to the previous tile, complete: S_b(j) was committed after that
+        // tile's PV_b,
         // and PV_b(j) is issued only after this thread arrives on the P barriers below
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
@@ -404,8 +431,8 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       tc_fence_after();
       const float inv1 = 1.f / l_xchg[r];
       const float inv2 = 1.f / l_xchg[BM + r];
-      const bool row_valid = qi < p.S;
-      const size_t row_off = (static_cast<size_t>(b) * p.S + (row_valid ? qi : 0)) * n_pairs + pair;
+      const bool row_valid = qi < S;
+      const size_t row_off = (row_base + (row_valid ? qi : 0)) * n_pairs + pair;
       const float lam = row_valid ? __ldg(p.lambda + row_off) : 0.f;
 #pragma unroll 1
       for (int cc = 0; cc < 2; ++cc) {
@@ -449,7 +476,7 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 
 cudaError_t launch_prefill(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                            const float* lambda, __nv_bfloat16* out, int* err, int B, int S, int Hq, int Hkv,
-                           int causal, cudaStream_t stream) {
+                           int causal, int window, const int* cu_seqlens, cudaStream_t stream) {
   using namespace prefill;
   Params p;
   p.lambda = lambda;
@@ -460,12 +487,16 @@ cudaError_t launch_prefill(const CUtensorMap& tmQ, const CUtensorMap& tmK, const
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.causal = causal;
+  p.window = window;
+  p.cu_seqlens = cu_seqlens;  // with packed sequences S is the longest sequence's length
   p.n_row_tiles = (S + BM - 1) / BM;
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HD));
-  cudaError_t e = cudaFuncSetAttribute(diffattn_prefill_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  auto kernel = cu_seqlens ? diffattn_prefill_sm100<true, false>
+                           : (window > 0 ? diffattn_prefill_sm100<false, true> : diffattn_prefill_sm100<false, false>);
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(B * (Hq / 2), p.n_row_tiles);
-  diffattn_prefill_sm100<<<grid, kThreads, kSmemBytes, stream>>>(tmQ, tmK, tmV, p);
+  kernel<<<grid, kThreads, kSmemBytes, stream>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError();
 }
 

@@ -92,6 +92,36 @@ DA2_API int diffattn_v2_prefill(const void* q, const void* k, const void* v, con
                         da2_stream_t stream);
 
 /*
+ * Causal prefill with a sliding window, bf16 in / bf16 out: query i sees keys
+ * max(0, i - window + 1) .. i (the window holds the query's own key). This is DiffAttn in a
+ * sliding-window layer, the hybrid the "Differential Attention (V2)" lesson's "Use it"
+ * section names, with the window mask of the "Attention variants" lesson, "Build it",
+ * Step 2. Arguments, layout and semantics as diffattn_v2_prefill with causal = 1;
+ * window >= 1 (window >= S is the plain causal prefill); window < 1 gives DA2_ERR_INVALID.
+ * Only the KV tiles that intersect a query tile's windows are read.
+ */
+DA2_API int diffattn_v2_prefill_window(const void* q, const void* k, const void* v, const float* lambda,
+                                       void* out, int B, int S, int Hq, int Hkv, int D, int window,
+                                       da2_stream_t stream);
+
+/*
+ * Prefill of B sequences of different lengths packed along the token axis (the layout of
+ * serving engines), bf16 in / bf16 out. Sequence b is tokens cu_seqlens[b] ..
+ * cu_seqlens[b+1]-1; each sequence is an independent prefill (its queries see only its own
+ * keys, causally when causal = 1).
+ *   q bf16 [T,Hq,D]   k, v bf16 [T,Hkv,D]   lambda fp32 [T,Hq/2]   out bf16 [T,Hq/2,D]
+ *   cu_seqlens int32 [B+1] (device), non-decreasing, cu_seqlens[0] = 0, cu_seqlens[B] = T
+ *   max_seqlen >= the longest sequence (sizes the grid; longer values only add idle CTAs)
+ *   total_tokens = T
+ * The caller guarantees the cu_seqlens contract; the kernel reads it on the device, so the
+ * call needs no host synchronisation. Supported: D == 128. Zero-length sequences are allowed.
+ */
+DA2_API int diffattn_v2_prefill_varlen(const void* q, const void* k, const void* v, const float* lambda,
+                                       void* out, const int32_t* cu_seqlens, int B, int max_seqlen,
+                                       int total_tokens, int Hq, int Hkv, int D, int causal,
+                                       da2_stream_t stream);
+
+/*
  * The same operator in fp32 end to end (CUDA-core arithmetic, no tensor cores), for
  * callers that need results within ~1e-5 of exact. q, k, v, out are fp32 with the prefill
  * layout above. Supported: D in {64, 128}. Same argument checks and semantics.
@@ -128,6 +158,26 @@ DA2_API int diffattn_v2_decode(const void* q, const void* kcache, const void* vc
                        const int32_t* seqlens, const float* lambda, void* out, int B, int Smax,
                        int Hq, int Hkv, int D, void* workspace, size_t workspace_bytes,
                        da2_stream_t stream);
+
+/*
+ * The bf16 decode step over a paged KV cache (the layout serving engines keep): the caches
+ * are pages of page_size tokens, and logical token t of sequence b is row t % page_size of
+ * page block_table[b * max_pages + t / page_size].
+ *   kpages, vpages bf16 [num_pages, page_size, Hkv, D]    block_table int32 [B, max_pages]
+ *   q, seqlens, lambda, out as in diffattn_v2_decode; seqlens[b] is clamped to
+ *   [0, max_pages * page_size]
+ *   workspace: diffattn_v2_decode_workspace_size(B, max_pages * page_size, Hq, Hkv, D) bytes
+ * page_size is a power of two in [8, 4096]. Entries of block_table past a sequence's last
+ * page are never read. Same kernels, arithmetic and results as diffattn_v2_decode on the
+ * gathered cache with Smax = max_pages * page_size (bit for bit). Source: the lesson's "Use
+ * it" section (integration into the vLLM and SGLang serving engines) and "V1 vs V2" (the
+ * cache is read once per step).
+ */
+DA2_API int diffattn_v2_decode_paged(const void* q, const void* kpages, const void* vpages,
+                                     const int32_t* block_table, const int32_t* seqlens,
+                                     const float* lambda, void* out, int B, int max_pages, int page_size,
+                                     int num_pages, int Hq, int Hkv, int D, void* workspace,
+                                     size_t workspace_bytes, da2_stream_t stream);
 
 /*
  * The decode step in fp32 end to end (CUDA cores), same layout with fp32 q, caches and

@@ -31,8 +31,11 @@ def _softmax(row):
     return [e / total for e in exps]
 
 
-def prefill(q, k, v, lam, causal=True):
-    """q[b][i][h][d], k/v[b][j][g][d], lam[b][i][p] -> out[b][i][p][d] (lists of floats)."""
+def prefill(q, k, v, lam, causal=True, window=None):
+    """q[b][i][h][d], k/v[b][j][g][d], lam[b][i][p] -> out[b][i][p][d] (lists of floats).
+
+    window (causal only): query i sees keys max(0, i - window + 1) .. i, the sliding-window
+    mask of the "Attention variants" lesson, Step 2."""
     B = len(q)
     S = len(q[0])
     Hq = len(q[0][0])
@@ -45,6 +48,8 @@ def prefill(q, k, v, lam, causal=True):
         for i in range(S):
             heads = []
             visible = list(range(i + 1)) if causal else list(range(S))
+            if window is not None:
+                visible = [j for j in visible if j >= i - window + 1]
             for p in range(Hq // 2):
                 h1, h2 = 2 * p, 2 * p + 1
                 g = (h1 * Hkv) // Hq

@@ -37,11 +37,14 @@ import numpy as np
 __all__ = [
     "stable_softmax",
     "causal_mask",
+    "window_mask",
     "pair_layout",
     "diff_attention_block",
     "prefill",
     "prefill_rows",
+    "prefill_varlen",
     "decode",
+    "decode_paged",
     "lambda_v1",
     "branch_weights",
     "snr",
@@ -69,6 +72,17 @@ def causal_mask(n_q: int, n_k: int, q_offset: int = 0) -> np.ndarray:
     i = np.arange(q_offset, q_offset + n_q)[:, None]
     j = np.arange(n_k)[None, :]
     return np.where(j <= i, 0.0, -np.inf)
+
+
+def window_mask(n_q: int, n_k: int, window: int, q_offset: int = 0) -> np.ndarray:
+    """Additive causal sliding-window mask of [L07] Step 2: key j is visible from query i
+    when max(0, i - window + 1) <= j <= i (the window holds the query's own key); 0.0 there,
+    -inf elsewhere. window >= n gives the full causal mask; window = 1 leaves only j = i."""
+    if window < 1:
+        raise ValueError("window must be >= 1")
+    i = np.arange(q_offset, q_offset + n_q)[:, None]
+    j = np.arange(n_k)[None, :]
+    return np.where((j <= i) & (j >= i - window + 1), 0.0, -np.inf)
 
 
 def pair_layout(Hq: int, Hkv: int):
@@ -114,13 +128,17 @@ def _f64(t) -> np.ndarray:
     return np.asarray(t, dtype=np.float64)
 
 
-def prefill(q, k, v, lam, causal: bool = True, row_block: int = 512) -> np.ndarray:
+def prefill(q, k, v, lam, causal: bool = True, row_block: int = 512, window=None) -> np.ndarray:
     """Forward prefill over the whole batch: out[B, S, Hq/2, D] in float64.
 
     q [B,S,Hq,D], k/v [B,S,Hkv,D], lam [B,S,Hq/2]. For every batch b and pair p the rows are
     processed in blocks of `row_block` (a memory bound only: every row is computed exactly
-    as the definition states, over all its visible keys).
+    as the definition states, over all its visible keys). `window` (causal only) restricts
+    each query to its last `window` keys, the DiffAttn + sliding-window combination that the
+    lesson's "Use it" section names for hybrid layers, with the mask of [L07] Step 2.
     """
+    if window is not None and not causal:
+        raise ValueError("a sliding window is defined for causal attention")
     q, k, v, lam = _f64(q), _f64(k), _f64(v), _f64(lam)
     B, S, Hq, D = q.shape
     Hkv = k.shape[2]
@@ -131,9 +149,26 @@ def prefill(q, k, v, lam, causal: bool = True, row_block: int = 512) -> np.ndarr
             for r0 in range(0, S, row_block):
                 r1 = min(S, r0 + row_block)
                 n_k = r1 if causal else S
-                mask = causal_mask(r1 - r0, n_k, r0) if causal else np.zeros((r1 - r0, S))
+                if window is not None:
+                    mask = window_mask(r1 - r0, n_k, window, r0)
+                else:
+                    mask = causal_mask(r1 - r0, n_k, r0) if causal else np.zeros((r1 - r0, S))
                 out[b, r0:r1, p] = diff_attention_block(
                     q[b, r0:r1, h1], q[b, r0:r1, h2], kk[:n_k], vv[:n_k], lam[b, r0:r1, p], mask)
+    return out
+
+
+def prefill_varlen(q, k, v, lam, cu_seqlens, causal: bool = True) -> np.ndarray:
+    """Prefill of sequences packed along the token axis: q [T,Hq,D], k/v [T,Hkv,D],
+    lam [T,Hq/2], sequence b = tokens cu_seqlens[b] .. cu_seqlens[b+1]-1. Every sequence is an
+    independent prefill (its queries see only its own keys). Returns out [T,Hq/2,D]."""
+    cu = [int(x) for x in cu_seqlens]
+    T = int(q.shape[0])
+    out = np.zeros((T, q.shape[1] // 2, q.shape[2]), dtype=np.float64)
+    for b in range(len(cu) - 1):
+        s0, s1 = cu[b], cu[b + 1]
+        if s1 > s0:
+            out[s0:s1] = prefill(q[None, s0:s1], k[None, s0:s1], v[None, s0:s1], lam[None, s0:s1], causal=causal)[0]
     return out
 
 
@@ -192,6 +227,23 @@ def decode(q, kcache, vcache, seqlens, lam) -> np.ndarray:
                 lm = np.array([float(lam[b, p])], dtype=np.float64)
                 out[b, p] = diff_attention_block(q1, q2, kk, vv, lm, np.zeros((1, n)))[0]
     return out
+
+
+def decode_paged(q, kpages, vpages, block_table, seqlens, lam) -> np.ndarray:
+    """Decode step over a paged cache: kpages/vpages [P, page_size, Hkv, D]; logical token t
+    of sequence b lives in page block_table[b][t // page_size] at row t % page_size. The
+    sequence's logical cache is gathered page by page, then `decode` applies as written."""
+    page_size = int(kpages.shape[1])
+    B = q.shape[0]
+    outs = []
+    for b in range(B):
+        n = int(seqlens[b])
+        n_pages = (n + page_size - 1) // page_size
+        pages = [int(block_table[b][i]) for i in range(n_pages)]
+        kc = np.concatenate([_f64(kpages[pg]) for pg in pages], axis=0)[:n] if n else np.zeros((0,) + tuple(kpages.shape[2:]))
+        vc = np.concatenate([_f64(vpages[pg]) for pg in pages], axis=0)[:n] if n else np.zeros((0,) + tuple(vpages.shape[2:]))
+        outs.append(decode(q[b:b + 1], kc[None], vc[None], [n], lam[b:b + 1])[0])
+    return np.stack(outs)
 
 
 def lambda_v1(lq1, lk1, lq2, lk2, lambda_init: float = 0.8) -> np.ndarray:

@@ -74,6 +74,22 @@ def test_prefill_host_checks(lib, args, expect):
     assert lib.diffattn_v2_prefill(*args, None) == expect
 
 
+def test_prefill_window_host_checks(lib):
+    assert lib.diffattn_v2_prefill_window(Q, K, V, L, O, 1, 64, 8, 2, 128, 0, None) == -1   # window 0
+    assert lib.diffattn_v2_prefill_window(Q, K, V, L, O, 1, 64, 6, 2, 128, 8, None) == -1   # straddling pair
+    assert lib.diffattn_v2_prefill_window(Q, K, V, L, O, 1, 64, 8, 2, 64, 8, None) == -2    # D = 64
+    assert lib.diffattn_v2_prefill_window(Q, K, V, L, O, 0, 64, 8, 2, 128, 8, None) == 0    # B = 0
+
+
+def test_prefill_varlen_host_checks(lib):
+    C = P + 28672
+    assert lib.diffattn_v2_prefill_varlen(Q, K, V, L, O, None, 2, 64, 100, 8, 2, 128, 1, None) == -1  # no cu_seqlens
+    assert lib.diffattn_v2_prefill_varlen(Q, K, V, L, O, C, 2, 64, 100, 8, 2, 64, 1, None) == -2      # D = 64
+    assert lib.diffattn_v2_prefill_varlen(Q, K, V, L, O, C, 2, 64, 100, 6, 2, 128, 1, None) == -1     # straddling
+    assert lib.diffattn_v2_prefill_varlen(Q, K, V, L, O, C, 0, 64, 100, 8, 2, 128, 1, None) == 0      # no sequences
+    assert lib.diffattn_v2_prefill_varlen(Q, K, V, L, O, C, 2, 64, 100, 8, 2, 128, 3, None) == -1     # causal flag
+
+
 def test_prefill_f32_host_checks(lib):
     assert lib.diffattn_v2_prefill_f32(Q, K, V, L, O, 1, 16, 4, 1, 96, 1, None) == -2
     assert lib.diffattn_v2_prefill_f32(Q, K, V, L, O, 1, 16, 4, 3, 64, 1, None) == -1
@@ -110,6 +126,24 @@ def test_decode_host_checks(lib):
     assert lib.diffattn_v2_decode(*b0) == 0
     assert lib.diffattn_v2_decode(Q, K, V, S, L, O, 2, 0, 16, 2, 128, W, ws, None) == -1
     assert lib.diffattn_v2_decode_f32(Q, K, V, S, L, O, 2, 1024, 16, 3, 64, None) == -1
+
+
+def test_decode_paged_host_checks(lib):
+    T = P + 32768
+    W = P + 65536
+    S_ = P + 24576
+    ws = lib.diffattn_v2_decode_workspace_size(2, 1024, 16, 2, 128)
+    ok = (Q, K, V, T, S_, L, O, 2, 16, 64, 40, 16, 2, 128, W, ws, None)
+    bad_ps = ok[:9] + (48,) + ok[10:]
+    assert lib.diffattn_v2_decode_paged(*bad_ps) == -1                  # page size not a power of two
+    small = ok[:9] + (4,) + ok[10:]
+    assert lib.diffattn_v2_decode_paged(*small) == -1                   # page size below 8
+    no_table = ok[:3] + (None,) + ok[4:]
+    assert lib.diffattn_v2_decode_paged(*no_table) == -1
+    short_ws = ok[:15] + (ws - 16,) + ok[16:]
+    assert lib.diffattn_v2_decode_paged(*short_ws) == -1
+    d64 = ok[:13] + (64,) + ok[14:]
+    assert lib.diffattn_v2_decode_paged(*d64[:15] + (1 << 30,) + d64[16:]) == -2
 
 
 def test_lambda_v1_host_checks(lib):

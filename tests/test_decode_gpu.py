@@ -113,3 +113,35 @@ def test_decode_equal_heads_cancel_exactly(da):
     inp["lam"].fill_(1.0)
     out = _run(da, inp)
     assert torch.count_nonzero(out).item() == 0
+
+
+def _paged(kc, vc, page_size, seed):
+    """Scatter contiguous caches [B,Smax,Hkv,D] into shuffled pages; returns pages + table."""
+    B, Smax = kc.shape[:2]
+    max_pages = Smax // page_size
+    n_pages = B * max_pages + 3
+    perm = torch.randperm(n_pages, generator=torch.Generator().manual_seed(seed))[: B * max_pages]
+    table = perm.view(B, max_pages).to(torch.int32)
+    kp = torch.zeros(n_pages, page_size, *kc.shape[2:], dtype=kc.dtype)
+    vp = torch.zeros_like(kp)
+    for b in range(B):
+        for i in range(max_pages):
+            kp[table[b, i]] = kc[b, i * page_size:(i + 1) * page_size]
+            vp[table[b, i]] = vc[b, i * page_size:(i + 1) * page_size]
+    return kp, vp, table
+
+
+@pytest.mark.parametrize("page_size,lens", [(16, [1024, 17, 0, 1000]), (64, [1024, 640, 65, 1]),
+                                            (256, [1024, 1023, 300, 257]), (8, [512, 9, 100, 511])])
+def test_decode_paged_matches_contiguous_and_oracle(da, page_size, lens):
+    B, Hq, Hkv = len(lens), 16, 2
+    Smax = ((max(lens) + page_size - 1) // page_size) * page_size
+    inp = _decode_case(B, Smax, Hq, Hkv, lens, seed=page_size)
+    kp, vp, table = _paged(inp["kcache"], inp["vcache"], page_size, seed=page_size)
+    got = da.decode_paged(inp["q"].cuda(), kp.cuda(), vp.cuda(), table.cuda(), inp["seqlens"].cuda(),
+                          inp["lam"].cuda())
+    assert da.device_error() == 0
+    contiguous = _run(da, inp)
+    assert torch.equal(got, contiguous)  # same splits, same arithmetic
+    ref = ora.decode_paged(inp["q"], kp, vp, table.tolist(), inp["seqlens"], inp["lam"])
+    bf16_close(got, ref, f"paged decode page_size={page_size}")

@@ -227,6 +227,79 @@ def pin_weights_rows_sum():
     return bool(ok)
 
 
+def pin_window_reduces_to_causal_and_self():
+    """A window at least S long is the causal mask; window 1 leaves each query only its own
+    key, so out[b,i,p] = (1 - lam) v[b,i,g]."""
+    q, k, v, lam = _rand_prefill(seed=13)
+    S = q.shape[1]
+    ok = np.allclose(ora.prefill(q, k, v, lam, window=S), ora.prefill(q, k, v, lam), atol=1e-13)
+    ok &= np.allclose(ora.prefill(q, k, v, lam, window=10 * S), ora.prefill(q, k, v, lam), atol=1e-13)
+    one = ora.prefill(q, k, v, lam, window=1)
+    G = q.shape[2] // k.shape[2]
+    for p in range(q.shape[2] // 2):
+        ok &= np.allclose(one[:, :, p], (1.0 - lam[:, :, p])[..., None] * v[:, :, (2 * p) // G], atol=1e-13)
+    return bool(ok)
+
+
+def pin_window_brute_force():
+    q, k, v, lam = _rand_prefill(B=1, S=11, Hq=4, Hkv=1, D=4, seed=14)
+    ok = True
+    for w in (2, 3, 7):
+        ref = np.array(brute.prefill(q.tolist(), k.tolist(), v.tolist(), lam.tolist(), window=w))
+        ok &= np.allclose(ora.prefill(q, k, v, lam, window=w, row_block=4), ref, atol=1e-12)
+    return bool(ok)
+
+
+def pin_window_mask_definition():
+    """The lesson's worked picture: n = 8, window 4 keeps the last 4 keys of each row."""
+    m = ora.window_mask(8, 8, 4)
+    vis = (m == 0.0)
+    ok = all(vis[i].sum() == min(i + 1, 4) for i in range(8))
+    ok &= bool(vis[7, 4:].all() and not vis[7, :4].any() and vis[2, :3].all())
+    return bool(ok)
+
+
+def pin_varlen_is_per_sequence_prefill():
+    """Packed sequences: each equals its own prefill, and a packing of equal lengths equals
+    the batched prefill (the brute force checks the batched one)."""
+    q, k, v, lam = _rand_prefill(B=3, S=13, Hq=8, Hkv=2, D=6, seed=15)
+    flat = lambda t: t.reshape(-1, *t.shape[2:])
+    cu = [0, 13, 26, 39]
+    ok = np.allclose(ora.prefill_varlen(flat(q), flat(k), flat(v), flat(lam), cu).reshape(3, 13, 4, 6),
+                     ora.prefill(q, k, v, lam), atol=1e-13)
+    cu2 = [0, 5, 5, 20, 39]  # lengths 5, 0, 15, 19
+    out = ora.prefill_varlen(flat(q), flat(k), flat(v), flat(lam), cu2)
+    for a, b_ in zip(cu2[:-1], cu2[1:]):
+        if b_ > a:
+            ref = np.array(brute.prefill(*(flat(t)[None, a:b_].tolist() for t in (q, k, v, lam))))[0]
+            ok &= np.allclose(out[a:b_], ref, atol=1e-12)
+    return bool(ok)
+
+
+def pin_paged_decode_gathers_pages():
+    """A paged cache with a shuffled block table decodes like the contiguous cache it holds
+    (and, through `decode`, like the brute force)."""
+    rng = np.random.default_rng(16)
+    B, Hq, Hkv, D, ps = 3, 8, 2, 6, 4
+    lens = [9, 1, 0]
+    n_pages = 12
+    kp = rng.standard_normal((n_pages, ps, Hkv, D))
+    vp = rng.standard_normal((n_pages, ps, Hkv, D))
+    perm = rng.permutation(n_pages)
+    table = [perm[0:3].tolist(), perm[3:4].tolist() + [0, 0], [0, 0, 0]]
+    q = rng.standard_normal((B, Hq, D))
+    lam = rng.uniform(-1, 2, size=(B, Hq // 2))
+    out = ora.decode_paged(q, kp, vp, table, lens, lam)
+    ok = True
+    for b in range(B):
+        n = lens[b]
+        kc = np.concatenate([kp[pg] for pg in table[b]], axis=0)[None, :max(n, 1)]
+        vc = np.concatenate([vp[pg] for pg in table[b]], axis=0)[None, :max(n, 1)]
+        ref = np.array(brute.decode(q[b:b + 1].tolist(), kc.tolist(), vc.tolist(), [n], lam[b:b + 1].tolist()))
+        ok &= np.allclose(out[b], ref[0], atol=1e-12)
+    return bool(ok)
+
+
 ALL_PINS = {
     "softmax_library": pin_softmax_library,
     "lambda0_is_softmax_attention": pin_lambda0_is_softmax_attention,
@@ -245,6 +318,11 @@ ALL_PINS = {
     "noise_mass_golden": pin_noise_mass_golden,
     "uniform_logits": pin_uniform_logits,
     "weights_rows_sum": pin_weights_rows_sum,
+    "window_reduces_to_causal_and_self": pin_window_reduces_to_causal_and_self,
+    "window_brute_force": pin_window_brute_force,
+    "window_mask_definition": pin_window_mask_definition,
+    "varlen_is_per_sequence_prefill": pin_varlen_is_per_sequence_prefill,
+    "paged_decode_gathers_pages": pin_paged_decode_gathers_pages,
 }
 
 

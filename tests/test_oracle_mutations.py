@@ -84,6 +84,12 @@ def _mask_transposed(n_q, n_k, q_offset=0):
     return np.where(j >= i, 0.0, -np.inf)
 
 
+def _window_off_by_one(n_q, n_k, window, q_offset=0):
+    i = np.arange(q_offset, q_offset + n_q)[:, None]
+    j = np.arange(n_k)[None, :]
+    return np.where((j <= i) & (j >= i - window), 0.0, -np.inf)
+
+
 def _softmax_no_max(x):
     x = np.asarray(x, dtype=np.float64)
     e = np.exp(x)
@@ -117,6 +123,7 @@ MUTANTS = {
     "softmax_unstable": ("stable_softmax", _softmax_no_max),
     "softmax_epsilon": ("stable_softmax", _softmax_off),
     "lambda_v1_plus": ("lambda_v1", _lambda_v1_plus),
+    "window_off_by_one": ("window_mask", _window_off_by_one),
 }
 
 

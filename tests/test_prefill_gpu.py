@@ -118,6 +118,68 @@ def test_prefill_f32_matches_oracle(da, B, S, Hq, Hkv, D, causal):
     f32_close(out, ref, f"fp32 prefill S={S} D={D}")
 
 
+@pytest.mark.parametrize("B,S,Hq,Hkv,window", [
+    (1, 300, 8, 2, 1),       # each query sees only itself
+    (1, 300, 8, 2, 17),      # window inside one tile
+    (2, 700, 8, 1, 128),     # exactly one tile wide
+    (1, 700, 16, 2, 129),    # one more than a tile
+    (1, 1000, 8, 2, 300),    # spans several tiles, ragged sequence
+    (1, 257, 8, 2, 5000),    # wider than the sequence: plain causal
+])
+def test_prefill_window_matches_oracle(da, B, S, Hq, Hkv, window):
+    inp = workloads.make_prefill(workloads.PrefillCase(B=B, S=S, Hq=Hq, Hkv=Hkv, D=128, seed=window + S))
+    d = _dev(inp)
+    out = da.prefill_window(d["q"], d["k"], d["v"], d["lam"], window)
+    assert da.device_error() == 0
+    ref = ora.prefill(inp["q"], inp["k"], inp["v"], inp["lam"], window=window)
+    bf16_close(out, ref, f"window={window} S={S}")
+
+
+def test_prefill_window_at_full_size_sampled(da):
+    """The 4 x 4k workload with a 1024-key window (a hybrid sliding-window layer), sampled rows."""
+    case = workloads.CONFIGS["c2_bf16_prefill"]
+    inp = workloads.make_prefill(case)
+    out = da.prefill_window(*(inp[x].cuda() for x in ("q", "k", "v", "lam")), 1024).cpu()
+    assert da.device_error() == 0
+    rows = sample_rows(case.B, case.S, case.Hq // 2, n=512, seed=5)
+    # the row's window is the causal prefix of the slice that ends at the row
+    ref = np.concatenate([ora.prefill_rows(*(inp[x][b:b + 1, max(0, i - 1023):i + 1] for x in ("q", "k", "v", "lam")),
+                                           [(0, i - max(0, i - 1023), p)]) for b, i, p in rows])
+    got = torch.stack([out[b, i, p] for b, i, p in rows])
+    bf16_close(got, ref, "window 1024 sampled rows")
+
+
+@pytest.mark.parametrize("lens,Hq,Hkv,causal", [
+    ([300, 1, 0, 129, 128, 77], 8, 2, True),       # ragged, single token, empty, tile edges
+    ([1000, 513], 16, 2, True),
+    ([200, 64, 390], 8, 1, False),                 # non-causal packed sequences
+])
+def test_prefill_varlen_matches_oracle(da, lens, Hq, Hkv, causal):
+    T = sum(lens)
+    g = torch.Generator().manual_seed(T)
+    q = torch.randn(T, Hq, 128, generator=g).bfloat16()
+    k = torch.randn(T, Hkv, 128, generator=g).bfloat16()
+    v = torch.randn(T, Hkv, 128, generator=g).bfloat16()
+    lam = torch.sigmoid(torch.randn(T, Hq // 2, generator=g))
+    cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32)
+    out = da.prefill_varlen(q.cuda(), k.cuda(), v.cuda(), lam.cuda(), cu.cuda(), max(lens), causal=causal)
+    assert da.device_error() == 0
+    ref = ora.prefill_varlen(q, k, v, lam, cu.tolist(), causal=causal)
+    bf16_close(out, ref, f"varlen {lens}")
+
+
+def test_prefill_varlen_equals_batched(da):
+    """Equal-length packed sequences give the batched prefill's output bit for bit."""
+    case = workloads.PrefillCase(B=3, S=333, Hq=16, Hkv=2, D=128, seed=8)
+    inp = workloads.make_prefill(case)
+    d = _dev(inp)
+    batched = da.prefill(d["q"], d["k"], d["v"], d["lam"])
+    flat = lambda t: t.reshape(-1, *t.shape[2:]).contiguous()
+    cu = torch.tensor([0, 333, 666, 999], dtype=torch.int32, device="cuda")
+    packed = da.prefill_varlen(flat(d["q"]), flat(d["k"]), flat(d["v"]), flat(d["lam"]), cu, 333)
+    assert torch.equal(packed.view(3, 333, 8, 128), batched)
+
+
 def test_prefill_rejects_bad_arguments_on_gpu(da):
     q = torch.zeros(1, 16, 6, 128, dtype=torch.bfloat16, device="cuda")
     k = torch.zeros(1, 16, 2, 128, dtype=torch.bfloat16, device="cuda")
