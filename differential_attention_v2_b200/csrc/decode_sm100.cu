@@ -75,6 +75,8 @@ diffattn_decode_split(const __grid_constant__ CUtensorMap tmK, const __grid_cons
   auto empty = [&](int s) -> uint32_t { return sbase + kOffBar + 8u * (kStages + s); };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc);
 
+  // the combine kernel may be scheduled now; it waits for this grid's results before reading
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int split = blockIdx.x;
   const int g = blockIdx.y;
   const int b = blockIdx.z;
@@ -330,6 +332,9 @@ __global__ void __launch_bounds__(128)
 diffattn_decode_combine(const float* __restrict__ ws_o, const float* __restrict__ ws_ml,
                         const int32_t* __restrict__ seqlens, const float* __restrict__ lambda,
                         __nv_bfloat16* __restrict__ out, int B, int Smax, int Hq, int nsplit, int split_len) {
+  // launched as a programmatic dependent of the split kernel: wait until its partials are
+  // complete and visible
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int n_pairs = Hq >> 1;
   const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -411,10 +416,20 @@ cudaError_t launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const 
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  // the combine overlaps its launch with the split kernel's tail (programmatic dependent launch)
   const int warps = B * (Hq / 2);
-  diffattn_decode_combine<<<(warps + 3) / 4, 128, 0, stream>>>(ws_o, ws_ml, seqlens, lambda, out, B, Smax, Hq,
-                                                               nsplit, split_len);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((warps + 3) / 4);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, diffattn_decode_combine, static_cast<const float*>(ws_o),
+                            static_cast<const float*>(ws_ml), seqlens, lambda, out, B, Smax, Hq, nsplit, split_len);
 }
 
 }  // namespace da2
