@@ -53,7 +53,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # reported as null once the source differs from the one captured.
 NCU_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one launch (B=4 x 4k causal prefill)
-    "prefill": {"bytes": 766537216, "source_sha": "cc174fd0353f516e"},
+    "prefill": {"bytes": 620974848, "source_sha": "a32175841b489c66"},
     # split (1.228e9 + 9.13e6) + combine (6.62e6) of one B=64 decode step
     "decode": {"bytes": 1243700000, "source_sha": "bbed945a81dc3b45"},
 }
@@ -491,6 +491,136 @@ def run_reference(args):
     }
 
 
+# ------------------------------------------------------------ single-operation lines
+def _time_op(fn, steps, warmup, stream):
+    for _ in range(max(warmup, 3)):
+        fn()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        fn()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    return t0.elapsed_time(t1) / steps
+
+
+def run_workload(args):
+    """One operation of the operator's scope on one GPU, timed alone (CUDA events over
+    `steps` back-to-back launches after `warmup`): the second prefill and decode workloads
+    and the next rows (sliding window, packed prefill, paged and multi-token decode, the V2
+    lambda projection). Prints one JSON line with its own metric, work count and roofline."""
+    import differential_attention_v2_b200 as da
+
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    peaks, peak_src = _peaks()
+    name = args.workload
+    D = 128
+    if name in ("prefill_long", "window", "varlen"):
+        if name == "varlen":
+            g = torch.Generator().manual_seed(1010)
+            lens = torch.randint(512, 3585, (8,), generator=g).tolist()
+            T = sum(lens)
+            case = workloads.PrefillCase(B=1, S=T, Hq=64, Hkv=8, D=D, seed=1010)
+            inp = workloads.make_prefill(case)
+            q, k, v, lam = (inp[x][0].to(dev) for x in ("q", "k", "v", "lam"))
+            cu = torch.tensor([0] + list(torch.tensor(lens).cumsum(0).tolist()), dtype=torch.int32, device=dev)
+            out = torch.empty(T, 32, D, dtype=torch.bfloat16, device=dev)
+            fn = lambda: da.prefill_varlen(q, k, v, lam, cu, max(lens), out=out, stream=stream)
+            flops = sum(4 * D * 64 * L * (L + 1) // 2 for L in lens)
+            cfg = {"workload": f"packed causal prefill of 8 sequences, lengths U[512,3584] (total {T}), Hq=64 Hkv=8 D=128",
+                   "lengths": lens}
+        else:
+            case = workloads.CONFIGS["c3_long_bf16_prefill"] if name == "prefill_long" else workloads.CONFIGS["c2_bf16_prefill"]
+            inp = workloads.make_prefill(case)
+            q, k, v, lam = (inp[x].to(dev) for x in ("q", "k", "v", "lam"))
+            out = torch.empty(case.B, case.S, case.Hq // 2, D, dtype=torch.bfloat16, device=dev)
+            if name == "window":
+                W = 1024
+                fn = lambda: da.prefill_window(q, k, v, lam, W, out=out, stream=stream)
+                flops = 4 * D * case.Hq * case.B * sum(min(i + 1, W) for i in range(case.S))
+                cfg = {"workload": f"sliding-window causal prefill, window {W}, B=4 S=4096 Hq=64 Hkv=8 D=128"}
+            else:
+                fn = lambda: da.prefill(q, k, v, lam, out=out, stream=stream)
+                flops = workloads.prefill_flops(case.B, case.S, case.Hq, D)
+                cfg = {"workload": "causal prefill B=1 S=32768 Hq=64 Hkv=8 D=128"}
+        ms = _time_op(fn, args.steps, args.warmup, stream)
+        val = flops / (ms * 1e-3) / 1e12
+        unit, peak, bound = "TFLOP/s", peaks["bf16_tflops"], "tensor"
+        launches = 1
+    elif name in ("decode_needle", "paged", "multi"):
+        case = workloads.CONFIGS["c5_needle_decode"] if name == "decode_needle" else workloads.CONFIGS["c4_bf16_decode"]
+        inp = workloads.make_decode(case)
+        kc, vc, sl = (inp[x].to(dev) for x in ("kcache", "vcache", "seqlens"))
+        if inp["lam"] is None:
+            lam = da.lambda_v1(*(inp[x].to(dev) for x in ("lq1", "lk1", "lq2", "lk2")), inp["lambda_init"], rows=case.B)
+        else:
+            lam = inp["lam"].to(dev)
+        q = inp["q"].to(dev)
+        nbytes = workloads.decode_bytes(inp["seqlens"].tolist(), case.Hkv, D, case.Hq)
+        launches = 2
+        if name == "paged":
+            ps = 64
+            max_pages = case.Smax // ps
+            perm = torch.randperm(case.B * max_pages, generator=torch.Generator().manual_seed(7))
+            table = perm.view(case.B, max_pages).to(torch.int32).to(dev)
+            kp = torch.empty(case.B * max_pages, ps, case.Hkv, D, dtype=torch.bfloat16, device=dev)
+            vp = torch.empty_like(kp)
+            kp[perm.to(dev)] = kc.view(case.B * max_pages, ps, case.Hkv, D)
+            vp[perm.to(dev)] = vc.view(case.B * max_pages, ps, case.Hkv, D)
+            del kc, vc
+            out = torch.empty(case.B, case.Hq // 2, D, dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(da.decode_workspace_size(case.B, case.Smax, case.Hq, case.Hkv, D), dtype=torch.uint8, device=dev)
+            fn = lambda: da.decode_paged(q, kp, vp, table, sl, lam, out=out, workspace=ws, stream=stream)
+            nbytes += case.B * max_pages * 4
+            cfg = {"workload": "paged decode (page size 64, shuffled pages) of B=64, lengths U[1024,8192], Hq=64 Hkv=8"}
+        elif name == "multi":
+            Tn = 2
+            g = torch.Generator().manual_seed(11)
+            qm = torch.randn(case.B, Tn, case.Hq, D, generator=g).bfloat16().to(dev)
+            lm = torch.sigmoid(torch.randn(case.B, Tn, case.Hq // 2, generator=g)).to(dev)
+            out = torch.empty(case.B, Tn, case.Hq // 2, D, dtype=torch.bfloat16, device=dev)
+            fn = lambda: da.decode_multi(qm, kc, vc, sl, lm, out=out, stream=stream)
+            nbytes += (Tn - 1) * case.B * (case.Hq * D * 2 + case.Hq // 2 * (4 + D * 2))
+            cfg = {"workload": "2-token (speculative) decode of B=64, lengths U[1024,8192], Hq=64 Hkv=8"}
+        else:
+            out = torch.empty(case.B, case.Hq // 2, D, dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(da.decode_workspace_size(case.B, case.Smax, case.Hq, case.Hkv, D), dtype=torch.uint8, device=dev)
+            fn = lambda: da.decode(q, kc, vc, sl, lam, out=out, workspace=ws, stream=stream)
+            cfg = {"workload": "needle decode B=8, 131072 cached tokens each, V1 lambda, Hq=64 Hkv=8"}
+        ms = _time_op(fn, args.steps, args.warmup, stream)
+        val = nbytes / (ms * 1e-3) / 1e9
+        unit, peak, bound = "GB/s", peaks["hbm_gbs"], "hbm"
+    elif name == "lambda_v2":
+        T, dm, npair = 16384, 4096, 32
+        g = torch.Generator().manual_seed(12)
+        x = torch.randn(T, dm, generator=g).bfloat16().to(dev)
+        w = (torch.randn(dm, npair, generator=g) / dm ** 0.5).bfloat16().to(dev)
+        b = torch.randn(npair, generator=g).to(dev)
+        out = torch.empty(T, npair, dtype=torch.float32, device=dev)
+        fn = lambda: da.lambda_v2(x, w, b, out=out, stream=stream)
+        nbytes = T * dm * 2 + dm * npair * 2 + npair * 4 + T * npair * 4
+        ms = _time_op(fn, args.steps, args.warmup, stream)
+        val = nbytes / (ms * 1e-3) / 1e9
+        unit, peak, bound = "GB/s", peaks["hbm_gbs"], "hbm"
+        launches = 1
+        cfg = {"workload": "V2 lambda projection sigmoid(x W + b): T=16384 tokens, d_model=4096, 32 pairs"}
+    else:
+        raise SystemExit(f"unknown workload {name}")
+    err = da.device_error(stream)
+    if err:
+        raise RuntimeError(f"kernel reported device error {err}")
+    line = {"metric": f"{name}: {unit}", "value": round(val, 2), "unit": unit, "n_gpus": 1, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic, seeded", "config": cfg,
+            "roofline": {"bound": bound, "achieved": round(val, 2), "peak": peak, "unit": unit,
+                         "frac": round(val / peak, 4), "traffic": None,
+                         "peak_source": f"{peak_src} {'bf16_tflops (burst)' if bound == 'tensor' else 'hbm_gbs'}"},
+            "gpu_launches": launches * args.steps, "workload": name}
+    print(json.dumps(line), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -501,6 +631,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=120.0,
                     help="host-time budget of the whole reference run (warm-up and timed steps)")
+    ap.add_argument("--workload", choices=("prefill_long", "decode_needle", "window", "varlen", "paged", "multi",
+                                           "lambda_v2"), default=None,
+                    help="time one other operation alone instead of the default step")
     ap.add_argument("--scaling", choices=("weak", "strong"), default="weak",
                     help="weak: each GPU runs the full per-GPU workload; strong: the heads of one workload "
                          "are split over the GPUs")
@@ -508,6 +641,9 @@ def main(argv=None):
                     help="run one half of the step (for profiling a single kernel on less device memory)")
     args = ap.parse_args(argv)
 
+    if args.workload:
+        run_workload(args)
+        return 0
     if args.impl == "reference":
         if int(os.environ.get("RANK", "0")) != 0:
             return 0

@@ -33,7 +33,10 @@ _SIGNATURES = {
     "diffattn_v2_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "diffattn_v2_decode_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
     "diffattn_v2_decode_paged": (_i, [_vp] * 7 + [_i] * 7 + [_vp, _sz, _vp]),
+    "diffattn_v2_decode_multi_workspace_size": (_sz, [_i] * 6),
+    "diffattn_v2_decode_multi": (_i, [_vp] * 6 + [_i] * 6 + [_vp, _sz, _vp]),
     "diffattn_v2_lambda_v1": (_i, [_vp, _vp, _vp, _vp, _f, _i, _i, _i, _vp, _vp]),
+    "diffattn_v2_lambda_v2": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
     "diffattn_v2_device_error": (_i, [ctypes.POINTER(_i), _vp]),
     "diffattn_v2_decode_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
 }
@@ -186,6 +189,29 @@ def decode(q, kcache, vcache, seqlens, lam, out=None, workspace=None, stream=Non
     return out
 
 
+def decode_multi(q, kcache, vcache, seqlens, lam, out=None, workspace=None, stream=None):
+    """bf16 decode of T new tokens per sequence: q [B,T,Hq,D], lam fp32 [B,T,Hq/2] ->
+    out bf16 [B,T,Hq/2,D]; token t sees keys [0, seqlens[b] - T + t + 1)."""
+    _need(q, "q", torch.bfloat16, 4)
+    _need(kcache, "kcache", torch.bfloat16, 4)
+    _need(vcache, "vcache", torch.bfloat16, 4)
+    _need(seqlens, "seqlens", torch.int32, 1)
+    _need(lam, "lam", torch.float32, 3)
+    B, T, Hq, D = q.shape
+    Smax, Hkv = kcache.shape[1], kcache.shape[2]
+    if out is None:
+        out = torch.empty((B, T, Hq // 2, D), dtype=torch.bfloat16, device=q.device)
+    _need(out, "out", torch.bfloat16, 4)
+    need = int(LIB.diffattn_v2_decode_multi_workspace_size(B, T, Smax, Hq, Hkv, D))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    st = LIB.diffattn_v2_decode_multi(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(lam), _ptr(out), B, T,
+                                      Smax, Hq, Hkv, D, _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                      _stream(stream, q.device))
+    _check(st, "diffattn_v2_decode_multi")
+    return out
+
+
 def decode_paged(q, kpages, vpages, block_table, seqlens, lam, out=None, workspace=None, stream=None):
     """bf16 decode over a paged cache: kpages/vpages [num_pages, page_size, Hkv, D],
     block_table int32 [B, max_pages], seqlens int32 [B], lam fp32 [B, Hq/2]."""
@@ -241,6 +267,23 @@ def lambda_v1(lq1, lk1, lq2, lk2, lambda_init=0.8, rows=1, out=None, stream=None
     st = LIB.diffattn_v2_lambda_v1(_ptr(lq1), _ptr(lk1), _ptr(lq2), _ptr(lk2), float(lambda_init), n_pairs, d, rows,
                                    _ptr(out), _stream(stream, lq1.device))
     _check(st, "diffattn_v2_lambda_v1")
+    return out
+
+
+def lambda_v2(x, w_lambda, bias=None, out=None, stream=None):
+    """V2 lambda sigmoid(x @ w_lambda + bias): x bf16 [T, d_model], w_lambda bf16
+    [d_model, n_pairs], bias fp32 [n_pairs] or None -> fp32 [T, n_pairs]."""
+    _need(x, "x", torch.bfloat16, 2)
+    _need(w_lambda, "w_lambda", torch.bfloat16, 2)
+    if bias is not None:
+        _need(bias, "bias", torch.float32, 1)
+    T, d = x.shape
+    n_pairs = w_lambda.shape[1]
+    if out is None:
+        out = torch.empty((T, n_pairs), dtype=torch.float32, device=x.device)
+    st = LIB.diffattn_v2_lambda_v2(_ptr(x), _ptr(w_lambda), _ptr(bias), T, d, n_pairs, _ptr(out),
+                                   _stream(stream, x.device))
+    _check(st, "diffattn_v2_lambda_v2")
     return out
 
 

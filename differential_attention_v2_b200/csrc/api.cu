@@ -231,7 +231,7 @@ int diffattn_v2_decode(const void* q, const void* kcache, const void* vcache, co
   float* ws_ml = ws_o + static_cast<size_t>(B) * Hq * nsplit * D;
   e = da2::launch_decode(tk, tv, static_cast<const __nv_bfloat16*>(q), seqlens, lambda,
                          static_cast<__nv_bfloat16*>(out), ws_o, ws_ml, err, B, Smax, Hq, Hkv, nsplit, split_len,
-                         nullptr, 0, 0, reinterpret_cast<cudaStream_t>(stream));
+                         nullptr, 0, 0, 1, reinterpret_cast<cudaStream_t>(stream));
   return status_of(e);
 }
 
@@ -267,7 +267,45 @@ int diffattn_v2_decode_paged(const void* q, const void* kpages, const void* vpag
   float* ws_ml = ws_o + static_cast<size_t>(B) * Hq * nsplit * D;
   e = da2::launch_decode(tk, tv, static_cast<const __nv_bfloat16*>(q), seqlens, lambda,
                          static_cast<__nv_bfloat16*>(out), ws_o, ws_ml, err, B, Smax, Hq, Hkv, nsplit, split_len,
-                         block_table, max_pages, page_shift, reinterpret_cast<cudaStream_t>(stream));
+                         block_table, max_pages, page_shift, 1, reinterpret_cast<cudaStream_t>(stream));
+  return status_of(e);
+}
+
+size_t diffattn_v2_decode_multi_workspace_size(int B, int T, int Smax, int Hq, int Hkv, int D) {
+  if (B <= 0 || T <= 0 || Smax <= 0 || D <= 0 || !heads_ok(Hq, Hkv)) return 0;
+  int split_len = 0, nsplit = 0;
+  da2::decode_split_plan(B, Smax, Hkv, &split_len, &nsplit);
+  const size_t rows = static_cast<size_t>(B) * T * Hq * nsplit;
+  return rows * static_cast<size_t>(D) * sizeof(float) + rows * 2 * sizeof(float);
+}
+
+int diffattn_v2_decode_multi(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens,
+                             const float* lambda, void* out, int B, int T, int Smax, int Hq, int Hkv, int D,
+                             void* workspace, size_t workspace_bytes, da2_stream_t stream) {
+  if (B < 0 || T <= 0 || Smax <= 0 || D <= 0 || !heads_ok(Hq, Hkv)) return DA2_ERR_INVALID;
+  if (B == 0) return DA2_OK;
+  if (!q || !kcache || !vcache || !seqlens || !lambda || !out || !workspace) return DA2_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(seqlens) || !aligned16(lambda) ||
+      !aligned16(out) || !aligned16(workspace))
+    return DA2_ERR_INVALID;
+  if (workspace_bytes < diffattn_v2_decode_multi_workspace_size(B, T, Smax, Hq, Hkv, D)) return DA2_ERR_INVALID;
+  const int group = Hq / Hkv;
+  if (D != 128 || !(group == 2 || group == 4 || group == 8 || group == 16) || T * group > 16)
+    return DA2_ERR_UNSUPPORTED;
+  if (B > 65535 || Hkv > 65535) return DA2_ERR_UNSUPPORTED;
+  int* err = nullptr;
+  cudaError_t e = device_error_ptr(&err);
+  if (e != cudaSuccess) return DA2_ERR_CUDA;
+  int split_len = 0, nsplit = 0;
+  da2::decode_split_plan(B, Smax, Hkv, &split_len, &nsplit);
+  CUtensorMap tk, tv;
+  if (encode_bshd(&tk, kcache, D, Hkv, Smax, B, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
+  if (encode_bshd(&tv, vcache, D, Hkv, Smax, B, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
+  float* ws_o = static_cast<float*>(workspace);
+  float* ws_ml = ws_o + static_cast<size_t>(B) * T * Hq * nsplit * D;
+  e = da2::launch_decode(tk, tv, static_cast<const __nv_bfloat16*>(q), seqlens, lambda,
+                         static_cast<__nv_bfloat16*>(out), ws_o, ws_ml, err, B, Smax, Hq, Hkv, nsplit, split_len,
+                         nullptr, 0, 0, T, reinterpret_cast<cudaStream_t>(stream));
   return status_of(e);
 }
 
@@ -294,6 +332,19 @@ int diffattn_v2_lambda_v1(const float* lq1, const float* lk1, const float* lq2, 
     return DA2_ERR_INVALID;
   return status_of(da2::launch_lambda_v1(lq1, lk1, lq2, lk2, lambda_init, n_pairs, d, rows, lambda_out,
                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int diffattn_v2_lambda_v2(const void* x, const void* w_lambda, const float* bias, int T, int d_model, int n_pairs,
+                          float* lambda_out, da2_stream_t stream) {
+  if (T < 0 || d_model <= 0 || n_pairs <= 0) return DA2_ERR_INVALID;
+  if (T == 0) return DA2_OK;
+  if (!x || !w_lambda || !lambda_out) return DA2_ERR_INVALID;
+  if (!aligned16(x) || !aligned16(w_lambda) || !aligned16(lambda_out) || (bias && !aligned16(bias)))
+    return DA2_ERR_INVALID;
+  if (d_model % 64 != 0 || n_pairs % 8 != 0 || n_pairs > 64) return DA2_ERR_UNSUPPORTED;
+  return status_of(da2::launch_lambda_v2(static_cast<const __nv_bfloat16*>(x),
+                                         static_cast<const __nv_bfloat16*>(w_lambda), bias, T, d_model, n_pairs,
+                                         lambda_out, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int diffattn_v2_device_error(int* code, da2_stream_t stream) {

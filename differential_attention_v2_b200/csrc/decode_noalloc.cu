@@ -87,6 +87,6 @@ extern "C" int diffattn_v2_decode_noalloc(const void* q, const void* kcache, con
   float* ws_ml = ws_o + static_cast<size_t>(B) * Hq * nsplit * D;
   cudaError_t e = da2::launch_decode(tk, tv, static_cast<const __nv_bfloat16*>(q), seqlens, lambda,
                                      static_cast<__nv_bfloat16*>(out), ws_o, ws_ml, err, B, Smax, Hq, Hkv, nsplit,
-                                     split_len, nullptr, 0, 0, reinterpret_cast<cudaStream_t>(stream));
+                                     split_len, nullptr, 0, 0, 1, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? DA2_OK : DA2_ERR_CUDA;
 }

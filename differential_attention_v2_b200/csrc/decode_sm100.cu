@@ -56,6 +56,7 @@ struct Params {
   float* ws_ml;             // [B,Hq,nsplit,2]
   int* err;
   int B, Smax, Hq, Hkv, nsplit, split_len;
+  int T;                    // new tokens per sequence (1: plain decode); T * group <= 16
   float scale_log2;
   // paged caches [num_pages, page_size, Hkv, D]: logical token t of sequence b is row
   // t % page_size of page block_table[b * max_pages + t / page_size]; null = [B, Smax] caches
@@ -68,6 +69,8 @@ template <int NT>
 __global__ void __launch_bounds__(kThreads, 2)
 diffattn_decode_split(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const Params p) {
+  // The MMA's N dimension holds the (new token, query head) columns of the group: column
+  // n is token n / group, head n % group; q is [B,T,Hq,D] and the partials are per column.
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -158,15 +161,16 @@ diffattn_decode_split(const __grid_constant__ CUtensorMap tmK, const __grid_cons
   float o[NT][8][4];
   float m_run[NT][2], l_part[NT][2];
   if (warp < kConsumerWarps) {
-    // Q^T as B fragments: head column n = gl of tile nt, k = d
+    // Q^T as B fragments: column n = 8 nt + gl (token n / group, head n % group), k = d
     uint32_t qf[NT][8][2];
     const int hq0 = g * group;  // first query head of the group
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      const int h = nt * 8 + gl;
-      const bool hv = h < group;
+      const int n = nt * 8 + gl;
+      const bool hv = n < p.T * group;
+      const int tok = hv ? n / group : 0, h = hv ? n % group : 0;
       const uint32_t* qrow =
-          reinterpret_cast<const uint32_t*>(p.q + (static_cast<size_t>(b) * p.Hq + hq0 + (hv ? h : 0)) * HD);
+          reinterpret_cast<const uint32_t*>(p.q + ((static_cast<size_t>(b) * p.T + tok) * p.Hq + hq0 + h) * HD);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         qf[nt][kk][0] = hv ? __ldg(qrow + (16 * kk + 2 * tq) / 2) : 0u;
@@ -211,10 +215,14 @@ diffattn_decode_split(const __grid_constant__ CUtensorMap tmK, const __grid_cons
       // scale, mask tokens outside [t0, t1), online softmax per head column
       const int tok_a = t0 + i * kTok + 16 * warp + gl;
       const int tok_b = tok_a + 8;
-      const bool va = tok_a < t1, vb_ = tok_b < t1;
       uint32_t pb[NT][2];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
+        // this thread's two columns belong to one new token, which sees keys below
+        // seqlen - T + token + 1 (causal among the new tokens)
+        const int col_tok = (8 * nt + 2 * tq) / group;
+        const int lim = col_tok < p.T ? min(t1, seqlen - p.T + col_tok + 1) : t1;
+        const bool va = tok_a < lim, vb_ = tok_b < lim;
         float x[4];
         x[0] = va ? sacc[nt][0] * p.scale_log2 : -INFINITY;
         x[1] = va ? sacc[nt][1] * p.scale_log2 : -INFINITY;
@@ -304,8 +312,8 @@ diffattn_decode_split(const __grid_constant__ CUtensorMap tmK, const __grid_cons
   }
   if (warp < kConsumerWarps) {
     const int d = threadIdx.x;  // 0..127
-    const int nh = min(group, 8 * NT);
-    for (int h = 0; h < nh; ++h) {
+    const int nh = min(p.T * group, 8 * NT);
+    for (int h = 0; h < nh; ++h) {  // h: column (token h / group, head h % group)
       float M = -INFINITY;
 #pragma unroll
       for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, w_ml[(w * 8 * NT + h) * 2]);
@@ -317,7 +325,8 @@ diffattn_decode_split(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         O += w_o[(w * 8 * NT + h) * HD + d] * sc;
         L += w_ml[(w * 8 * NT + h) * 2 + 1] * sc;
       }
-      const size_t row = (static_cast<size_t>(b) * p.Hq + g * group + h) * p.nsplit + split;
+      const size_t row =
+          ((static_cast<size_t>(b) * p.T + h / group) * p.Hq + g * group + h % group) * p.nsplit + split;
       p.ws_o[row * HD + d] = O;
       if (d == 0) {
         p.ws_ml[row * 2 + 0] = M;
@@ -327,26 +336,28 @@ diffattn_decode_split(const __grid_constant__ CUtensorMap tmK, const __grid_cons
   }
 }
 
-// One warp per (b, pair): merge the splits of both heads and apply the lambda subtraction.
+// One warp per (b, new token, pair): merge the splits of both heads and apply the lambda
+// subtraction. Splits past a token's visible keys hold (m = -inf, l = 0, O = 0) and weigh 0.
 __global__ void __launch_bounds__(128)
 diffattn_decode_combine(const float* __restrict__ ws_o, const float* __restrict__ ws_ml,
                         const int32_t* __restrict__ seqlens, const float* __restrict__ lambda,
-                        __nv_bfloat16* __restrict__ out, int B, int Smax, int Hq, int nsplit, int split_len) {
+                        __nv_bfloat16* __restrict__ out, int B, int T, int Smax, int Hq, int nsplit, int split_len) {
   // launched as a programmatic dependent of the split kernel: wait until its partials are
   // complete and visible
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int n_pairs = Hq >> 1;
   const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (wid >= B * n_pairs) return;
-  const int b = wid / n_pairs;
+  if (wid >= B * T * n_pairs) return;
+  const int bt = wid / n_pairs;  // b * T + token
+  const int b = bt / T;
   const int pair = wid % n_pairs;
   const int n = min(max(__ldg(seqlens + b), 0), Smax);
   const int ns = (n + split_len - 1) / split_len;
   float res[2][4];
 #pragma unroll
   for (int br = 0; br < 2; ++br) {
-    const size_t row0 = (static_cast<size_t>(b) * Hq + 2 * pair + br) * nsplit;
+    const size_t row0 = (static_cast<size_t>(bt) * Hq + 2 * pair + br) * nsplit;
     float M = -INFINITY;
     for (int s = lane; s < ns; s += 32) M = fmaxf(M, __ldg(ws_ml + (row0 + s) * 2));
 #pragma unroll
@@ -370,11 +381,11 @@ diffattn_decode_combine(const float* __restrict__ ws_o, const float* __restrict_
     res[br][2] = __fmul_rn(acc.z, inv);
     res[br][3] = __fmul_rn(acc.w, inv);
   }
-  const float lam = __ldg(lambda + static_cast<size_t>(b) * n_pairs + pair);
+  const float lam = __ldg(lambda + static_cast<size_t>(bt) * n_pairs + pair);
   uint2 packed;
   packed.x = pack_bf16x2(__fmaf_rn(-lam, res[1][0], res[0][0]), __fmaf_rn(-lam, res[1][1], res[0][1]));
   packed.y = pack_bf16x2(__fmaf_rn(-lam, res[1][2], res[0][2]), __fmaf_rn(-lam, res[1][3], res[0][3]));
-  reinterpret_cast<uint2*>(out + (static_cast<size_t>(b) * n_pairs + pair) * HD)[lane] = packed;
+  reinterpret_cast<uint2*>(out + (static_cast<size_t>(bt) * n_pairs + pair) * HD)[lane] = packed;
 }
 
 }  // namespace decode
@@ -382,7 +393,7 @@ diffattn_decode_combine(const float* __restrict__ ws_o, const float* __restrict_
 cudaError_t launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const __nv_bfloat16* q,
                           const int32_t* seqlens, const float* lambda, __nv_bfloat16* out, float* ws_o,
                           float* ws_ml, int* err, int B, int Smax, int Hq, int Hkv, int nsplit,
-                          int split_len, const int32_t* block_table, int max_pages, int page_shift,
+                          int split_len, const int32_t* block_table, int max_pages, int page_shift, int T,
                           cudaStream_t stream) {
   using namespace decode;
   Params p;
@@ -398,6 +409,7 @@ cudaError_t launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const 
   p.nsplit = nsplit;
   p.split_len = split_len;
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HD));
+  p.T = T;
   p.block_table = block_table;
   p.max_pages = max_pages;
   p.page_shift = page_shift;
@@ -405,7 +417,7 @@ cudaError_t launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const 
   const int group = Hq / Hkv;
   dim3 grid(nsplit, Hkv, B);
   cudaError_t e;
-  if (group > 8) {
+  if (T * group > 8) {
     e = cudaFuncSetAttribute(diffattn_decode_split<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     diffattn_decode_split<2><<<grid, kThreads, kSmemBytes, stream>>>(tmK, tmV, p);
@@ -417,7 +429,7 @@ cudaError_t launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const 
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // the combine overlaps its launch with the split kernel's tail (programmatic dependent launch)
-  const int warps = B * (Hq / 2);
+  const int warps = B * T * (Hq / 2);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((warps + 3) / 4);
   cfg.blockDim = dim3(128);
@@ -429,7 +441,7 @@ cudaError_t launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, diffattn_decode_combine, static_cast<const float*>(ws_o),
-                            static_cast<const float*>(ws_ml), seqlens, lambda, out, B, Smax, Hq, nsplit, split_len);
+                            static_cast<const float*>(ws_ml), seqlens, lambda, out, B, T, Smax, Hq, nsplit, split_len);
 }
 
 }  // namespace da2

@@ -20,11 +20,11 @@ cudaError_t launch_prefill(const CUtensorMap& tmQ, const CUtensorMap& tmK, const
 // bf16 decode (D = 128): split kernel + combine. Tensor maps over the caches [B,Smax,Hkv,D],
 // boxes of 64 (d) x 1 x 64 (tokens) x 1, 128-byte swizzle. With block_table the maps cover
 // pages [num_pages, 1 << page_shift, Hkv, D] with boxes of min(page_size, 64) tokens and
-// Smax = max_pages << page_shift.
+// Smax = max_pages << page_shift. T new tokens per sequence (q [B,T,Hq,D]); T * Hq/Hkv <= 16.
 cudaError_t launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const __nv_bfloat16* q,
                           const int32_t* seqlens, const float* lambda, __nv_bfloat16* out, float* ws_o,
                           float* ws_ml, int* err, int B, int Smax, int Hq, int Hkv, int nsplit,
-                          int split_len, const int32_t* block_table, int max_pages, int page_shift,
+                          int split_len, const int32_t* block_table, int max_pages, int page_shift, int T,
                           cudaStream_t stream);
 
 // Tokens per split and number of splits of the bf16 decode for these sizes.
@@ -47,5 +47,10 @@ cudaError_t device_error_word(int** out);
 // 4-D bf16 tensor map over a row-major [B,S,H,D] array, box {box0, 1, box2, 1}, 128-byte swizzle.
 cudaError_t encode_bshd_bf16(CUtensorMap* map, const void* base, uint64_t D, uint64_t H, uint64_t S, uint64_t B,
                              uint32_t box0, uint32_t box2);
+
+// V2 lambda projection sigmoid(x W + bias), x [T, d_model] bf16, W [d_model, n_pairs] bf16,
+// bias fp32 [n_pairs] or null; d_model % 64 == 0, n_pairs % 8 == 0 and <= 64.
+cudaError_t launch_lambda_v2(const __nv_bfloat16* x, const __nv_bfloat16* w, const float* bias, int T, int d_model,
+                             int n_pairs, float* out, cudaStream_t stream);
 
 }  // namespace da2

@@ -180,6 +180,25 @@ DA2_API int diffattn_v2_decode_paged(const void* q, const void* kpages, const vo
                                      size_t workspace_bytes, da2_stream_t stream);
 
 /*
+ * Decode of T new tokens per sequence in one step (e.g. verifying T speculative tokens),
+ * bf16 in / bf16 out. The caches already hold all T new keys; new token t of sequence b
+ * attends to keys [0, seqlens[b] - T + t + 1), i.e. causally among the new tokens. Source:
+ * the lesson's compatibility table (speculative decoding works with DIFF V2: the attention
+ * change is invisible to the decoding loop) and the DiffAttn equation.
+ *   q bf16 [B,T,Hq,D]   lambda fp32 [B,T,Hq/2]   out bf16 [B,T,Hq/2,D]
+ *   caches, seqlens as in diffattn_v2_decode (seqlens[b] >= T; a token without visible keys
+ *   gets a zero output)
+ *   workspace: diffattn_v2_decode_multi_workspace_size(B, T, Smax, Hq, Hkv, D) bytes
+ * The (token, head) pairs of a GQA group share one pass over the cache. Supported: D == 128,
+ * group size Hq/Hkv in {2, 4, 8, 16} with T * group <= 16. T == 1 equals diffattn_v2_decode.
+ */
+DA2_API size_t diffattn_v2_decode_multi_workspace_size(int B, int T, int Smax, int Hq, int Hkv, int D);
+DA2_API int diffattn_v2_decode_multi(const void* q, const void* kcache, const void* vcache,
+                                     const int32_t* seqlens, const float* lambda, void* out, int B, int T,
+                                     int Smax, int Hq, int Hkv, int D, void* workspace, size_t workspace_bytes,
+                                     da2_stream_t stream);
+
+/*
  * The decode step in fp32 end to end (CUDA cores), same layout with fp32 q, caches and
  * out, no workspace. Supported: D in {64, 128}.
  */
@@ -227,6 +246,22 @@ DA2_API int diffattn_v2_lambda_v1(const float* lq1, const float* lk1, const floa
 DA2_API int diffattn_v2_decode_noalloc(const void* q, const void* kcache, const void* vcache,
                                        const int32_t* seqlens, const float* lambda, void* out, int B,
                                        int Smax, int Hq, int Hkv, int D, da2_stream_t stream);
+
+/*
+ * V2 lambda: lambda[t, p] = sigmoid(x[t] . w_lambda[:, p] + bias[p]), one value per token and
+ * per pair, bounded to (0, 1). Source: "Differential Transformer V2 soll KI-Training stabiler
+ * machen", section "Weniger Ausreisser und Gradientenspitzen" (V2 projects a sigmoid-bounded
+ * lambda for every token and head instead of V1's per-head normalisation). The projection
+ * input is the token's hidden state; whether it has a bias is not fixed by the pages, so
+ * bias may be NULL.
+ *   x        bf16 [T, d_model]         w_lambda bf16 [d_model, n_pairs]
+ *   bias     fp32 [n_pairs] or NULL    lambda_out fp32 [T, n_pairs] (the prefill/decode
+ *                                      lambda layout when T = B*S or T = B)
+ * bf16 products accumulated in fp32 on the tensor cores; sigmoid with the accurate expf.
+ * Supported: d_model % 64 == 0, n_pairs % 8 == 0 and n_pairs <= 64 (else DA2_ERR_UNSUPPORTED).
+ */
+DA2_API int diffattn_v2_lambda_v2(const void* x, const void* w_lambda, const float* bias, int T, int d_model,
+                                  int n_pairs, float* lambda_out, da2_stream_t stream);
 
 /*
  * Synchronise `stream`, then read and clear the device error word that kernels set when a

@@ -43,9 +43,12 @@ __all__ = [
     "prefill",
     "prefill_rows",
     "prefill_varlen",
+    "prefill_backward",
     "decode",
     "decode_paged",
+    "decode_multi",
     "lambda_v1",
+    "lambda_v2_projection",
     "branch_weights",
     "snr",
 ]
@@ -172,6 +175,47 @@ def prefill_varlen(q, k, v, lam, cu_seqlens, causal: bool = True) -> np.ndarray:
     return out
 
 
+def prefill_backward(q, k, v, lam, dout, causal: bool = True):
+    """Gradients of the prefill: returns (dq [B,S,Hq,D], dk, dv [B,S,Hkv,D], dlam [B,S,Hq/2])
+    for an upstream gradient dout [B,S,Hq/2,D], all float64.
+
+    The chain rule applied to the definition of `diff_attention_block`, per pair p (heads h1,
+    h2 over KV head g) and batch b, with A_b = softmax(S_b), S_b = Q_b K^T / sqrt(D) + mask,
+    O_b = A_b V and out = O_1 - lam * O_2:
+      dlam_i  = -dout_i . O_2,i
+      dV     += A_1^T dout - A_2^T (lam * dout)
+      dA_1    = dout V^T,            dA_2 = -lam * (dout V^T)
+      dS_b    = A_b * (dA_b - rowsum(A_b * dA_b))           (softmax backward)
+      dQ_b    = dS_b K / sqrt(D),    dK += (dS_1^T Q_1 + dS_2^T Q_2) / sqrt(D)
+    KV heads accumulate over every pair of their group.
+    """
+    q, k, v, lam, dout = _f64(q), _f64(k), _f64(v), _f64(lam), _f64(dout)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    inv = 1.0 / math.sqrt(D)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    dlam = np.zeros_like(lam)
+    mask = causal_mask(S, S) if causal else np.zeros((S, S))
+    for b in range(B):
+        for p, h1, h2, g in pair_layout(Hq, Hkv):
+            kk, vv = k[b, :, g], v[b, :, g]
+            a1 = stable_softmax(q[b, :, h1] @ kk.T * inv + mask)
+            a2 = stable_softmax(q[b, :, h2] @ kk.T * inv + mask)
+            lm = lam[b, :, p][:, None]
+            do = dout[b, :, p]
+            o2 = a2 @ vv
+            dlam[b, :, p] = -np.sum(do * o2, axis=1)
+            dv[b, :, g] += a1.T @ do - a2.T @ (lm * do)
+            dpv = do @ vv.T
+            for a, da, h in ((a1, dpv, h1), (a2, -lm * dpv, h2)):
+                ds = a * (da - np.sum(a * da, axis=1, keepdims=True))
+                dq[b, :, h] = ds @ kk * inv
+                dk[b, :, g] += ds.T @ q[b, :, h] * inv
+    return dq, dk, dv, dlam
+
+
 def prefill_rows(q, k, v, lam, rows, causal: bool = True) -> np.ndarray:
     """Selected output rows of a prefill: rows is a list of (b, i, p); returns [len(rows), D].
 
@@ -246,6 +290,19 @@ def decode_paged(q, kpages, vpages, block_table, seqlens, lam) -> np.ndarray:
     return np.stack(outs)
 
 
+def decode_multi(q, kcache, vcache, seqlens, lam) -> np.ndarray:
+    """Decode of T new tokens per sequence (a speculative-decoding verification step):
+    q [B,T,Hq,D], lam [B,T,Hq/2]; the caches already hold all T new keys, and new token t
+    of sequence b attends to keys [0, seqlens[b] - T + t + 1) -- causal among the new tokens.
+    Each token is one `decode` over its visible prefix. Returns out [B,T,Hq/2,D]."""
+    B, T = q.shape[0], q.shape[1]
+    out = np.zeros((B, T, q.shape[2] // 2, q.shape[3]), dtype=np.float64)
+    for t in range(T):
+        n_t = [max(0, int(seqlens[b]) - T + t + 1) for b in range(B)]
+        out[:, t] = decode(q[:, t], kcache, vcache, n_t, lam[:, t])
+    return out
+
+
 def lambda_v1(lq1, lk1, lq2, lk2, lambda_init: float = 0.8) -> np.ndarray:
     """V1 lambda re-parameterisation of [L16] "The differential concept":
     lambda = exp(lq1 . lk1) - exp(lq2 . lk2) + lambda_init, one scalar per pair.
@@ -255,6 +312,17 @@ def lambda_v1(lq1, lk1, lq2, lk2, lambda_init: float = 0.8) -> np.ndarray:
     """
     a, b, c, e = (_f64(x) for x in (lq1, lk1, lq2, lk2))
     return np.exp(np.sum(a * b, axis=-1)) - np.exp(np.sum(c * e, axis=-1)) + float(lambda_init)
+
+
+def lambda_v2_projection(x, w, bias=None) -> np.ndarray:
+    """V2 lambda of [HF] (section "Weniger Ausreisser und Gradientenspitzen"): projected from
+    each token's hidden state for each head (pair) and bounded by a sigmoid,
+    lambda[t, p] = 1 / (1 + exp(-(x[t] . w[:, p] + bias[p]))). x [T, d_model], w [d_model,
+    n_pairs], bias [n_pairs] or None (no bias). Returns [T, n_pairs] in (0, 1)."""
+    z = _f64(x) @ _f64(w)
+    if bias is not None:
+        z = z + _f64(bias)[None, :]
+    return 1.0 / (1.0 + np.exp(-z))
 
 
 def branch_weights(q1, q2, k, lam, n_visible=None):

@@ -146,6 +146,24 @@ def test_decode_paged_host_checks(lib):
     assert lib.diffattn_v2_decode_paged(*d64[:15] + (1 << 30,) + d64[16:]) == -2
 
 
+def test_decode_multi_host_checks(lib):
+    W = P + 65536
+    S_ = P + 24576
+    ws = lib.diffattn_v2_decode_multi_workspace_size(2, 2, 1024, 16, 2, 128)
+    assert ws >= lib.diffattn_v2_decode_workspace_size(2, 1024, 16, 2, 128)
+    assert lib.diffattn_v2_decode_multi(Q, K, V, S_, L, O, 2, 4, 1024, 16, 2, 128, W, 1 << 30, None) == -2  # T*G > 16
+    assert lib.diffattn_v2_decode_multi(Q, K, V, S_, L, O, 2, 0, 1024, 16, 2, 128, W, ws, None) == -1       # T = 0
+    assert lib.diffattn_v2_decode_multi(Q, K, V, S_, L, O, 2, 2, 1024, 16, 2, 128, W, ws - 16, None) == -1  # workspace
+
+
+def test_lambda_v2_host_checks(lib):
+    assert lib.diffattn_v2_lambda_v2(Q, K, None, 10, 100, 32, O, None) == -2   # d_model % 64
+    assert lib.diffattn_v2_lambda_v2(Q, K, None, 10, 128, 20, O, None) == -2   # n_pairs % 8
+    assert lib.diffattn_v2_lambda_v2(Q, K, None, 10, 128, 72, O, None) == -2   # n_pairs > 64
+    assert lib.diffattn_v2_lambda_v2(None, K, None, 10, 128, 32, O, None) == -1
+    assert lib.diffattn_v2_lambda_v2(Q, K, None, 0, 128, 32, O, None) == 0
+
+
 def test_lambda_v1_host_checks(lib):
     assert lib.diffattn_v2_lambda_v1(Q, K, V, L, 0.8, 0, 128, 1, O, None) == -1
     assert lib.diffattn_v2_lambda_v1(Q, K, V, L, 0.8, 4, 0, 1, O, None) == -1

@@ -145,3 +145,37 @@ def test_decode_paged_matches_contiguous_and_oracle(da, page_size, lens):
     assert torch.equal(got, contiguous)  # same splits, same arithmetic
     ref = ora.decode_paged(inp["q"], kp, vp, table.tolist(), inp["seqlens"], inp["lam"])
     bf16_close(got, ref, f"paged decode page_size={page_size}")
+
+
+@pytest.mark.parametrize("T,d_model,n_pairs,with_bias", [
+    (1, 64, 8, False), (100, 256, 32, True), (4096, 4096, 32, True), (333, 512, 64, False), (70, 128, 40, True)])
+def test_lambda_v2_projection_matches_oracle(da, T, d_model, n_pairs, with_bias):
+    g = torch.Generator().manual_seed(T + n_pairs)
+    x = torch.randn(T, d_model, generator=g).bfloat16()
+    w = (torch.randn(d_model, n_pairs, generator=g) / d_model ** 0.5).bfloat16()
+    bias = torch.randn(n_pairs, generator=g) if with_bias else None
+    got = da.lambda_v2(x.cuda(), w.cuda(), None if bias is None else bias.cuda())
+    ref = ora.lambda_v2_projection(x, w, bias)
+    np.testing.assert_allclose(got.cpu().double().numpy(), ref, rtol=0, atol=1e-5)
+    assert torch.all((got > 0) & (got < 1))
+
+
+@pytest.mark.parametrize("B,T,Smax,Hq,Hkv,lens", [
+    (3, 2, 700, 16, 2, [700, 2, 301]),       # group 8, two tokens (two column tiles)
+    (2, 4, 900, 8, 2, [900, 65]),            # group 4, four tokens
+    (2, 8, 500, 4, 2, [500, 8]),             # group 2, eight tokens
+    (2, 1, 600, 16, 2, [600, 1]),            # one token: the plain decode
+])
+def test_decode_multi_matches_oracle(da, B, T, Smax, Hq, Hkv, lens):
+    inp = _decode_case(B, Smax, Hq, Hkv, lens, seed=T * 100 + Smax)
+    g = torch.Generator().manual_seed(T)
+    q = torch.randn(B, T, Hq, 128, generator=g).bfloat16()
+    lam = torch.sigmoid(torch.randn(B, T, Hq // 2, generator=g))
+    out = da.decode_multi(q.cuda(), inp["kcache"].cuda(), inp["vcache"].cuda(), inp["seqlens"].cuda(), lam.cuda())
+    assert da.device_error() == 0
+    ref = ora.decode_multi(q, inp["kcache"], inp["vcache"], inp["seqlens"], lam)
+    bf16_close(out, ref, f"decode_multi T={T}")
+    if T == 1:
+        single = da.decode(q[:, 0].contiguous().cuda(), inp["kcache"].cuda(), inp["vcache"].cuda(),
+                           inp["seqlens"].cuda(), lam[:, 0].contiguous().cuda())
+        assert torch.equal(out[:, 0], single)

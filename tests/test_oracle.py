@@ -300,6 +300,76 @@ def pin_paged_decode_gathers_pages():
     return bool(ok)
 
 
+def pin_lambda_v2_projection():
+    """sigmoid(x W + b): W = 0 gives sigmoid(b) (0.5 without bias, 0.75 for b = ln 3); one
+    nonzero weight gives sigmoid(x_k w_k); random inputs match torch.sigmoid(x @ W + b)."""
+    rng = np.random.default_rng(17)
+    x = rng.standard_normal((5, 12))
+    w0 = np.zeros((12, 4))
+    ok = np.allclose(ora.lambda_v2_projection(x, w0), 0.5, rtol=0, atol=0)
+    ok &= np.allclose(ora.lambda_v2_projection(x, w0, np.full(4, math.log(3.0))), 0.75, atol=1e-15)
+    w1 = w0.copy()
+    w1[3, 2] = 0.7
+    ok &= np.allclose(ora.lambda_v2_projection(x, w1)[:, 2], 1.0 / (1.0 + np.exp(-0.7 * x[:, 3])), atol=1e-15)
+    w = rng.standard_normal((12, 4))
+    b = rng.standard_normal(4)
+    ref = torch.sigmoid(torch.from_numpy(x) @ torch.from_numpy(w) + torch.from_numpy(b)).numpy()
+    lam = ora.lambda_v2_projection(x, w, b)
+    ok &= np.allclose(lam, ref, atol=1e-14) and bool(np.all((lam > 0) & (lam < 1)))
+    return bool(ok)
+
+
+def pin_multi_token_decode_is_prefill_tail():
+    """T new tokens decoded together equal the last T rows of a causal prefill."""
+    q, k, v, lam = _rand_prefill(B=2, S=15, Hq=8, Hkv=2, D=6, seed=18)
+    T = 3
+    full = ora.prefill(q, k, v, lam)
+    dec = ora.decode_multi(q[:, -T:], k, v, [15, 15], lam[:, -T:])
+    return bool(np.allclose(dec, full[:, -T:], atol=1e-13))
+
+
+def _torch_forward(q, k, v, lam, causal=True):
+    """An independent float64 torch forward (for autograd): heads 2p and 2p+1 over KV head
+    2p // G, scores / sqrt(D), causal mask, torch.softmax, out = A1 V - lam A2 V."""
+    B, S, Hq, D = q.shape
+    G = Hq // k.shape[2]
+    kv = torch.arange(Hq) // G
+    kk = k[:, :, kv].permute(0, 2, 1, 3)
+    vv = v[:, :, kv].permute(0, 2, 1, 3)
+    s_ = q.permute(0, 2, 1, 3) @ kk.transpose(-1, -2) / math.sqrt(D)
+    if causal:
+        s_ = s_.masked_fill(torch.triu(torch.ones(S, S, dtype=torch.bool), 1), float("-inf"))
+    o = torch.softmax(s_, dim=-1) @ vv  # [B, Hq, S, D]
+    return (o[:, 0::2] - lam.permute(0, 2, 1)[..., None] * o[:, 1::2]).permute(0, 2, 1, 3)
+
+
+def pin_backward_matches_autograd(causal=True):
+    q, k, v, lam = _rand_prefill(B=2, S=11, Hq=8, Hkv=2, D=6, seed=19)
+    dout = np.random.default_rng(20).standard_normal((2, 11, 4, 6))
+    ts = [torch.tensor(x, requires_grad=True) for x in (q, k, v, lam)]
+    _torch_forward(*ts, causal=causal).backward(torch.tensor(dout))
+    got = ora.prefill_backward(q, k, v, lam, dout, causal=causal)
+    return bool(all(np.allclose(g, t.grad.numpy(), atol=1e-11) for g, t in zip(got, ts)))
+
+
+def pin_backward_finite_differences():
+    """Central differences of <dout, prefill(.)> on a few entries of every input."""
+    q, k, v, lam = _rand_prefill(B=1, S=6, Hq=4, Hkv=1, D=3, seed=21)
+    dout = np.random.default_rng(22).standard_normal((1, 6, 2, 3))
+    grads = ora.prefill_backward(q, k, v, lam, dout)
+    f = lambda q_, k_, v_, l_: float(np.sum(ora.prefill(q_, k_, v_, l_) * dout))
+    eps = 1e-6
+    ok = True
+    for which, idx in ((0, (0, 4, 1, 2)), (1, (0, 3, 0, 1)), (2, (0, 5, 0, 0)), (3, (0, 2, 1))):
+        args = [q.copy(), k.copy(), v.copy(), lam.copy()]
+        args[which][idx] += eps
+        up = f(*args)
+        args[which][idx] -= 2 * eps
+        dn = f(*args)
+        ok &= abs((up - dn) / (2 * eps) - grads[which][idx]) < 1e-6
+    return bool(ok)
+
+
 ALL_PINS = {
     "softmax_library": pin_softmax_library,
     "lambda0_is_softmax_attention": pin_lambda0_is_softmax_attention,
@@ -323,6 +393,11 @@ ALL_PINS = {
     "window_mask_definition": pin_window_mask_definition,
     "varlen_is_per_sequence_prefill": pin_varlen_is_per_sequence_prefill,
     "paged_decode_gathers_pages": pin_paged_decode_gathers_pages,
+    "lambda_v2_projection": pin_lambda_v2_projection,
+    "multi_token_decode_is_prefill_tail": pin_multi_token_decode_is_prefill_tail,
+    "backward_matches_autograd": pin_backward_matches_autograd,
+    "backward_matches_autograd_noncausal": lambda: pin_backward_matches_autograd(causal=False),
+    "backward_finite_differences": pin_backward_finite_differences,
 }
 
 

@@ -108,6 +108,11 @@ def _lambda_v1_plus(lq1, lk1, lq2, lk2, lambda_init=0.8):
     return np.exp(np.sum(a * b, -1)) + np.exp(np.sum(c * e, -1)) + lambda_init
 
 
+def _lambda_v2_no_sigmoid(x, w, bias=None):
+    z = np.asarray(x, dtype=np.float64) @ np.asarray(w, dtype=np.float64)
+    return z if bias is None else z + np.asarray(bias)[None, :]
+
+
 MUTANTS = {
     "plus_sign": ("diff_attention_block", _block_plus_sign),
     "no_scale": ("diff_attention_block", _block_no_scale),
@@ -124,6 +129,7 @@ MUTANTS = {
     "softmax_epsilon": ("stable_softmax", _softmax_off),
     "lambda_v1_plus": ("lambda_v1", _lambda_v1_plus),
     "window_off_by_one": ("window_mask", _window_off_by_one),
+    "lambda_v2_no_sigmoid": ("lambda_v2_projection", _lambda_v2_no_sigmoid),
 }
 
 
