@@ -592,6 +592,29 @@ def run_workload(args):
         ms = _time_op(fn, args.steps, args.warmup, stream)
         val = nbytes / (ms * 1e-3) / 1e9
         unit, peak, bound = "GB/s", peaks["hbm_gbs"], "hbm"
+    elif name == "backward":
+        case = workloads.CONFIGS["c2_bf16_prefill"]
+        inp = workloads.make_prefill(case)
+        q, k, v, lam = (inp[x].to(dev) for x in ("q", "k", "v", "lam"))
+        dout = workloads.make_prefill_grad(case).to(dev)
+        out, ob, lse = da.prefill_train(q, k, v, lam, stream=stream)
+        grads = [torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(lam)]
+        ws = torch.empty(da.backward_workspace_size(case.B, case.S, case.Hq), dtype=torch.uint8, device=dev)
+        fwd_ms = _time_op(lambda: da.prefill_train(q, k, v, lam, out=out, o_branch=ob, lse=lse, stream=stream),
+                          args.steps, args.warmup, stream)
+        fn = lambda: da.backward(q, k, v, lam, ob, lse, dout, dq=grads[0], dk=grads[1], dv=grads[2], dlam=grads[3],
+                                 workspace=ws, stream=stream)
+        # chain-rule products per pair and visible (query, key): S_1, S_2 recomputed, dP shared
+        # by both branches, dV from the combined weights, dK and dQ of both heads: 8 products
+        # of 2*D flops each, twice the forward's 4
+        flops = 2 * workloads.prefill_flops(case.B, case.S, case.Hq, D)
+        ms = _time_op(fn, args.steps, args.warmup, stream)
+        val = flops / (ms * 1e-3) / 1e12
+        unit, peak, bound = "TFLOP/s", peaks["bf16_tflops"], "tensor"
+        launches = 3
+        cfg = {"workload": "backward of the causal prefill B=4 S=4096 Hq=64 Hkv=8 D=128 (dQ, dK, dV, dlambda)",
+               "train_forward_ms": round(fwd_ms, 4),
+               "train_forward_tflops": round(workloads.prefill_flops(case.B, case.S, case.Hq, D) / (fwd_ms * 1e-3) / 1e12, 2)}
     elif name == "lambda_v2":
         T, dm, npair = 16384, 4096, 32
         g = torch.Generator().manual_seed(12)
@@ -632,7 +655,7 @@ def main(argv=None):
     ap.add_argument("--ref-seconds", type=float, default=120.0,
                     help="host-time budget of the whole reference run (warm-up and timed steps)")
     ap.add_argument("--workload", choices=("prefill_long", "decode_needle", "window", "varlen", "paged", "multi",
-                                           "lambda_v2"), default=None,
+                                           "lambda_v2", "backward"), default=None,
                     help="time one other operation alone instead of the default step")
     ap.add_argument("--scaling", choices=("weak", "strong"), default="weak",
                     help="weak: each GPU runs the full per-GPU workload; strong: the heads of one workload "

@@ -29,6 +29,9 @@ _SIGNATURES = {
     "diffattn_v2_prefill_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
     "diffattn_v2_prefill_window": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
     "diffattn_v2_prefill_varlen": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]),
+    "diffattn_v2_prefill_train": (_i, [_vp] * 7 + [_i] * 6 + [_vp]),
+    "diffattn_v2_backward_workspace_size": (_sz, [_i, _i, _i]),
+    "diffattn_v2_backward": (_i, [_vp] * 11 + [_i] * 6 + [_vp, _sz, _vp]),
     "diffattn_v2_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "diffattn_v2_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "diffattn_v2_decode_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
@@ -161,6 +164,60 @@ def prefill_f32(q, k, v, lam, out=None, causal=True, stream=None):
                                      1 if causal else 0, _stream(stream, q.device))
     _check(st, "diffattn_v2_prefill_f32")
     return out
+
+
+def prefill_train(q, k, v, lam, out=None, o_branch=None, lse=None, causal=True, stream=None):
+    """Training forward: prefill plus the per-head normalised O_b (bf16 [B,S,Hq,D]) and the
+    log2-domain row log-sum-exp (fp32 [B,S,Hq]) that backward reads. Returns (out, o_branch, lse)."""
+    for t, n, nd in ((q, "q", 4), (k, "k", 4), (v, "v", 4)):
+        _need(t, n, torch.bfloat16, nd)
+    _need(lam, "lam", torch.float32, 3)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if out is None:
+        out = torch.empty((B, S, Hq // 2, D), dtype=torch.bfloat16, device=q.device)
+    if o_branch is None:
+        o_branch = torch.empty((B, S, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, S, Hq), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.bfloat16, 4)
+    _need(o_branch, "o_branch", torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    st = LIB.diffattn_v2_prefill_train(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(out), _ptr(o_branch), _ptr(lse),
+                                       B, S, Hq, Hkv, D, 1 if causal else 0, _stream(stream, q.device))
+    _check(st, "diffattn_v2_prefill_train")
+    return out, o_branch, lse
+
+
+def backward_workspace_size(B, S, Hq) -> int:
+    return int(LIB.diffattn_v2_backward_workspace_size(B, S, Hq))
+
+
+def backward(q, k, v, lam, o_branch, lse, dout, causal=True, dq=None, dk=None, dv=None, dlam=None,
+             workspace=None, stream=None):
+    """Gradients of the bf16 prefill: returns (dq, dk, dv, dlam) with the layouts of q, k, v, lam."""
+    for t, n, nd in ((q, "q", 4), (k, "k", 4), (v, "v", 4), (o_branch, "o_branch", 4), (dout, "dout", 4)):
+        _need(t, n, torch.bfloat16, nd)
+    _need(lam, "lam", torch.float32, 3)
+    _need(lse, "lse", torch.float32, 3)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    dlam = torch.empty_like(lam) if dlam is None else dlam
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _need(t, n, torch.bfloat16, 4)
+    _need(dlam, "dlam", torch.float32, 3)
+    ws_bytes = backward_workspace_size(B, S, Hq)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+    st = LIB.diffattn_v2_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(o_branch), _ptr(lse), _ptr(dout),
+                                  _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlam), B, S, Hq, Hkv, D, 1 if causal else 0,
+                                  _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                  _stream(stream, q.device))
+    _check(st, "diffattn_v2_backward")
+    return dq, dk, dv, dlam
 
 
 def decode_workspace_size(B, Smax, Hq, Hkv, D) -> int:

@@ -198,6 +198,59 @@ int diffattn_v2_prefill_f32(const float* q, const float* k, const float* v, cons
                                            reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int diffattn_v2_prefill_train(const void* q, const void* k, const void* v, const float* lambda, void* out,
+                              void* o_branch, float* lse, int B, int S, int Hq, int Hkv, int D, int causal,
+                              da2_stream_t stream) {
+  if (B < 0 || S < 0 || D <= 0 || !heads_ok(Hq, Hkv)) return DA2_ERR_INVALID;
+  if (causal != 0 && causal != 1) return DA2_ERR_INVALID;
+  if (B == 0 || S == 0) return DA2_OK;
+  if (!q || !k || !v || !lambda || !out || !o_branch || !lse) return DA2_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(lambda) || !aligned16(out) ||
+      !aligned16(o_branch) || !aligned16(lse))
+    return DA2_ERR_INVALID;
+  if (D != 128) return DA2_ERR_UNSUPPORTED;
+  if ((S + 127) / 128 > 65535) return DA2_ERR_UNSUPPORTED;
+  int* err = nullptr;
+  cudaError_t e = device_error_ptr(&err);
+  if (e != cudaSuccess) return DA2_ERR_CUDA;
+  CUtensorMap tq, tk, tv;
+  if (encode_bshd(&tq, q, D, Hq, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  if (encode_bshd(&tk, k, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  if (encode_bshd(&tv, v, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  e = da2::launch_prefill(tq, tk, tv, lambda, static_cast<__nv_bfloat16*>(out), err, B, S, Hq, Hkv, causal, 0,
+                          nullptr, reinterpret_cast<cudaStream_t>(stream), static_cast<__nv_bfloat16*>(o_branch),
+                          lse);
+  return status_of(e);
+}
+
+size_t diffattn_v2_backward_workspace_size(int B, int S, int Hq) {
+  if (B <= 0 || S <= 0 || Hq <= 0) return 0;
+  return static_cast<size_t>(B) * S * Hq * sizeof(float);
+}
+
+int diffattn_v2_backward(const void* q, const void* k, const void* v, const float* lambda, const void* o_branch,
+                         const float* lse, const void* dout, void* dq, void* dk, void* dv, float* dlambda, int B,
+                         int S, int Hq, int Hkv, int D, int causal, void* workspace, size_t workspace_bytes,
+                         da2_stream_t stream) {
+  if (B < 0 || S < 0 || D <= 0 || !heads_ok(Hq, Hkv)) return DA2_ERR_INVALID;
+  if (causal != 0 && causal != 1) return DA2_ERR_INVALID;
+  if (B == 0 || S == 0) return DA2_OK;
+  const void* ptrs[] = {q, k, v, lambda, o_branch, lse, dout, dq, dk, dv, dlambda, workspace};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return DA2_ERR_INVALID;
+  if (workspace_bytes < diffattn_v2_backward_workspace_size(B, S, Hq)) return DA2_ERR_INVALID;
+  if (D != 128) return DA2_ERR_UNSUPPORTED;
+  // grid limits: heads and batch on grid y / z; the preprocess runs 4 (token, pair) warps per CTA
+  if (B > 65535 || Hq > 65535) return DA2_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * S * (Hq / 2) > 4LL * 2147483647LL) return DA2_ERR_UNSUPPORTED;
+  using bf = __nv_bfloat16;
+  return status_of(da2::launch_backward(
+      static_cast<const bf*>(q), static_cast<const bf*>(k), static_cast<const bf*>(v), lambda,
+      static_cast<const bf*>(o_branch), lse, static_cast<const bf*>(dout), static_cast<bf*>(dq), static_cast<bf*>(dk),
+      static_cast<bf*>(dv), dlambda, static_cast<float*>(workspace), B, S, Hq, Hkv, causal,
+      reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t diffattn_v2_decode_workspace_size(int B, int Smax, int Hq, int Hkv, int D) {
   if (B <= 0 || Smax <= 0 || D <= 0 || !heads_ok(Hq, Hkv)) return 0;
   int split_len = 0, nsplit = 0;

@@ -15,7 +15,16 @@ namespace da2 {
 // boxes of 64 (d) x 1 (head) x 128 (rows) x 1, 128-byte swizzle.
 cudaError_t launch_prefill(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                            const float* lambda, __nv_bfloat16* out, int* err, int B, int S, int Hq, int Hkv,
-                           int causal, int window, const int* cu_seqlens, cudaStream_t stream);
+                           int causal, int window, const int* cu_seqlens, cudaStream_t stream,
+                           __nv_bfloat16* o_branch = nullptr, float* lse = nullptr);
+
+// Backward of the bf16 [B,S] prefill (D = 128): preprocess (E, dlambda), dK/dV, dQ. o_branch
+// [B,S,Hq,D] and lse [B,S,Hq] come from the training forward; E is fp32 [B,S,Hq] scratch.
+cudaError_t launch_backward(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
+                            const float* lambda, const __nv_bfloat16* o_branch, const float* lse,
+                            const __nv_bfloat16* dout, __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv,
+                            float* dlambda, float* E, int B, int S, int Hq, int Hkv, int causal,
+                            cudaStream_t stream);
 
 // bf16 decode (D = 128): split kernel + combine. Tensor maps over the caches [B,Smax,Hkv,D],
 // boxes of 64 (d) x 1 x 64 (tokens) x 1, 128-byte swizzle. With block_table the maps cover

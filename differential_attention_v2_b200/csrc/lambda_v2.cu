@@ -7,8 +7,9 @@
 //
 // x [T, d_model] bf16 and W [d_model, n_pairs] bf16 give a skinny GEMM (n_pairs <= 64); the
 // kernel reads x once. A CTA takes 64 tokens; four warps each take 16 tokens and all pairs
-// on mma.sync m16n8k16 (bf16 in, fp32 accumulate); x and W chunks of 64 along d_model are
-// double-buffered in shared memory with cp.async. The epilogue adds the bias and applies the
+// on mma.sync m16n8k16 (bf16 in, fp32 accumulate); x and W chunks of 64 along d_model stream
+// through a ring of kStages shared-memory stages filled by cp.async, so that about 40 KB per
+// CTA is in flight (the read is HBM-latency-bound with fewer). The epilogue adds the bias and applies the
 // sigmoid with the accurate expf, writing fp32 lambda [T, n_pairs] -- the layout of the
 // prefill ([B*S, Hq/2]) and decode ([B, Hq/2]) lambda arguments.
 
@@ -20,7 +21,11 @@ namespace lambda2 {
 
 constexpr int kTok = 64;     // tokens per CTA
 constexpr int kChunk = 64;   // d_model per stage
+constexpr int kStages = 6;   // ring depth
 constexpr int kThreads = 128;
+
+template <int NT>
+constexpr int smem_bytes() { return kStages * (kTok * kChunk * 2 + kChunk * (NT + 1) * 16); }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
@@ -37,9 +42,9 @@ lambda_v2_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __res
   constexpr int kWChunks = NT + 1;                     // 16-byte chunks per W row (+1 padding)
   constexpr uint32_t kXBytes = kTok * kChunk * 2;      // 8 KB per x stage
   constexpr uint32_t kWBytes = kChunk * kWChunks * 16; // per W stage
-  __shared__ __align__(128) uint8_t smem[2 * kXBytes + 2 * kWBytes];
+  extern __shared__ __align__(128) uint8_t smem[];
   const uint32_t sx = smem_u32(smem);
-  const uint32_t sw = sx + 2 * kXBytes;
+  const uint32_t sw = sx + kStages * kXBytes;
 
   const int tok0 = blockIdx.x * kTok;
   const int tid = threadIdx.x;
@@ -75,16 +80,18 @@ lambda_v2_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __res
   const int b_krow = (lane & 7) + (lane >> 3 & 1) * 8;                 // W: (k0,n0)(k8,n0)(k0,n8)(k8,n8)
   const int b_nsel = (lane >> 4) & 1;
 
-  load_stage(0, 0);
+  // one commit group per chunk (empty groups past the end keep the count uniform)
+#pragma unroll
+  for (int s = 0; s < kStages - 1; ++s) {
+    if (s < n_chunks) load_stage(s, s);
+    else cp_async_commit();
+  }
   for (int kc = 0; kc < n_chunks; ++kc) {
-    const int st = kc & 1;
-    if (kc + 1 < n_chunks) {
-      load_stage(st ^ 1, kc + 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
+    const int st = kc % kStages;
+    cp_async_wait<kStages - 2>();  // chunk kc has landed (this thread's copies)
+    __syncthreads();               // ... everyone's; and chunk kc-1's stage is free
+    if (kc + kStages - 1 < n_chunks) load_stage((kc + kStages - 1) % kStages, kc + kStages - 1);
+    else cp_async_commit();
 #pragma unroll
     for (int ks = 0; ks < kChunk / 16; ++ks) {
       const int chunk = 2 * ks + a_csel;
@@ -99,7 +106,6 @@ lambda_v2_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __res
         mma_m16n8k16_bf16(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
       }
     }
-    __syncthreads();  // the stage is overwritten by the next iteration's loads
   }
 
   const int gl = lane >> 2, tq = lane & 3;
@@ -130,14 +136,19 @@ cudaError_t launch_lambda_v2(const __nv_bfloat16* x, const __nv_bfloat16* w, con
   using namespace lambda2;
   const dim3 grid((T + kTok - 1) / kTok);
   const int nt = (n_pairs + 15) / 16 * 2;  // 8-pair tiles, even
+  auto run = [&](auto kernel, int smem) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kernel<<<grid, kThreads, smem, stream>>>(x, w, bias, out, T, d_model, n_pairs);
+    return cudaGetLastError();
+  };
   switch (nt) {
-    case 2: lambda_v2_kernel<2><<<grid, kThreads, 0, stream>>>(x, w, bias, out, T, d_model, n_pairs); break;
-    case 4: lambda_v2_kernel<4><<<grid, kThreads, 0, stream>>>(x, w, bias, out, T, d_model, n_pairs); break;
-    case 6: lambda_v2_kernel<6><<<grid, kThreads, 0, stream>>>(x, w, bias, out, T, d_model, n_pairs); break;
-    case 8: lambda_v2_kernel<8><<<grid, kThreads, 0, stream>>>(x, w, bias, out, T, d_model, n_pairs); break;
+    case 2: return run(lambda_v2_kernel<2>, smem_bytes<2>());
+    case 4: return run(lambda_v2_kernel<4>, smem_bytes<4>());
+    case 6: return run(lambda_v2_kernel<6>, smem_bytes<6>());
+    case 8: return run(lambda_v2_kernel<8>, smem_bytes<8>());
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 }  // namespace da2

@@ -75,6 +75,8 @@ constexpr uint32_t kTmS1 = 0, kTmS2 = 128, kTmO1 = 256, kTmO2 = 384;
 struct Params {
   const float* lambda;    // [B,S,Hq/2]
   __nv_bfloat16* out;     // [B,S,Hq/2,D]
+  __nv_bfloat16* o_branch;  // training forward: [B,S,Hq,D] per-head normalised O_b (null = inference)
+  float* lse;             // training forward: [B,S,Hq] log2-domain log-sum-exp of the scaled scores
   int* err;               // device error word
   int B, S, Hq, Hkv, causal;
   int window;             // causal sliding window (keys i-window+1 .. i); 0 = none
@@ -426,6 +428,9 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 
     if (ok) ok = mbar_wait(bar(kOFull), 0, abort_flag);
     l_xchg[br * BM + r] = l_run;
+    // training forward: A_b = 2^(s * scale_log2 - lse) recomputes the probabilities later
+    if (p.lse != nullptr && qi < S)
+      p.lse[(row_base + qi) * p.Hq + 2 * pair + br] = (m_run == -INFINITY ? 0.f : m_run) + __log2f(l_run);
     asm volatile("bar.sync 1, 256;" ::: "memory");
     if (__all_sync(0xffffffffu, ok && !*abort_flag)) {
       tc_fence_after();
@@ -442,6 +447,21 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         tmem_ld_32x32b_x32(trow + kTmO2 + col, o2);
         tmem_ld_wait(o1);
         reg_fence(o2);
+        if (p.o_branch != nullptr && row_valid) {
+          // per-head normalised O_1, O_2 of the pair, same columns as this thread's out slice
+#pragma unroll
+          for (int hb = 0; hb < 2; ++hb) {
+            const uint32_t* o = hb ? o2 : o1;
+            const float inv = hb ? inv2 : inv1;
+            uint4* dst = reinterpret_cast<uint4*>(p.o_branch + ((row_base + qi) * p.Hq + 2 * pair + hb) * HD + col);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv),
+                                  pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv),
+                                  pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv),
+                                  pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv));
+          }
+        }
         uint32_t packed[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
@@ -476,11 +496,14 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 
 cudaError_t launch_prefill(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                            const float* lambda, __nv_bfloat16* out, int* err, int B, int S, int Hq, int Hkv,
-                           int causal, int window, const int* cu_seqlens, cudaStream_t stream) {
+                           int causal, int window, const int* cu_seqlens, cudaStream_t stream,
+                           __nv_bfloat16* o_branch, float* lse) {
   using namespace prefill;
   Params p;
   p.lambda = lambda;
   p.out = out;
+  p.o_branch = o_branch;
+  p.lse = lse;
   p.err = err;
   p.B = B;
   p.S = S;

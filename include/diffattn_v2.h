@@ -131,6 +131,45 @@ DA2_API int diffattn_v2_prefill_f32(const float* q, const float* k, const float*
                             int D, int causal, da2_stream_t stream);
 
 /*
+ * Training forward: diffattn_v2_prefill (same arguments, checks and out) that also writes
+ * what the backward pass needs ("Differential Transformer V2 soll KI-Training stabiler
+ * machen": V2 is meant for pretraining, so the operator carries gradients):
+ *   o_branch bf16 [B,S,Hq,D]  O_b = softmax(Q_b K^T / sqrt(D)) V of every query head, each
+ *                             normalised on its own (head 2p is branch 1 of pair p, 2p+1
+ *                             branch 2), so out = O_{2p} - lambda * O_{2p+1} up to rounding
+ *   lse      fp32 [B,S,Hq]    log2-domain log-sum-exp of the head's scaled scores:
+ *                             softmax row = 2^(s * log2(e) / sqrt(D) - lse)
+ * Caller-owned device buffers, 16-byte aligned; D == 128.
+ */
+DA2_API int diffattn_v2_prefill_train(const void* q, const void* k, const void* v, const float* lambda,
+                                      void* out, void* o_branch, float* lse, int B, int S, int Hq,
+                                      int Hkv, int D, int causal, da2_stream_t stream);
+
+/* Scratch (bytes) diffattn_v2_backward needs: fp32 [B,S,Hq] row terms; 0 for invalid sizes. */
+DA2_API size_t diffattn_v2_backward_workspace_size(int B, int S, int Hq);
+
+/*
+ * Gradients of the bf16 prefill given dout = dL/d(out), bf16 [B,S,Hq/2,D]. Chain rule of
+ * out = softmax(Q_1 K^T/sqrt(D)) V - lambda * softmax(Q_2 K^T/sqrt(D)) V ("Differential
+ * Attention (V2)" lesson, "The differential concept"; causal mask of the "Attention
+ * variants" lesson):
+ *   dq bf16 [B,S,Hq,D]    dL/dQ of every query head (both branches of every pair)
+ *   dk, dv bf16 [B,S,Hkv,D]  summed over the query heads of each KV head's group
+ *   dlambda fp32 [B,S,Hq/2]  dL/dlambda = -dout . O_2 per token and pair
+ * Inputs: q, k, v, lambda as given to diffattn_v2_prefill_train, and the o_branch and lse it
+ * wrote. workspace: at least diffattn_v2_backward_workspace_size(B, S, Hq) bytes of device
+ * memory, no state between calls. Every output is overwritten (nothing accumulates into
+ * it); the result is deterministic (no atomics). Supported: D == 128, causal 0 or 1.
+ * Errors: DA2_ERR_INVALID for bad sizes, null or unaligned pointers, short workspace;
+ * DA2_ERR_UNSUPPORTED for other D or grids past the launch limits (B or Hq > 65535).
+ */
+DA2_API int diffattn_v2_backward(const void* q, const void* k, const void* v, const float* lambda,
+                                 const void* o_branch, const float* lse, const void* dout, void* dq,
+                                 void* dk, void* dv, float* dlambda, int B, int S, int Hq, int Hkv, int D,
+                                 int causal, void* workspace, size_t workspace_bytes,
+                                 da2_stream_t stream);
+
+/*
  * Workspace (bytes) that diffattn_v2_decode needs for these sizes: the per-split partial
  * results (running max, running sum and unnormalised output of each head), fp32. Returns 0
  * for invalid sizes. The workspace holds no state between calls.

@@ -44,6 +44,7 @@ __all__ = [
     "prefill_rows",
     "prefill_varlen",
     "prefill_backward",
+    "prefill_branches",
     "decode",
     "decode_paged",
     "decode_multi",
@@ -214,6 +215,32 @@ def prefill_backward(q, k, v, lam, dout, causal: bool = True):
                 dq[b, :, h] = ds @ kk * inv
                 dk[b, :, g] += ds.T @ q[b, :, h] * inv
     return dq, dk, dv, dlam
+
+
+def prefill_branches(q, k, v, causal: bool = True):
+    """Per-head pieces of the prefill that a training forward keeps for the backward pass:
+    O_h = softmax(Q_h K_g^T / sqrt(D) + mask) V_g for every query head h (float64
+    [B,S,Hq,D]), and the row log-sum-exp of the head's scaled scores in base 2,
+    lse2_h[i] = log2(sum_j 2^(s_ij * log2(e))) with s = Q_h K_g^T / sqrt(D) (float64
+    [B,S,Hq]), so that softmax row i equals 2^(s_ij * log2(e) - lse2_h[i]).
+
+    Heads map to KV heads as in `pair_layout`; out = O_{2p} - lam * O_{2p+1} ("Differential
+    Attention (V2)" lesson, "The differential concept")."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    inv = 1.0 / math.sqrt(D)
+    mask = causal_mask(S, S) if causal else np.zeros((S, S))
+    o = np.zeros_like(q)
+    lse2 = np.zeros((B, S, Hq))
+    for b in range(B):
+        for p, h1, h2, g in pair_layout(Hq, Hkv):
+            for h in (h1, h2):
+                s_ = q[b, :, h] @ k[b, :, g].T * inv + mask
+                o[b, :, h] = stable_softmax(s_) @ v[b, :, g]
+                m = np.max(s_, axis=1, keepdims=True)
+                lse2[b, :, h] = (m[:, 0] + np.log(np.sum(np.exp(s_ - m), axis=1))) / math.log(2.0)
+    return o, lse2
 
 
 def prefill_rows(q, k, v, lam, rows, causal: bool = True) -> np.ndarray:

@@ -49,3 +49,25 @@ def sample_rows(B, S, n_pairs, n=1024, seed=0, tile=128):
     while len(rows) < n + len(special) * B * n_pairs:
         rows.append((int(rng.integers(B)), int(rng.integers(S)), int(rng.integers(n_pairs))))
     return rows
+
+
+# Gradients (bf16 backward): relative Frobenius 1e-2 and max-abs 2e-2 of the largest
+# reference entry. P and dS are rounded to bf16 before their products (relative 2^-9 each),
+# the branch outputs O_b that E = dO . O_b reads are stored in bf16, and every gradient is
+# rounded once to bf16: each term is ~2e-3 relative, so 1e-2 leaves a factor ~3 of margin.
+GRAD_REL_FRO = 1e-2
+GRAD_MAX_REL = 2e-2
+
+
+def grad_close(got, ref, what=""):
+    got = to64(got) if hasattr(got, "detach") else np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite gradient"
+    scale = float(np.abs(ref).max()) if ref.size else 0.0
+    max_abs = float(np.abs(got - ref).max()) if ref.size else 0.0
+    den = float(np.linalg.norm(ref))
+    rel = float(np.linalg.norm(got - ref) / den) if den > 0 else float(np.linalg.norm(got))
+    assert max_abs <= GRAD_MAX_REL * max(scale, 1e-30), f"{what}: max-abs {max_abs:.3e} > {GRAD_MAX_REL} x {scale:.3e}"
+    assert rel <= GRAD_REL_FRO, f"{what}: rel-Frobenius {rel:.3e} > {GRAD_REL_FRO}"
+    return max_abs, rel

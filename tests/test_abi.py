@@ -169,3 +169,38 @@ def test_lambda_v1_host_checks(lib):
     assert lib.diffattn_v2_lambda_v1(Q, K, V, L, 0.8, 4, 0, 1, O, None) == -1
     assert lib.diffattn_v2_lambda_v1(Q, K, V, L, 0.8, 4, 128, 0, O, None) == 0
     assert lib.diffattn_v2_lambda_v1(None, K, V, L, 0.8, 4, 128, 1, O, None) == -1
+
+
+def test_package_exposes_every_binding_name(lib):
+    """Each wrapper of the binding module is reachable from the package namespace."""
+    import differential_attention_v2_b200 as da
+    from differential_attention_v2_b200 import _lib
+
+    public = [n for n in dir(_lib) if not n.startswith("_") and callable(getattr(_lib, n))
+              and getattr(getattr(_lib, n), "__module__", "") == _lib.__name__ and n != "DiffAttnError"]
+    for name in public:
+        assert getattr(da, name) is getattr(_lib, name), name
+
+
+def test_prefill_train_host_checks(lib):
+    OB, LS = P + 32768, P + 40960
+    assert lib.diffattn_v2_prefill_train(Q, K, V, L, O, OB, LS, 2, 256, 7, 1, 128, 1, None) == -1  # odd Hq
+    assert lib.diffattn_v2_prefill_train(Q, K, V, L, O, None, LS, 2, 256, 8, 1, 128, 1, None) == -1  # no o_branch
+    assert lib.diffattn_v2_prefill_train(Q, K, V, L, O, OB, LS + 4, 2, 256, 8, 1, 128, 1, None) == -1  # unaligned
+    assert lib.diffattn_v2_prefill_train(Q, K, V, L, O, OB, LS, 2, 256, 8, 1, 64, 1, None) == -2  # D = 64
+    assert lib.diffattn_v2_prefill_train(Q, K, V, L, O, OB, LS, 0, 256, 8, 1, 128, 1, None) == 0   # empty
+
+
+def test_backward_host_checks(lib):
+    OB, LS, DO, DQ, DK, DV, DL, W = (P + 32768 * i for i in range(1, 9))
+    ws = lib.diffattn_v2_backward_workspace_size(2, 256, 8)
+    assert ws == 2 * 256 * 8 * 4
+    assert lib.diffattn_v2_backward_workspace_size(0, 256, 8) == 0
+    ok = (Q, K, V, L, OB, LS, DO, DQ, DK, DV, DL, 2, 256, 8, 2, 128, 1, W, ws, None)
+    assert lib.diffattn_v2_backward(*ok[:18], ws - 4, None) == -1                  # short workspace
+    assert lib.diffattn_v2_backward(*ok[:6], None, *ok[7:]) == -1                  # no dout
+    assert lib.diffattn_v2_backward(*ok[:9], DV + 8, *ok[10:]) == -1               # unaligned dv
+    assert lib.diffattn_v2_backward(*ok[:13], 6, *ok[14:]) == -1                   # pair straddles KV heads
+    assert lib.diffattn_v2_backward(*ok[:16], 2, *ok[17:]) == -1                   # causal not 0/1
+    assert lib.diffattn_v2_backward(*ok[:15], 64, *ok[16:]) == -2                  # D = 64
+    assert lib.diffattn_v2_backward(*ok[:11], 0, *ok[12:]) == 0                    # B = 0

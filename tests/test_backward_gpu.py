@@ -1,0 +1,114 @@
+"""GPU parity of the training forward and the backward pass against the float64 oracle
+(through the C ABI)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from oracle import diffattn_f64 as ora
+from tests.parity import bf16_close, grad_close, to64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def da():
+    import differential_attention_v2_b200 as m
+
+    assert torch.cuda.is_available()
+    return m
+
+
+def _case(B, S, Hq, Hkv, seed):
+    case = workloads.PrefillCase(B=B, S=S, Hq=Hq, Hkv=Hkv, D=128, seed=seed)
+    inp = workloads.make_prefill(case)
+    inp["dout"] = workloads.make_prefill_grad(case)
+    return inp
+
+
+def _gpu_grads(da, inp, causal):
+    d = {k: v.cuda() for k, v in inp.items()}
+    out, ob, lse = da.prefill_train(d["q"], d["k"], d["v"], d["lam"], causal=causal)
+    dq, dk, dv, dlam = da.backward(d["q"], d["k"], d["v"], d["lam"], ob, lse, d["dout"], causal=causal)
+    torch.cuda.synchronize()
+    assert da.device_error() == 0
+    return (out, ob, lse), (dq, dk, dv, dlam)
+
+
+def _check_grads(got, inp, causal, what):
+    ref = ora.prefill_backward(inp["q"], inp["k"], inp["v"], inp["lam"], inp["dout"], causal=causal)
+    for g, r, name in zip(got, ref, ("dq", "dk", "dv", "dlam")):
+        grad_close(g, r, f"{what} {name}")
+
+
+@pytest.mark.parametrize("B,S,Hq,Hkv,causal", [
+    (1, 128, 4, 1, True),      # one tile, group of 4
+    (2, 300, 8, 2, True),      # ragged tail (64-key and 32-row steps, 128-row forward tiles)
+    (1, 1, 2, 1, True),        # a single token
+    (1, 129, 16, 1, True),     # tile boundary + 1, group of 16
+    (1, 640, 32, 4, True),     # several tiles, group of 8
+    (2, 200, 8, 2, False),     # non-causal with ragged tiles
+    (1, 513, 4, 2, False),     # non-causal, group of 2
+])
+def test_backward_matches_oracle(da, B, S, Hq, Hkv, causal):
+    inp = _case(B, S, Hq, Hkv, seed=31 + S + Hq)
+    _, grads = _gpu_grads(da, inp, causal)
+    _check_grads(grads, inp, causal, f"B={B} S={S} Hq={Hq} Hkv={Hkv} causal={causal}")
+
+
+def test_training_forward_outputs(da):
+    """out equals the inference prefill bit for bit; O_b and lse match the oracle."""
+    inp = _case(2, 300, 8, 2, seed=41)
+    for causal in (True, False):
+        (out, ob, lse), _ = _gpu_grads(da, inp, causal)
+        d = {k: v.cuda() for k, v in inp.items()}
+        assert torch.equal(out, da.prefill(d["q"], d["k"], d["v"], d["lam"], causal=causal))
+        o_ref, lse_ref = ora.prefill_branches(inp["q"], inp["k"], inp["v"], causal=causal)
+        bf16_close(ob, o_ref, f"o_branch causal={causal}")
+        assert float(np.abs(to64(lse) - lse_ref).max()) < 1e-3, "lse"
+
+
+def test_backward_lambda_edge_values(da):
+    inp = _case(1, 200, 8, 1, seed=43)
+    g = torch.Generator().manual_seed(4)
+    inp["lam"] = (torch.rand(inp["lam"].shape, generator=g) * 4.0 - 1.5).float()
+    inp["lam"][0, :10] = 0.0
+    _, grads = _gpu_grads(da, inp, True)
+    _check_grads(grads, inp, True, "lambda in [-1.5, 2.5]")
+
+
+def test_backward_equal_branches_are_antisymmetric(da):
+    """Q1 == Q2 and lambda == 1: the two heads of a pair get exactly opposite dQ."""
+    inp = _case(1, 300, 8, 2, seed=47)
+    inp["q"][:, :, 1::2] = inp["q"][:, :, 0::2]
+    inp["lam"][:] = 1.0
+    _, (dq, dk, dv, dlam) = _gpu_grads(da, inp, True)
+    assert torch.equal(dq[:, :, 1::2], -dq[:, :, 0::2])
+
+
+def test_backward_is_deterministic(da):
+    inp = _case(2, 300, 16, 2, seed=53)
+    _, g1 = _gpu_grads(da, inp, True)
+    _, g2 = _gpu_grads(da, inp, True)
+    for a, b in zip(g1, g2):
+        assert torch.equal(a, b)
+
+
+def test_backward_full_size_one_group(da):
+    """B=4 S=4096 Hq=64 Hkv=8: gradients of one (batch, KV group) slice against the oracle on
+    that slice (dK, dV of the KV head; dQ of its 8 query heads; dlambda of its 4 pairs)."""
+    case = workloads.CONFIGS["c2_bf16_prefill"]
+    inp = workloads.make_prefill(case)
+    inp["dout"] = workloads.make_prefill_grad(case)
+    _, (dq, dk, dv, dlam) = _gpu_grads(da, inp, True)
+    b, g = 3, 5
+    G = case.Hq // case.Hkv
+    heads = slice(g * G, (g + 1) * G)
+    pairs = slice(g * G // 2, (g + 1) * G // 2)
+    sl = {"q": inp["q"][b:b + 1, :, heads], "k": inp["k"][b:b + 1, :, g:g + 1],
+          "v": inp["v"][b:b + 1, :, g:g + 1], "lam": inp["lam"][b:b + 1, :, pairs],
+          "dout": inp["dout"][b:b + 1, :, pairs]}
+    got = (dq[b:b + 1, :, heads], dk[b:b + 1, :, g:g + 1], dv[b:b + 1, :, g:g + 1], dlam[b:b + 1, :, pairs])
+    _check_grads(got, sl, True, "c2 slice b=3 g=5")

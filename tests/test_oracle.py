@@ -370,6 +370,30 @@ def pin_backward_finite_differences():
     return bool(ok)
 
 
+def pin_branches_recombine_and_normalise():
+    """O_{2p} - lam * O_{2p+1} is the prefill; 2^(s log2(e) - lse2) rows sum to one and
+    equal the library softmax (scipy) of the scaled scores."""
+    from scipy.special import softmax as sp_softmax
+    q, k, v, lam = _rand_prefill(B=2, S=9, Hq=8, Hkv=2, D=5, seed=23)
+    ok = True
+    for causal in (True, False):
+        o, lse2 = ora.prefill_branches(q, k, v, causal=causal)
+        full = ora.prefill(q, k, v, lam, causal=causal)
+        ok &= np.allclose(o[:, :, 0::2] - lam[..., None] * o[:, :, 1::2], full, atol=1e-13)
+        # head 5 reads KV head 1 (group 4)
+        s_ = q[1, :, 5] @ k[1, :, 1].T / math.sqrt(5)
+        if causal:
+            s_ = np.where(np.tril(np.ones((9, 9))) > 0, s_, -np.inf)
+        a = np.exp2(s_ * math.log2(math.e) - lse2[1, :, 5][:, None])
+        ok &= np.allclose(a.sum(axis=1), 1.0, atol=1e-13)
+        ok &= np.allclose(a, sp_softmax(s_, axis=1), atol=1e-13)
+    # the first causal row sees one key: its lse is that key's scaled score in base 2
+    o, lse2 = ora.prefill_branches(q, k, v)
+    ok &= math.isclose(lse2[0, 0, 3], float(q[0, 0, 3] @ k[0, 0, 0]) / math.sqrt(5) * math.log2(math.e),
+                       rel_tol=1e-12, abs_tol=1e-12)
+    return bool(ok)
+
+
 ALL_PINS = {
     "softmax_library": pin_softmax_library,
     "lambda0_is_softmax_attention": pin_lambda0_is_softmax_attention,
@@ -398,6 +422,7 @@ ALL_PINS = {
     "backward_matches_autograd": pin_backward_matches_autograd,
     "backward_matches_autograd_noncausal": lambda: pin_backward_matches_autograd(causal=False),
     "backward_finite_differences": pin_backward_finite_differences,
+    "branches_recombine_and_normalise": pin_branches_recombine_and_normalise,
 }
 
 

@@ -113,6 +113,49 @@ def _lambda_v2_no_sigmoid(x, w, bias=None):
     return z if bias is None else z + np.asarray(bias)[None, :]
 
 
+def _backward_variant(drop_rowsum=False, dlam_sign=-1.0, dk_first_only=False, dv_no_lambda=False,
+                      dq_unscaled=False):
+    """The chain rule of the prefill with one planted mistake (a flag set)."""
+    def fn(q, k, v, lam, dout, causal=True):
+        q, k, v, lam, dout = (np.asarray(x, dtype=np.float64) for x in (q, k, v, lam, dout))
+        B, S, Hq, D = q.shape
+        inv = 1.0 / math.sqrt(D)
+        dq, dk, dv, dlam = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v), np.zeros_like(lam)
+        mask = ora.causal_mask(S, S) if causal else np.zeros((S, S))
+        for b in range(B):
+            for p, h1, h2, g in ora.pair_layout(Hq, k.shape[2]):
+                kk, vv = k[b, :, g], v[b, :, g]
+                a1 = ora.stable_softmax(q[b, :, h1] @ kk.T * inv + mask)
+                a2 = ora.stable_softmax(q[b, :, h2] @ kk.T * inv + mask)
+                lm = lam[b, :, p][:, None]
+                do = dout[b, :, p]
+                dlam[b, :, p] = dlam_sign * np.sum(do * (a2 @ vv), axis=1)
+                dv[b, :, g] += a1.T @ do - a2.T @ ((1.0 if dv_no_lambda else lm) * do)
+                dpv = do @ vv.T
+                for a, da, h in ((a1, dpv, h1), (a2, -lm * dpv, h2)):
+                    rs = 0.0 if drop_rowsum else np.sum(a * da, axis=1, keepdims=True)
+                    ds = a * (da - rs)
+                    dq[b, :, h] = ds @ kk * (1.0 if dq_unscaled else inv)
+                    if not (dk_first_only and h == h2):
+                        dk[b, :, g] += ds.T @ q[b, :, h] * inv
+        return dq, dk, dv, dlam
+    return fn
+
+
+def _branches_natural_log(q, k, v, causal=True):
+    o, lse2 = _ORIG_BRANCHES(q, k, v, causal)
+    return o, lse2 * math.log(2.0)
+
+
+def _branches_swapped(q, k, v, causal=True):
+    o, lse2 = _ORIG_BRANCHES(q, k, v, causal)
+    o2 = o.copy()
+    o2[:, :, 0::2], o2[:, :, 1::2] = o[:, :, 1::2], o[:, :, 0::2]
+    return o2, lse2
+
+
+_ORIG_BRANCHES = ora.prefill_branches
+
 MUTANTS = {
     "plus_sign": ("diff_attention_block", _block_plus_sign),
     "no_scale": ("diff_attention_block", _block_no_scale),
@@ -130,6 +173,13 @@ MUTANTS = {
     "lambda_v1_plus": ("lambda_v1", _lambda_v1_plus),
     "window_off_by_one": ("window_mask", _window_off_by_one),
     "lambda_v2_no_sigmoid": ("lambda_v2_projection", _lambda_v2_no_sigmoid),
+    "backward_no_softmax_rowsum": ("prefill_backward", _backward_variant(drop_rowsum=True)),
+    "backward_dlambda_sign": ("prefill_backward", _backward_variant(dlam_sign=1.0)),
+    "backward_dk_first_branch_only": ("prefill_backward", _backward_variant(dk_first_only=True)),
+    "backward_dv_without_lambda": ("prefill_backward", _backward_variant(dv_no_lambda=True)),
+    "backward_dq_unscaled": ("prefill_backward", _backward_variant(dq_unscaled=True)),
+    "branches_lse_natural_log": ("prefill_branches", _branches_natural_log),
+    "branches_heads_swapped": ("prefill_branches", _branches_swapped),
 }
 
 

@@ -118,6 +118,13 @@ def make_prefill(case: PrefillCase):
     return {"q": q, "k": k, "v": v, "lam": lam}
 
 
+def make_prefill_grad(case: PrefillCase):
+    """Upstream gradient dL/d(out) for a prefill case: standard normal, shape [B,S,Hq/2,D],
+    in the case's dtype, from its own seeded stream (seed + 7919)."""
+    gen = _gen(case.seed + 7919)
+    return _randn((case.B, case.S, case.Hq // 2, case.D), gen, _DT[case.dtype])
+
+
 def plant_signal_row(inp, b=0, row=None, pair=0, signal_key=7, logit_gain=4.0, seed=77):
     """Plant the signal-plus-shared-noise query row of the lesson's noise-cancellation toy.
 
