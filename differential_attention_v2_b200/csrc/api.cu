@@ -224,8 +224,8 @@ int diffattn_v2_prefill_train(const void* q, const void* k, const void* v, const
 }
 
 size_t diffattn_v2_backward_workspace_size(int B, int S, int Hq) {
-  if (B <= 0 || S <= 0 || Hq <= 0) return 0;
-  return static_cast<size_t>(B) * S * Hq * sizeof(float);
+  if (B <= 0 || S <= 0 || Hq <= 0 || (Hq % 2) != 0) return 0;
+  return da2::backward_stats_bytes(B, S, Hq);
 }
 
 int diffattn_v2_backward(const void* q, const void* k, const void* v, const float* lambda, const void* o_branch,
@@ -240,15 +240,23 @@ int diffattn_v2_backward(const void* q, const void* k, const void* v, const floa
     if (!ptr || !aligned16(ptr)) return DA2_ERR_INVALID;
   if (workspace_bytes < diffattn_v2_backward_workspace_size(B, S, Hq)) return DA2_ERR_INVALID;
   if (D != 128) return DA2_ERR_UNSUPPORTED;
-  // grid limits: heads and batch on grid y / z; the preprocess runs 4 (token, pair) warps per CTA
-  if (B > 65535 || Hq > 65535) return DA2_ERR_UNSUPPORTED;
-  if (static_cast<long long>(B) * S * (Hq / 2) > 4LL * 2147483647LL) return DA2_ERR_UNSUPPORTED;
+  // grid limits: 128-row tiles on grid y; the preprocess runs 4 (token, pair) warps per CTA
+  if ((S + 127) / 128 > 65535) return DA2_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * ((S + 127) / 128 * 128) * (Hq / 2) > 4LL * 2147483647LL) return DA2_ERR_UNSUPPORTED;
+  int* err = nullptr;
+  if (device_error_ptr(&err) != cudaSuccess) return DA2_ERR_CUDA;
+  CUtensorMap q64, q128, o64, o128, k64, k128, v64, v128;
+  if (encode_bshd(&q64, q, D, Hq, S, B, 64, 64) != cudaSuccess || encode_bshd(&q128, q, D, Hq, S, B, 64, 128) != cudaSuccess ||
+      encode_bshd(&o64, dout, D, Hq / 2, S, B, 64, 64) != cudaSuccess ||
+      encode_bshd(&o128, dout, D, Hq / 2, S, B, 64, 128) != cudaSuccess ||
+      encode_bshd(&k64, k, D, Hkv, S, B, 64, 64) != cudaSuccess || encode_bshd(&k128, k, D, Hkv, S, B, 64, 128) != cudaSuccess ||
+      encode_bshd(&v64, v, D, Hkv, S, B, 64, 64) != cudaSuccess || encode_bshd(&v128, v, D, Hkv, S, B, 64, 128) != cudaSuccess)
+    return DA2_ERR_CUDA;
   using bf = __nv_bfloat16;
-  return status_of(da2::launch_backward(
-      static_cast<const bf*>(q), static_cast<const bf*>(k), static_cast<const bf*>(v), lambda,
-      static_cast<const bf*>(o_branch), lse, static_cast<const bf*>(dout), static_cast<bf*>(dq), static_cast<bf*>(dk),
-      static_cast<bf*>(dv), dlambda, static_cast<float*>(workspace), B, S, Hq, Hkv, causal,
-      reinterpret_cast<cudaStream_t>(stream)));
+  return status_of(da2::launch_backward_sm100(
+      q64, q128, o64, o128, k64, k128, v64, v128, lambda, static_cast<const bf*>(o_branch), lse,
+      static_cast<const bf*>(dout), static_cast<bf*>(dq), static_cast<bf*>(dk), static_cast<bf*>(dv), dlambda,
+      static_cast<float*>(workspace), err, B, S, Hq, Hkv, causal, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 size_t diffattn_v2_decode_workspace_size(int B, int Smax, int Hq, int Hkv, int D) {

@@ -1,0 +1,578 @@
+// backward_sm100.cu -- gradients of the bf16 DiffAttn V2 prefill on the 5th-generation tensor
+// cores (sm_100a).
+//
+// Chain rule of out = A_1 V - lambda A_2 V, A_b = softmax(Q_b K^T / sqrt(D)) ("Differential
+// Attention (V2)" lesson, "The differential concept"; causal mask of the "Attention variants"
+// lesson), per pair of heads (2p, 2p+1) over KV head g, with dO the upstream gradient:
+//   dP   = dO V^T                       (one product per pair: both branches read dO and V)
+//   W    = A_1 - lambda A_2             (the combined weights, rounded to bf16 once)
+//   dS_1 = A_1 (dP - E_1),  dS_2 = -lambda A_2 (dP - E_2),   E_b = dO . O_b per row
+//   dV  += W^T dO,   dK += (dS_1^T Q_1 + dS_2^T Q_2) / sqrt(D),   dQ_b = dS_b K / sqrt(D)
+//   dlambda = -dO . O_2
+// A_b is recomputed from the forward's base-2 row log-sum-exp: A_b = 2^(s log2(e)/sqrt(D) - lse_b).
+//
+// Three launches, no atomics (the result is deterministic):
+//   preprocess   one warp per (token, pair): E_1, E_2, dlambda, and a 32-byte record
+//                {lse_1, lse_2, E_1, E_2, lambda} per (pair, row) that the other kernels
+//                stream; rows past S (to a multiple of 128) get lse = +inf so their
+//                probabilities are exactly 0 without per-element row checks
+//   dkdv_sm100   a CTA owns 128 keys of one KV head (the TMEM lanes) and walks every pair of
+//                the group and every 64-row query block that sees the keys
+//   dq_sm100     a CTA owns 128 query rows of one pair (the TMEM lanes) and walks the 64-key
+//                blocks they see
+// Both tile kernels have the forward prefill's shape: a TMA producer warp, an MMA warp (one
+// thread issues tcgen05.mma), 8 elementwise warps that read fp32 scores from TMEM and write
+// bf16 operands back over them. A step's scores are produced in two 32-column halves so that
+// the elementwise work on one half overlaps the MMAs of the other.
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace da2 {
+namespace bwd_tc {
+
+constexpr int HD = 128;
+constexpr int kThreads = 320;
+constexpr int kStages = 2;
+constexpr int kStatFloats = 8;                 // {lse1, lse2, E1, E2, lambda, 0, 0, 0}
+constexpr int kRowPad = 128;                   // stats rows padded to a multiple of this
+
+constexpr uint32_t kIdescS = idesc_bf16_f32(128, 32, false);   // scores: N = 32 columns per half
+constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, 128, true);  // accumulators: B MN-major, N = d
+
+// TMEM columns
+constexpr uint32_t kTmS1 = 0, kTmS2 = 64, kTmDP = 128, kTmAcc0 = 256, kTmAcc1 = 384;
+
+// K-major SW128 operand of R rows: K-step kk (16 of d) -> chunk kk/4, +32 bytes per 16 elements
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, uint32_t chunk_bytes, int kk) {
+  return sdesc_sw128(base + (kk >> 2) * chunk_bytes + (kk & 3) * 32, 16, 1024);
+}
+// MN-major SW128 B operand (rows = reduction dim, d = N): K-step of 16 rows from `row`
+__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t base, uint32_t chunk_bytes, int row) {
+  return sdesc_sw128(base + row * 128, chunk_bytes, 1024);
+}
+
+struct Params {
+  const float* stats;        // [B, Hq/2, S_pad, 8]
+  __nv_bfloat16* dq;         // [B,S,Hq,D]
+  __nv_bfloat16* dk;         // [B,S,Hkv,D]
+  __nv_bfloat16* dv;
+  int* err;
+  int B, S, S_pad, Hq, Hkv, causal;
+  int n_tiles;               // 128-row tiles
+  float scale, scale_log2;
+};
+
+// ------------------------------------------------------------------------ preprocess
+__global__ void __launch_bounds__(128)
+preprocess_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ o_branch,
+                  const float* __restrict__ lse, const float* __restrict__ lambda, float* __restrict__ stats,
+                  float* __restrict__ dlam, int B, int S, int S_pad, int n_pairs) {
+  const long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= static_cast<long long>(B) * S_pad * n_pairs) return;
+  // warp w: row i of pair p of batch b, rows fastest (records of a pair are contiguous)
+  const int i = static_cast<int>(w % S_pad);
+  const long long bp = w / S_pad;
+  const int p = static_cast<int>(bp % n_pairs);
+  const int b = static_cast<int>(bp / n_pairs);
+  float* rec = stats + w * kStatFloats;
+  if (i >= S) {
+    if (lane < kStatFloats) rec[lane] = lane < 2 ? INFINITY : 0.f;
+    return;
+  }
+  const long long row = static_cast<long long>(b) * S + i;
+  const uint2 g = __ldg(reinterpret_cast<const uint2*>(dout + (row * n_pairs + p) * HD) + lane);
+  const float2 g0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&g.x));
+  const float2 g1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&g.y));
+  float e[2];
+#pragma unroll
+  for (int br = 0; br < 2; ++br) {
+    const uint2 o = __ldg(reinterpret_cast<const uint2*>(o_branch + (row * (2 * n_pairs) + 2 * p + br) * HD) + lane);
+    const float2 o0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o.x));
+    const float2 o1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o.y));
+    float v = g0.x * o0.x + g0.y * o0.y + g1.x * o1.x + g1.y * o1.y;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    e[br] = v;
+  }
+  if (lane == 0) {
+    const float l1 = __ldg(lse + row * (2 * n_pairs) + 2 * p);
+    const float l2 = __ldg(lse + row * (2 * n_pairs) + 2 * p + 1);
+    const float lam = __ldg(lambda + row * n_pairs + p);
+    reinterpret_cast<float4*>(rec)[0] = make_float4(l1, l2, e[0], e[1]);
+    reinterpret_cast<float4*>(rec)[1] = make_float4(lam, 0.f, 0.f, 0.f);
+    dlam[row * n_pairs + p] = -e[1];
+  }
+}
+
+// Shared-memory layouts (byte offsets from a 1024-aligned base). Both tile kernels hold
+// three "fixed" tiles of 128 rows and stream 64-row tiles through a 2-stage ring.
+constexpr uint32_t kFixedTile = 128 * 256;     // 128 rows x 128 bf16
+constexpr uint32_t kFixedChunk = 128 * 128;    // one 64-wide d half of it
+constexpr uint32_t kStreamTile = 64 * 256;     // 64 rows x 128 bf16
+constexpr uint32_t kStreamChunk = 64 * 128;
+constexpr uint32_t kStatBytes = 64 * kStatFloats * 4;
+
+// mbarriers
+enum Bar : int {
+  kFixedFull = 0,
+  kXFull = 1,    // +stage
+  kXEmpty = 3,   // +stage
+  kSFull = 5,    // +half
+  kPReady = 7,   // +half
+  kDFull = 9,
+  kDrain = 10,
+  kNumBars = 11
+};
+
+// dK/dV: fixed K, V (128 keys); stream Q1, Q2, dO (64 query rows) + their 64 stat records
+constexpr uint32_t kKvOffK = 0;
+constexpr uint32_t kKvOffV = kFixedTile;
+constexpr uint32_t kKvOffX = 2 * kFixedTile;
+constexpr uint32_t kKvStage = 3 * kStreamTile + kStatBytes;
+constexpr uint32_t kKvOffBar = kKvOffX + kStages * kKvStage;
+constexpr uint32_t kKvSmem = kKvOffBar + 256 + 1024;
+
+// dQ: fixed Q1, Q2, dO (128 query rows); stream K, V (64 keys)
+constexpr uint32_t kQOffQ1 = 0;
+constexpr uint32_t kQOffQ2 = kFixedTile;
+constexpr uint32_t kQOffO = 2 * kFixedTile;
+constexpr uint32_t kQOffX = 3 * kFixedTile;
+constexpr uint32_t kQStage = 2 * kStreamTile;
+constexpr uint32_t kQOffBar = kQOffX + kStages * kQStage;
+constexpr uint32_t kQSmem = kQOffBar + 256 + 1024;
+
+__device__ __forceinline__ void tmem_ld_x32_wait(uint32_t taddr, uint32_t (&r)[32]) {
+  tmem_ld_32x32b_x32(taddr, r);
+  tmem_ld_wait(r);
+}
+
+// Common set-up: barriers, TMEM (512 columns, by warp 9). Returns the TMEM base.
+__device__ __forceinline__ uint32_t setup(uint32_t bar0, uint32_t* tmem_slot, volatile int* abort_flag, int warp) {
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kNumBars; ++i) {
+      const uint32_t count = (i == kPReady || i == kPReady + 1) ? 128u : 1u;
+      mbar_init(bar0 + 8u * i, count);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  return *tmem_slot;
+}
+
+__device__ __forceinline__ void teardown(uint32_t tmem, const volatile int* abort_flag, int* err, int warp) {
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) atomicCAS(err, 0, kErrBackwardWait);
+  if (warp == 9) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// Write 64 fp32 accumulator columns of this thread's row (TMEM) as bf16, times `mul`.
+__device__ __forceinline__ void store_row64(uint32_t taddr, __nv_bfloat16* dst, float mul, bool valid) {
+#pragma unroll 1
+  for (int c = 0; c < 2; ++c) {
+    uint32_t a[32];
+    tmem_ld_x32_wait(taddr + 32 * c, a);
+    if (valid) {
+      uint4* d = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+      for (int v = 0; v < 4; ++v)
+        d[v] = make_uint4(pack_bf16x2(__uint_as_float(a[8 * v + 0]) * mul, __uint_as_float(a[8 * v + 1]) * mul),
+                          pack_bf16x2(__uint_as_float(a[8 * v + 2]) * mul, __uint_as_float(a[8 * v + 3]) * mul),
+                          pack_bf16x2(__uint_as_float(a[8 * v + 4]) * mul, __uint_as_float(a[8 * v + 5]) * mul),
+                          pack_bf16x2(__uint_as_float(a[8 * v + 6]) * mul, __uint_as_float(a[8 * v + 7]) * mul));
+    }
+  }
+}
+
+// --------------------------------------------------------------------------- dK / dV
+__global__ void __launch_bounds__(kThreads, 1)
+dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+           const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + kKvOffBar;
+  auto bar = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kKvOffBar + 128);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kKvOffBar + 136);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_pairs = p.Hq >> 1, group = p.Hq / p.Hkv, gpairs = group >> 1;
+  const int g = static_cast<int>(blockIdx.x) % p.Hkv;
+  const int b = static_cast<int>(blockIdx.x) / p.Hkv;
+  const int tile = static_cast<int>(blockIdx.y);  // tile 0 (most query blocks when causal) first
+  const int k0 = tile * 128;
+  const int nq = (p.S + 63) / 64;                   // 64-row query blocks
+  const int q_first = p.causal ? k0 / 64 : 0;
+  const int steps_per_pair = nq - q_first;
+  const int n_steps = gpairs * steps_per_pair;
+
+  const uint32_t tmem = setup(bar0, tmem_slot, abort_flag, warp);
+
+  if (warp == 8) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmO);
+      mbar_arrive_expect_tx(bar(kFixedFull), 2 * kFixedTile);
+      for (int c = 0; c < 2; ++c) {
+        tma_load_4d(sbase + kKvOffK + c * kFixedChunk, &tmK, bar(kFixedFull), c * 64, g, k0, b);
+        tma_load_4d(sbase + kKvOffV + c * kFixedChunk, &tmV, bar(kFixedFull), c * 64, g, k0, b);
+      }
+      int issued = 0;
+      for (int t = 0; t < n_steps; ++t) {
+        const int s = t & 1;
+        if (!mbar_wait(bar(kXEmpty + s), ((t >> 1) & 1) ^ 1, abort_flag)) break;
+        const int pair = g * gpairs + t / steps_per_pair;
+        const int q0 = (q_first + t % steps_per_pair) * 64;
+        const uint32_t st = sbase + kKvOffX + s * kKvStage;
+        mbar_arrive_expect_tx(bar(kXFull + s), 3 * kStreamTile + kStatBytes);
+        for (int c = 0; c < 2; ++c) {
+          tma_load_4d(st + c * kStreamChunk, &tmQ, bar(kXFull + s), c * 64, 2 * pair, q0, b);
+          tma_load_4d(st + kStreamTile + c * kStreamChunk, &tmQ, bar(kXFull + s), c * 64, 2 * pair + 1, q0, b);
+          tma_load_4d(st + 2 * kStreamTile + c * kStreamChunk, &tmO, bar(kXFull + s), c * 64, pair, q0, b);
+        }
+        bulk_load(st + 3 * kStreamTile,
+                  p.stats + ((static_cast<size_t>(b) * n_pairs + pair) * p.S_pad + q0) * kStatFloats, kStatBytes,
+                  bar(kXFull + s));
+        issued = t + 1;
+      }
+      if (*abort_flag) {
+        volatile int no_abort = 0;
+        mbar_wait(bar(kFixedFull), 0, &no_abort);
+        for (int t = max(0, issued - kStages); t < issued; ++t) mbar_wait(bar(kXFull + (t & 1)), (t >> 1) & 1, &no_abort);
+      }
+    }
+  } else if (warp == 9) {
+    // -------------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(bar(kFixedFull), 0, abort_flag);
+      for (int t = 0; ok && t < n_steps; ++t) {
+        const int s = t & 1;
+        if (!(ok = mbar_wait(bar(kXFull + s), (t >> 1) & 1, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t st = sbase + kKvOffX + s * kKvStage;
+        const uint32_t sQ1 = st, sQ2 = st + kStreamTile, sO = st + 2 * kStreamTile;
+        // S_1^T = K Q_1^T, S_2^T = K Q_2^T, dP^T = V dO^T; queries 32h .. 32h+31 per half
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint64_t a_k = desc_kmajor(sbase + kKvOffK, kFixedChunk, kk);
+            const uint64_t a_v = desc_kmajor(sbase + kKvOffV, kFixedChunk, kk);
+            const uint32_t acc = kk > 0 ? 1u : 0u;
+            mma_bf16_ss(tmem + kTmS1 + 32 * h, a_k, desc_kmajor(sQ1 + h * 4096, kStreamChunk, kk), kIdescS, acc);
+            mma_bf16_ss(tmem + kTmS2 + 32 * h, a_k, desc_kmajor(sQ2 + h * 4096, kStreamChunk, kk), kIdescS, acc);
+            mma_bf16_ss(tmem + kTmDP + 32 * h, a_v, desc_kmajor(sO + h * 4096, kStreamChunk, kk), kIdescS, acc);
+          }
+          tc_commit(bar(kSFull + h));
+        }
+        // dV += W^T dO, dK += dS_1^T Q_1 + dS_2^T Q_2 (bf16 operands written over the scores)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (!(ok = mbar_wait(bar(kPReady + h), t & 1, abort_flag))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int k2 = 0; k2 < 2; ++k2) {
+            const int row = 32 * h + 16 * k2;
+            const uint32_t first = (t == 0 && h == 0 && k2 == 0) ? 0u : 1u;
+            mma_bf16_ts(tmem + kTmAcc0, tmem + kTmS1 + 32 * h + 8 * k2, desc_mnmajor(sO, kStreamChunk, row), kIdescAcc,
+                        first);
+            mma_bf16_ts(tmem + kTmAcc1, tmem + kTmS2 + 32 * h + 8 * k2, desc_mnmajor(sQ1, kStreamChunk, row),
+                        kIdescAcc, first);
+            mma_bf16_ts(tmem + kTmAcc1, tmem + kTmDP + 32 * h + 8 * k2, desc_mnmajor(sQ2, kStreamChunk, row),
+                        kIdescAcc, 1u);
+          }
+        }
+        if (!ok) break;
+        tc_commit(bar(kXEmpty + s));
+      }
+      if (ok) tc_commit(bar(kDFull));
+      tc_commit(bar(kDrain));
+      volatile int no_abort = 0;
+      mbar_wait(bar(kDrain), 0, &no_abort);
+    }
+  } else {
+    // ------------------------------------------------------------------ elementwise
+    const int hc = warp >> 2;                 // query half of each step
+    const int r = 32 * (warp & 3) + lane;     // key row of the tile == TMEM lane
+    const int key = k0 + r;
+    const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    bool ok = true;
+    for (int t = 0; t < n_steps; ++t) {
+      const int s = t & 1;
+      const int q0 = (q_first + t % steps_per_pair) * 64;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(kSFull + hc), t & 1, abort_flag));
+      // the stage's stat records came by bulk copy: observe its completion directly (the
+      // stage is refilled only after this step's operands have been consumed)
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(kXFull + s), (t >> 1) & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t s1[32], s2[32], dp[32];
+      tmem_ld_32x32b_x32(trow + kTmS1 + 32 * hc, s1);
+      tmem_ld_32x32b_x32(trow + kTmS2 + 32 * hc, s2);
+      tmem_ld_32x32b_x32(trow + kTmDP + 32 * hc, dp);
+      tmem_ld_wait(s1);
+      reg_fence(s2);
+      reg_fence(dp);
+      const float4* rec = reinterpret_cast<const float4*>(smem + kKvOffX + s * kKvStage + 3 * kStreamTile) + 2 * (32 * hc);
+      // causal: only the two query blocks that overlap the key tile hold keys past a query
+      const bool diag = p.causal && q0 < k0 + 128;
+      const int qbase = q0 + 32 * hc;
+      uint32_t w_pk[16], d1_pk[16], d2_pk[16];
+#pragma unroll
+      for (int c = 0; c < 32; c += 2) {
+        float w[2], d1[2], d2[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float4 ra = rec[2 * (c + e)];
+          const float lam = rec[2 * (c + e) + 1].x;
+          float p1 = fast_exp2(__uint_as_float(s1[c + e]) * p.scale_log2 - ra.x);
+          float p2 = fast_exp2(__uint_as_float(s2[c + e]) * p.scale_log2 - ra.y);
+          if (diag && key > qbase + c + e) p1 = p2 = 0.f;
+          const float dpv = __uint_as_float(dp[c + e]);
+          w[e] = __fmaf_rn(-lam, p2, p1);
+          d1[e] = p1 * (dpv - ra.z);
+          d2[e] = -lam * p2 * (dpv - ra.w);
+        }
+        w_pk[c >> 1] = pack_bf16x2(w[0], w[1]);
+        d1_pk[c >> 1] = pack_bf16x2(d1[0], d1[1]);
+        d2_pk[c >> 1] = pack_bf16x2(d2[0], d2[1]);
+      }
+      tmem_st_32x32b_x16(trow + kTmS1 + 32 * hc, w_pk);
+      tmem_st_32x32b_x16(trow + kTmS2 + 32 * hc, d1_pk);
+      tmem_st_32x32b_x16(trow + kTmDP + 32 * hc, d2_pk);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(kPReady + hc));
+    }
+    if (ok) ok = mbar_wait(bar(kDFull), 0, abort_flag);
+    if (__all_sync(0xffffffffu, ok && !*abort_flag)) {
+      tc_fence_after();
+      const bool valid = key < p.S;
+      const size_t off = ((static_cast<size_t>(b) * p.S + (valid ? key : 0)) * p.Hkv + g) * HD + 64 * hc;
+      store_row64(trow + kTmAcc0 + 64 * hc, p.dv + off, 1.f, valid);
+      store_row64(trow + kTmAcc1 + 64 * hc, p.dk + off, p.scale, valid);
+    }
+  }
+  teardown(tmem, abort_flag, p.err, warp);
+}
+
+// --------------------------------------------------------------------------------- dQ
+__global__ void __launch_bounds__(kThreads, 1)
+dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+         const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + kQOffBar;
+  auto bar = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kQOffBar + 128);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kQOffBar + 136);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_pairs = p.Hq >> 1, group = p.Hq / p.Hkv;
+  const int pair = static_cast<int>(blockIdx.x) % n_pairs;
+  const int b = static_cast<int>(blockIdx.x) / n_pairs;
+  const int g = (2 * pair) / group;
+  const int tile = p.causal ? p.n_tiles - 1 - static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.y);
+  const int m0 = tile * 128;
+  const int nk = (p.S + 63) / 64;
+  const int n_steps = p.causal ? min(nk, (m0 + 128) / 64) : nk;
+
+  const uint32_t tmem = setup(bar0, tmem_slot, abort_flag, warp);
+
+  if (warp == 8) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      mbar_arrive_expect_tx(bar(kFixedFull), 3 * kFixedTile);
+      for (int c = 0; c < 2; ++c) {
+        tma_load_4d(sbase + kQOffQ1 + c * kFixedChunk, &tmQ, bar(kFixedFull), c * 64, 2 * pair, m0, b);
+        tma_load_4d(sbase + kQOffQ2 + c * kFixedChunk, &tmQ, bar(kFixedFull), c * 64, 2 * pair + 1, m0, b);
+        tma_load_4d(sbase + kQOffO + c * kFixedChunk, &tmO, bar(kFixedFull), c * 64, pair, m0, b);
+      }
+      int issued = 0;
+      for (int t = 0; t < n_steps; ++t) {
+        const int s = t & 1;
+        if (!mbar_wait(bar(kXEmpty + s), ((t >> 1) & 1) ^ 1, abort_flag)) break;
+        const uint32_t st = sbase + kQOffX + s * kQStage;
+        mbar_arrive_expect_tx(bar(kXFull + s), 2 * kStreamTile);
+        for (int c = 0; c < 2; ++c) {
+          tma_load_4d(st + c * kStreamChunk, &tmK, bar(kXFull + s), c * 64, g, 64 * t, b);
+          tma_load_4d(st + kStreamTile + c * kStreamChunk, &tmV, bar(kXFull + s), c * 64, g, 64 * t, b);
+        }
+        issued = t + 1;
+      }
+      if (*abort_flag) {
+        volatile int no_abort = 0;
+        mbar_wait(bar(kFixedFull), 0, &no_abort);
+        for (int t = max(0, issued - kStages); t < issued; ++t) mbar_wait(bar(kXFull + (t & 1)), (t >> 1) & 1, &no_abort);
+      }
+    }
+  } else if (warp == 9) {
+    if (lane == 0) {
+      bool ok = mbar_wait(bar(kFixedFull), 0, abort_flag);
+      for (int t = 0; ok && t < n_steps; ++t) {
+        const int s = t & 1;
+        if (!(ok = mbar_wait(bar(kXFull + s), (t >> 1) & 1, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t sK = sbase + kQOffX + s * kQStage, sV = sK + kStreamTile;
+        // S_1 = Q_1 K^T, S_2 = Q_2 K^T, dP = dO V^T; keys 32h .. 32h+31 per half
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint64_t b_k = desc_kmajor(sK + h * 4096, kStreamChunk, kk);
+            const uint32_t acc = kk > 0 ? 1u : 0u;
+            mma_bf16_ss(tmem + kTmS1 + 32 * h, desc_kmajor(sbase + kQOffQ1, kFixedChunk, kk), b_k, kIdescS, acc);
+            mma_bf16_ss(tmem + kTmS2 + 32 * h, desc_kmajor(sbase + kQOffQ2, kFixedChunk, kk), b_k, kIdescS, acc);
+            mma_bf16_ss(tmem + kTmDP + 32 * h, desc_kmajor(sbase + kQOffO, kFixedChunk, kk),
+                        desc_kmajor(sV + h * 4096, kStreamChunk, kk), kIdescS, acc);
+          }
+          tc_commit(bar(kSFull + h));
+        }
+        // dQ_1 += dS_1 K, dQ_2 += dS_2 K
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (!(ok = mbar_wait(bar(kPReady + h), t & 1, abort_flag))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int k2 = 0; k2 < 2; ++k2) {
+            const int row = 32 * h + 16 * k2;
+            const uint32_t first = (t == 0 && h == 0 && k2 == 0) ? 0u : 1u;
+            const uint64_t b_k = desc_mnmajor(sK, kStreamChunk, row);
+            mma_bf16_ts(tmem + kTmAcc0, tmem + kTmS1 + 32 * h + 8 * k2, b_k, kIdescAcc, first);
+            mma_bf16_ts(tmem + kTmAcc1, tmem + kTmS2 + 32 * h + 8 * k2, b_k, kIdescAcc, first);
+          }
+        }
+        if (!ok) break;
+        tc_commit(bar(kXEmpty + s));
+      }
+      if (ok) tc_commit(bar(kDFull));
+      tc_commit(bar(kDrain));
+      volatile int no_abort = 0;
+      mbar_wait(bar(kDrain), 0, &no_abort);
+    }
+  } else {
+    const int hc = warp >> 2;                 // key half of each step
+    const int r = 32 * (warp & 3) + lane;     // query row of the tile == TMEM lane
+    const int qi = m0 + r;
+    const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    // this row's record (rows past S carry lse = +inf: probabilities 0)
+    const float4* rec =
+        reinterpret_cast<const float4*>(p.stats + ((static_cast<size_t>(b) * n_pairs + pair) * p.S_pad + qi) * kStatFloats);
+    const float4 ra = __ldg(rec);
+    const float lam = __ldg(rec + 1).x;
+    bool ok = true;
+    for (int t = 0; t < n_steps; ++t) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(kSFull + hc), t & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t s1[32], s2[32], dp[32];
+      tmem_ld_32x32b_x32(trow + kTmS1 + 32 * hc, s1);
+      tmem_ld_32x32b_x32(trow + kTmS2 + 32 * hc, s2);
+      tmem_ld_32x32b_x32(trow + kTmDP + 32 * hc, dp);
+      tmem_ld_wait(s1);
+      reg_fence(s2);
+      reg_fence(dp);
+      const int kbase = 64 * t + 32 * hc;
+      // tile-uniform: keys past the query (causal diagonal) or past S (ragged last block)
+      const bool masked = (p.causal && 64 * t + 63 > m0) || (64 * t + 64 > p.S);
+      const int lim = p.causal ? min(qi, p.S - 1) : p.S - 1;
+      uint32_t d1_pk[16], d2_pk[16];
+#pragma unroll
+      for (int c = 0; c < 32; c += 2) {
+        float d1[2], d2[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          float p1 = fast_exp2(__uint_as_float(s1[c + e]) * p.scale_log2 - ra.x);
+          float p2 = fast_exp2(__uint_as_float(s2[c + e]) * p.scale_log2 - ra.y);
+          if (masked && kbase + c + e > lim) p1 = p2 = 0.f;
+          const float dpv = __uint_as_float(dp[c + e]);
+          d1[e] = p1 * (dpv - ra.z);
+          d2[e] = -lam * p2 * (dpv - ra.w);
+        }
+        d1_pk[c >> 1] = pack_bf16x2(d1[0], d1[1]);
+        d2_pk[c >> 1] = pack_bf16x2(d2[0], d2[1]);
+      }
+      tmem_st_32x32b_x16(trow + kTmS1 + 32 * hc, d1_pk);
+      tmem_st_32x32b_x16(trow + kTmS2 + 32 * hc, d2_pk);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(kPReady + hc));
+    }
+    if (ok) ok = mbar_wait(bar(kDFull), 0, abort_flag);
+    if (__all_sync(0xffffffffu, ok && !*abort_flag)) {
+      tc_fence_after();
+      const bool valid = qi < p.S;
+      const size_t off = ((static_cast<size_t>(b) * p.S + (valid ? qi : 0)) * p.Hq + 2 * pair) * HD + 64 * hc;
+      store_row64(trow + kTmAcc0 + 64 * hc, p.dq + off, p.scale, valid);
+      store_row64(trow + kTmAcc1 + 64 * hc, p.dq + off + HD, p.scale, valid);
+    }
+  }
+  teardown(tmem, abort_flag, p.err, warp);
+}
+
+}  // namespace bwd_tc
+
+size_t backward_stats_bytes(int B, int S, int Hq) {
+  const size_t s_pad = (static_cast<size_t>(S) + bwd_tc::kRowPad - 1) / bwd_tc::kRowPad * bwd_tc::kRowPad;
+  return static_cast<size_t>(B) * (Hq / 2) * s_pad * bwd_tc::kStatFloats * sizeof(float);
+}
+
+cudaError_t launch_backward_sm100(const CUtensorMap& tmQ64, const CUtensorMap& tmQ128, const CUtensorMap& tmO64,
+                                  const CUtensorMap& tmO128, const CUtensorMap& tmK64, const CUtensorMap& tmK128,
+                                  const CUtensorMap& tmV64, const CUtensorMap& tmV128, const float* lambda,
+                                  const __nv_bfloat16* o_branch, const float* lse, const __nv_bfloat16* dout,
+                                  __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv, float* dlambda,
+                                  float* stats, int* err, int B, int S, int Hq, int Hkv, int causal,
+                                  cudaStream_t stream) {
+  using namespace bwd_tc;
+  const int n_pairs = Hq / 2;
+  const int S_pad = (S + kRowPad - 1) / kRowPad * kRowPad;
+  const long long warps = static_cast<long long>(B) * S_pad * n_pairs;
+  preprocess_kernel<<<static_cast<unsigned>((warps + 3) / 4), 128, 0, stream>>>(dout, o_branch, lse, lambda, stats,
+                                                                                  dlambda, B, S, S_pad, n_pairs);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  Params p;
+  p.stats = stats;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.err = err;
+  p.B = B;
+  p.S = S;
+  p.S_pad = S_pad;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.causal = causal;
+  p.n_tiles = S_pad / 128;
+  p.scale = 1.f / sqrtf(static_cast<float>(HD));
+  p.scale_log2 = 1.4426950408889634f * p.scale;
+  e = cudaFuncSetAttribute(dkdv_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(dq_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmem);
+  if (e != cudaSuccess) return e;
+  dkdv_sm100<<<dim3(B * Hkv, p.n_tiles), kThreads, kKvSmem, stream>>>(tmQ64, tmO64, tmK128, tmV128, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  dq_sm100<<<dim3(B * n_pairs, p.n_tiles), kThreads, kQSmem, stream>>>(tmQ128, tmO128, tmK64, tmV64, p);
+  return cudaGetLastError();
+}
+
+}  // namespace da2

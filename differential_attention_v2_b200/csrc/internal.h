@@ -18,13 +18,17 @@ cudaError_t launch_prefill(const CUtensorMap& tmQ, const CUtensorMap& tmK, const
                            int causal, int window, const int* cu_seqlens, cudaStream_t stream,
                            __nv_bfloat16* o_branch = nullptr, float* lse = nullptr);
 
-// Backward of the bf16 [B,S] prefill (D = 128): preprocess (E, dlambda), dK/dV, dQ. o_branch
-// [B,S,Hq,D] and lse [B,S,Hq] come from the training forward; E is fp32 [B,S,Hq] scratch.
-cudaError_t launch_backward(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
-                            const float* lambda, const __nv_bfloat16* o_branch, const float* lse,
-                            const __nv_bfloat16* dout, __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv,
-                            float* dlambda, float* E, int B, int S, int Hq, int Hkv, int causal,
-                            cudaStream_t stream);
+// tcgen05 backward of the bf16 [B,S] prefill (D = 128): preprocess into `stats`
+// (backward_stats_bytes), then the dK/dV and dQ tile kernels. Tensor maps over q [B,S,Hq,D],
+// dout [B,S,Hq/2,D], k and v [B,S,Hkv,D] with 64- and 128-row boxes (64 d x 1 head).
+size_t backward_stats_bytes(int B, int S, int Hq);
+cudaError_t launch_backward_sm100(const CUtensorMap& tmQ64, const CUtensorMap& tmQ128, const CUtensorMap& tmO64,
+                                  const CUtensorMap& tmO128, const CUtensorMap& tmK64, const CUtensorMap& tmK128,
+                                  const CUtensorMap& tmV64, const CUtensorMap& tmV128, const float* lambda,
+                                  const __nv_bfloat16* o_branch, const float* lse, const __nv_bfloat16* dout,
+                                  __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv, float* dlambda,
+                                  float* stats, int* err, int B, int S, int Hq, int Hkv, int causal,
+                                  cudaStream_t stream);
 
 // bf16 decode (D = 128): split kernel + combine. Tensor maps over the caches [B,Smax,Hkv,D],
 // boxes of 64 (d) x 1 x 64 (tokens) x 1, 128-byte swizzle. With block_table the maps cover

@@ -15,7 +15,7 @@ namespace da2 {
 // reports through the device error word and then returns without trapping.
 constexpr uint64_t kWaitLimitNs = 250ull * 1000ull * 1000ull;
 
-enum DeviceError : int { kErrNone = 0, kErrPrefillWait = 1, kErrDecodeWait = 2 };
+enum DeviceError : int { kErrNone = 0, kErrPrefillWait = 1, kErrDecodeWait = 2, kErrBackwardWait = 3 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -86,6 +86,14 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
+}
+
+// Untiled bulk copy global -> shared of `bytes` (multiple of 16; both addresses 16-byte
+// aligned), completion counted on `bar` in bytes.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
 }
 
 // ------------------------------------------------------------------------------ tcgen05
