@@ -51,6 +51,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic per launch from an ncu capture, keyed by the kernel source it was taken on;
 # reported as null once the source differs from the one captured.
+# B200 data-sheet figures (dense bf16 tensor throughput, HBM3e bandwidth), reported beside
+# the measured peaks
+SPEC_BF16_TFLOPS = 2250.0
+SPEC_HBM_GBS = 8000.0
+
 NCU_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one launch (B=4 x 4k causal prefill)
     "prefill": {"bytes": 620974848, "source_sha": "a32175841b489c66"},
@@ -355,13 +360,15 @@ def run_ours(args, rank, world, local, dist):
             "value": round(dec_value, 1), "unit": "GB/s", "us_per_step": round(1000 * dec_launch_ms, 2),
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": traffic_d,
-                         "peak_source": f"{peak_src} hbm_gbs"},
+                         "peak_source": f"{peak_src} hbm_gbs",
+                         "frac_of_spec": round(gbs / SPEC_HBM_GBS, 4), "spec_peak": SPEC_HBM_GBS},
         },
         "roofline": {
             "bound": "tensor", "achieved": round(tflops, 2), "peak": peak_t, "unit": "TFLOP/s",
             "frac": round(tflops / peak_t, 4), "traffic": traffic,
             "kernel": "diffattn_prefill_sm100", "flops_per_launch": flops,
             "launch_ms": round(pre_launch_ms, 4), "peak_source": f"{peak_src} bf16_tflops (burst)",
+            "frac_of_spec": round(tflops / SPEC_BF16_TFLOPS, 4), "spec_peak": SPEC_BF16_TFLOPS,
         },
         "e2e": {
             "value": round(world * flops * e2e_steps / (e2e_ms * 1e-3) / 1e12, 3) if do_pre else None,
@@ -639,6 +646,7 @@ def run_workload(args):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic, seeded", "config": cfg,
             "roofline": {"bound": bound, "achieved": round(val, 2), "peak": peak, "unit": unit,
                          "frac": round(val / peak, 4), "traffic": None,
+                         "frac_of_spec": round(val / (SPEC_BF16_TFLOPS if bound == "tensor" else SPEC_HBM_GBS), 4),
                          "peak_source": f"{peak_src} {'bf16_tflops (burst)' if bound == 'tensor' else 'hbm_gbs'}"},
             "gpu_launches": launches * args.steps, "workload": name}
     print(json.dumps(line), flush=True)

@@ -12,10 +12,11 @@
 // A_b is recomputed from the forward's base-2 row log-sum-exp: A_b = 2^(s log2(e)/sqrt(D) - lse_b).
 //
 // Three launches, no atomics (the result is deterministic):
-//   preprocess   one warp per (token, pair): E_1, E_2, dlambda, and a 32-byte record
-//                {lse_1, lse_2, E_1, E_2, lambda} per (pair, row) that the other kernels
-//                stream; rows past S (to a multiple of 128) get lse = +inf so their
-//                probabilities are exactly 0 without per-element row checks
+//   preprocess   one warp per (token, pair): E_1, E_2, dlambda, and the row terms the other
+//                kernels stream, negated and stored per 64-row block as five arrays of 64
+//                fp32 (-lse_1, -lse_2, -E_1, -E_2, -lambda); rows past S (to a multiple of
+//                128) get -lse = -inf so their probabilities are exactly 0 without
+//                per-element row checks
 //   dkdv_sm100   a CTA owns 128 keys of one KV head (the TMEM lanes) and walks every pair of
 //                the group and every 64-row query block that sees the keys
 //   dq_sm100     a CTA owns 128 query rows of one pair (the TMEM lanes) and walks the 64-key
@@ -32,16 +33,36 @@ namespace da2 {
 namespace bwd_tc {
 
 constexpr int HD = 128;
-constexpr int kThreads = 320;
 constexpr int kStages = 2;
-constexpr int kStatFloats = 8;                 // {lse1, lse2, E1, E2, lambda, 0, 0, 0}
+
+// Elementwise warps: 8 (each thread takes 32 columns of a step) or 16 (16 columns). Warps
+// w and w+4k read the same TMEM lanes (w % 4 picks the lane quarter) and split the columns.
+#ifndef DA2_BWD_EW_WARPS
+#define DA2_BWD_EW_WARPS 16
+#endif
+constexpr int kEwWarps = DA2_BWD_EW_WARPS;
+static_assert(kEwWarps == 8 || kEwWarps == 16, "elementwise warps");
+constexpr int kGroups = kEwWarps / 4;      // column groups of a 64-column step
+constexpr int kCols = 64 / kGroups;        // columns per elementwise thread
+constexpr int kProducerWarp = kEwWarps;
+constexpr int kMmaWarp = kEwWarps + 1;
+constexpr int kThreads = 32 * (kEwWarps + 2);
+
+// A column group writes its bf16 results (two per 32-bit column) over the first half of
+// its own fp32 columns. TMEM column of the bf16 operand for columns 32h+16k2 .. +15.
+__host__ __device__ constexpr uint32_t packed_col(int h, int k2) {
+  return static_cast<uint32_t>(((32 * h + 16 * k2) / kCols) * kCols + ((32 * h + 16 * k2) % kCols) / 2);
+}
+constexpr int kStatArrays = 5;                 // -lse1, -lse2, -E1, -E2, -lambda
+constexpr int kStatBlock = 64;                 // rows per block of the five arrays
 constexpr int kRowPad = 128;                   // stats rows padded to a multiple of this
 
 constexpr uint32_t kIdescS = idesc_bf16_f32(128, 32, false);   // scores: N = 32 columns per half
 constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, 128, true);  // accumulators: B MN-major, N = d
 
-// TMEM columns
-constexpr uint32_t kTmS1 = 0, kTmS2 = 64, kTmDP = 128, kTmAcc0 = 256, kTmAcc1 = 384;
+// TMEM columns. kTmA holds one resident 128 x 128 operand (bf16 pairs) read as the A
+// operand of a score MMA: K in the dK/dV kernel, Q_1 in the dQ kernel.
+constexpr uint32_t kTmS1 = 0, kTmS2 = 64, kTmDP = 128, kTmA = 192, kTmAcc0 = 256, kTmAcc1 = 384;
 
 // K-major SW128 operand of R rows: K-step kk (16 of d) -> chunk kk/4, +32 bytes per 16 elements
 __device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, uint32_t chunk_bytes, int kk) {
@@ -53,7 +74,7 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t base, uint32_t chunk_b
 }
 
 struct Params {
-  const float* stats;        // [B, Hq/2, S_pad, 8]
+  const float* stats;        // [B, Hq/2, S_pad/64, 5, 64]
   __nv_bfloat16* dq;         // [B,S,Hq,D]
   __nv_bfloat16* dk;         // [B,S,Hkv,D]
   __nv_bfloat16* dv;
@@ -64,6 +85,11 @@ struct Params {
 };
 
 // ------------------------------------------------------------------------ preprocess
+// Offset of row i's term k in the stats of (b, pair).
+__host__ __device__ __forceinline__ size_t stat_index(size_t bp, int S_pad, int i, int k) {
+  return (bp * (S_pad / kStatBlock) + i / kStatBlock) * (kStatArrays * kStatBlock) + k * kStatBlock + i % kStatBlock;
+}
+
 __global__ void __launch_bounds__(128)
 preprocess_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ o_branch,
                   const float* __restrict__ lse, const float* __restrict__ lambda, float* __restrict__ stats,
@@ -71,14 +97,13 @@ preprocess_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
   const long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (w >= static_cast<long long>(B) * S_pad * n_pairs) return;
-  // warp w: row i of pair p of batch b, rows fastest (records of a pair are contiguous)
+  // warp w: row i of pair p of batch b, rows fastest
   const int i = static_cast<int>(w % S_pad);
   const long long bp = w / S_pad;
   const int p = static_cast<int>(bp % n_pairs);
   const int b = static_cast<int>(bp / n_pairs);
-  float* rec = stats + w * kStatFloats;
   if (i >= S) {
-    if (lane < kStatFloats) rec[lane] = lane < 2 ? INFINITY : 0.f;
+    if (lane < kStatArrays) stats[stat_index(bp, S_pad, i, lane)] = lane < 2 ? -INFINITY : 0.f;
     return;
   }
   const long long row = static_cast<long long>(b) * S + i;
@@ -96,14 +121,14 @@ preprocess_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
     for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
     e[br] = v;
   }
-  if (lane == 0) {
-    const float l1 = __ldg(lse + row * (2 * n_pairs) + 2 * p);
-    const float l2 = __ldg(lse + row * (2 * n_pairs) + 2 * p + 1);
-    const float lam = __ldg(lambda + row * n_pairs + p);
-    reinterpret_cast<float4*>(rec)[0] = make_float4(l1, l2, e[0], e[1]);
-    reinterpret_cast<float4*>(rec)[1] = make_float4(lam, 0.f, 0.f, 0.f);
-    dlam[row * n_pairs + p] = -e[1];
+  if (lane < kStatArrays) {
+    float t;
+    if (lane < 2) t = -__ldg(lse + row * (2 * n_pairs) + 2 * p + lane);
+    else if (lane < 4) t = -e[lane - 2];
+    else t = -__ldg(lambda + row * n_pairs + p);
+    stats[stat_index(bp, S_pad, i, lane)] = t;
   }
+  if (lane == 0) dlam[row * n_pairs + p] = -e[1];
 }
 
 // Shared-memory layouts (byte offsets from a 1024-aligned base). Both tile kernels hold
@@ -112,7 +137,7 @@ constexpr uint32_t kFixedTile = 128 * 256;     // 128 rows x 128 bf16
 constexpr uint32_t kFixedChunk = 128 * 128;    // one 64-wide d half of it
 constexpr uint32_t kStreamTile = 64 * 256;     // 64 rows x 128 bf16
 constexpr uint32_t kStreamChunk = 64 * 128;
-constexpr uint32_t kStatBytes = 64 * kStatFloats * 4;
+constexpr uint32_t kStatBytes = kStatArrays * kStatBlock * 4;  // one 64-row block
 
 // mbarriers
 enum Bar : int {
@@ -123,14 +148,15 @@ enum Bar : int {
   kPReady = 7,   // +half
   kDFull = 9,
   kDrain = 10,
-  kNumBars = 11
+  kAReady = 11,  // the resident A operand is in TMEM
+  kNumBars = 12
 };
 
 // dK/dV: fixed K, V (128 keys); stream Q1, Q2, dO (64 query rows) + their 64 stat records
 constexpr uint32_t kKvOffK = 0;
 constexpr uint32_t kKvOffV = kFixedTile;
 constexpr uint32_t kKvOffX = 2 * kFixedTile;
-constexpr uint32_t kKvStage = 3 * kStreamTile + kStatBytes;
+constexpr uint32_t kKvStage = (3 * kStreamTile + kStatBytes + 1023) / 1024 * 1024;  // tiles stay 1024-aligned
 constexpr uint32_t kKvOffBar = kKvOffX + kStages * kKvStage;
 constexpr uint32_t kKvSmem = kKvOffBar + 256 + 1024;
 
@@ -142,6 +168,8 @@ constexpr uint32_t kQOffX = 3 * kFixedTile;
 constexpr uint32_t kQStage = 2 * kStreamTile;
 constexpr uint32_t kQOffBar = kQOffX + kStages * kQStage;
 constexpr uint32_t kQSmem = kQOffBar + 256 + 1024;
+static_assert(kKvStage % 1024 == 0 && kQStage % 1024 == 0, "128-byte-swizzled tiles need 1024-byte alignment");
+static_assert(kKvSmem <= 232448 && kQSmem <= 232448, "shared memory per CTA");
 
 __device__ __forceinline__ void tmem_ld_x32_wait(uint32_t taddr, uint32_t (&r)[32]) {
   tmem_ld_32x32b_x32(taddr, r);
@@ -152,13 +180,13 @@ __device__ __forceinline__ void tmem_ld_x32_wait(uint32_t taddr, uint32_t (&r)[3
 __device__ __forceinline__ uint32_t setup(uint32_t bar0, uint32_t* tmem_slot, volatile int* abort_flag, int warp) {
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i) {
-      const uint32_t count = (i == kPReady || i == kPReady + 1) ? 128u : 1u;
+      const uint32_t count = (i == kPReady || i == kPReady + 1) ? 32u * kEwWarps / 2 : (i == kAReady ? 32u * kEwWarps : 1u);
       mbar_init(bar0 + 8u * i, count);
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -172,17 +200,17 @@ __device__ __forceinline__ void teardown(uint32_t tmem, const volatile int* abor
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag) atomicCAS(err, 0, kErrBackwardWait);
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
 }
 
-// Write 64 fp32 accumulator columns of this thread's row (TMEM) as bf16, times `mul`.
-__device__ __forceinline__ void store_row64(uint32_t taddr, __nv_bfloat16* dst, float mul, bool valid) {
+// Write this thread's 128 / kGroups accumulator columns of its row (TMEM) as bf16, times `mul`.
+__device__ __forceinline__ void store_row(uint32_t taddr, __nv_bfloat16* dst, float mul, bool valid) {
 #pragma unroll 1
-  for (int c = 0; c < 2; ++c) {
+  for (int c = 0; c < 128 / kGroups / 32; ++c) {
     uint32_t a[32];
     tmem_ld_x32_wait(taddr + 32 * c, a);
     if (valid) {
@@ -195,6 +223,59 @@ __device__ __forceinline__ void store_row64(uint32_t taddr, __nv_bfloat16* dst, 
                           pack_bf16x2(__uint_as_float(a[8 * v + 6]) * mul, __uint_as_float(a[8 * v + 7]) * mul));
     }
   }
+}
+
+// N (kCols) consecutive fp32 columns of this warp's 32 lanes; the wait completes them.
+template <int N>
+__device__ __forceinline__ void ld_cols(uint32_t taddr, uint32_t (&r)[N]) {
+  if constexpr (N == 32) {
+    tmem_ld_32x32b_x32(taddr, r);
+  } else {
+    tmem_ld_32x32b_x16(taddr, r);
+  }
+}
+template <int N>
+__device__ __forceinline__ void ld_cols_wait(uint32_t (&r)[N]) {
+  if constexpr (N == 32) {
+    tmem_ld_wait(r);
+  } else {
+    tmem_ld_wait16(r);
+  }
+}
+// N = 16 or 32 consecutive 32-bit columns of this warp's 32 lanes
+template <int N>
+__device__ __forceinline__ void st_cols(uint32_t taddr, const uint32_t (&r)[N]) {
+  if constexpr (N == 32) {
+    tmem_st_32x32b_x32(taddr, r);
+  } else {
+    tmem_st_32x32b_x16(taddr, r);
+  }
+}
+// N packed bf16x2 columns (N = kCols / 2)
+template <int N>
+__device__ __forceinline__ void st_packed(uint32_t taddr, const uint32_t (&r)[N]) {
+  if constexpr (N == 16) {
+    tmem_st_32x32b_x16(taddr, r);
+  } else {
+    tmem_st_32x32b_x8(taddr, r);
+  }
+}
+
+// Copy this thread's share of a resident 128-row K-major SW128 tile (row r = TMEM lane)
+// into TMEM from column kTmA on, as packed bf16 pairs along d (element 2j in the low half
+// of column j): the A-operand layout of a TS MMA. Each column group takes 128 / kGroups d.
+__device__ __forceinline__ void tile_to_tmem(uint32_t tile, uint32_t trow, int r, int cg) {
+  constexpr int kD = 128 / kGroups;
+  uint32_t v[kD / 2];
+#pragma unroll
+  for (int u = 0; u < kD / 8; ++u) {
+    const int du = (kD / 8) * cg + u;  // 16-byte unit along d, 0..15
+    const uint32_t addr = tile + (du >> 3) * kFixedChunk + r * 128 + (((du & 7) ^ (r & 7)) << 4);
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v[4 * u]), "=r"(v[4 * u + 1]), "=r"(v[4 * u + 2]), "=r"(v[4 * u + 3])
+                 : "r"(addr));
+  }
+  st_cols(trow + kTmA + (kD / 2) * cg, v);
 }
 
 // --------------------------------------------------------------------------- dK / dV
@@ -222,7 +303,7 @@ dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 
   const uint32_t tmem = setup(bar0, tmem_slot, abort_flag, warp);
 
-  if (warp == 8) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
@@ -245,9 +326,8 @@ dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           tma_load_4d(st + kStreamTile + c * kStreamChunk, &tmQ, bar(kXFull + s), c * 64, 2 * pair + 1, q0, b);
           tma_load_4d(st + 2 * kStreamTile + c * kStreamChunk, &tmO, bar(kXFull + s), c * 64, pair, q0, b);
         }
-        bulk_load(st + 3 * kStreamTile,
-                  p.stats + ((static_cast<size_t>(b) * n_pairs + pair) * p.S_pad + q0) * kStatFloats, kStatBytes,
-                  bar(kXFull + s));
+        bulk_load(st + 3 * kStreamTile, p.stats + stat_index(static_cast<size_t>(b) * n_pairs + pair, p.S_pad, q0, 0),
+                  kStatBytes, bar(kXFull + s));
         issued = t + 1;
       }
       if (*abort_flag) {
@@ -256,30 +336,41 @@ dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         for (int t = max(0, issued - kStages); t < issued; ++t) mbar_wait(bar(kXFull + (t & 1)), (t >> 1) & 1, &no_abort);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == kMmaWarp) {
     // -------------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      bool ok = mbar_wait(bar(kFixedFull), 0, abort_flag);
+      // S_1^T = K Q_1^T, S_2^T = K Q_2^T, dP^T = V dO^T of step t, queries 32h .. 32h+31
+      auto issue_scores = [&](int t, int h) {
+        const uint32_t st = sbase + kKvOffX + (t & 1) * kKvStage;
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t a_k = tmem + kTmA + 8 * kk;  // K, resident in TMEM
+          const uint64_t a_v = desc_kmajor(sbase + kKvOffV, kFixedChunk, kk);
+          const uint32_t acc = kk > 0 ? 1u : 0u;
+          mma_bf16_ts(tmem + kTmS1 + 32 * h, a_k, desc_kmajor(st + h * 4096, kStreamChunk, kk), kIdescS, acc);
+          mma_bf16_ts(tmem + kTmS2 + 32 * h, a_k, desc_kmajor(st + kStreamTile + h * 4096, kStreamChunk, kk), kIdescS,
+                      acc);
+          mma_bf16_ss(tmem + kTmDP + 32 * h, a_v, desc_kmajor(st + 2 * kStreamTile + h * 4096, kStreamChunk, kk),
+                      kIdescS, acc);
+        }
+        tc_commit(bar(kSFull + h));
+      };
+      // Issue order: scores(0); then per step t and half h: [wait P_h(t)] dV, dK of half h;
+      // scores(t+1, h). Scores of step t+1, half h overwrite only half h's columns, which the
+      // accumulations just issued read first (MMAs execute in issue order), so half h of the
+      // next step starts while the elementwise warps still work on the other half.
+      bool ok = mbar_wait(bar(kFixedFull), 0, abort_flag) && mbar_wait(bar(kAReady), 0, abort_flag) &&
+                mbar_wait(bar(kXFull), 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_scores(0, 0);
+        issue_scores(0, 1);
+      }
       for (int t = 0; ok && t < n_steps; ++t) {
         const int s = t & 1;
-        if (!(ok = mbar_wait(bar(kXFull + s), (t >> 1) & 1, abort_flag))) break;
-        tc_fence_after();
         const uint32_t st = sbase + kKvOffX + s * kKvStage;
         const uint32_t sQ1 = st, sQ2 = st + kStreamTile, sO = st + 2 * kStreamTile;
-        // S_1^T = K Q_1^T, S_2^T = K Q_2^T, dP^T = V dO^T; queries 32h .. 32h+31 per half
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-#pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint64_t a_k = desc_kmajor(sbase + kKvOffK, kFixedChunk, kk);
-            const uint64_t a_v = desc_kmajor(sbase + kKvOffV, kFixedChunk, kk);
-            const uint32_t acc = kk > 0 ? 1u : 0u;
-            mma_bf16_ss(tmem + kTmS1 + 32 * h, a_k, desc_kmajor(sQ1 + h * 4096, kStreamChunk, kk), kIdescS, acc);
-            mma_bf16_ss(tmem + kTmS2 + 32 * h, a_k, desc_kmajor(sQ2 + h * 4096, kStreamChunk, kk), kIdescS, acc);
-            mma_bf16_ss(tmem + kTmDP + 32 * h, a_v, desc_kmajor(sO + h * 4096, kStreamChunk, kk), kIdescS, acc);
-          }
-          tc_commit(bar(kSFull + h));
-        }
+        const bool next = t + 1 < n_steps;
         // dV += W^T dO, dK += dS_1^T Q_1 + dS_2^T Q_2 (bf16 operands written over the scores)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -289,12 +380,17 @@ dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           for (int k2 = 0; k2 < 2; ++k2) {
             const int row = 32 * h + 16 * k2;
             const uint32_t first = (t == 0 && h == 0 && k2 == 0) ? 0u : 1u;
-            mma_bf16_ts(tmem + kTmAcc0, tmem + kTmS1 + 32 * h + 8 * k2, desc_mnmajor(sO, kStreamChunk, row), kIdescAcc,
+            mma_bf16_ts(tmem + kTmAcc0, tmem + kTmS1 + packed_col(h, k2), desc_mnmajor(sO, kStreamChunk, row), kIdescAcc,
                         first);
-            mma_bf16_ts(tmem + kTmAcc1, tmem + kTmS2 + 32 * h + 8 * k2, desc_mnmajor(sQ1, kStreamChunk, row),
+            mma_bf16_ts(tmem + kTmAcc1, tmem + kTmS2 + packed_col(h, k2), desc_mnmajor(sQ1, kStreamChunk, row),
                         kIdescAcc, first);
-            mma_bf16_ts(tmem + kTmAcc1, tmem + kTmDP + 32 * h + 8 * k2, desc_mnmajor(sQ2, kStreamChunk, row),
+            mma_bf16_ts(tmem + kTmAcc1, tmem + kTmDP + packed_col(h, k2), desc_mnmajor(sQ2, kStreamChunk, row),
                         kIdescAcc, 1u);
+          }
+          if (next) {
+            if (h == 0 && !(ok = mbar_wait(bar(kXFull + (s ^ 1)), ((t + 1) >> 1) & 1, abort_flag))) break;
+            tc_fence_after();
+            issue_scores(t + 1, h);
           }
         }
         if (!ok) break;
@@ -307,12 +403,21 @@ dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     }
   } else {
     // ------------------------------------------------------------------ elementwise
-    const int hc = warp >> 2;                 // query half of each step
+    const int cg = warp >> 2;                 // column group: queries kCols*cg .. of each step
+    const int hc = cg / (kGroups / 2);        // the step half those columns belong to
+    const int col0 = kCols * cg;
     const int r = 32 * (warp & 3) + lane;     // key row of the tile == TMEM lane
     const int key = k0 + r;
     const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    bool ok = true;
-    for (int t = 0; t < n_steps; ++t) {
+    // K into TMEM for the score MMAs
+    bool ok = __all_sync(0xffffffffu, mbar_wait(bar(kFixedFull), 0, abort_flag));
+    if (ok) {
+      tile_to_tmem(sbase + kKvOffK, trow, r, cg);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(kAReady));
+    }
+    for (int t = 0; ok && t < n_steps; ++t) {
       const int s = t & 1;
       const int q0 = (q_first + t % steps_per_pair) * 64;
       ok = __all_sync(0xffffffffu, mbar_wait(bar(kSFull + hc), t & 1, abort_flag));
@@ -321,40 +426,58 @@ dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(kXFull + s), (t >> 1) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      uint32_t s1[32], s2[32], dp[32];
-      tmem_ld_32x32b_x32(trow + kTmS1 + 32 * hc, s1);
-      tmem_ld_32x32b_x32(trow + kTmS2 + 32 * hc, s2);
-      tmem_ld_32x32b_x32(trow + kTmDP + 32 * hc, dp);
-      tmem_ld_wait(s1);
-      reg_fence(s2);
-      reg_fence(dp);
-      const float4* rec = reinterpret_cast<const float4*>(smem + kKvOffX + s * kKvStage + 3 * kStreamTile) + 2 * (32 * hc);
+      uint32_t s1[kCols], s2[kCols], dp[kCols];
+      ld_cols(trow + kTmS1 + col0, s1);
+      ld_cols(trow + kTmS2 + col0, s2);
+      ld_cols(trow + kTmDP + col0, dp);
+      ld_cols_wait(s1);
+      ld_cols_wait(s2);
+      ld_cols_wait(dp);
+      // this group's columns of the five row-term arrays (shared, filled by bulk copy)
+      const uint32_t rec = sbase + kKvOffX + s * kKvStage + 3 * kStreamTile + 4 * col0;
       // causal: only the two query blocks that overlap the key tile hold keys past a query
       const bool diag = p.causal && q0 < k0 + 128;
-      const int qbase = q0 + 32 * hc;
-      uint32_t w_pk[16], d1_pk[16], d2_pk[16];
+      const int qbase = q0 + col0;
+      const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
+      uint32_t w_pk[kCols / 2], d1_pk[kCols / 2], d2_pk[kCols / 2];
 #pragma unroll
-      for (int c = 0; c < 32; c += 2) {
-        float w[2], d1[2], d2[2];
+      for (int c4 = 0; c4 < kCols; c4 += 4) {
+        uint64_t nl1[2], nl2[2], ne1[2], ne2[2], nlam[2];
+        lds_f32x4(rec + 0 * 256 + 4 * c4, nl1[0], nl1[1]);
+        lds_f32x4(rec + 1 * 256 + 4 * c4, nl2[0], nl2[1]);
+        lds_f32x4(rec + 2 * 256 + 4 * c4, ne1[0], ne1[1]);
+        lds_f32x4(rec + 3 * 256 + 4 * c4, ne2[0], ne2[1]);
+        lds_f32x4(rec + 4 * 256 + 4 * c4, nlam[0], nlam[1]);
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float4 ra = rec[2 * (c + e)];
-          const float lam = rec[2 * (c + e) + 1].x;
-          float p1 = fast_exp2(__uint_as_float(s1[c + e]) * p.scale_log2 - ra.x);
-          float p2 = fast_exp2(__uint_as_float(s2[c + e]) * p.scale_log2 - ra.y);
-          if (diag && key > qbase + c + e) p1 = p2 = 0.f;
-          const float dpv = __uint_as_float(dp[c + e]);
-          w[e] = __fmaf_rn(-lam, p2, p1);
-          d1[e] = p1 * (dpv - ra.z);
-          d2[e] = -lam * p2 * (dpv - ra.w);
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int c = c4 + 2 * h2;  // columns c, c+1
+          const uint64_t a1 = f2_fma(f2_pack(__uint_as_float(s1[c]), __uint_as_float(s1[c + 1])), sc2, nl1[h2]);
+          const uint64_t a2 = f2_fma(f2_pack(__uint_as_float(s2[c]), __uint_as_float(s2[c + 1])), sc2, nl2[h2]);
+          float x0, x1, y0, y1;
+          f2_unpack(a1, x0, x1);
+          f2_unpack(a2, y0, y1);
+          float p10 = fast_exp2(x0), p11 = fast_exp2(x1), p20 = fast_exp2(y0), p21 = fast_exp2(y1);
+          if (diag) {
+            if (key > qbase + c) p10 = p20 = 0.f;
+            if (key > qbase + c + 1) p11 = p21 = 0.f;
+          }
+          const uint64_t P1 = f2_pack(p10, p11), P2 = f2_pack(p20, p21);
+          const uint64_t dpp = f2_pack(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1]));
+          const uint64_t w = f2_fma(nlam[h2], P2, P1);                           // P1 - lambda P2
+          const uint64_t d1 = f2_mul(P1, f2_add(dpp, ne1[h2]));                  // P1 (dP - E1)
+          const uint64_t d2 = f2_mul(f2_mul(nlam[h2], P2), f2_add(dpp, ne2[h2]));  // -lambda P2 (dP - E2)
+          float u0, u1;
+          f2_unpack(w, u0, u1);
+          w_pk[c >> 1] = pack_bf16x2(u0, u1);
+          f2_unpack(d1, u0, u1);
+          d1_pk[c >> 1] = pack_bf16x2(u0, u1);
+          f2_unpack(d2, u0, u1);
+          d2_pk[c >> 1] = pack_bf16x2(u0, u1);
         }
-        w_pk[c >> 1] = pack_bf16x2(w[0], w[1]);
-        d1_pk[c >> 1] = pack_bf16x2(d1[0], d1[1]);
-        d2_pk[c >> 1] = pack_bf16x2(d2[0], d2[1]);
       }
-      tmem_st_32x32b_x16(trow + kTmS1 + 32 * hc, w_pk);
-      tmem_st_32x32b_x16(trow + kTmS2 + 32 * hc, d1_pk);
-      tmem_st_32x32b_x16(trow + kTmDP + 32 * hc, d2_pk);
+      st_packed(trow + kTmS1 + col0, w_pk);
+      st_packed(trow + kTmS2 + col0, d1_pk);
+      st_packed(trow + kTmDP + col0, d2_pk);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(kPReady + hc));
@@ -363,9 +486,10 @@ dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     if (__all_sync(0xffffffffu, ok && !*abort_flag)) {
       tc_fence_after();
       const bool valid = key < p.S;
-      const size_t off = ((static_cast<size_t>(b) * p.S + (valid ? key : 0)) * p.Hkv + g) * HD + 64 * hc;
-      store_row64(trow + kTmAcc0 + 64 * hc, p.dv + off, 1.f, valid);
-      store_row64(trow + kTmAcc1 + 64 * hc, p.dk + off, p.scale, valid);
+      const int d0 = (128 / kGroups) * cg;
+      const size_t off = ((static_cast<size_t>(b) * p.S + (valid ? key : 0)) * p.Hkv + g) * HD + d0;
+      store_row(trow + kTmAcc0 + d0, p.dv + off, 1.f, valid);
+      store_row(trow + kTmAcc1 + d0, p.dk + off, p.scale, valid);
     }
   }
   teardown(tmem, abort_flag, p.err, warp);
@@ -395,7 +519,7 @@ dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
 
   const uint32_t tmem = setup(bar0, tmem_slot, abort_flag, warp);
 
-  if (warp == 8) {
+  if (warp == kProducerWarp) {
     if (lane == 0) {
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
@@ -423,28 +547,34 @@ dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         for (int t = max(0, issued - kStages); t < issued; ++t) mbar_wait(bar(kXFull + (t & 1)), (t >> 1) & 1, &no_abort);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == kMmaWarp) {
     if (lane == 0) {
-      bool ok = mbar_wait(bar(kFixedFull), 0, abort_flag);
+      // S_1 = Q_1 K^T, S_2 = Q_2 K^T, dP = dO V^T of key block t, keys 32h .. 32h+31
+      auto issue_scores = [&](int t, int h) {
+        const uint32_t sK = sbase + kQOffX + (t & 1) * kQStage, sV = sK + kStreamTile;
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint64_t b_k = desc_kmajor(sK + h * 4096, kStreamChunk, kk);
+          const uint32_t acc = kk > 0 ? 1u : 0u;
+          mma_bf16_ts(tmem + kTmS1 + 32 * h, tmem + kTmA + 8 * kk, b_k, kIdescS, acc);  // Q_1 resident in TMEM
+          mma_bf16_ss(tmem + kTmS2 + 32 * h, desc_kmajor(sbase + kQOffQ2, kFixedChunk, kk), b_k, kIdescS, acc);
+          mma_bf16_ss(tmem + kTmDP + 32 * h, desc_kmajor(sbase + kQOffO, kFixedChunk, kk),
+                      desc_kmajor(sV + h * 4096, kStreamChunk, kk), kIdescS, acc);
+        }
+        tc_commit(bar(kSFull + h));
+      };
+      // same issue order as the dK/dV kernel
+      bool ok = mbar_wait(bar(kFixedFull), 0, abort_flag) && mbar_wait(bar(kAReady), 0, abort_flag) &&
+                mbar_wait(bar(kXFull), 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_scores(0, 0);
+        issue_scores(0, 1);
+      }
       for (int t = 0; ok && t < n_steps; ++t) {
         const int s = t & 1;
-        if (!(ok = mbar_wait(bar(kXFull + s), (t >> 1) & 1, abort_flag))) break;
-        tc_fence_after();
-        const uint32_t sK = sbase + kQOffX + s * kQStage, sV = sK + kStreamTile;
-        // S_1 = Q_1 K^T, S_2 = Q_2 K^T, dP = dO V^T; keys 32h .. 32h+31 per half
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-#pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint64_t b_k = desc_kmajor(sK + h * 4096, kStreamChunk, kk);
-            const uint32_t acc = kk > 0 ? 1u : 0u;
-            mma_bf16_ss(tmem + kTmS1 + 32 * h, desc_kmajor(sbase + kQOffQ1, kFixedChunk, kk), b_k, kIdescS, acc);
-            mma_bf16_ss(tmem + kTmS2 + 32 * h, desc_kmajor(sbase + kQOffQ2, kFixedChunk, kk), b_k, kIdescS, acc);
-            mma_bf16_ss(tmem + kTmDP + 32 * h, desc_kmajor(sbase + kQOffO, kFixedChunk, kk),
-                        desc_kmajor(sV + h * 4096, kStreamChunk, kk), kIdescS, acc);
-          }
-          tc_commit(bar(kSFull + h));
-        }
+        const uint32_t sK = sbase + kQOffX + s * kQStage;
+        const bool next = t + 1 < n_steps;
         // dQ_1 += dS_1 K, dQ_2 += dS_2 K
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -455,8 +585,13 @@ dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
             const int row = 32 * h + 16 * k2;
             const uint32_t first = (t == 0 && h == 0 && k2 == 0) ? 0u : 1u;
             const uint64_t b_k = desc_mnmajor(sK, kStreamChunk, row);
-            mma_bf16_ts(tmem + kTmAcc0, tmem + kTmS1 + 32 * h + 8 * k2, b_k, kIdescAcc, first);
-            mma_bf16_ts(tmem + kTmAcc1, tmem + kTmS2 + 32 * h + 8 * k2, b_k, kIdescAcc, first);
+            mma_bf16_ts(tmem + kTmAcc0, tmem + kTmS1 + packed_col(h, k2), b_k, kIdescAcc, first);
+            mma_bf16_ts(tmem + kTmAcc1, tmem + kTmS2 + packed_col(h, k2), b_k, kIdescAcc, first);
+          }
+          if (next) {
+            if (h == 0 && !(ok = mbar_wait(bar(kXFull + (s ^ 1)), ((t + 1) >> 1) & 1, abort_flag))) break;
+            tc_fence_after();
+            issue_scores(t + 1, h);
           }
         }
         if (!ok) break;
@@ -468,49 +603,68 @@ dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
       mbar_wait(bar(kDrain), 0, &no_abort);
     }
   } else {
-    const int hc = warp >> 2;                 // key half of each step
+    const int cg = warp >> 2;                 // column group: keys kCols*cg .. of each step
+    const int hc = cg / (kGroups / 2);        // the step half those columns belong to
+    const int col0 = kCols * cg;
     const int r = 32 * (warp & 3) + lane;     // query row of the tile == TMEM lane
     const int qi = m0 + r;
     const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    // this row's record (rows past S carry lse = +inf: probabilities 0)
-    const float4* rec =
-        reinterpret_cast<const float4*>(p.stats + ((static_cast<size_t>(b) * n_pairs + pair) * p.S_pad + qi) * kStatFloats);
-    const float4 ra = __ldg(rec);
-    const float lam = __ldg(rec + 1).x;
-    bool ok = true;
-    for (int t = 0; t < n_steps; ++t) {
+    // Q_1 into TMEM for the score MMAs
+    bool ok = __all_sync(0xffffffffu, mbar_wait(bar(kFixedFull), 0, abort_flag));
+    if (ok) {
+      tile_to_tmem(sbase + kQOffQ1, trow, r, cg);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(kAReady));
+    }
+    // this row's terms (rows past S carry -lse = -inf: probabilities 0)
+    const size_t bp = static_cast<size_t>(b) * n_pairs + pair;
+    const float nl1 = __ldg(p.stats + stat_index(bp, p.S_pad, qi, 0));
+    const float nl2 = __ldg(p.stats + stat_index(bp, p.S_pad, qi, 1));
+    const uint64_t ne1 = f2_pack(__ldg(p.stats + stat_index(bp, p.S_pad, qi, 2)), __ldg(p.stats + stat_index(bp, p.S_pad, qi, 2)));
+    const uint64_t ne2 = f2_pack(__ldg(p.stats + stat_index(bp, p.S_pad, qi, 3)), __ldg(p.stats + stat_index(bp, p.S_pad, qi, 3)));
+    const float nlam_s = __ldg(p.stats + stat_index(bp, p.S_pad, qi, 4));
+    const uint64_t nl1_2 = f2_pack(nl1, nl1), nl2_2 = f2_pack(nl2, nl2), nlam = f2_pack(nlam_s, nlam_s);
+    const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
+    for (int t = 0; ok && t < n_steps; ++t) {
       ok = __all_sync(0xffffffffu, mbar_wait(bar(kSFull + hc), t & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      uint32_t s1[32], s2[32], dp[32];
-      tmem_ld_32x32b_x32(trow + kTmS1 + 32 * hc, s1);
-      tmem_ld_32x32b_x32(trow + kTmS2 + 32 * hc, s2);
-      tmem_ld_32x32b_x32(trow + kTmDP + 32 * hc, dp);
-      tmem_ld_wait(s1);
-      reg_fence(s2);
-      reg_fence(dp);
-      const int kbase = 64 * t + 32 * hc;
+      uint32_t s1[kCols], s2[kCols], dp[kCols];
+      ld_cols(trow + kTmS1 + col0, s1);
+      ld_cols(trow + kTmS2 + col0, s2);
+      ld_cols(trow + kTmDP + col0, dp);
+      ld_cols_wait(s1);
+      ld_cols_wait(s2);
+      ld_cols_wait(dp);
+      const int kbase = 64 * t + col0;
       // tile-uniform: keys past the query (causal diagonal) or past S (ragged last block)
       const bool masked = (p.causal && 64 * t + 63 > m0) || (64 * t + 64 > p.S);
       const int lim = p.causal ? min(qi, p.S - 1) : p.S - 1;
-      uint32_t d1_pk[16], d2_pk[16];
+      uint32_t d1_pk[kCols / 2], d2_pk[kCols / 2];
 #pragma unroll
-      for (int c = 0; c < 32; c += 2) {
-        float d1[2], d2[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          float p1 = fast_exp2(__uint_as_float(s1[c + e]) * p.scale_log2 - ra.x);
-          float p2 = fast_exp2(__uint_as_float(s2[c + e]) * p.scale_log2 - ra.y);
-          if (masked && kbase + c + e > lim) p1 = p2 = 0.f;
-          const float dpv = __uint_as_float(dp[c + e]);
-          d1[e] = p1 * (dpv - ra.z);
-          d2[e] = -lam * p2 * (dpv - ra.w);
+      for (int c = 0; c < kCols; c += 2) {
+        const uint64_t a1 = f2_fma(f2_pack(__uint_as_float(s1[c]), __uint_as_float(s1[c + 1])), sc2, nl1_2);
+        const uint64_t a2 = f2_fma(f2_pack(__uint_as_float(s2[c]), __uint_as_float(s2[c + 1])), sc2, nl2_2);
+        float x0, x1, y0, y1;
+        f2_unpack(a1, x0, x1);
+        f2_unpack(a2, y0, y1);
+        float p10 = fast_exp2(x0), p11 = fast_exp2(x1), p20 = fast_exp2(y0), p21 = fast_exp2(y1);
+        if (masked) {
+          if (kbase + c > lim) p10 = p20 = 0.f;
+          if (kbase + c + 1 > lim) p11 = p21 = 0.f;
         }
-        d1_pk[c >> 1] = pack_bf16x2(d1[0], d1[1]);
-        d2_pk[c >> 1] = pack_bf16x2(d2[0], d2[1]);
+        const uint64_t dpp = f2_pack(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1]));
+        const uint64_t d1 = f2_mul(f2_pack(p10, p11), f2_add(dpp, ne1));
+        const uint64_t d2 = f2_mul(f2_mul(nlam, f2_pack(p20, p21)), f2_add(dpp, ne2));
+        float u0, u1;
+        f2_unpack(d1, u0, u1);
+        d1_pk[c >> 1] = pack_bf16x2(u0, u1);
+        f2_unpack(d2, u0, u1);
+        d2_pk[c >> 1] = pack_bf16x2(u0, u1);
       }
-      tmem_st_32x32b_x16(trow + kTmS1 + 32 * hc, d1_pk);
-      tmem_st_32x32b_x16(trow + kTmS2 + 32 * hc, d2_pk);
+      st_packed(trow + kTmS1 + col0, d1_pk);
+      st_packed(trow + kTmS2 + col0, d2_pk);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(kPReady + hc));
@@ -519,9 +673,10 @@ dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     if (__all_sync(0xffffffffu, ok && !*abort_flag)) {
       tc_fence_after();
       const bool valid = qi < p.S;
-      const size_t off = ((static_cast<size_t>(b) * p.S + (valid ? qi : 0)) * p.Hq + 2 * pair) * HD + 64 * hc;
-      store_row64(trow + kTmAcc0 + 64 * hc, p.dq + off, p.scale, valid);
-      store_row64(trow + kTmAcc1 + 64 * hc, p.dq + off + HD, p.scale, valid);
+      const int d0 = (128 / kGroups) * cg;
+      const size_t off = ((static_cast<size_t>(b) * p.S + (valid ? qi : 0)) * p.Hq + 2 * pair) * HD + d0;
+      store_row(trow + kTmAcc0 + d0, p.dq + off, p.scale, valid);
+      store_row(trow + kTmAcc1 + d0, p.dq + off + HD, p.scale, valid);
     }
   }
   teardown(tmem, abort_flag, p.err, warp);
@@ -531,7 +686,7 @@ dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
 
 size_t backward_stats_bytes(int B, int S, int Hq) {
   const size_t s_pad = (static_cast<size_t>(S) + bwd_tc::kRowPad - 1) / bwd_tc::kRowPad * bwd_tc::kRowPad;
-  return static_cast<size_t>(B) * (Hq / 2) * s_pad * bwd_tc::kStatFloats * sizeof(float);
+  return static_cast<size_t>(B) * (Hq / 2) * s_pad * bwd_tc::kStatArrays * sizeof(float);
 }
 
 cudaError_t launch_backward_sm100(const CUtensorMap& tmQ64, const CUtensorMap& tmQ128, const CUtensorMap& tmO64,

@@ -194,8 +194,8 @@ def test_prefill_train_host_checks(lib):
 def test_backward_host_checks(lib):
     OB, LS, DO, DQ, DK, DV, DL, W = (P + 32768 * i for i in range(1, 9))
     ws = lib.diffattn_v2_backward_workspace_size(2, 256, 8)
-    assert ws == 2 * (8 // 2) * 256 * 32                   # one 32-byte record per (b, pair, row)
-    assert lib.diffattn_v2_backward_workspace_size(1, 300, 8) == 4 * 384 * 32  # rows padded to 128
+    assert ws == 2 * (8 // 2) * 256 * 20                   # five fp32 row terms per (b, pair, row)
+    assert lib.diffattn_v2_backward_workspace_size(1, 300, 8) == 4 * 384 * 20  # rows padded to 128
     assert lib.diffattn_v2_backward_workspace_size(0, 256, 8) == 0
     ok = (Q, K, V, L, OB, LS, DO, DQ, DK, DV, DL, 2, 256, 8, 2, 128, 1, W, ws, None)
     assert lib.diffattn_v2_backward(*ok[:18], ws - 4, None) == -1                  # short workspace
