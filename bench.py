@@ -57,10 +57,11 @@ SPEC_BF16_TFLOPS = 2250.0
 SPEC_HBM_GBS = 8000.0
 
 NCU_TRAFFIC = {
-    # dram__bytes_read.sum + dram__bytes_write.sum of one launch (B=4 x 4k causal prefill)
-    "prefill": {"bytes": 620974848, "source_sha": "a32175841b489c66"},
-    # split (1.228e9 + 9.13e6) + combine (6.62e6) of one B=64 decode step
-    "decode": {"bytes": 1243700000, "source_sha": "bbed945a81dc3b45"},
+    # dram__bytes_read.sum + dram__bytes_write.sum of one launch (B=4 x 4k causal prefill),
+    # mean of two captured launches
+    "prefill": {"bytes": 764522752, "source_sha": "385877f446c46b12"},
+    # split + combine of one B=64 decode step, mean of two captured steps
+    "decode": {"bytes": 1240836992, "source_sha": "5a98bc5cb2987830"},
 }
 
 

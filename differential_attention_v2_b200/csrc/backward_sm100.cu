@@ -44,20 +44,31 @@ constexpr int kEwWarps = DA2_BWD_EW_WARPS;
 static_assert(kEwWarps == 8 || kEwWarps == 16, "elementwise warps");
 constexpr int kGroups = kEwWarps / 4;      // column groups of a 64-column step
 constexpr int kCols = 64 / kGroups;        // columns per elementwise thread
+// Pipeline chains per step: the score MMAs of a chain cover 64 / kChains columns (their N)
+// and are committed together; the groups of a chain turn them into operands together.
+#ifndef DA2_BWD_CHAINS
+#define DA2_BWD_CHAINS 1
+#endif
+constexpr int kChains = DA2_BWD_CHAINS;
+static_assert(kChains >= 1 && kGroups % kChains == 0, "chains");
+constexpr int kChainCols = 64 / kChains;
+constexpr int kGroupsPerChain = kGroups / kChains;
 constexpr int kProducerWarp = kEwWarps;
 constexpr int kMmaWarp = kEwWarps + 1;
 constexpr int kThreads = 32 * (kEwWarps + 2);
 
-// A column group writes its bf16 results (two per 32-bit column) over the first half of
-// its own fp32 columns. TMEM column of the bf16 operand for columns 32h+16k2 .. +15.
-__host__ __device__ constexpr uint32_t packed_col(int h, int k2) {
-  return static_cast<uint32_t>(((32 * h + 16 * k2) / kCols) * kCols + ((32 * h + 16 * k2) % kCols) / 2);
+// Per chain: the MMA warp issues the chain's scores, the four warps of each of its column
+// groups turn them into bf16 operands written (two per 32-bit column) over the first half of
+// the group's own fp32 columns, and the MMA warp accumulates from them. TMEM column of the
+// bf16 operands of the 16 columns from column q (a K-step of an accumulation MMA):
+__host__ __device__ constexpr uint32_t operand_col(int q) {
+  return static_cast<uint32_t>((q / kCols) * kCols + (q % kCols) / 2);
 }
 constexpr int kStatArrays = 5;                 // -lse1, -lse2, -E1, -E2, -lambda
 constexpr int kStatBlock = 64;                 // rows per block of the five arrays
 constexpr int kRowPad = 128;                   // stats rows padded to a multiple of this
 
-constexpr uint32_t kIdescS = idesc_bf16_f32(128, 32, false);   // scores: N = 32 columns per half
+constexpr uint32_t kIdescS = idesc_bf16_f32(128, kChainCols, false);  // scores: N = one chain's columns
 constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, 128, true);  // accumulators: B MN-major, N = d
 
 // TMEM columns. kTmA holds one resident 128 x 128 operand (bf16 pairs) read as the A
@@ -144,12 +155,12 @@ enum Bar : int {
   kFixedFull = 0,
   kXFull = 1,    // +stage
   kXEmpty = 3,   // +stage
-  kSFull = 5,    // +half
-  kPReady = 7,   // +half
-  kDFull = 9,
-  kDrain = 10,
-  kAReady = 11,  // the resident A operand is in TMEM
-  kNumBars = 12
+  kSFull = 5,    // +column group: its scores are in TMEM
+  kPReady = 9,   // +column group: its bf16 operands are in TMEM
+  kDFull = 13,
+  kDrain = 14,
+  kAReady = 15,  // the resident A operand is in TMEM
+  kNumBars = 16
 };
 
 // dK/dV: fixed K, V (128 keys); stream Q1, Q2, dO (64 query rows) + their 64 stat records
@@ -180,7 +191,8 @@ __device__ __forceinline__ void tmem_ld_x32_wait(uint32_t taddr, uint32_t (&r)[3
 __device__ __forceinline__ uint32_t setup(uint32_t bar0, uint32_t* tmem_slot, volatile int* abort_flag, int warp) {
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i) {
-      const uint32_t count = (i == kPReady || i == kPReady + 1) ? 32u * kEwWarps / 2 : (i == kAReady ? 32u * kEwWarps : 1u);
+      const uint32_t count =
+          (i >= kPReady && i < kPReady + kChains) ? 128u * kGroupsPerChain : (i == kAReady ? 32u * kEwWarps : 1u);
       mbar_init(bar0 + 8u * i, count);
     }
     *abort_flag = 0;
@@ -339,32 +351,31 @@ dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   } else if (warp == kMmaWarp) {
     // -------------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      // S_1^T = K Q_1^T, S_2^T = K Q_2^T, dP^T = V dO^T of step t, queries 32h .. 32h+31
-      auto issue_scores = [&](int t, int h) {
+      // S_1^T = K Q_1^T, S_2^T = K Q_2^T, dP^T = V dO^T of step t for the queries of group c
+      auto issue_scores = [&](int t, int c) {
         const uint32_t st = sbase + kKvOffX + (t & 1) * kKvStage;
+        const uint32_t ro = kChainCols * c * 128;  // the chain's first query row in the stream tiles
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t a_k = tmem + kTmA + 8 * kk;  // K, resident in TMEM
           const uint64_t a_v = desc_kmajor(sbase + kKvOffV, kFixedChunk, kk);
           const uint32_t acc = kk > 0 ? 1u : 0u;
-          mma_bf16_ts(tmem + kTmS1 + 32 * h, a_k, desc_kmajor(st + h * 4096, kStreamChunk, kk), kIdescS, acc);
-          mma_bf16_ts(tmem + kTmS2 + 32 * h, a_k, desc_kmajor(st + kStreamTile + h * 4096, kStreamChunk, kk), kIdescS,
+          mma_bf16_ts(tmem + kTmS1 + kChainCols * c, a_k, desc_kmajor(st + ro, kStreamChunk, kk), kIdescS, acc);
+          mma_bf16_ts(tmem + kTmS2 + kChainCols * c, a_k, desc_kmajor(st + kStreamTile + ro, kStreamChunk, kk), kIdescS, acc);
+          mma_bf16_ss(tmem + kTmDP + kChainCols * c, a_v, desc_kmajor(st + 2 * kStreamTile + ro, kStreamChunk, kk), kIdescS,
                       acc);
-          mma_bf16_ss(tmem + kTmDP + 32 * h, a_v, desc_kmajor(st + 2 * kStreamTile + h * 4096, kStreamChunk, kk),
-                      kIdescS, acc);
         }
-        tc_commit(bar(kSFull + h));
+        tc_commit(bar(kSFull + c));
       };
-      // Issue order: scores(0); then per step t and half h: [wait P_h(t)] dV, dK of half h;
-      // scores(t+1, h). Scores of step t+1, half h overwrite only half h's columns, which the
-      // accumulations just issued read first (MMAs execute in issue order), so half h of the
-      // next step starts while the elementwise warps still work on the other half.
+      // Issue order: scores(0); then per step t and group c: [wait P_c(t)] dV, dK of group c;
+      // scores(t+1, c). Scores of step t+1 for group c overwrite only group c's columns, which
+      // the accumulations just issued read first (MMAs execute in issue order), so each group
+      // runs its own chain and the chains interleave on the tensor core.
       bool ok = mbar_wait(bar(kFixedFull), 0, abort_flag) && mbar_wait(bar(kAReady), 0, abort_flag) &&
                 mbar_wait(bar(kXFull), 0, abort_flag);
       if (ok) {
         tc_fence_after();
-        issue_scores(0, 0);
-        issue_scores(0, 1);
+        for (int c = 0; c < kChains; ++c) issue_scores(0, c);
       }
       for (int t = 0; ok && t < n_steps; ++t) {
         const int s = t & 1;
@@ -373,24 +384,22 @@ dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         const bool next = t + 1 < n_steps;
         // dV += W^T dO, dK += dS_1^T Q_1 + dS_2^T Q_2 (bf16 operands written over the scores)
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (!(ok = mbar_wait(bar(kPReady + h), t & 1, abort_flag))) break;
+        for (int c = 0; c < kChains; ++c) {
+          if (!(ok = mbar_wait(bar(kPReady + c), t & 1, abort_flag))) break;
           tc_fence_after();
 #pragma unroll
-          for (int k2 = 0; k2 < 2; ++k2) {
-            const int row = 32 * h + 16 * k2;
-            const uint32_t first = (t == 0 && h == 0 && k2 == 0) ? 0u : 1u;
-            mma_bf16_ts(tmem + kTmAcc0, tmem + kTmS1 + packed_col(h, k2), desc_mnmajor(sO, kStreamChunk, row), kIdescAcc,
-                        first);
-            mma_bf16_ts(tmem + kTmAcc1, tmem + kTmS2 + packed_col(h, k2), desc_mnmajor(sQ1, kStreamChunk, row),
-                        kIdescAcc, first);
-            mma_bf16_ts(tmem + kTmAcc1, tmem + kTmDP + packed_col(h, k2), desc_mnmajor(sQ2, kStreamChunk, row),
-                        kIdescAcc, 1u);
+          for (int k2 = 0; k2 < kChainCols / 16; ++k2) {
+            const int row = kChainCols * c + 16 * k2;                 // queries of this K-step
+            const uint32_t col = operand_col(row);                    // their bf16 operands
+            const uint32_t first = (t == 0 && c == 0 && k2 == 0) ? 0u : 1u;
+            mma_bf16_ts(tmem + kTmAcc0, tmem + kTmS1 + col, desc_mnmajor(sO, kStreamChunk, row), kIdescAcc, first);
+            mma_bf16_ts(tmem + kTmAcc1, tmem + kTmS2 + col, desc_mnmajor(sQ1, kStreamChunk, row), kIdescAcc, first);
+            mma_bf16_ts(tmem + kTmAcc1, tmem + kTmDP + col, desc_mnmajor(sQ2, kStreamChunk, row), kIdescAcc, 1u);
           }
           if (next) {
-            if (h == 0 && !(ok = mbar_wait(bar(kXFull + (s ^ 1)), ((t + 1) >> 1) & 1, abort_flag))) break;
+            if (c == 0 && !(ok = mbar_wait(bar(kXFull + (s ^ 1)), ((t + 1) >> 1) & 1, abort_flag))) break;
             tc_fence_after();
-            issue_scores(t + 1, h);
+            issue_scores(t + 1, c);
           }
         }
         if (!ok) break;
@@ -404,7 +413,6 @@ dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   } else {
     // ------------------------------------------------------------------ elementwise
     const int cg = warp >> 2;                 // column group: queries kCols*cg .. of each step
-    const int hc = cg / (kGroups / 2);        // the step half those columns belong to
     const int col0 = kCols * cg;
     const int r = 32 * (warp & 3) + lane;     // key row of the tile == TMEM lane
     const int key = k0 + r;
@@ -420,7 +428,7 @@ dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     for (int t = 0; ok && t < n_steps; ++t) {
       const int s = t & 1;
       const int q0 = (q_first + t % steps_per_pair) * 64;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(kSFull + hc), t & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(kSFull + cg / kGroupsPerChain), t & 1, abort_flag));
       // the stage's stat records came by bulk copy: observe its completion directly (the
       // stage is refilled only after this step's operands have been consumed)
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(kXFull + s), (t >> 1) & 1, abort_flag));
@@ -480,7 +488,7 @@ dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       st_packed(trow + kTmDP + col0, d2_pk);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(kPReady + hc));
+      mbar_arrive(bar(kPReady + cg / kGroupsPerChain));
     }
     if (ok) ok = mbar_wait(bar(kDFull), 0, abort_flag);
     if (__all_sync(0xffffffffu, ok && !*abort_flag)) {
@@ -550,26 +558,26 @@ dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
       // S_1 = Q_1 K^T, S_2 = Q_2 K^T, dP = dO V^T of key block t, keys 32h .. 32h+31
-      auto issue_scores = [&](int t, int h) {
+      auto issue_scores = [&](int t, int c) {
         const uint32_t sK = sbase + kQOffX + (t & 1) * kQStage, sV = sK + kStreamTile;
+        const uint32_t ro = kChainCols * c * 128;  // the chain's first key row in the stream tiles
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint64_t b_k = desc_kmajor(sK + h * 4096, kStreamChunk, kk);
+          const uint64_t b_k = desc_kmajor(sK + ro, kStreamChunk, kk);
           const uint32_t acc = kk > 0 ? 1u : 0u;
-          mma_bf16_ts(tmem + kTmS1 + 32 * h, tmem + kTmA + 8 * kk, b_k, kIdescS, acc);  // Q_1 resident in TMEM
-          mma_bf16_ss(tmem + kTmS2 + 32 * h, desc_kmajor(sbase + kQOffQ2, kFixedChunk, kk), b_k, kIdescS, acc);
-          mma_bf16_ss(tmem + kTmDP + 32 * h, desc_kmajor(sbase + kQOffO, kFixedChunk, kk),
-                      desc_kmajor(sV + h * 4096, kStreamChunk, kk), kIdescS, acc);
+          mma_bf16_ts(tmem + kTmS1 + kChainCols * c, tmem + kTmA + 8 * kk, b_k, kIdescS, acc);  // Q_1 resident in TMEM
+          mma_bf16_ss(tmem + kTmS2 + kChainCols * c, desc_kmajor(sbase + kQOffQ2, kFixedChunk, kk), b_k, kIdescS, acc);
+          mma_bf16_ss(tmem + kTmDP + kChainCols * c, desc_kmajor(sbase + kQOffO, kFixedChunk, kk),
+                      desc_kmajor(sV + ro, kStreamChunk, kk), kIdescS, acc);
         }
-        tc_commit(bar(kSFull + h));
+        tc_commit(bar(kSFull + c));
       };
       // same issue order as the dK/dV kernel
       bool ok = mbar_wait(bar(kFixedFull), 0, abort_flag) && mbar_wait(bar(kAReady), 0, abort_flag) &&
                 mbar_wait(bar(kXFull), 0, abort_flag);
       if (ok) {
         tc_fence_after();
-        issue_scores(0, 0);
-        issue_scores(0, 1);
+        for (int c = 0; c < kChains; ++c) issue_scores(0, c);
       }
       for (int t = 0; ok && t < n_steps; ++t) {
         const int s = t & 1;
@@ -577,21 +585,22 @@ dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         const bool next = t + 1 < n_steps;
         // dQ_1 += dS_1 K, dQ_2 += dS_2 K
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (!(ok = mbar_wait(bar(kPReady + h), t & 1, abort_flag))) break;
+        for (int c = 0; c < kChains; ++c) {
+          if (!(ok = mbar_wait(bar(kPReady + c), t & 1, abort_flag))) break;
           tc_fence_after();
 #pragma unroll
-          for (int k2 = 0; k2 < 2; ++k2) {
-            const int row = 32 * h + 16 * k2;
-            const uint32_t first = (t == 0 && h == 0 && k2 == 0) ? 0u : 1u;
+          for (int k2 = 0; k2 < kChainCols / 16; ++k2) {
+            const int row = kChainCols * c + 16 * k2;                 // keys of this K-step
+            const uint32_t col = operand_col(row);                    // their bf16 operands
+            const uint32_t first = (t == 0 && c == 0 && k2 == 0) ? 0u : 1u;
             const uint64_t b_k = desc_mnmajor(sK, kStreamChunk, row);
-            mma_bf16_ts(tmem + kTmAcc0, tmem + kTmS1 + packed_col(h, k2), b_k, kIdescAcc, first);
-            mma_bf16_ts(tmem + kTmAcc1, tmem + kTmS2 + packed_col(h, k2), b_k, kIdescAcc, first);
+            mma_bf16_ts(tmem + kTmAcc0, tmem + kTmS1 + col, b_k, kIdescAcc, first);
+            mma_bf16_ts(tmem + kTmAcc1, tmem + kTmS2 + col, b_k, kIdescAcc, first);
           }
           if (next) {
-            if (h == 0 && !(ok = mbar_wait(bar(kXFull + (s ^ 1)), ((t + 1) >> 1) & 1, abort_flag))) break;
+            if (c == 0 && !(ok = mbar_wait(bar(kXFull + (s ^ 1)), ((t + 1) >> 1) & 1, abort_flag))) break;
             tc_fence_after();
-            issue_scores(t + 1, h);
+            issue_scores(t + 1, c);
           }
         }
         if (!ok) break;
@@ -604,7 +613,6 @@ dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     }
   } else {
     const int cg = warp >> 2;                 // column group: keys kCols*cg .. of each step
-    const int hc = cg / (kGroups / 2);        // the step half those columns belong to
     const int col0 = kCols * cg;
     const int r = 32 * (warp & 3) + lane;     // query row of the tile == TMEM lane
     const int qi = m0 + r;
@@ -627,7 +635,7 @@ dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     const uint64_t nl1_2 = f2_pack(nl1, nl1), nl2_2 = f2_pack(nl2, nl2), nlam = f2_pack(nlam_s, nlam_s);
     const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
     for (int t = 0; ok && t < n_steps; ++t) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(kSFull + hc), t & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(kSFull + cg / kGroupsPerChain), t & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
       uint32_t s1[kCols], s2[kCols], dp[kCols];
@@ -667,7 +675,7 @@ dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
       st_packed(trow + kTmS2 + col0, d2_pk);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(kPReady + hc));
+      mbar_arrive(bar(kPReady + cg / kGroupsPerChain));
     }
     if (ok) ok = mbar_wait(bar(kDFull), 0, abort_flag);
     if (__all_sync(0xffffffffu, ok && !*abort_flag)) {
