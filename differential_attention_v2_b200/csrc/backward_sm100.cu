@@ -38,7 +38,7 @@ constexpr int kStages = 2;
 // Elementwise warps: 8 (each thread takes 32 columns of a step) or 16 (16 columns). Warps
 // w and w+4k read the same TMEM lanes (w % 4 picks the lane quarter) and split the columns.
 #ifndef DA2_BWD_EW_WARPS
-#define DA2_BWD_EW_WARPS 16
+#define DA2_BWD_EW_WARPS 8
 #endif
 constexpr int kEwWarps = DA2_BWD_EW_WARPS;
 static_assert(kEwWarps == 8 || kEwWarps == 16, "elementwise warps");
