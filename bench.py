@@ -442,6 +442,18 @@ def _decode_seqs(inp, case, n_seqs, seed):
     return byts, time.perf_counter() - t0
 
 
+def _blas_name():
+    """Name of the BLAS library NumPy was built against (the oracle's matrix products)."""
+    try:
+        import numpy as np
+
+        cfg = np.show_config(mode="dicts")
+        blas = cfg.get("Build Dependencies", {}).get("blas", {})
+        return f"{blas.get('name', '?')} {blas.get('version', '')}".strip()
+    except Exception:  # older NumPy: no dict mode
+        return "unknown"
+
+
 def cpu_baseline(seconds=15.0, inputs=None):
     """The float64 oracle on a bounded sample of the same workload, timed on the host."""
     pc = workloads.CONFIGS[PREFILL_CFG]
@@ -457,7 +469,7 @@ def cpu_baseline(seconds=15.0, inputs=None):
     return {"value": round(f / t / 1e12, 6), "unit": "TFLOP/s", "cores": _oracle_threads(), "kind": "oracle",
             "sample": f"{n} random (batch, pair, 128-row tile) units of the B=4 S=4096 prefill "
                       f"({t:.1f} s); decode: 2 full sequences of the B=64 decode ({td:.1f} s)",
-            "decode_gbs": round(b / td / 1e9, 4)}
+            "decode_gbs": round(b / td / 1e9, 4), "blas": _blas_name()}
 
 
 def run_reference(args):
