@@ -635,6 +635,25 @@ def run_workload(args):
         cfg = {"workload": "backward of the causal prefill B=4 S=4096 Hq=64 Hkv=8 D=128 (dQ, dK, dV, dlambda)",
                "train_forward_ms": round(fwd_ms, 4),
                "train_forward_tflops": round(workloads.prefill_flops(case.B, case.S, case.Hq, D) / (fwd_ms * 1e-3) / 1e12, 2)}
+    elif name == "backward_varlen":
+        g = torch.Generator().manual_seed(1010)
+        lens = torch.randint(512, 3585, (8,), generator=g).tolist()
+        T = sum(lens)
+        case = workloads.PrefillCase(B=1, S=T, Hq=64, Hkv=8, D=D, seed=1010)
+        inp = workloads.make_prefill(case)
+        q, k, v, lam = (inp[x][0].to(dev) for x in ("q", "k", "v", "lam"))
+        dout = workloads.make_prefill_grad(case)[0].to(dev)
+        cu = torch.tensor([0] + list(torch.tensor(lens).cumsum(0).tolist()), dtype=torch.int32, device=dev)
+        out, ob, lse = da.prefill_varlen_train(q, k, v, lam, cu, max(lens), stream=stream)
+        ws = torch.empty(da.backward_varlen_workspace_size(len(lens), T, 64), dtype=torch.uint8, device=dev)
+        fn = lambda: da.backward_varlen(q, k, v, lam, ob, lse, dout, cu, max(lens), workspace=ws, stream=stream)
+        flops = 2 * sum(4 * D * 64 * L * (L + 1) // 2 for L in lens)
+        ms = _time_op(fn, args.steps, args.warmup, stream)
+        val = flops / (ms * 1e-3) / 1e12
+        unit, peak, bound = "TFLOP/s", peaks["bf16_tflops"], "tensor"
+        launches = 4
+        cfg = {"workload": f"backward of the packed causal prefill of 8 sequences, lengths U[512,3584] (total {T}), "
+                           "Hq=64 Hkv=8 D=128", "lengths": lens}
     elif name == "lambda_v2":
         T, dm, npair = 16384, 4096, 32
         g = torch.Generator().manual_seed(12)
@@ -676,7 +695,7 @@ def main(argv=None):
     ap.add_argument("--ref-seconds", type=float, default=120.0,
                     help="host-time budget of the whole reference run (warm-up and timed steps)")
     ap.add_argument("--workload", choices=("prefill_long", "decode_needle", "window", "varlen", "paged", "multi",
-                                           "lambda_v2", "backward"), default=None,
+                                           "lambda_v2", "backward", "backward_varlen"), default=None,
                     help="time one other operation alone instead of the default step")
     ap.add_argument("--scaling", choices=("weak", "strong"), default="weak",
                     help="weak: each GPU runs the full per-GPU workload; strong: the heads of one workload "

@@ -32,6 +32,9 @@ _SIGNATURES = {
     "diffattn_v2_prefill_train": (_i, [_vp] * 7 + [_i] * 6 + [_vp]),
     "diffattn_v2_backward_workspace_size": (_sz, [_i, _i, _i]),
     "diffattn_v2_backward": (_i, [_vp] * 11 + [_i] * 6 + [_vp, _sz, _vp]),
+    "diffattn_v2_prefill_varlen_train": (_i, [_vp] * 8 + [_i] * 7 + [_vp]),
+    "diffattn_v2_backward_varlen_workspace_size": (_sz, [_i, _i, _i]),
+    "diffattn_v2_backward_varlen": (_i, [_vp] * 12 + [_i] * 7 + [_vp, _sz, _vp]),
     "diffattn_v2_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "diffattn_v2_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "diffattn_v2_decode_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
@@ -217,6 +220,57 @@ def backward(q, k, v, lam, o_branch, lse, dout, causal=True, dq=None, dk=None, d
                                   _ptr(workspace), workspace.numel() * workspace.element_size(),
                                   _stream(stream, q.device))
     _check(st, "diffattn_v2_backward")
+    return dq, dk, dv, dlam
+
+
+def prefill_varlen_train(q, k, v, lam, cu_seqlens, max_seqlen, out=None, o_branch=None, lse=None, causal=True,
+                         stream=None):
+    """Training forward of packed sequences (layouts of prefill_varlen): returns
+    (out [T,Hq/2,D], o_branch [T,Hq,D], lse [T,Hq])."""
+    for t, n, nd in ((q, "q", 3), (k, "k", 3), (v, "v", 3)):
+        _need(t, n, torch.bfloat16, nd)
+    _need(lam, "lam", torch.float32, 2)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    T, Hq, D = q.shape
+    Hkv = k.shape[1]
+    B = cu_seqlens.numel() - 1
+    out = torch.empty((T, Hq // 2, D), dtype=torch.bfloat16, device=q.device) if out is None else out
+    o_branch = torch.empty((T, Hq, D), dtype=torch.bfloat16, device=q.device) if o_branch is None else o_branch
+    lse = torch.empty((T, Hq), dtype=torch.float32, device=q.device) if lse is None else lse
+    _need(out, "out", torch.bfloat16, 3)
+    _need(o_branch, "o_branch", torch.bfloat16, 3)
+    _need(lse, "lse", torch.float32, 2)
+    st = LIB.diffattn_v2_prefill_varlen_train(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(out), _ptr(o_branch),
+                                              _ptr(lse), _ptr(cu_seqlens), B, int(max_seqlen), T, Hq, Hkv, D,
+                                              1 if causal else 0, _stream(stream, q.device))
+    _check(st, "diffattn_v2_prefill_varlen_train")
+    return out, o_branch, lse
+
+
+def backward_varlen_workspace_size(B, total_tokens, Hq) -> int:
+    return int(LIB.diffattn_v2_backward_varlen_workspace_size(B, total_tokens, Hq))
+
+
+def backward_varlen(q, k, v, lam, o_branch, lse, dout, cu_seqlens, max_seqlen, causal=True, workspace=None,
+                    stream=None):
+    """Gradients of the packed-sequence prefill: returns (dq, dk, dv, dlam) in the packed layouts."""
+    for t, n, nd in ((q, "q", 3), (k, "k", 3), (v, "v", 3), (o_branch, "o_branch", 3), (dout, "dout", 3)):
+        _need(t, n, torch.bfloat16, nd)
+    _need(lam, "lam", torch.float32, 2)
+    _need(lse, "lse", torch.float32, 2)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    T, Hq, D = q.shape
+    Hkv = k.shape[1]
+    B = cu_seqlens.numel() - 1
+    dq, dk, dv, dlam = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(lam)
+    ws_bytes = backward_varlen_workspace_size(B, T, Hq)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+    st = LIB.diffattn_v2_backward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(o_branch), _ptr(lse),
+                                         _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlam), _ptr(cu_seqlens), B,
+                                         int(max_seqlen), T, Hq, Hkv, D, 1 if causal else 0, _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(), _stream(stream, q.device))
+    _check(st, "diffattn_v2_backward_varlen")
     return dq, dk, dv, dlam
 
 

@@ -259,6 +259,69 @@ int diffattn_v2_backward(const void* q, const void* k, const void* v, const floa
       static_cast<float*>(workspace), err, B, S, Hq, Hkv, causal, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int diffattn_v2_prefill_varlen_train(const void* q, const void* k, const void* v, const float* lambda, void* out,
+                                     void* o_branch, float* lse, const int32_t* cu_seqlens, int B, int max_seqlen,
+                                     int total_tokens, int Hq, int Hkv, int D, int causal, da2_stream_t stream) {
+  if (B < 0 || max_seqlen < 0 || total_tokens < 0 || D <= 0 || !heads_ok(Hq, Hkv)) return DA2_ERR_INVALID;
+  if (causal != 0 && causal != 1) return DA2_ERR_INVALID;
+  if (B == 0 || max_seqlen == 0 || total_tokens == 0) return DA2_OK;
+  const void* ptrs[] = {q, k, v, lambda, out, o_branch, lse, cu_seqlens};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return DA2_ERR_INVALID;
+  if (D != 128) return DA2_ERR_UNSUPPORTED;
+  if ((max_seqlen + 127) / 128 > 65535) return DA2_ERR_UNSUPPORTED;
+  int* err = nullptr;
+  cudaError_t e = device_error_ptr(&err);
+  if (e != cudaSuccess) return DA2_ERR_CUDA;
+  CUtensorMap tq, tk, tv;  // the packed tokens as one batch of total_tokens rows
+  if (encode_bshd(&tq, q, D, Hq, total_tokens, 1, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  if (encode_bshd(&tk, k, D, Hkv, total_tokens, 1, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  if (encode_bshd(&tv, v, D, Hkv, total_tokens, 1, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  e = da2::launch_prefill(tq, tk, tv, lambda, static_cast<__nv_bfloat16*>(out), err, B, max_seqlen, Hq, Hkv, causal,
+                          0, cu_seqlens, reinterpret_cast<cudaStream_t>(stream), static_cast<__nv_bfloat16*>(o_branch),
+                          lse);
+  return status_of(e);
+}
+
+size_t diffattn_v2_backward_varlen_workspace_size(int B, int total_tokens, int Hq) {
+  if (B <= 0 || total_tokens <= 0 || Hq <= 0 || (Hq % 2) != 0) return 0;
+  return da2::backward_varlen_workspace_bytes(B, total_tokens, Hq);
+}
+
+int diffattn_v2_backward_varlen(const void* q, const void* k, const void* v, const float* lambda,
+                                const void* o_branch, const float* lse, const void* dout, void* dq, void* dk,
+                                void* dv, float* dlambda, const int32_t* cu_seqlens, int B, int max_seqlen,
+                                int total_tokens, int Hq, int Hkv, int D, int causal, void* workspace,
+                                size_t workspace_bytes, da2_stream_t stream) {
+  if (B < 0 || max_seqlen < 0 || total_tokens < 0 || D <= 0 || !heads_ok(Hq, Hkv)) return DA2_ERR_INVALID;
+  if (causal != 0 && causal != 1) return DA2_ERR_INVALID;
+  if (B == 0 || max_seqlen == 0 || total_tokens == 0) return DA2_OK;
+  const void* ptrs[] = {q, k, v, lambda, o_branch, lse, dout, dq, dk, dv, dlambda, cu_seqlens, workspace};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return DA2_ERR_INVALID;
+  if (workspace_bytes < diffattn_v2_backward_varlen_workspace_size(B, total_tokens, Hq)) return DA2_ERR_INVALID;
+  if (D != 128) return DA2_ERR_UNSUPPORTED;
+  // grid limits: 128-row tiles on grid y; the preprocess runs 4 (row, pair) warps per CTA
+  if ((max_seqlen + 127) / 128 > 65535) return DA2_ERR_UNSUPPORTED;
+  if ((static_cast<long long>(total_tokens) + 128LL * B + 128) * (Hq / 2) > 4LL * 2147483647LL) return DA2_ERR_UNSUPPORTED;
+  int* err = nullptr;
+  if (device_error_ptr(&err) != cudaSuccess) return DA2_ERR_CUDA;
+  const int T = total_tokens;
+  CUtensorMap q64, q128, o64, o128, k64, k128, v64, v128;
+  if (encode_bshd(&q64, q, D, Hq, T, 1, 64, 64) != cudaSuccess || encode_bshd(&q128, q, D, Hq, T, 1, 64, 128) != cudaSuccess ||
+      encode_bshd(&o64, dout, D, Hq / 2, T, 1, 64, 64) != cudaSuccess ||
+      encode_bshd(&o128, dout, D, Hq / 2, T, 1, 64, 128) != cudaSuccess ||
+      encode_bshd(&k64, k, D, Hkv, T, 1, 64, 64) != cudaSuccess || encode_bshd(&k128, k, D, Hkv, T, 1, 64, 128) != cudaSuccess ||
+      encode_bshd(&v64, v, D, Hkv, T, 1, 64, 64) != cudaSuccess || encode_bshd(&v128, v, D, Hkv, T, 1, 64, 128) != cudaSuccess)
+    return DA2_ERR_CUDA;
+  using bf = __nv_bfloat16;
+  return status_of(da2::launch_backward_sm100(
+      q64, q128, o64, o128, k64, k128, v64, v128, lambda, static_cast<const bf*>(o_branch), lse,
+      static_cast<const bf*>(dout), static_cast<bf*>(dq), static_cast<bf*>(dk), static_cast<bf*>(dv), dlambda,
+      static_cast<float*>(workspace), err, B, max_seqlen, Hq, Hkv, causal, reinterpret_cast<cudaStream_t>(stream),
+      cu_seqlens, T));
+}
+
 size_t diffattn_v2_decode_workspace_size(int B, int Smax, int Hq, int Hkv, int D) {
   if (B <= 0 || Smax <= 0 || D <= 0 || !heads_ok(Hq, Hkv)) return 0;
   int split_len = 0, nsplit = 0;

@@ -92,6 +92,8 @@ struct Params {
   int* err;
   int B, S, S_pad, Hq, Hkv, causal;
   int n_tiles;               // 128-row tiles
+  const int* cu_seqlens;     // packed sequences: sequence b is rows cu[b] .. cu[b+1]-1 (null: [B,S])
+  const int* pad_off;        // packed sequences: first row of sequence b in the row terms (128-aligned)
   float scale, scale_log2;
 };
 
@@ -138,6 +140,69 @@ preprocess_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
     else if (lane < 4) t = -e[lane - 2];
     else t = -__ldg(lambda + row * n_pairs + p);
     stats[stat_index(bp, S_pad, i, lane)] = t;
+  }
+  if (lane == 0) dlam[row * n_pairs + p] = -e[1];
+}
+
+// Packed sequences: sequence b's row terms start at pad_off[b], each sequence padded to a
+// multiple of 128 rows (pad_off[B] = the padded total). One thread: the scan is over B.
+__global__ void pad_offsets_kernel(const int* __restrict__ cu, int* __restrict__ pad_off, int B) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    int acc = 0;
+    for (int b = 0; b < B; ++b) {
+      pad_off[b] = acc;
+      acc += (cu[b + 1] - cu[b] + kRowPad - 1) / kRowPad * kRowPad;
+    }
+    pad_off[B] = acc;
+  }
+}
+
+// The preprocess for packed sequences: warp w is padded row pr of pair p (rows of all pairs
+// laid out as one batch of S_pad rows). Rows past a sequence's end, and past the padded
+// total, get -lse = -inf.
+__global__ void __launch_bounds__(128)
+preprocess_varlen_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ o_branch,
+                         const float* __restrict__ lse, const float* __restrict__ lambda, float* __restrict__ stats,
+                         float* __restrict__ dlam, const int* __restrict__ cu, const int* __restrict__ pad_off, int B,
+                         int S_pad, int n_pairs) {
+  const long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= static_cast<long long>(S_pad) * n_pairs) return;
+  const int pr = static_cast<int>(w % S_pad);
+  const int p = static_cast<int>(w / S_pad);
+  // the sequence whose padded rows hold pr: last b with pad_off[b] <= pr (b = B: past the end)
+  int lo = 0, hi = B;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(pad_off + mid) <= pr) lo = mid; else hi = mid - 1;
+  }
+  const int b = lo;
+  const int i = pr - (b < B ? __ldg(pad_off + b) : 0);
+  if (b >= B || i >= __ldg(cu + b + 1) - __ldg(cu + b)) {
+    if (lane < kStatArrays) stats[stat_index(p, S_pad, pr, lane)] = lane < 2 ? -INFINITY : 0.f;
+    return;
+  }
+  const long long row = static_cast<long long>(__ldg(cu + b)) + i;
+  const uint2 g = __ldg(reinterpret_cast<const uint2*>(dout + (row * n_pairs + p) * HD) + lane);
+  const float2 g0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&g.x));
+  const float2 g1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&g.y));
+  float e[2];
+#pragma unroll
+  for (int br = 0; br < 2; ++br) {
+    const uint2 o = __ldg(reinterpret_cast<const uint2*>(o_branch + (row * (2 * n_pairs) + 2 * p + br) * HD) + lane);
+    const float2 o0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o.x));
+    const float2 o1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o.y));
+    float v = g0.x * o0.x + g0.y * o0.y + g1.x * o1.x + g1.y * o1.y;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    e[br] = v;
+  }
+  if (lane < kStatArrays) {
+    float t;
+    if (lane < 2) t = -__ldg(lse + row * (2 * n_pairs) + 2 * p + lane);
+    else if (lane < 4) t = -e[lane - 2];
+    else t = -__ldg(lambda + row * n_pairs + p);
+    stats[stat_index(p, S_pad, pr, lane)] = t;
   }
   if (lane == 0) dlam[row * n_pairs + p] = -e[1];
 }
@@ -291,6 +356,7 @@ __device__ __forceinline__ void tile_to_tmem(uint32_t tile, uint32_t trow, int r
 }
 
 // --------------------------------------------------------------------------- dK / dV
+template <bool kVarlen>
 __global__ void __launch_bounds__(kThreads, 1)
 dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
            const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const Params p) {
@@ -308,7 +374,21 @@ dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   const int b = static_cast<int>(blockIdx.x) / p.Hkv;
   const int tile = static_cast<int>(blockIdx.y);  // tile 0 (most query blocks when causal) first
   const int k0 = tile * 128;
-  const int nq = (p.S + 63) / 64;                   // 64-row query blocks
+  // sequence extent: a [B,S] batch, or packed sequences whose tensors are one [1,T] batch
+  // (tok0: the sequence's first row; tb: the batch coordinate of the tensor maps; sb, srow0:
+  // where the sequence's row terms start)
+  int S = p.S, tok0 = 0, tb = b, srow0 = 0;
+  size_t sb = static_cast<size_t>(b) * n_pairs;
+  if (kVarlen) {
+    tok0 = __ldg(p.cu_seqlens + b);
+    S = __ldg(p.cu_seqlens + b + 1) - tok0;
+    tb = 0;
+    sb = 0;
+    srow0 = __ldg(p.pad_off + b);
+  }
+  if (k0 >= S) return;  // uniform over the CTA: the key tile lies past the sequence's end
+  const size_t row_base = kVarlen ? static_cast<size_t>(tok0) : static_cast<size_t>(b) * p.S;
+  const int nq = (S + 63) / 64;                     // 64-row query blocks
   const int q_first = p.causal ? k0 / 64 : 0;
   const int steps_per_pair = nq - q_first;
   const int n_steps = gpairs * steps_per_pair;
@@ -322,8 +402,8 @@ dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       tma_prefetch_desc(&tmO);
       mbar_arrive_expect_tx(bar(kFixedFull), 2 * kFixedTile);
       for (int c = 0; c < 2; ++c) {
-        tma_load_4d(sbase + kKvOffK + c * kFixedChunk, &tmK, bar(kFixedFull), c * 64, g, k0, b);
-        tma_load_4d(sbase + kKvOffV + c * kFixedChunk, &tmV, bar(kFixedFull), c * 64, g, k0, b);
+        tma_load_4d(sbase + kKvOffK + c * kFixedChunk, &tmK, bar(kFixedFull), c * 64, g, tok0 + k0, tb);
+        tma_load_4d(sbase + kKvOffV + c * kFixedChunk, &tmV, bar(kFixedFull), c * 64, g, tok0 + k0, tb);
       }
       int issued = 0;
       for (int t = 0; t < n_steps; ++t) {
@@ -334,11 +414,11 @@ dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         const uint32_t st = sbase + kKvOffX + s * kKvStage;
         mbar_arrive_expect_tx(bar(kXFull + s), 3 * kStreamTile + kStatBytes);
         for (int c = 0; c < 2; ++c) {
-          tma_load_4d(st + c * kStreamChunk, &tmQ, bar(kXFull + s), c * 64, 2 * pair, q0, b);
-          tma_load_4d(st + kStreamTile + c * kStreamChunk, &tmQ, bar(kXFull + s), c * 64, 2 * pair + 1, q0, b);
-          tma_load_4d(st + 2 * kStreamTile + c * kStreamChunk, &tmO, bar(kXFull + s), c * 64, pair, q0, b);
+          tma_load_4d(st + c * kStreamChunk, &tmQ, bar(kXFull + s), c * 64, 2 * pair, tok0 + q0, tb);
+          tma_load_4d(st + kStreamTile + c * kStreamChunk, &tmQ, bar(kXFull + s), c * 64, 2 * pair + 1, tok0 + q0, tb);
+          tma_load_4d(st + 2 * kStreamTile + c * kStreamChunk, &tmO, bar(kXFull + s), c * 64, pair, tok0 + q0, tb);
         }
-        bulk_load(st + 3 * kStreamTile, p.stats + stat_index(static_cast<size_t>(b) * n_pairs + pair, p.S_pad, q0, 0),
+        bulk_load(st + 3 * kStreamTile, p.stats + stat_index(sb + pair, p.S_pad, srow0 + q0, 0),
                   kStatBytes, bar(kXFull + s));
         issued = t + 1;
       }
@@ -493,9 +573,9 @@ dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     if (ok) ok = mbar_wait(bar(kDFull), 0, abort_flag);
     if (__all_sync(0xffffffffu, ok && !*abort_flag)) {
       tc_fence_after();
-      const bool valid = key < p.S;
+      const bool valid = key < S;
       const int d0 = (128 / kGroups) * cg;
-      const size_t off = ((static_cast<size_t>(b) * p.S + (valid ? key : 0)) * p.Hkv + g) * HD + d0;
+      const size_t off = ((row_base + (valid ? key : 0)) * p.Hkv + g) * HD + d0;
       store_row(trow + kTmAcc0 + d0, p.dv + off, 1.f, valid);
       store_row(trow + kTmAcc1 + d0, p.dk + off, p.scale, valid);
     }
@@ -504,6 +584,7 @@ dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 }
 
 // --------------------------------------------------------------------------------- dQ
+template <bool kVarlen>
 __global__ void __launch_bounds__(kThreads, 1)
 dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
          const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const Params p) {
@@ -522,7 +603,19 @@ dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
   const int g = (2 * pair) / group;
   const int tile = p.causal ? p.n_tiles - 1 - static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.y);
   const int m0 = tile * 128;
-  const int nk = (p.S + 63) / 64;
+  // sequence extent, as in the dK/dV kernel
+  int S = p.S, tok0 = 0, tb = b, srow0 = 0;
+  size_t sb = static_cast<size_t>(b) * n_pairs;
+  if (kVarlen) {
+    tok0 = __ldg(p.cu_seqlens + b);
+    S = __ldg(p.cu_seqlens + b + 1) - tok0;
+    tb = 0;
+    sb = 0;
+    srow0 = __ldg(p.pad_off + b);
+  }
+  if (m0 >= S) return;  // uniform over the CTA: the row tile lies past the sequence's end
+  const size_t row_base = kVarlen ? static_cast<size_t>(tok0) : static_cast<size_t>(b) * p.S;
+  const int nk = (S + 63) / 64;
   const int n_steps = p.causal ? min(nk, (m0 + 128) / 64) : nk;
 
   const uint32_t tmem = setup(bar0, tmem_slot, abort_flag, warp);
@@ -533,9 +626,9 @@ dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
       tma_prefetch_desc(&tmV);
       mbar_arrive_expect_tx(bar(kFixedFull), 3 * kFixedTile);
       for (int c = 0; c < 2; ++c) {
-        tma_load_4d(sbase + kQOffQ1 + c * kFixedChunk, &tmQ, bar(kFixedFull), c * 64, 2 * pair, m0, b);
-        tma_load_4d(sbase + kQOffQ2 + c * kFixedChunk, &tmQ, bar(kFixedFull), c * 64, 2 * pair + 1, m0, b);
-        tma_load_4d(sbase + kQOffO + c * kFixedChunk, &tmO, bar(kFixedFull), c * 64, pair, m0, b);
+        tma_load_4d(sbase + kQOffQ1 + c * kFixedChunk, &tmQ, bar(kFixedFull), c * 64, 2 * pair, tok0 + m0, tb);
+        tma_load_4d(sbase + kQOffQ2 + c * kFixedChunk, &tmQ, bar(kFixedFull), c * 64, 2 * pair + 1, tok0 + m0, tb);
+        tma_load_4d(sbase + kQOffO + c * kFixedChunk, &tmO, bar(kFixedFull), c * 64, pair, tok0 + m0, tb);
       }
       int issued = 0;
       for (int t = 0; t < n_steps; ++t) {
@@ -544,8 +637,8 @@ dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         const uint32_t st = sbase + kQOffX + s * kQStage;
         mbar_arrive_expect_tx(bar(kXFull + s), 2 * kStreamTile);
         for (int c = 0; c < 2; ++c) {
-          tma_load_4d(st + c * kStreamChunk, &tmK, bar(kXFull + s), c * 64, g, 64 * t, b);
-          tma_load_4d(st + kStreamTile + c * kStreamChunk, &tmV, bar(kXFull + s), c * 64, g, 64 * t, b);
+          tma_load_4d(st + c * kStreamChunk, &tmK, bar(kXFull + s), c * 64, g, tok0 + 64 * t, tb);
+          tma_load_4d(st + kStreamTile + c * kStreamChunk, &tmV, bar(kXFull + s), c * 64, g, tok0 + 64 * t, tb);
         }
         issued = t + 1;
       }
@@ -626,12 +719,13 @@ dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
       mbar_arrive(bar(kAReady));
     }
     // this row's terms (rows past S carry -lse = -inf: probabilities 0)
-    const size_t bp = static_cast<size_t>(b) * n_pairs + pair;
-    const float nl1 = __ldg(p.stats + stat_index(bp, p.S_pad, qi, 0));
-    const float nl2 = __ldg(p.stats + stat_index(bp, p.S_pad, qi, 1));
-    const uint64_t ne1 = f2_pack(__ldg(p.stats + stat_index(bp, p.S_pad, qi, 2)), __ldg(p.stats + stat_index(bp, p.S_pad, qi, 2)));
-    const uint64_t ne2 = f2_pack(__ldg(p.stats + stat_index(bp, p.S_pad, qi, 3)), __ldg(p.stats + stat_index(bp, p.S_pad, qi, 3)));
-    const float nlam_s = __ldg(p.stats + stat_index(bp, p.S_pad, qi, 4));
+    const size_t bp = sb + pair;
+    const int sr = srow0 + qi;  // this row in the row terms (past the sequence: -lse = -inf)
+    const float nl1 = __ldg(p.stats + stat_index(bp, p.S_pad, sr, 0));
+    const float nl2 = __ldg(p.stats + stat_index(bp, p.S_pad, sr, 1));
+    const uint64_t ne1 = f2_pack(__ldg(p.stats + stat_index(bp, p.S_pad, sr, 2)), __ldg(p.stats + stat_index(bp, p.S_pad, sr, 2)));
+    const uint64_t ne2 = f2_pack(__ldg(p.stats + stat_index(bp, p.S_pad, sr, 3)), __ldg(p.stats + stat_index(bp, p.S_pad, sr, 3)));
+    const float nlam_s = __ldg(p.stats + stat_index(bp, p.S_pad, sr, 4));
     const uint64_t nl1_2 = f2_pack(nl1, nl1), nl2_2 = f2_pack(nl2, nl2), nlam = f2_pack(nlam_s, nlam_s);
     const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
     for (int t = 0; ok && t < n_steps; ++t) {
@@ -647,8 +741,8 @@ dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
       ld_cols_wait(dp);
       const int kbase = 64 * t + col0;
       // tile-uniform: keys past the query (causal diagonal) or past S (ragged last block)
-      const bool masked = (p.causal && 64 * t + 63 > m0) || (64 * t + 64 > p.S);
-      const int lim = p.causal ? min(qi, p.S - 1) : p.S - 1;
+      const bool masked = (p.causal && 64 * t + 63 > m0) || (64 * t + 64 > S);
+      const int lim = p.causal ? min(qi, S - 1) : S - 1;
       uint32_t d1_pk[kCols / 2], d2_pk[kCols / 2];
 #pragma unroll
       for (int c = 0; c < kCols; c += 2) {
@@ -680,9 +774,9 @@ dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     if (ok) ok = mbar_wait(bar(kDFull), 0, abort_flag);
     if (__all_sync(0xffffffffu, ok && !*abort_flag)) {
       tc_fence_after();
-      const bool valid = qi < p.S;
+      const bool valid = qi < S;
       const int d0 = (128 / kGroups) * cg;
-      const size_t off = ((static_cast<size_t>(b) * p.S + (valid ? qi : 0)) * p.Hq + 2 * pair) * HD + d0;
+      const size_t off = ((row_base + (valid ? qi : 0)) * p.Hq + 2 * pair) * HD + d0;
       store_row(trow + kTmAcc0 + d0, p.dq + off, p.scale, valid);
       store_row(trow + kTmAcc1 + d0, p.dq + off + HD, p.scale, valid);
     }
@@ -697,45 +791,77 @@ size_t backward_stats_bytes(int B, int S, int Hq) {
   return static_cast<size_t>(B) * (Hq / 2) * s_pad * bwd_tc::kStatArrays * sizeof(float);
 }
 
+// Packed sequences: rows of the row terms for T tokens in B sequences, each padded to 128.
+static size_t varlen_stat_rows(int B, int T) {
+  return (static_cast<size_t>(T) + static_cast<size_t>(bwd_tc::kRowPad) * B + bwd_tc::kRowPad - 1) /
+         bwd_tc::kRowPad * bwd_tc::kRowPad;
+}
+
+size_t backward_varlen_workspace_bytes(int B, int T, int Hq) {
+  const size_t stats = static_cast<size_t>(Hq / 2) * varlen_stat_rows(B, T) * bwd_tc::kStatArrays * sizeof(float);
+  return stats + (static_cast<size_t>(B) + 1 + 3) / 4 * 16;  // + the B+1 padded offsets
+}
+
 cudaError_t launch_backward_sm100(const CUtensorMap& tmQ64, const CUtensorMap& tmQ128, const CUtensorMap& tmO64,
                                   const CUtensorMap& tmO128, const CUtensorMap& tmK64, const CUtensorMap& tmK128,
                                   const CUtensorMap& tmV64, const CUtensorMap& tmV128, const float* lambda,
                                   const __nv_bfloat16* o_branch, const float* lse, const __nv_bfloat16* dout,
                                   __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv, float* dlambda,
-                                  float* stats, int* err, int B, int S, int Hq, int Hkv, int causal,
-                                  cudaStream_t stream) {
+                                  float* workspace, int* err, int B, int S, int Hq, int Hkv, int causal,
+                                  cudaStream_t stream, const int32_t* cu_seqlens, int total_tokens) {
   using namespace bwd_tc;
   const int n_pairs = Hq / 2;
-  const int S_pad = (S + kRowPad - 1) / kRowPad * kRowPad;
-  const long long warps = static_cast<long long>(B) * S_pad * n_pairs;
-  preprocess_kernel<<<static_cast<unsigned>((warps + 3) / 4), 128, 0, stream>>>(dout, o_branch, lse, lambda, stats,
-                                                                                  dlambda, B, S, S_pad, n_pairs);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
   Params p;
-  p.stats = stats;
+  cudaError_t e;
+  if (cu_seqlens) {
+    // S is the longest sequence; the row terms of all sequences form one padded batch
+    const int S_pad = static_cast<int>(varlen_stat_rows(B, total_tokens));
+    int* pad_off = reinterpret_cast<int*>(workspace + static_cast<size_t>(n_pairs) * S_pad * kStatArrays);
+    pad_offsets_kernel<<<1, 32, 0, stream>>>(cu_seqlens, pad_off, B);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const long long warps = static_cast<long long>(S_pad) * n_pairs;
+    preprocess_varlen_kernel<<<static_cast<unsigned>((warps + 3) / 4), 128, 0, stream>>>(
+        dout, o_branch, lse, lambda, workspace, dlambda, cu_seqlens, pad_off, B, S_pad, n_pairs);
+    p.S_pad = S_pad;
+    p.pad_off = pad_off;
+  } else {
+    const int S_pad = (S + kRowPad - 1) / kRowPad * kRowPad;
+    const long long warps = static_cast<long long>(B) * S_pad * n_pairs;
+    preprocess_kernel<<<static_cast<unsigned>((warps + 3) / 4), 128, 0, stream>>>(dout, o_branch, lse, lambda,
+                                                                                    workspace, dlambda, B, S, S_pad,
+                                                                                    n_pairs);
+    p.S_pad = S_pad;
+    p.pad_off = nullptr;
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  p.stats = workspace;
   p.dq = dq;
   p.dk = dk;
   p.dv = dv;
   p.err = err;
   p.B = B;
   p.S = S;
-  p.S_pad = S_pad;
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.causal = causal;
-  p.n_tiles = S_pad / 128;
+  p.cu_seqlens = cu_seqlens;
+  p.n_tiles = (S + 127) / 128;
   p.scale = 1.f / sqrtf(static_cast<float>(HD));
   p.scale_log2 = 1.4426950408889634f * p.scale;
-  e = cudaFuncSetAttribute(dkdv_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmem);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(dq_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmem);
-  if (e != cudaSuccess) return e;
-  dkdv_sm100<<<dim3(B * Hkv, p.n_tiles), kThreads, kKvSmem, stream>>>(tmQ64, tmO64, tmK128, tmV128, p);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  dq_sm100<<<dim3(B * n_pairs, p.n_tiles), kThreads, kQSmem, stream>>>(tmQ128, tmO128, tmK64, tmV64, p);
-  return cudaGetLastError();
+  auto run = [&](auto kdkdv, auto kdq) {
+    cudaError_t r = cudaFuncSetAttribute(kdkdv, cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmem);
+    if (r != cudaSuccess) return r;
+    r = cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmem);
+    if (r != cudaSuccess) return r;
+    kdkdv<<<dim3(B * Hkv, p.n_tiles), kThreads, kKvSmem, stream>>>(tmQ64, tmO64, tmK128, tmV128, p);
+    r = cudaGetLastError();
+    if (r != cudaSuccess) return r;
+    kdq<<<dim3(B * n_pairs, p.n_tiles), kThreads, kQSmem, stream>>>(tmQ128, tmO128, tmK64, tmV64, p);
+    return cudaGetLastError();
+  };
+  return cu_seqlens ? run(dkdv_sm100<true>, dq_sm100<true>) : run(dkdv_sm100<false>, dq_sm100<false>);
 }
 
 }  // namespace da2

@@ -170,6 +170,31 @@ DA2_API int diffattn_v2_backward(const void* q, const void* k, const void* v, co
                                  da2_stream_t stream);
 
 /*
+ * Training forward and backward for B sequences packed along the token axis (the layout of
+ * diffattn_v2_prefill_varlen; pretraining on packed documents). Every sequence is an
+ * independent prefill, so its gradients are those of its own prefill:
+ *   q bf16 [T,Hq,D]  k, v bf16 [T,Hkv,D]  lambda fp32 [T,Hq/2]  out, dout bf16 [T,Hq/2,D]
+ *   o_branch bf16 [T,Hq,D]  lse fp32 [T,Hq]   (written by the training forward, read back)
+ *   dq bf16 [T,Hq,D]  dk, dv bf16 [T,Hkv,D]  dlambda fp32 [T,Hq/2]   (overwritten)
+ *   cu_seqlens int32 [B+1] (device): sequence b is tokens cu_seqlens[b] .. cu_seqlens[b+1]-1;
+ *   max_seqlen >= the longest sequence; total_tokens = T.
+ * The backward's workspace: diffattn_v2_backward_varlen_workspace_size(B, T, Hq) bytes of
+ * device memory (the row terms of every sequence padded to 128 rows, and B+1 offsets);
+ * sizes depend on host-known B and T only, so no host synchronisation is needed. Same
+ * checks, semantics and determinism as the [B,S] calls; D == 128.
+ */
+DA2_API int diffattn_v2_prefill_varlen_train(const void* q, const void* k, const void* v, const float* lambda,
+                                             void* out, void* o_branch, float* lse, const int32_t* cu_seqlens,
+                                             int B, int max_seqlen, int total_tokens, int Hq, int Hkv, int D,
+                                             int causal, da2_stream_t stream);
+DA2_API size_t diffattn_v2_backward_varlen_workspace_size(int B, int total_tokens, int Hq);
+DA2_API int diffattn_v2_backward_varlen(const void* q, const void* k, const void* v, const float* lambda,
+                                        const void* o_branch, const float* lse, const void* dout, void* dq,
+                                        void* dk, void* dv, float* dlambda, const int32_t* cu_seqlens, int B,
+                                        int max_seqlen, int total_tokens, int Hq, int Hkv, int D, int causal,
+                                        void* workspace, size_t workspace_bytes, da2_stream_t stream);
+
+/*
  * Workspace (bytes) that diffattn_v2_decode needs for these sizes: the per-split partial
  * results (running max, running sum and unnormalised output of each head), fp32. Returns 0
  * for invalid sizes. The workspace holds no state between calls.

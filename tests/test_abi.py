@@ -205,3 +205,22 @@ def test_backward_host_checks(lib):
     assert lib.diffattn_v2_backward(*ok[:16], 2, *ok[17:]) == -1                   # causal not 0/1
     assert lib.diffattn_v2_backward(*ok[:15], 64, *ok[16:]) == -2                  # D = 64
     assert lib.diffattn_v2_backward(*ok[:11], 0, *ok[12:]) == 0                    # B = 0
+
+
+def test_varlen_training_host_checks(lib):
+    OB, LS, CU = P + 32768, P + 40960, P + 49152
+    args = (Q, K, V, L, O, OB, LS, CU, 2, 256, 300, 8, 2, 128, 1, None)
+    assert lib.diffattn_v2_prefill_varlen_train(*args[:7], None, *args[8:]) == -1   # no cu_seqlens
+    assert lib.diffattn_v2_prefill_varlen_train(*args[:11], 6, *args[12:]) == -1    # pair straddles KV heads
+    assert lib.diffattn_v2_prefill_varlen_train(*args[:13], 64, *args[14:]) == -2   # D = 64
+    assert lib.diffattn_v2_prefill_varlen_train(*args[:8], 0, *args[9:]) == 0       # no sequences
+    ws = lib.diffattn_v2_backward_varlen_workspace_size(3, 500, 8)
+    assert ws >= 4 * (500 + 3 * 128) * 20                                            # padded row terms
+    assert lib.diffattn_v2_backward_varlen_workspace_size(0, 500, 8) == 0
+    DO, DQ, DK, DV, DL, W = (P + 65536 + 32768 * i for i in range(6))
+    ok = (Q, K, V, L, OB, LS, DO, DQ, DK, DV, DL, CU, 3, 256, 500, 8, 2, 128, 1, W, ws, None)
+    assert lib.diffattn_v2_backward_varlen(*ok[:20], ws - 16, None) == -1            # short workspace
+    assert lib.diffattn_v2_backward_varlen(*ok[:11], None, *ok[12:]) == -1           # no cu_seqlens
+    assert lib.diffattn_v2_backward_varlen(*ok[:18], 2, *ok[19:]) == -1              # causal not 0/1
+    assert lib.diffattn_v2_backward_varlen(*ok[:17], 64, *ok[18:]) == -2             # D = 64
+    assert lib.diffattn_v2_backward_varlen(*ok[:12], 0, *ok[13:]) == 0               # B = 0

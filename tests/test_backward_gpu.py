@@ -112,3 +112,57 @@ def test_backward_full_size_one_group(da):
           "dout": inp["dout"][b:b + 1, :, pairs]}
     got = (dq[b:b + 1, :, heads], dk[b:b + 1, :, g:g + 1], dv[b:b + 1, :, g:g + 1], dlam[b:b + 1, :, pairs])
     _check_grads(got, sl, True, "c2 slice b=3 g=5")
+
+
+def _packed(lens, Hq, Hkv, seed):
+    T = sum(lens)
+    case = workloads.PrefillCase(B=1, S=max(T, 1), Hq=Hq, Hkv=Hkv, D=128, seed=seed)
+    inp = workloads.make_prefill(case)
+    inp["dout"] = workloads.make_prefill_grad(case)
+    packed = {k: v[0, :T].contiguous() for k, v in inp.items()}
+    cu = [0]
+    for L in lens:
+        cu.append(cu[-1] + L)
+    return packed, cu
+
+
+def _gpu_varlen(da, inp, cu, causal):
+    d = {k: v.cuda() for k, v in inp.items()}
+    cu_t = torch.tensor(cu, dtype=torch.int32, device="cuda")
+    mx = max(b - a for a, b in zip(cu[:-1], cu[1:]))
+    out, ob, lse = da.prefill_varlen_train(d["q"], d["k"], d["v"], d["lam"], cu_t, mx, causal=causal)
+    grads = da.backward_varlen(d["q"], d["k"], d["v"], d["lam"], ob, lse, d["dout"], cu_t, mx, causal=causal)
+    torch.cuda.synchronize()
+    assert da.device_error() == 0
+    return (out, ob, lse), grads
+
+
+@pytest.mark.parametrize("lens,Hq,Hkv,causal", [
+    ([300, 1, 0, 200, 129], 8, 2, True),   # ragged, a single token, an empty sequence, tile + 1
+    ([64, 65, 127, 128], 16, 2, True),     # offsets that are not multiples of 64 or 128
+    ([513, 37], 4, 2, True),               # several tiles, group of 2
+    ([300, 90, 200], 8, 1, False),         # full attention inside each sequence, group of 8
+])
+def test_backward_varlen_matches_oracle(da, lens, Hq, Hkv, causal):
+    inp, cu = _packed(lens, Hq, Hkv, seed=61 + len(lens) + Hq)
+    (out, ob, lse), grads = _gpu_varlen(da, inp, cu, causal)
+    d = {k: v.cuda() for k, v in inp.items()}
+    cu_t = torch.tensor(cu, dtype=torch.int32, device="cuda")
+    mx = max(lens)
+    assert torch.equal(out, da.prefill_varlen(d["q"], d["k"], d["v"], d["lam"], cu_t, mx, causal=causal))
+    ref = ora.prefill_backward_varlen(inp["q"], inp["k"], inp["v"], inp["lam"], inp["dout"], cu, causal=causal)
+    for g, r, name in zip(grads, ref, ("dq", "dk", "dv", "dlam")):
+        grad_close(g, r, f"varlen {lens} causal={causal} {name}")
+
+
+def test_backward_varlen_equal_lengths_equals_batched(da):
+    """Packed sequences of equal (ragged) length give bit-identical gradients to the batch."""
+    B, S, Hq, Hkv = 3, 300, 8, 2
+    case = workloads.PrefillCase(B=B, S=S, Hq=Hq, Hkv=Hkv, D=128, seed=67)
+    inp = workloads.make_prefill(case)
+    inp["dout"] = workloads.make_prefill_grad(case)
+    _, g_batched = _gpu_grads(da, inp, True)
+    packed = {k: v.reshape((B * S,) + v.shape[2:]).contiguous() for k, v in inp.items()}
+    _, g_packed = _gpu_varlen(da, packed, [0, S, 2 * S, 3 * S], True)
+    for a, b in zip(g_batched, g_packed):
+        assert torch.equal(a.reshape(b.shape), b)

@@ -394,6 +394,43 @@ def pin_branches_recombine_and_normalise():
     return bool(ok)
 
 
+def pin_backward_varlen_finite_differences():
+    """Central differences of <dout, prefill_varlen(.)> for packed sequences of lengths
+    3, 0, 5: entries inside a sequence match, and a key of the first sequence has exactly
+    zero gradient through the second."""
+    rng = np.random.default_rng(24)
+    T, Hq, Hkv, D = 8, 4, 2, 3
+    q, k, v = (rng.standard_normal((T, h, D)) for h in (Hq, Hkv, Hkv))
+    lam = rng.uniform(0.2, 0.9, (T, Hq // 2))
+    dout = rng.standard_normal((T, Hq // 2, D))
+    cu = [0, 3, 3, 8]
+    grads = ora.prefill_backward_varlen(q, k, v, lam, dout, cu)
+    f = lambda q_, k_, v_, l_: float(np.sum(ora.prefill_varlen(q_, k_, v_, l_, cu) * dout))
+    eps = 1e-6
+    ok = True
+    for which, idx in ((0, (6, 3, 1)), (1, (4, 1, 2)), (2, (2, 0, 0)), (3, (7, 1)), (1, (1, 0, 1))):
+        args = [q.copy(), k.copy(), v.copy(), lam.copy()]
+        args[which][idx] += eps
+        up = f(*args)
+        args[which][idx] -= 2 * eps
+        dn = f(*args)
+        ok &= abs((up - dn) / (2 * eps) - grads[which][idx]) < 1e-6
+    # perturbing key 1 (first sequence) leaves the second sequence's outputs unchanged
+    k2 = k.copy()
+    k2[1] += 1.0
+    ok &= np.array_equal(ora.prefill_varlen(q, k2, v, lam, cu)[3:], ora.prefill_varlen(q, k, v, lam, cu)[3:])
+    return bool(ok)
+
+
+def pin_backward_varlen_equal_lengths_is_batched():
+    """Two packed sequences of equal length give the batched backward of the same data."""
+    q, k, v, lam = _rand_prefill(B=2, S=6, Hq=8, Hkv=2, D=4, seed=25)
+    dout = np.random.default_rng(26).standard_normal((2, 6, 4, 4))
+    batched = ora.prefill_backward(q, k, v, lam, dout)
+    packed = ora.prefill_backward_varlen(*(x.reshape((12,) + x.shape[2:]) for x in (q, k, v, lam, dout)), [0, 6, 12])
+    return bool(all(np.allclose(a.reshape(p_.shape), p_, atol=1e-13) for a, p_ in zip(batched, packed)))
+
+
 ALL_PINS = {
     "softmax_library": pin_softmax_library,
     "lambda0_is_softmax_attention": pin_lambda0_is_softmax_attention,
@@ -423,6 +460,8 @@ ALL_PINS = {
     "backward_matches_autograd_noncausal": lambda: pin_backward_matches_autograd(causal=False),
     "backward_finite_differences": pin_backward_finite_differences,
     "branches_recombine_and_normalise": pin_branches_recombine_and_normalise,
+    "backward_varlen_finite_differences": pin_backward_varlen_finite_differences,
+    "backward_varlen_equal_lengths_is_batched": pin_backward_varlen_equal_lengths_is_batched,
 }
 
 
