@@ -635,6 +635,21 @@ def run_workload(args):
         cfg = {"workload": "backward of the causal prefill B=4 S=4096 Hq=64 Hkv=8 D=128 (dQ, dK, dV, dlambda)",
                "train_forward_ms": round(fwd_ms, 4),
                "train_forward_tflops": round(workloads.prefill_flops(case.B, case.S, case.Hq, D) / (fwd_ms * 1e-3) / 1e12, 2)}
+    elif name == "backward_window":
+        case = workloads.CONFIGS["c2_bf16_prefill"]
+        W = 1024
+        inp = workloads.make_prefill(case)
+        q, k, v, lam = (inp[x].to(dev) for x in ("q", "k", "v", "lam"))
+        dout = workloads.make_prefill_grad(case).to(dev)
+        out, ob, lse = da.prefill_train(q, k, v, lam, window=W, stream=stream)
+        ws = torch.empty(da.backward_workspace_size(case.B, case.S, case.Hq), dtype=torch.uint8, device=dev)
+        fn = lambda: da.backward(q, k, v, lam, ob, lse, dout, workspace=ws, window=W, stream=stream)
+        flops = 2 * 4 * D * case.Hq * case.B * sum(min(i + 1, W) for i in range(case.S))
+        ms = _time_op(fn, args.steps, args.warmup, stream)
+        val = flops / (ms * 1e-3) / 1e12
+        unit, peak, bound = "TFLOP/s", peaks["bf16_tflops"], "tensor"
+        launches = 3
+        cfg = {"workload": f"backward of the sliding-window causal prefill, window {W}, B=4 S=4096 Hq=64 Hkv=8 D=128"}
     elif name == "backward_varlen":
         g = torch.Generator().manual_seed(1010)
         lens = torch.randint(512, 3585, (8,), generator=g).tolist()
@@ -695,7 +710,8 @@ def main(argv=None):
     ap.add_argument("--ref-seconds", type=float, default=120.0,
                     help="host-time budget of the whole reference run (warm-up and timed steps)")
     ap.add_argument("--workload", choices=("prefill_long", "decode_needle", "window", "varlen", "paged", "multi",
-                                           "lambda_v2", "backward", "backward_varlen"), default=None,
+                                           "lambda_v2", "backward", "backward_varlen", "backward_window"),
+                    default=None,
                     help="time one other operation alone instead of the default step")
     ap.add_argument("--scaling", choices=("weak", "strong"), default="weak",
                     help="weak: each GPU runs the full per-GPU workload; strong: the heads of one workload "

@@ -32,6 +32,8 @@ _SIGNATURES = {
     "diffattn_v2_prefill_train": (_i, [_vp] * 7 + [_i] * 6 + [_vp]),
     "diffattn_v2_backward_workspace_size": (_sz, [_i, _i, _i]),
     "diffattn_v2_backward": (_i, [_vp] * 11 + [_i] * 6 + [_vp, _sz, _vp]),
+    "diffattn_v2_prefill_window_train": (_i, [_vp] * 7 + [_i] * 6 + [_vp]),
+    "diffattn_v2_backward_window": (_i, [_vp] * 11 + [_i] * 6 + [_vp, _sz, _vp]),
     "diffattn_v2_prefill_varlen_train": (_i, [_vp] * 8 + [_i] * 7 + [_vp]),
     "diffattn_v2_backward_varlen_workspace_size": (_sz, [_i, _i, _i]),
     "diffattn_v2_backward_varlen": (_i, [_vp] * 12 + [_i] * 7 + [_vp, _sz, _vp]),
@@ -169,9 +171,10 @@ def prefill_f32(q, k, v, lam, out=None, causal=True, stream=None):
     return out
 
 
-def prefill_train(q, k, v, lam, out=None, o_branch=None, lse=None, causal=True, stream=None):
+def prefill_train(q, k, v, lam, out=None, o_branch=None, lse=None, causal=True, window=None, stream=None):
     """Training forward: prefill plus the per-head normalised O_b (bf16 [B,S,Hq,D]) and the
-    log2-domain row log-sum-exp (fp32 [B,S,Hq]) that backward reads. Returns (out, o_branch, lse)."""
+    log2-domain row log-sum-exp (fp32 [B,S,Hq]) that backward reads. Returns (out, o_branch, lse).
+    With `window` the causal sliding-window prefill (query i sees keys i-window+1 .. i)."""
     for t, n, nd in ((q, "q", 4), (k, "k", 4), (v, "v", 4)):
         _need(t, n, torch.bfloat16, nd)
     _need(lam, "lam", torch.float32, 3)
@@ -186,6 +189,11 @@ def prefill_train(q, k, v, lam, out=None, o_branch=None, lse=None, causal=True, 
     _need(out, "out", torch.bfloat16, 4)
     _need(o_branch, "o_branch", torch.bfloat16, 4)
     _need(lse, "lse", torch.float32, 3)
+    if window is not None:
+        st = LIB.diffattn_v2_prefill_window_train(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(out), _ptr(o_branch),
+                                                  _ptr(lse), B, S, Hq, Hkv, D, int(window), _stream(stream, q.device))
+        _check(st, "diffattn_v2_prefill_window_train")
+        return out, o_branch, lse
     st = LIB.diffattn_v2_prefill_train(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(out), _ptr(o_branch), _ptr(lse),
                                        B, S, Hq, Hkv, D, 1 if causal else 0, _stream(stream, q.device))
     _check(st, "diffattn_v2_prefill_train")
@@ -197,8 +205,9 @@ def backward_workspace_size(B, S, Hq) -> int:
 
 
 def backward(q, k, v, lam, o_branch, lse, dout, causal=True, dq=None, dk=None, dv=None, dlam=None,
-             workspace=None, stream=None):
-    """Gradients of the bf16 prefill: returns (dq, dk, dv, dlam) with the layouts of q, k, v, lam."""
+             workspace=None, window=None, stream=None):
+    """Gradients of the bf16 prefill: returns (dq, dk, dv, dlam) with the layouts of q, k, v, lam.
+    With `window` the gradients of the causal sliding-window prefill."""
     for t, n, nd in ((q, "q", 4), (k, "k", 4), (v, "v", 4), (o_branch, "o_branch", 4), (dout, "dout", 4)):
         _need(t, n, torch.bfloat16, nd)
     _need(lam, "lam", torch.float32, 3)
@@ -215,6 +224,13 @@ def backward(q, k, v, lam, o_branch, lse, dout, causal=True, dq=None, dk=None, d
     ws_bytes = backward_workspace_size(B, S, Hq)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+    if window is not None:
+        st = LIB.diffattn_v2_backward_window(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(o_branch), _ptr(lse),
+                                             _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlam), B, S, Hq, Hkv, D,
+                                             int(window), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                             _stream(stream, q.device))
+        _check(st, "diffattn_v2_backward_window")
+        return dq, dk, dv, dlam
     st = LIB.diffattn_v2_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(o_branch), _ptr(lse), _ptr(dout),
                                   _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlam), B, S, Hq, Hkv, D, 1 if causal else 0,
                                   _ptr(workspace), workspace.numel() * workspace.element_size(),

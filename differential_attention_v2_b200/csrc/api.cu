@@ -228,10 +228,13 @@ size_t diffattn_v2_backward_workspace_size(int B, int S, int Hq) {
   return da2::backward_stats_bytes(B, S, Hq);
 }
 
-int diffattn_v2_backward(const void* q, const void* k, const void* v, const float* lambda, const void* o_branch,
-                         const float* lse, const void* dout, void* dq, void* dk, void* dv, float* dlambda, int B,
-                         int S, int Hq, int Hkv, int D, int causal, void* workspace, size_t workspace_bytes,
-                         da2_stream_t stream) {
+namespace {
+
+// The [B,S] backward: causal 0/1, window > 0 only with causal (window >= S: plain causal).
+int backward_bshd(const void* q, const void* k, const void* v, const float* lambda, const void* o_branch,
+                  const float* lse, const void* dout, void* dq, void* dk, void* dv, float* dlambda, int B, int S,
+                  int Hq, int Hkv, int D, int causal, int window, void* workspace, size_t workspace_bytes,
+                  da2_stream_t stream) {
   if (B < 0 || S < 0 || D <= 0 || !heads_ok(Hq, Hkv)) return DA2_ERR_INVALID;
   if (causal != 0 && causal != 1) return DA2_ERR_INVALID;
   if (B == 0 || S == 0) return DA2_OK;
@@ -256,7 +259,51 @@ int diffattn_v2_backward(const void* q, const void* k, const void* v, const floa
   return status_of(da2::launch_backward_sm100(
       q64, q128, o64, o128, k64, k128, v64, v128, lambda, static_cast<const bf*>(o_branch), lse,
       static_cast<const bf*>(dout), static_cast<bf*>(dq), static_cast<bf*>(dk), static_cast<bf*>(dv), dlambda,
-      static_cast<float*>(workspace), err, B, S, Hq, Hkv, causal, reinterpret_cast<cudaStream_t>(stream)));
+      static_cast<float*>(workspace), err, B, S, Hq, Hkv, causal, reinterpret_cast<cudaStream_t>(stream), nullptr, 0,
+      window));
+}
+
+}  // namespace
+
+int diffattn_v2_backward(const void* q, const void* k, const void* v, const float* lambda, const void* o_branch,
+                         const float* lse, const void* dout, void* dq, void* dk, void* dv, float* dlambda, int B,
+                         int S, int Hq, int Hkv, int D, int causal, void* workspace, size_t workspace_bytes,
+                         da2_stream_t stream) {
+  return backward_bshd(q, k, v, lambda, o_branch, lse, dout, dq, dk, dv, dlambda, B, S, Hq, Hkv, D, causal, 0,
+                       workspace, workspace_bytes, stream);
+}
+
+int diffattn_v2_prefill_window_train(const void* q, const void* k, const void* v, const float* lambda, void* out,
+                                     void* o_branch, float* lse, int B, int S, int Hq, int Hkv, int D, int window,
+                                     da2_stream_t stream) {
+  if (B < 0 || S < 0 || D <= 0 || !heads_ok(Hq, Hkv) || window < 1) return DA2_ERR_INVALID;
+  if (B == 0 || S == 0) return DA2_OK;
+  const void* ptrs[] = {q, k, v, lambda, out, o_branch, lse};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return DA2_ERR_INVALID;
+  if (D != 128) return DA2_ERR_UNSUPPORTED;
+  if ((S + 127) / 128 > 65535) return DA2_ERR_UNSUPPORTED;
+  int* err = nullptr;
+  cudaError_t e = device_error_ptr(&err);
+  if (e != cudaSuccess) return DA2_ERR_CUDA;
+  CUtensorMap tq, tk, tv;
+  if (encode_bshd(&tq, q, D, Hq, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  if (encode_bshd(&tk, k, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  if (encode_bshd(&tv, v, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  // a window of S or more keys is the plain causal mask
+  e = da2::launch_prefill(tq, tk, tv, lambda, static_cast<__nv_bfloat16*>(out), err, B, S, Hq, Hkv, 1,
+                          window >= S ? 0 : window, nullptr, reinterpret_cast<cudaStream_t>(stream),
+                          static_cast<__nv_bfloat16*>(o_branch), lse);
+  return status_of(e);
+}
+
+int diffattn_v2_backward_window(const void* q, const void* k, const void* v, const float* lambda,
+                                const void* o_branch, const float* lse, const void* dout, void* dq, void* dk,
+                                void* dv, float* dlambda, int B, int S, int Hq, int Hkv, int D, int window,
+                                void* workspace, size_t workspace_bytes, da2_stream_t stream) {
+  if (window < 1) return DA2_ERR_INVALID;
+  return backward_bshd(q, k, v, lambda, o_branch, lse, dout, dq, dk, dv, dlambda, B, S, Hq, Hkv, D, 1,
+                       window >= S ? 0 : window, workspace, workspace_bytes, stream);
 }
 
 int diffattn_v2_prefill_varlen_train(const void* q, const void* k, const void* v, const float* lambda, void* out,

@@ -91,6 +91,7 @@ struct Params {
   __nv_bfloat16* dv;
   int* err;
   int B, S, S_pad, Hq, Hkv, causal;
+  int window;                // causal sliding window: query i sees keys i-window+1 .. i (0: none)
   int n_tiles;               // 128-row tiles
   const int* cu_seqlens;     // packed sequences: sequence b is rows cu[b] .. cu[b+1]-1 (null: [B,S])
   const int* pad_off;        // packed sequences: first row of sequence b in the row terms (128-aligned)
@@ -356,7 +357,9 @@ __device__ __forceinline__ void tile_to_tmem(uint32_t tile, uint32_t trow, int r
 }
 
 // --------------------------------------------------------------------------- dK / dV
-template <bool kVarlen>
+// kVarlen: packed sequences (p.cu_seqlens); kWindow: causal sliding window (p.window). The
+// plain [B,S] backward is the <false, false> instance and carries neither.
+template <bool kVarlen, bool kWindow>
 __global__ void __launch_bounds__(kThreads, 1)
 dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
            const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const Params p) {
@@ -390,7 +393,9 @@ dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   const size_t row_base = kVarlen ? static_cast<size_t>(tok0) : static_cast<size_t>(b) * p.S;
   const int nq = (S + 63) / 64;                     // 64-row query blocks
   const int q_first = p.causal ? k0 / 64 : 0;
-  const int steps_per_pair = nq - q_first;
+  // with a window the tile's keys k0 .. k0+127 are seen by queries up to k0+127+window-1
+  const int q_end = kWindow ? min(nq, (k0 + 126 + p.window) / 64 + 1) : nq;
+  const int steps_per_pair = q_end - q_first;
   const int n_steps = gpairs * steps_per_pair;
 
   const uint32_t tmem = setup(bar0, tmem_slot, abort_flag, warp);
@@ -523,8 +528,11 @@ dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       ld_cols_wait(dp);
       // this group's columns of the five row-term arrays (shared, filled by bulk copy)
       const uint32_t rec = sbase + kKvOffX + s * kKvStage + 3 * kStreamTile + 4 * col0;
-      // causal: only the two query blocks that overlap the key tile hold keys past a query
+      // causal: only the two query blocks that overlap the key tile hold keys past a query;
+      // window: blocks whose last query is window or more past the tile's first key hold
+      // pairs outside the window
       const bool diag = p.causal && q0 < k0 + 128;
+      const bool wedge = kWindow && q0 + 63 - k0 >= p.window;
       const int qbase = q0 + col0;
       const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
       uint32_t w_pk[kCols / 2], d1_pk[kCols / 2], d2_pk[kCols / 2];
@@ -548,6 +556,10 @@ dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           if (diag) {
             if (key > qbase + c) p10 = p20 = 0.f;
             if (key > qbase + c + 1) p11 = p21 = 0.f;
+          }
+          if (kWindow && wedge) {
+            if (qbase + c - key >= p.window) p10 = p20 = 0.f;
+            if (qbase + c + 1 - key >= p.window) p11 = p21 = 0.f;
           }
           const uint64_t P1 = f2_pack(p10, p11), P2 = f2_pack(p20, p21);
           const uint64_t dpp = f2_pack(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1]));
@@ -584,7 +596,7 @@ dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 }
 
 // --------------------------------------------------------------------------------- dQ
-template <bool kVarlen>
+template <bool kVarlen, bool kWindow>
 __global__ void __launch_bounds__(kThreads, 1)
 dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
          const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const Params p) {
@@ -616,7 +628,10 @@ dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
   if (m0 >= S) return;  // uniform over the CTA: the row tile lies past the sequence's end
   const size_t row_base = kVarlen ? static_cast<size_t>(tok0) : static_cast<size_t>(b) * p.S;
   const int nk = (S + 63) / 64;
-  const int n_steps = p.causal ? min(nk, (m0 + 128) / 64) : nk;
+  // key blocks kb_first .. kb_first+n_steps-1 (64 keys each); with a window the rows
+  // m0 .. m0+127 see keys from m0-window+1 on
+  const int kb_first = kWindow ? max(0, m0 - p.window + 1) / 64 : 0;
+  const int n_steps = (p.causal ? min(nk, (m0 + 128) / 64) : nk) - kb_first;
 
   const uint32_t tmem = setup(bar0, tmem_slot, abort_flag, warp);
 
@@ -637,8 +652,9 @@ dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         const uint32_t st = sbase + kQOffX + s * kQStage;
         mbar_arrive_expect_tx(bar(kXFull + s), 2 * kStreamTile);
         for (int c = 0; c < 2; ++c) {
-          tma_load_4d(st + c * kStreamChunk, &tmK, bar(kXFull + s), c * 64, g, tok0 + 64 * t, tb);
-          tma_load_4d(st + kStreamTile + c * kStreamChunk, &tmV, bar(kXFull + s), c * 64, g, tok0 + 64 * t, tb);
+          tma_load_4d(st + c * kStreamChunk, &tmK, bar(kXFull + s), c * 64, g, tok0 + 64 * (kb_first + t), tb);
+          tma_load_4d(st + kStreamTile + c * kStreamChunk, &tmV, bar(kXFull + s), c * 64, g,
+                      tok0 + 64 * (kb_first + t), tb);
         }
         issued = t + 1;
       }
@@ -739,10 +755,14 @@ dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
       ld_cols_wait(s1);
       ld_cols_wait(s2);
       ld_cols_wait(dp);
-      const int kbase = 64 * t + col0;
-      // tile-uniform: keys past the query (causal diagonal) or past S (ragged last block)
-      const bool masked = (p.causal && 64 * t + 63 > m0) || (64 * t + 64 > S);
-      const int lim = p.causal ? min(qi, S - 1) : S - 1;
+      const int kb = kb_first + t;  // key block (t drives the stages and barriers)
+      const int kbase = 64 * kb + col0;
+      // tile-uniform: keys past the query (causal diagonal) or past S (ragged last block);
+      // keys before some row's window start (the window's lower edge)
+      const bool masked = (p.causal && 64 * kb + 63 > m0) || (64 * kb + 64 > S);
+      const bool wedge = kWindow && 64 * kb < m0 + 128 - p.window;
+      const int lim = p.causal ? min(qi, S - 1) : S - 1;  // last key this row sees
+      const int lo = qi - p.window + 1;                      // first key it sees with a window
       uint32_t d1_pk[kCols / 2], d2_pk[kCols / 2];
 #pragma unroll
       for (int c = 0; c < kCols; c += 2) {
@@ -755,6 +775,10 @@ dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         if (masked) {
           if (kbase + c > lim) p10 = p20 = 0.f;
           if (kbase + c + 1 > lim) p11 = p21 = 0.f;
+        }
+        if (kWindow && wedge) {
+          if (kbase + c < lo) p10 = p20 = 0.f;
+          if (kbase + c + 1 < lo) p11 = p21 = 0.f;
         }
         const uint64_t dpp = f2_pack(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1]));
         const uint64_t d1 = f2_mul(f2_pack(p10, p11), f2_add(dpp, ne1));
@@ -808,7 +832,7 @@ cudaError_t launch_backward_sm100(const CUtensorMap& tmQ64, const CUtensorMap& t
                                   const __nv_bfloat16* o_branch, const float* lse, const __nv_bfloat16* dout,
                                   __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv, float* dlambda,
                                   float* workspace, int* err, int B, int S, int Hq, int Hkv, int causal,
-                                  cudaStream_t stream, const int32_t* cu_seqlens, int total_tokens) {
+                                  cudaStream_t stream, const int32_t* cu_seqlens, int total_tokens, int window) {
   using namespace bwd_tc;
   const int n_pairs = Hq / 2;
   Params p;
@@ -846,6 +870,7 @@ cudaError_t launch_backward_sm100(const CUtensorMap& tmQ64, const CUtensorMap& t
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.causal = causal;
+  p.window = window;
   p.cu_seqlens = cu_seqlens;
   p.n_tiles = (S + 127) / 128;
   p.scale = 1.f / sqrtf(static_cast<float>(HD));
@@ -861,7 +886,9 @@ cudaError_t launch_backward_sm100(const CUtensorMap& tmQ64, const CUtensorMap& t
     kdq<<<dim3(B * n_pairs, p.n_tiles), kThreads, kQSmem, stream>>>(tmQ128, tmO128, tmK64, tmV64, p);
     return cudaGetLastError();
   };
-  return cu_seqlens ? run(dkdv_sm100<true>, dq_sm100<true>) : run(dkdv_sm100<false>, dq_sm100<false>);
+  if (cu_seqlens) return run(dkdv_sm100<true, false>, dq_sm100<true, false>);
+  if (window > 0) return run(dkdv_sm100<false, true>, dq_sm100<false, true>);
+  return run(dkdv_sm100<false, false>, dq_sm100<false, false>);
 }
 
 }  // namespace da2

@@ -23,7 +23,7 @@ cudaError_t launch_prefill(const CUtensorMap& tmQ, const CUtensorMap& tmK, const
 // dK/dV and dQ tile kernels. Tensor maps over q [B,S,Hq,D], dout [B,S,Hq/2,D], k and v
 // [B,S,Hkv,D] with 64- and 128-row boxes (64 d x 1 head). With cu_seqlens (device, B+1
 // entries) the tensors hold B packed sequences as one [1,T] batch (T = total_tokens) and S
-// is the longest sequence.
+// is the longest sequence. window > 0 (causal only): query i saw keys i-window+1 .. i.
 size_t backward_stats_bytes(int B, int S, int Hq);
 size_t backward_varlen_workspace_bytes(int B, int T, int Hq);
 cudaError_t launch_backward_sm100(const CUtensorMap& tmQ64, const CUtensorMap& tmQ128, const CUtensorMap& tmO64,
@@ -32,7 +32,8 @@ cudaError_t launch_backward_sm100(const CUtensorMap& tmQ64, const CUtensorMap& t
                                   const __nv_bfloat16* o_branch, const float* lse, const __nv_bfloat16* dout,
                                   __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv, float* dlambda,
                                   float* workspace, int* err, int B, int S, int Hq, int Hkv, int causal,
-                                  cudaStream_t stream, const int32_t* cu_seqlens = nullptr, int total_tokens = 0);
+                                  cudaStream_t stream, const int32_t* cu_seqlens = nullptr, int total_tokens = 0,
+                                  int window = 0);
 
 // bf16 decode (D = 128): split kernel + combine. Tensor maps over the caches [B,Smax,Hkv,D],
 // boxes of 64 (d) x 1 x 64 (tokens) x 1, 128-byte swizzle. With block_table the maps cover

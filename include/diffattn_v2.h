@@ -170,6 +170,22 @@ DA2_API int diffattn_v2_backward(const void* q, const void* k, const void* v, co
                                  da2_stream_t stream);
 
 /*
+ * Training forward and backward of the causal sliding-window prefill (hybrid layers; query
+ * i sees keys i-window+1 .. i, "Attention variants" lesson, Step 2): the arguments, layouts,
+ * workspace (diffattn_v2_backward_workspace_size) and semantics of diffattn_v2_prefill_train
+ * and diffattn_v2_backward with `window` (>= 1; window >= S is the plain causal pass) in place
+ * of `causal`. Only the KV tiles inside the windows are read.
+ */
+DA2_API int diffattn_v2_prefill_window_train(const void* q, const void* k, const void* v, const float* lambda,
+                                             void* out, void* o_branch, float* lse, int B, int S, int Hq,
+                                             int Hkv, int D, int window, da2_stream_t stream);
+DA2_API int diffattn_v2_backward_window(const void* q, const void* k, const void* v, const float* lambda,
+                                        const void* o_branch, const float* lse, const void* dout, void* dq,
+                                        void* dk, void* dv, float* dlambda, int B, int S, int Hq, int Hkv,
+                                        int D, int window, void* workspace, size_t workspace_bytes,
+                                        da2_stream_t stream);
+
+/*
  * Training forward and backward for B sequences packed along the token axis (the layout of
  * diffattn_v2_prefill_varlen; pretraining on packed documents). Every sequence is an
  * independent prefill, so its gradients are those of its own prefill:

@@ -177,9 +177,10 @@ def prefill_varlen(q, k, v, lam, cu_seqlens, causal: bool = True) -> np.ndarray:
     return out
 
 
-def prefill_backward(q, k, v, lam, dout, causal: bool = True):
+def prefill_backward(q, k, v, lam, dout, causal: bool = True, window=None):
     """Gradients of the prefill: returns (dq [B,S,Hq,D], dk, dv [B,S,Hkv,D], dlam [B,S,Hq/2])
-    for an upstream gradient dout [B,S,Hq/2,D], all float64.
+    for an upstream gradient dout [B,S,Hq/2,D], all float64. With `window` (causal only) the
+    mask is the sliding window of `window_mask`.
 
     The chain rule applied to the definition of `diff_attention_block`, per pair p (heads h1,
     h2 over KV head g) and batch b, with A_b = softmax(S_b), S_b = Q_b K^T / sqrt(D) + mask,
@@ -199,7 +200,10 @@ def prefill_backward(q, k, v, lam, dout, causal: bool = True):
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
     dlam = np.zeros_like(lam)
-    mask = causal_mask(S, S) if causal else np.zeros((S, S))
+    if window is not None:
+        mask = window_mask(S, S, int(window))
+    else:
+        mask = causal_mask(S, S) if causal else np.zeros((S, S))
     for b in range(B):
         for p, h1, h2, g in pair_layout(Hq, Hkv):
             kk, vv = k[b, :, g], v[b, :, g]

@@ -57,6 +57,11 @@ def sample_rows(B, S, n_pairs, n=1024, seed=0, tile=128):
 # rounded once to bf16: each term is ~2e-3 relative, so 1e-2 leaves a factor ~3 of margin.
 GRAD_REL_FRO = 1e-2
 GRAD_MAX_REL = 2e-2
+# A reference that is identically zero (e.g. dQ with a one-key window: P = 1, dS = dP - E = 0)
+# has no scale for a relative bound; the GPU's result there is fp32 rounding of O(1) terms
+# (dP from the MMA against E from a dot product), bounded absolutely far below the bf16
+# resolution of O(1) gradients (2^-9).
+GRAD_ZERO_ABS = 1e-4
 
 
 def grad_close(got, ref, what=""):
@@ -66,6 +71,9 @@ def grad_close(got, ref, what=""):
     assert np.all(np.isfinite(got)), f"{what}: non-finite gradient"
     scale = float(np.abs(ref).max()) if ref.size else 0.0
     max_abs = float(np.abs(got - ref).max()) if ref.size else 0.0
+    if scale == 0.0:
+        assert max_abs <= GRAD_ZERO_ABS, f"{what}: zero reference, max-abs {max_abs:.3e} > {GRAD_ZERO_ABS}"
+        return max_abs, 0.0
     den = float(np.linalg.norm(ref))
     rel = float(np.linalg.norm(got - ref) / den) if den > 0 else float(np.linalg.norm(got))
     assert max_abs <= GRAD_MAX_REL * max(scale, 1e-30), f"{what}: max-abs {max_abs:.3e} > {GRAD_MAX_REL} x {scale:.3e}"

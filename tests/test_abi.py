@@ -224,3 +224,15 @@ def test_varlen_training_host_checks(lib):
     assert lib.diffattn_v2_backward_varlen(*ok[:18], 2, *ok[19:]) == -1              # causal not 0/1
     assert lib.diffattn_v2_backward_varlen(*ok[:17], 64, *ok[18:]) == -2             # D = 64
     assert lib.diffattn_v2_backward_varlen(*ok[:12], 0, *ok[13:]) == 0               # B = 0
+
+
+def test_window_training_host_checks(lib):
+    OB, LS, DO, DQ, DK, DV, DL, W = (P + 32768 * i for i in range(1, 9))
+    assert lib.diffattn_v2_prefill_window_train(Q, K, V, L, O, OB, LS, 2, 256, 8, 2, 128, 0, None) == -1  # window < 1
+    assert lib.diffattn_v2_prefill_window_train(Q, K, V, L, O, OB, LS, 2, 256, 8, 2, 64, 64, None) == -2  # D = 64
+    assert lib.diffattn_v2_prefill_window_train(Q, K, V, L, O, OB, LS, 0, 256, 8, 2, 128, 64, None) == 0   # empty
+    ws = lib.diffattn_v2_backward_workspace_size(2, 256, 8)
+    ok = (Q, K, V, L, OB, LS, DO, DQ, DK, DV, DL, 2, 256, 8, 2, 128, 64, W, ws, None)
+    assert lib.diffattn_v2_backward_window(*ok[:16], 0, *ok[17:]) == -1           # window < 1
+    assert lib.diffattn_v2_backward_window(*ok[:18], ws - 4, None) == -1          # short workspace
+    assert lib.diffattn_v2_backward_window(*ok[:15], 64, *ok[16:]) == -2          # D = 64

@@ -166,3 +166,32 @@ def test_backward_varlen_equal_lengths_equals_batched(da):
     _, g_packed = _gpu_varlen(da, packed, [0, S, 2 * S, 3 * S], True)
     for a, b in zip(g_batched, g_packed):
         assert torch.equal(a.reshape(b.shape), b)
+
+
+@pytest.mark.parametrize("S,window,Hq,Hkv", [
+    (300, 1, 8, 2),       # every query sees only itself
+    (300, 64, 8, 2),      # window inside one 64-key block
+    (700, 100, 16, 2),    # window across block and tile edges, several tiles
+    (513, 300, 4, 2),     # window wider than a tile
+])
+def test_backward_window_matches_oracle(da, S, window, Hq, Hkv):
+    inp = _case(1, S, Hq, Hkv, seed=71 + window)
+    d = {k: v.cuda() for k, v in inp.items()}
+    out, ob, lse = da.prefill_train(d["q"], d["k"], d["v"], d["lam"], window=window)
+    assert torch.equal(out, da.prefill_window(d["q"], d["k"], d["v"], d["lam"], window))
+    grads = da.backward(d["q"], d["k"], d["v"], d["lam"], ob, lse, d["dout"], window=window)
+    torch.cuda.synchronize()
+    assert da.device_error() == 0
+    ref = ora.prefill_backward(inp["q"], inp["k"], inp["v"], inp["lam"], inp["dout"], window=window)
+    for g, r, name in zip(grads, ref, ("dq", "dk", "dv", "dlam")):
+        grad_close(g, r, f"window={window} S={S} {name}")
+
+
+def test_backward_window_wider_than_sequence_is_causal(da):
+    inp = _case(2, 300, 8, 2, seed=79)
+    d = {k: v.cuda() for k, v in inp.items()}
+    _, g_causal = _gpu_grads(da, inp, True)
+    out, ob, lse = da.prefill_train(d["q"], d["k"], d["v"], d["lam"], window=300)
+    g_win = da.backward(d["q"], d["k"], d["v"], d["lam"], ob, lse, d["dout"], window=300)
+    for a, b in zip(g_causal, g_win):
+        assert torch.equal(a, b)

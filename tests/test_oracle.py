@@ -431,6 +431,28 @@ def pin_backward_varlen_equal_lengths_is_batched():
     return bool(all(np.allclose(a.reshape(p_.shape), p_, atol=1e-13) for a, p_ in zip(batched, packed)))
 
 
+def pin_backward_window():
+    """Sliding-window gradients: central differences of <dout, prefill(., window=3)>, and a
+    window covering the whole sequence reduces to the causal backward."""
+    q, k, v, lam = _rand_prefill(B=1, S=7, Hq=4, Hkv=2, D=3, seed=27)
+    dout = np.random.default_rng(28).standard_normal((1, 7, 2, 3))
+    grads = ora.prefill_backward(q, k, v, lam, dout, window=3)
+    f = lambda q_, k_, v_, l_: float(np.sum(ora.prefill(q_, k_, v_, l_, window=3) * dout))
+    eps = 1e-6
+    ok = True
+    for which, idx in ((0, (0, 6, 1, 2)), (1, (0, 4, 1, 0)), (1, (0, 1, 0, 1)), (2, (0, 3, 0, 2)), (3, (0, 5, 1))):
+        args = [q.copy(), k.copy(), v.copy(), lam.copy()]
+        args[which][idx] += eps
+        up = f(*args)
+        args[which][idx] -= 2 * eps
+        dn = f(*args)
+        ok &= abs((up - dn) / (2 * eps) - grads[which][idx]) < 1e-6
+    full = ora.prefill_backward(q, k, v, lam, dout, window=7)
+    causal = ora.prefill_backward(q, k, v, lam, dout)
+    ok &= all(np.allclose(a, b, atol=1e-13) for a, b in zip(full, causal))
+    return bool(ok)
+
+
 ALL_PINS = {
     "softmax_library": pin_softmax_library,
     "lambda0_is_softmax_attention": pin_lambda0_is_softmax_attention,
@@ -462,6 +484,7 @@ ALL_PINS = {
     "branches_recombine_and_normalise": pin_branches_recombine_and_normalise,
     "backward_varlen_finite_differences": pin_backward_varlen_finite_differences,
     "backward_varlen_equal_lengths_is_batched": pin_backward_varlen_equal_lengths_is_batched,
+    "backward_window": pin_backward_window,
 }
 
 

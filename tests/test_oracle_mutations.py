@@ -116,12 +116,15 @@ def _lambda_v2_no_sigmoid(x, w, bias=None):
 def _backward_variant(drop_rowsum=False, dlam_sign=-1.0, dk_first_only=False, dv_no_lambda=False,
                       dq_unscaled=False):
     """The chain rule of the prefill with one planted mistake (a flag set)."""
-    def fn(q, k, v, lam, dout, causal=True):
+    def fn(q, k, v, lam, dout, causal=True, window=None):
         q, k, v, lam, dout = (np.asarray(x, dtype=np.float64) for x in (q, k, v, lam, dout))
         B, S, Hq, D = q.shape
         inv = 1.0 / math.sqrt(D)
         dq, dk, dv, dlam = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v), np.zeros_like(lam)
-        mask = ora.causal_mask(S, S) if causal else np.zeros((S, S))
+        if window is not None:
+            mask = ora.window_mask(S, S, int(window))
+        else:
+            mask = ora.causal_mask(S, S) if causal else np.zeros((S, S))
         for b in range(B):
             for p, h1, h2, g in ora.pair_layout(Hq, k.shape[2]):
                 kk, vv = k[b, :, g], v[b, :, g]
