@@ -42,8 +42,8 @@ if ROOT not in sys.path:
 import workloads  # noqa: E402
 
 METRIC = "DiffAttnV2 fwd: prefill TFLOP/s (% bf16 peak); decode GB/s (% HBM)"
-PREFILL_CFG = "c2_bf16_prefill"
-DECODE_CFG = "c4_bf16_decode"
+PREFILL_CFG = "prefill_b4_s4096"
+DECODE_CFG = "decode_b64_s8192"
 
 # Measured roofline denominators of this machine's B200s (measured copy bandwidth and
 # cuBLAS bf16 GEMM); used when the peaks file is absent.
@@ -552,7 +552,7 @@ def run_workload(args):
             cfg = {"workload": f"packed causal prefill of 8 sequences, lengths U[512,3584] (total {T}), Hq=64 Hkv=8 D=128",
                    "lengths": lens}
         else:
-            case = workloads.CONFIGS["c3_long_bf16_prefill"] if name == "prefill_long" else workloads.CONFIGS["c2_bf16_prefill"]
+            case = workloads.CONFIGS["prefill_b1_s32768"] if name == "prefill_long" else workloads.CONFIGS["prefill_b4_s4096"]
             inp = workloads.make_prefill(case)
             q, k, v, lam = (inp[x].to(dev) for x in ("q", "k", "v", "lam"))
             out = torch.empty(case.B, case.S, case.Hq // 2, D, dtype=torch.bfloat16, device=dev)
@@ -570,7 +570,7 @@ def run_workload(args):
         unit, peak, bound = "TFLOP/s", peaks["bf16_tflops"], "tensor"
         launches = 1
     elif name in ("decode_needle", "paged", "multi"):
-        case = workloads.CONFIGS["c5_needle_decode"] if name == "decode_needle" else workloads.CONFIGS["c4_bf16_decode"]
+        case = workloads.CONFIGS["needle_decode_b8_s131072"] if name == "decode_needle" else workloads.CONFIGS["decode_b64_s8192"]
         inp = workloads.make_decode(case)
         kc, vc, sl = (inp[x].to(dev) for x in ("kcache", "vcache", "seqlens"))
         if inp["lam"] is None:
@@ -613,7 +613,7 @@ def run_workload(args):
         val = nbytes / (ms * 1e-3) / 1e9
         unit, peak, bound = "GB/s", peaks["hbm_gbs"], "hbm"
     elif name == "backward":
-        case = workloads.CONFIGS["c2_bf16_prefill"]
+        case = workloads.CONFIGS["prefill_b4_s4096"]
         inp = workloads.make_prefill(case)
         q, k, v, lam = (inp[x].to(dev) for x in ("q", "k", "v", "lam"))
         dout = workloads.make_prefill_grad(case).to(dev)
@@ -636,7 +636,7 @@ def run_workload(args):
                "train_forward_ms": round(fwd_ms, 4),
                "train_forward_tflops": round(workloads.prefill_flops(case.B, case.S, case.Hq, D) / (fwd_ms * 1e-3) / 1e12, 2)}
     elif name == "backward_window":
-        case = workloads.CONFIGS["c2_bf16_prefill"]
+        case = workloads.CONFIGS["prefill_b4_s4096"]
         W = 1024
         inp = workloads.make_prefill(case)
         q, k, v, lam = (inp[x].to(dev) for x in ("q", "k", "v", "lam"))

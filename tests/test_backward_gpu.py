@@ -99,7 +99,7 @@ def test_backward_is_deterministic(da):
 def test_backward_full_size_one_group(da):
     """B=4 S=4096 Hq=64 Hkv=8: gradients of one (batch, KV group) slice against the oracle on
     that slice (dK, dV of the KV head; dQ of its 8 query heads; dlambda of its 4 pairs)."""
-    case = workloads.CONFIGS["c2_bf16_prefill"]
+    case = workloads.CONFIGS["prefill_b4_s4096"]
     inp = workloads.make_prefill(case)
     inp["dout"] = workloads.make_prefill_grad(case)
     _, (dq, dk, dv, dlam) = _gpu_grads(da, inp, True)
@@ -111,7 +111,7 @@ def test_backward_full_size_one_group(da):
           "v": inp["v"][b:b + 1, :, g:g + 1], "lam": inp["lam"][b:b + 1, :, pairs],
           "dout": inp["dout"][b:b + 1, :, pairs]}
     got = (dq[b:b + 1, :, heads], dk[b:b + 1, :, g:g + 1], dv[b:b + 1, :, g:g + 1], dlam[b:b + 1, :, pairs])
-    _check_grads(got, sl, True, "c2 slice b=3 g=5")
+    _check_grads(got, sl, True, "B=4 S=4096 slice b=3 g=5")
 
 
 def _packed(lens, Hq, Hkv, seed):

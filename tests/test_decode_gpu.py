@@ -64,15 +64,15 @@ def test_decode_matches_last_prefill_row(da):
 
 def test_decode_c4_full_size(da):
     """The 64-sequence decode workload (lengths uniform in [1024, 8192]) in full."""
-    inp = workloads.make_decode(workloads.CONFIGS["c4_bf16_decode"])
+    inp = workloads.make_decode(workloads.CONFIGS["decode_b64_s8192"])
     out = _run(da, inp)
     ref = ora.decode(inp["q"], inp["kcache"], inp["vcache"], inp["seqlens"], inp["lam"])
-    bf16_close(out, ref, "c4")
+    bf16_close(out, ref, "decode B=64 Smax=8192")
 
 
 def test_decode_c5_needle_with_v1_lambda(da):
     """The 128k needle workload with the V1 lambda computed on the GPU, in full."""
-    case = workloads.CONFIGS["c5_needle_decode"]
+    case = workloads.CONFIGS["needle_decode_b8_s131072"]
     inp = workloads.make_decode(case)
     B, n_pairs = case.B, case.Hq // 2
     lam = da.lambda_v1(inp["lq1"].cuda(), inp["lk1"].cuda(), inp["lq2"].cuda(), inp["lk2"].cuda(),
@@ -82,7 +82,7 @@ def test_decode_c5_needle_with_v1_lambda(da):
     inp["lam"] = lam.cpu()
     out = _run(da, inp)
     ref = ora.decode(inp["q"], inp["kcache"], inp["vcache"], inp["seqlens"], inp["lam"])
-    bf16_close(out, ref, "c5 needle")
+    bf16_close(out, ref, "needle decode B=8 L=131072")
 
 
 def test_lambda_v1_matches_oracle(da):

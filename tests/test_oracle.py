@@ -496,7 +496,7 @@ def test_pin(name):
 # ------------------------------------------------------------ the noise-cancellation toy
 
 def _planted_c1():
-    case = workloads.CONFIGS["c1_tiny_fp32_prefill"]
+    case = workloads.CONFIGS["tiny_fp32_prefill_b1_s128"]
     inp = workloads.make_prefill(case)
     row, sig = workloads.plant_signal_row(inp)
     return inp, row, sig

@@ -82,7 +82,7 @@ def test_prefill_bf16_repeatable(da):
     assert torch.equal(a, b)
 
 
-@pytest.mark.parametrize("name,n_rows", [("c2_bf16_prefill", 1024), ("c3_long_bf16_prefill", 1024)])
+@pytest.mark.parametrize("name,n_rows", [("prefill_b4_s4096", 1024), ("prefill_b1_s32768", 1024)])
 def test_prefill_bf16_full_size_sampled(da, name, n_rows):
     """Full-size workloads in the benchmark's launch configuration; a seeded stratified
     sample of rows (tile boundaries, first/last rows, every pair) checked against the oracle
@@ -99,13 +99,13 @@ def test_prefill_bf16_full_size_sampled(da, name, n_rows):
 
 def test_prefill_f32_c1_with_planted_row(da):
     """The tiny fp32 workload with the planted signal row: the whole output within 1e-5."""
-    inp = workloads.make_prefill(workloads.CONFIGS["c1_tiny_fp32_prefill"])
+    inp = workloads.make_prefill(workloads.CONFIGS["tiny_fp32_prefill_b1_s128"])
     row, sig = workloads.plant_signal_row(inp)
     d = _dev(inp)
     out = da.prefill_f32(d["q"], d["k"], d["v"], d["lam"])
     ref = ora.prefill(inp["q"], inp["k"], inp["v"], inp["lam"])
-    f32_close(out, ref, "c1 fp32")
-    f32_close(out[0, row, 0], ref[0, row, 0], "c1 planted row")
+    f32_close(out, ref, "tiny fp32 prefill")
+    f32_close(out[0, row, 0], ref[0, row, 0], "tiny fp32 planted row")
 
 
 @pytest.mark.parametrize("B,S,Hq,Hkv,D,causal", [
@@ -137,7 +137,7 @@ def test_prefill_window_matches_oracle(da, B, S, Hq, Hkv, window):
 
 def test_prefill_window_at_full_size_sampled(da):
     """The 4 x 4k workload with a 1024-key window (a hybrid sliding-window layer), sampled rows."""
-    case = workloads.CONFIGS["c2_bf16_prefill"]
+    case = workloads.CONFIGS["prefill_b4_s4096"]
     inp = workloads.make_prefill(case)
     out = da.prefill_window(*(inp[x].cuda() for x in ("q", "k", "v", "lam")), 1024).cpu()
     assert da.device_error() == 0

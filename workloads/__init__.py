@@ -66,16 +66,16 @@ class DecodeCase:
 # The five workloads of the operator's scope, with their seeds (1000 + index).
 CONFIGS = {
     # tiny fp32 causal prefill, with the planted signal-plus-noise row in pair 0
-    "c1_tiny_fp32_prefill": PrefillCase(B=1, S=128, Hq=4, Hkv=1, D=64, dtype="f32", seed=1000),
+    "tiny_fp32_prefill_b1_s128": PrefillCase(B=1, S=128, Hq=4, Hkv=1, D=64, dtype="f32", seed=1000),
     # bf16 causal prefill at 4 x 4k
-    "c2_bf16_prefill": PrefillCase(B=4, S=4096, Hq=64, Hkv=8, D=128, seed=1001),
+    "prefill_b4_s4096": PrefillCase(B=4, S=4096, Hq=64, Hkv=8, D=128, seed=1001),
     # long-context bf16 causal prefill at 32k
-    "c3_long_bf16_prefill": PrefillCase(B=1, S=32768, Hq=64, Hkv=8, D=128, seed=1002),
+    "prefill_b1_s32768": PrefillCase(B=1, S=32768, Hq=64, Hkv=8, D=128, seed=1002),
     # bf16 decode, one new token per sequence, lengths uniform in [1024, 8192]
-    "c4_bf16_decode": DecodeCase(B=64, Smax=8192, Hq=64, Hkv=8, D=128, len_lo=1024, len_hi=8192,
+    "decode_b64_s8192": DecodeCase(B=64, Smax=8192, Hq=64, Hkv=8, D=128, len_lo=1024, len_hi=8192,
                                  seed=1003),
     # long-context decode with one planted needle key per sequence and V1-style lambda
-    "c5_needle_decode": DecodeCase(B=8, Smax=131072, Hq=64, Hkv=8, D=128, len_lo=131072,
+    "needle_decode_b8_s131072": DecodeCase(B=8, Smax=131072, Hq=64, Hkv=8, D=128, len_lo=131072,
                                    len_hi=131072, seed=1004, needle=True, lambda_kind="v1"),
 }
 
