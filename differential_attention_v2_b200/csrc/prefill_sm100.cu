@@ -9,7 +9,7 @@
 // kernel is persistent: one CTA per SM walks its share of the items, ranked heaviest first
 // (last row tile first) and dealt out to the CTAs in snake order, so the next item's Q and
 // K/V loads and its first score GEMMs overlap the previous item's last softmax and its
-// epilogue (packed sequences launch one CTA per item instead, see launch_prefill). Each 128x128 K and V tile of the shared KV head is brought into shared memory by
+// epilogue. Packed sequences deal out only their non-empty items (see work_item). Each 128x128 K and V tile of the shared KV head is brought into shared memory by
 // TMA ONCE and feeds both heads. The four GEMM blocks per KV tile run on tcgen05 with fp32
 // accumulators in tensor memory:
 //
@@ -56,7 +56,10 @@ constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;      // V stages
 constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;    // mbarriers
 constexpr uint32_t kOffMisc = kOffBar + 256;                  // tmem slot, abort flag
 constexpr uint32_t kOffL = kOffMisc + 64;                     // [item parity][branch][row] fp32 row sums
-constexpr uint32_t kSmemUsed = kOffL + 2 * 2 * BM * 4;
+// packed sequences: sequence ids sorted by row-tile count (longest first), then the counts
+constexpr int kMaxSortedSeqs = 256;
+constexpr uint32_t kOffSeq = kOffL + 2 * 2 * BM * 4;
+constexpr uint32_t kSmemUsed = kOffSeq + 2 * kMaxSortedSeqs * 4;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;             // slack for 1024-B alignment
 
 // mbarrier slots (8 bytes each)
@@ -89,6 +92,7 @@ struct Params {
   const int* cu_seqlens;  // packed sequences: sequence b is tokens cu[b] .. cu[b+1]-1; null = [B,S]
   int n_row_tiles;
   int n_items;            // B * (Hq/2) * n_row_tiles
+  int sorted_seqs;        // packed sequences dealt as a dense list of non-empty items (B <= kMaxSortedSeqs)
   float scale_log2;       // log2(e)/sqrt(D)
 };
 
@@ -101,22 +105,52 @@ struct WorkItem {
   size_t row_base;        // first output row of the sequence
 };
 
+// Walk over the dense list of non-empty packed-sequence items: rank r holds row tile
+// t = n_row_tiles-1-r of the n_seq longest sequences (those with more than t row tiles, a
+// prefix of the sorted list), pair fastest; base is the list index of the rank's first item.
+struct SortedCursor {
+  int r = 0, base = 0, n_seq = 0;
+};
+
 // The k-th item of this CTA; false once they are exhausted. Items are ranked by row tile,
 // last tile first (causal work grows with the tile index), and band k of gridDim.x items goes
-// to the CTAs in ascending order for even k and descending order for odd k.
+// to the CTAs in ascending order for even k and descending order for odd k. With sorted
+// packed sequences only non-empty items are listed (seq_id, seq_nt: sorted ids and row-tile
+// counts; n_dense: the list's length); a role's item indices only grow, so its cursor only
+// moves forward.
 template <bool kVarlen, bool kWindow>
-__device__ __forceinline__ bool work_item(const Params& p, int k, WorkItem& w) {
+__device__ __forceinline__ bool work_item(const Params& p, int k, WorkItem& w, SortedCursor& cur,
+                                          const int* seq_id, const int* seq_nt, int n_dense) {
   const int n_ctas = static_cast<int>(gridDim.x);
   const int c = static_cast<int>(blockIdx.x);
   const int idx = k * n_ctas + ((k & 1) ? n_ctas - 1 - c : c);
-  if (idx >= p.n_items) return false;  // only in the last band; later bands are empty too
   const int n_pairs = p.Hq >> 1;
-  const int per_tile = p.B * n_pairs;
-  const int rank = idx / per_tile;
-  const int bp = idx - rank * per_tile;
-  w.tile = p.n_row_tiles - 1 - rank;
-  w.b = bp / n_pairs;
-  w.pair = bp - w.b * n_pairs;
+  if (kVarlen && p.sorted_seqs) {
+    if (idx >= n_dense) return false;
+    int t = p.n_row_tiles - 1 - cur.r;
+    while (true) {
+      if (t < 0) return false;  // unreachable: the ranks hold exactly n_dense items
+      while (cur.n_seq < p.B && seq_nt[cur.n_seq] > t) ++cur.n_seq;
+      const int n_rank = cur.n_seq * n_pairs;
+      if (idx < cur.base + n_rank) break;
+      cur.base += n_rank;
+      ++cur.r;
+      --t;
+    }
+    const int within = idx - cur.base;
+    const int si = within / n_pairs;
+    w.tile = t;
+    w.b = seq_id[si];
+    w.pair = within - si * n_pairs;
+  } else {
+    if (idx >= p.n_items) return false;  // only in the last band; later bands are empty too
+    const int per_tile = p.B * n_pairs;
+    const int rank = idx / per_tile;
+    const int bp = idx - rank * per_tile;
+    w.tile = p.n_row_tiles - 1 - rank;
+    w.b = bp / n_pairs;
+    w.pair = bp - w.b * n_pairs;
+  }
   w.m0 = w.tile * BM;
   w.S = p.S;
   w.tok0 = 0;
@@ -259,6 +293,9 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   const int n_pairs = p.Hq >> 1;
   const int group = p.Hq / p.Hkv;
 
+  int* seq_id = reinterpret_cast<int*>(smem + kOffSeq);
+  int* seq_nt = seq_id + kMaxSortedSeqs;
+  int* n_dense_slot = reinterpret_cast<int*>(smem + kOffMisc + 16);
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i) {
       uint32_t count = 1;
@@ -268,6 +305,30 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     }
     *abort_flag = 0;
     fence_mbar_init();
+  }
+  if (kVarlen && p.sorted_seqs) {
+    // Sequences by row-tile count, longest first (ties by index). Counts are clamped to
+    // [0, n_row_tiles]: rows past the longest length the caller declared are not computed,
+    // as in the one-CTA-per-item launch. The row-sum array is free until the first epilogue
+    // and holds the counts meanwhile.
+    int* nt = reinterpret_cast<int*>(l_xchg);
+    for (int b = threadIdx.x; b < p.B; b += kThreads) {
+      const int len = __ldg(p.cu_seqlens + b + 1) - __ldg(p.cu_seqlens + b);
+      nt[b] = min(max((len + BM - 1) / BM, 0), p.n_row_tiles);
+    }
+    __syncthreads();
+    for (int b = threadIdx.x; b < p.B; b += kThreads) {
+      const int nb = nt[b];
+      int rank = 0;
+      for (int b2 = 0; b2 < p.B; ++b2) rank += (nt[b2] > nb || (nt[b2] == nb && b2 < b)) ? 1 : 0;
+      seq_id[rank] = b;
+      seq_nt[rank] = nb;
+    }
+    if (threadIdx.x == 0) {
+      int total = 0;
+      for (int b = 0; b < p.B; ++b) total += nt[b];
+      *n_dense_slot = total * (p.Hq >> 1);
+    }
   }
   if (warp == 8 && lane == 0) {
     tma_prefetch_desc(&tmQ);
@@ -282,7 +343,9 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const int n_dense = (kVarlen && p.sorted_seqs) ? *n_dense_slot : 0;
   WorkItem w;
+  SortedCursor cur;
 
   if (warp == 8) {
     // ------------------------------------------------------------------ TMA producer
@@ -290,7 +353,7 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       // Counts over all items of this CTA: KV tiles (ring stage and phase) and Q tiles.
       int k_issued = 0, v_issued = 0, q_issued = 0;
       bool ok = true;
-      for (int k = 0; ok && work_item<kVarlen, kWindow>(p, k, w); ++k) {
+      for (int k = 0; ok && work_item<kVarlen, kWindow>(p, k, w, cur, seq_id, seq_nt, n_dense); ++k) {
         if (w.n_kv == 0) continue;
         // the single Q buffer is free once the previous item's last score GEMM has read it
         if (q_issued > 0 && !(ok = mbar_wait(bar(kQEmpty), (q_issued - 1) & 1, abort_flag))) break;
@@ -363,7 +426,7 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       int n0 = 0;       // KV tiles of earlier items
       int n_items = 0;  // items done
       bool ok = true;
-      for (int k = 0; ok && work_item<kVarlen, kWindow>(p, k, w); ++k) {
+      for (int k = 0; ok && work_item<kVarlen, kWindow>(p, k, w, cur, seq_id, seq_nt, n_dense); ++k) {
         if (w.n_kv == 0) continue;
         if (!(ok = mbar_wait(bar(kQFull), n_items & 1, abort_flag))) break;
         for (int j = 0; j < w.n_kv; ++j) {
@@ -419,7 +482,7 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     int n_items = 0;  // items done
     bool ok = true;
 
-    for (int k = 0; ok && work_item<kVarlen, kWindow>(p, k, w); ++k) {
+    for (int k = 0; ok && work_item<kVarlen, kWindow>(p, k, w, cur, seq_id, seq_nt, n_dense); ++k) {
       if (w.n_kv == 0) continue;
       const int qi = w.m0 + r;  // query index of this row within its sequence
       const int S = w.S;
@@ -596,6 +659,7 @@ cudaError_t launch_prefill(const CUtensorMap& tmQ, const CUtensorMap& tmK, const
   p.cu_seqlens = cu_seqlens;  // with packed sequences S is the longest sequence's length
   p.n_row_tiles = (S + BM - 1) / BM;
   p.n_items = B * (Hq / 2) * p.n_row_tiles;
+  p.sorted_seqs = (cu_seqlens != nullptr && B <= kMaxSortedSeqs) ? 1 : 0;
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HD));
   auto kernel = cu_seqlens ? diffattn_prefill_sm100<true, false>
                            : (window > 0 ? diffattn_prefill_sm100<false, true> : diffattn_prefill_sm100<false, false>);
@@ -608,10 +672,13 @@ cudaError_t launch_prefill(const CUtensorMap& tmQ, const CUtensorMap& tmK, const
   if (e != cudaSuccess) return e;
   if (p.n_items == 0) return cudaSuccess;
   // Persistent: one CTA per SM (the shared memory admits one), each walking its items. Packed
-  // sequences of mixed length leave many items empty (row tiles past a short sequence's end),
-  // which a static deal spreads unevenly; there every item gets its own CTA and the hardware's
-  // CTA scheduler balances them (measured: 800 vs 745 TFLOP/s for 8 sequences of 512-3584).
-  const int n_ctas = (cu_seqlens != nullptr || p.n_items < n_sms) ? p.n_items : n_sms;
+  // sequences of mixed length leave many items empty (row tiles past a short sequence's end);
+  // up to kMaxSortedSeqs sequences the CTAs deal out only the non-empty ones (p.sorted_seqs),
+  // beyond that every item of the full grid gets its own CTA and the hardware's CTA scheduler
+  // balances them (a static deal that includes the empty items measured 745 against 800
+  // TFLOP/s for 8 sequences of 512-3584 tokens).
+  const bool one_per_item = cu_seqlens != nullptr && !p.sorted_seqs;
+  const int n_ctas = (one_per_item || p.n_items < n_sms) ? p.n_items : n_sms;
   kernel<<<n_ctas, kThreads, kSmemBytes, stream>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError();
 }

@@ -111,10 +111,14 @@ DA2_API int diffattn_v2_prefill_window(const void* q, const void* k, const void*
  * keys, causally when causal = 1).
  *   q bf16 [T,Hq,D]   k, v bf16 [T,Hkv,D]   lambda fp32 [T,Hq/2]   out bf16 [T,Hq/2,D]
  *   cu_seqlens int32 [B+1] (device), non-decreasing, cu_seqlens[0] = 0, cu_seqlens[B] = T
- *   max_seqlen >= the longest sequence (sizes the grid; longer values only add idle CTAs)
+ *   max_seqlen >= the longest sequence (bounds the row tiles a sequence can have; rows of a
+ *   sequence past max_seqlen are not computed)
  *   total_tokens = T
  * The caller guarantees the cu_seqlens contract; the kernel reads it on the device, so the
  * call needs no host synchronisation. Supported: D == 128. Zero-length sequences are allowed.
+ * Schedule: up to 256 sequences, persistent CTAs (one per SM) sort the sequences by length
+ * on the device and deal out only the non-empty (sequence, pair, 128-row tile) items; with
+ * more sequences every item of the B x pairs x ceil(max_seqlen/128) grid gets its own CTA.
  */
 DA2_API int diffattn_v2_prefill_varlen(const void* q, const void* k, const void* v, const float* lambda,
                                        void* out, const int32_t* cu_seqlens, int B, int max_seqlen,

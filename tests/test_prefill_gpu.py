@@ -149,12 +149,19 @@ def test_prefill_window_at_full_size_sampled(da):
     bf16_close(got, ref, "window 1024 sampled rows")
 
 
-@pytest.mark.parametrize("lens,Hq,Hkv,causal", [
-    ([300, 1, 0, 129, 128, 77], 8, 2, True),       # ragged, single token, empty, tile edges
-    ([1000, 513], 16, 2, True),
-    ([200, 64, 390], 8, 1, False),                 # non-causal packed sequences
+_MANY_LENS = [int(x) for x in np.random.default_rng(300).integers(0, 41, size=300)]
+
+
+@pytest.mark.parametrize("lens,Hq,Hkv,causal,extra", [
+    ([300, 1, 0, 129, 128, 77], 8, 2, True, 0),       # ragged, single token, empty, tile edges
+    ([1000, 513], 16, 2, True, 0),
+    ([200, 64, 390], 8, 1, False, 0),                 # non-causal packed sequences
+    # longest length declared above the true one: the top row tiles hold no sequence
+    ([700, 5, 0, 1300, 260, 129], 8, 2, True, 400),
+    # more sequences than the kernel sorts in shared memory: one CTA per item
+    (_MANY_LENS, 4, 2, True, 0),
 ])
-def test_prefill_varlen_matches_oracle(da, lens, Hq, Hkv, causal):
+def test_prefill_varlen_matches_oracle(da, lens, Hq, Hkv, causal, extra):
     T = sum(lens)
     g = torch.Generator().manual_seed(T)
     q = torch.randn(T, Hq, 128, generator=g).bfloat16()
@@ -162,7 +169,7 @@ def test_prefill_varlen_matches_oracle(da, lens, Hq, Hkv, causal):
     v = torch.randn(T, Hkv, 128, generator=g).bfloat16()
     lam = torch.sigmoid(torch.randn(T, Hq // 2, generator=g))
     cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32)
-    out = da.prefill_varlen(q.cuda(), k.cuda(), v.cuda(), lam.cuda(), cu.cuda(), max(lens), causal=causal)
+    out = da.prefill_varlen(q.cuda(), k.cuda(), v.cuda(), lam.cuda(), cu.cuda(), max(lens) + extra, causal=causal)
     assert da.device_error() == 0
     ref = ora.prefill_varlen(q, k, v, lam, cu.tolist(), causal=causal)
     bf16_close(out, ref, f"varlen {lens}")
@@ -178,6 +185,19 @@ def test_prefill_varlen_equals_batched(da):
     cu = torch.tensor([0, 333, 666, 999], dtype=torch.int32, device="cuda")
     packed = da.prefill_varlen(flat(d["q"]), flat(d["k"]), flat(d["v"]), flat(d["lam"]), cu, 333)
     assert torch.equal(packed.view(3, 333, 8, 128), batched)
+
+
+def test_prefill_varlen_many_sequences_equals_batched(da):
+    """300 equal-length packed sequences (one CTA per item) give the batched output bit for bit."""
+    case = workloads.PrefillCase(B=300, S=150, Hq=4, Hkv=2, D=128, seed=9)
+    inp = workloads.make_prefill(case)
+    d = _dev(inp)
+    batched = da.prefill(d["q"], d["k"], d["v"], d["lam"])
+    flat = lambda t: t.reshape(-1, *t.shape[2:]).contiguous()
+    cu = torch.arange(0, 301 * 150, 150, dtype=torch.int32, device="cuda")
+    packed = da.prefill_varlen(flat(d["q"]), flat(d["k"]), flat(d["v"]), flat(d["lam"]), cu, 150)
+    assert da.device_error() == 0
+    assert torch.equal(packed.view(300, 150, 2, 128), batched)
 
 
 def test_prefill_rejects_bad_arguments_on_gpu(da):
