@@ -350,7 +350,8 @@ DA2_API int diffattn_v2_lambda_v2(const void* x, const void* w_lambda, const flo
 /*
  * Synchronise `stream`, then read and clear the device error word that kernels set when a
  * bounded wait expires. *code receives 0 when no kernel reported an error, else the code
- * of the first error recorded (1 = pipeline wait expired in prefill, 2 = in decode).
+ * of the first error recorded (a pipeline wait expired: 1 = in a prefill, 2 = in a decode,
+ * 3 = in a backward kernel).
  * Returns DA2_ERR_DEVICE when *code != 0, DA2_OK when it is 0, DA2_ERR_CUDA on a CUDA
  * failure. `code` is a HOST pointer and may be NULL.
  */
