@@ -18,11 +18,12 @@
 //                  [256,384) O1 += P1 V
 //                  [384,512) O2 += P2 V
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads):
 //   warps 0-3  softmax of branch 1 (head 2p): thread r owns query row r of the tile
 //   warps 4-7  softmax of branch 2 (head 2p+1)
 //   warp 8     TMA producer (Q per item, K/V tiles through a 2-stage ring across items)
 //   warp 9     tcgen05 MMA issuer; also allocates and frees tensor memory
+//   warps 10-11 idle: they complete warpgroup 2, which hands its registers to warps 0-7
 //
 // Issue order on the tensor core for KV tile j: S1_j, PV2_{j-1}, S2_j, PV1_j. Softmax of
 // branch 1 on S1_j overlaps PV2_{j-1} and S2_j; softmax of branch 2 on S2_j overlaps PV1_j
@@ -44,7 +45,15 @@ namespace prefill {
 constexpr int BM = 128;  // query rows per CTA
 constexpr int BN = 128;  // keys per KV tile
 constexpr int HD = 128;  // head dim
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+// Register split (setmaxnreg, per warpgroup): the kernel launches with kRegsLaunch per thread;
+// warpgroup 2 (producer, MMA issuer, two idle warps) gives registers back so the two softmax
+// warpgroups can hold a row's 128 scores and its packed P without spilling. The shares add up
+// to no more than the launch total (128 * 96 + 256 * 200 = 63,488 <= 384 * 168 = 64,512; per SM
+// sub-partition, whose warps are w, w+4, w+8: (200 + 200 + 96) * 32 <= 16,384). ptxas compiles
+// each role's code to its share: at 200 the softmax path has no spills (at 168 it spilled).
+constexpr int kRegsLaunch = 168, kRegsSmall = 96, kRegsSoftmax = 200;
+static_assert(128 * kRegsSmall + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split exceeds the launch");
 constexpr int kStages = 2;
 
 constexpr uint32_t kChunkBytes = 128 * 64 * 2;     // 128 rows x 64 bf16 (one swizzle-128B half)
@@ -347,6 +356,8 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   WorkItem w;
   SortedCursor cur;
 
+  if (warp >= 8) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsSmall));
   if (warp == 8) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -471,8 +482,10 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       volatile int no_abort = 0;
       mbar_wait(bar(kDrain), 0, &no_abort);
     }
+  }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     const int br = warp >> 2;               // branch 0 (head 2p) or 1 (head 2p+1)
     const int r = threadIdx.x & 127;        // row of the tile == TMEM lane
     const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
