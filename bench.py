@@ -59,7 +59,7 @@ SPEC_HBM_GBS = 8000.0
 NCU_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one launch (B=4 x 4k causal prefill),
     # mean of two captured launches
-    "prefill": {"bytes": 590108928, "source_sha": "444eb8eba10d43a2"},
+    "prefill": {"bytes": 567917696, "source_sha": "ab645937d13ae3b9"},
     # split + combine of one B=64 decode step, mean of two captured steps
     "decode": {"bytes": 1240836992, "source_sha": "5a98bc5cb2987830"},
 }
