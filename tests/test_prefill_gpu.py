@@ -46,6 +46,37 @@ def test_prefill_bf16_matches_oracle(da, B, S, Hq, Hkv, causal):
     bf16_close(out, ref, f"prefill B={B} S={S} Hq={Hq} Hkv={Hkv} causal={causal}")
 
 
+# Launches with several work items per CTA (one persistent CTA per SM on 148 SMs): item
+# boundaries, both parities of the per-item barriers and row-sum buffers, odd and even bands.
+@pytest.mark.parametrize("B,S,Hq,Hkv,causal,window", [
+    (8, 1024, 32, 4, True, 0),     # 1024 items, ~7 per CTA, causal work 1..8 KV tiles
+    (6, 700, 16, 2, False, 0),     # 288 items, all of equal work, ragged last key tile
+    (8, 1024, 32, 4, True, 200),   # sliding window over many items
+])
+def test_prefill_many_items_per_cta(da, B, S, Hq, Hkv, causal, window):
+    inp = workloads.make_prefill(workloads.PrefillCase(B=B, S=S, Hq=Hq, Hkv=Hkv, D=128, seed=3 * S + window))
+    d = _dev(inp)
+    if window:
+        out = da.prefill_window(d["q"], d["k"], d["v"], d["lam"], window)
+    else:
+        out = da.prefill(d["q"], d["k"], d["v"], d["lam"], causal=causal)
+    assert da.device_error() == 0
+    ref = ora.prefill(inp["q"], inp["k"], inp["v"], inp["lam"], causal=causal, window=window or None)
+    bf16_close(out, ref, f"many items B={B} S={S} Hq={Hq} causal={causal} window={window}")
+
+
+def test_prefill_train_many_items_per_cta(da):
+    """The training forward's per-head O_b and row lse over 256 items (~2 per CTA)."""
+    inp = workloads.make_prefill(workloads.PrefillCase(B=4, S=1024, Hq=16, Hkv=2, D=128, seed=77))
+    d = _dev(inp)
+    out, ob, lse = da.prefill_train(d["q"], d["k"], d["v"], d["lam"])
+    assert da.device_error() == 0
+    assert torch.equal(out, da.prefill(d["q"], d["k"], d["v"], d["lam"]))
+    o_ref, lse_ref = ora.prefill_branches(inp["q"], inp["k"], inp["v"])
+    bf16_close(ob, o_ref, "o_branch, many items")
+    assert float(np.abs(lse.double().cpu().numpy() - lse_ref).max()) < 1e-3, "lse"
+
+
 def test_prefill_bf16_lambda_edge_values(da):
     """lambda negative, zero and above one (V1 values may be any real number)."""
     inp = workloads.make_prefill(workloads.PrefillCase(B=1, S=200, Hq=8, Hkv=1, D=128, seed=5))
