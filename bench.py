@@ -6,7 +6,8 @@ One step is one pass of the whole hot path over one batch of synthetic input:
   * prefill: causal bf16 DiffAttn V2 over B=4 x S=4096, Hq=64 (32 pairs), Hkv=8, D=128
     (one tcgen05 kernel launch), then
   * decode: one bf16 decode step for 64 sequences with lengths uniform in [1024, 8192]
-    over an [64, 8192, 8, 128] KV cache (split kernel + combine kernel).
+    over an [64, 8192, 8, 128] KV cache (one split-KV kernel whose last split per (b, KV head)
+    merges the partials; a memset of its split counters precedes it).
 `value` is the prefill throughput in TFLOP/s (algorithmic FLOPs = 4*D*Hq*B*S(S+1)/2 over
 the prefill kernel's CUDA-event time inside the timed steps); the decode throughput in
 GB/s (every visible K/V row once, plus q, lambda and out) is reported beside it.
@@ -60,8 +61,8 @@ NCU_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one launch (B=4 x 4k causal prefill),
     # mean of two captured launches
     "prefill": {"bytes": 567917696, "source_sha": "ab645937d13ae3b9"},
-    # split + combine of one B=64 decode step, mean of two captured steps
-    "decode": {"bytes": 1240836992, "source_sha": "5a98bc5cb2987830"},
+    # one B=64 decode step (split kernel with the fused merge), mean of two captured steps
+    "decode": {"bytes": 1238145408, "source_sha": "d524185fe62fafcb"},
 }
 
 
@@ -380,7 +381,7 @@ def run_ours(args, rank, world, local, dist):
                     "from pinned host memory, runs both kernels through the C ABI and copies both "
                     "outputs back",
         },
-        "gpu_launches": (int(do_pre) + 2 * int(do_dec)) * K,
+        "gpu_launches": (int(do_pre) + int(do_dec)) * K,
         "clocks": clk,
     }
     if args.only:
@@ -579,7 +580,7 @@ def run_workload(args):
             lam = inp["lam"].to(dev)
         q = inp["q"].to(dev)
         nbytes = workloads.decode_bytes(inp["seqlens"].tolist(), case.Hkv, D, case.Hq)
-        launches = 2
+        launches = 1
         if name == "paged":
             ps = 64
             max_pages = case.Smax // ps

@@ -374,7 +374,9 @@ size_t diffattn_v2_decode_workspace_size(int B, int Smax, int Hq, int Hkv, int D
   int split_len = 0, nsplit = 0;
   da2::decode_split_plan(B, Smax, Hkv, &split_len, &nsplit);
   const size_t rows = static_cast<size_t>(B) * Hq * nsplit;
-  return rows * static_cast<size_t>(D) * sizeof(float) + rows * 2 * sizeof(float);
+  // partials O, (m, l), then one split counter per (b, KV head)
+  return rows * static_cast<size_t>(D) * sizeof(float) + rows * 2 * sizeof(float) +
+         (static_cast<size_t>(B) * Hkv * sizeof(int) + 15) / 16 * 16;
 }
 
 int diffattn_v2_decode(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens,
@@ -400,8 +402,10 @@ int diffattn_v2_decode(const void* q, const void* kcache, const void* vcache, co
   if (encode_bshd(&tv, vcache, D, Hkv, Smax, B, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
   float* ws_o = static_cast<float*>(workspace);
   float* ws_ml = ws_o + static_cast<size_t>(B) * Hq * nsplit * D;
+  int* counters = reinterpret_cast<int*>(ws_ml + static_cast<size_t>(B) * Hq * nsplit * 2);
   e = da2::launch_decode(tk, tv, static_cast<const __nv_bfloat16*>(q), seqlens, lambda,
-                         static_cast<__nv_bfloat16*>(out), ws_o, ws_ml, err, B, Smax, Hq, Hkv, nsplit, split_len,
+                         static_cast<__nv_bfloat16*>(out), ws_o, ws_ml, counters, err, B, Smax, Hq, Hkv, nsplit,
+                         split_len,
                          nullptr, 0, 0, 1, reinterpret_cast<cudaStream_t>(stream));
   return status_of(e);
 }
@@ -436,8 +440,10 @@ int diffattn_v2_decode_paged(const void* q, const void* kpages, const void* vpag
   if (encode_bshd(&tv, vpages, D, Hkv, page_size, num_pages, 64, box) != cudaSuccess) return DA2_ERR_CUDA;
   float* ws_o = static_cast<float*>(workspace);
   float* ws_ml = ws_o + static_cast<size_t>(B) * Hq * nsplit * D;
+  int* counters = reinterpret_cast<int*>(ws_ml + static_cast<size_t>(B) * Hq * nsplit * 2);
   e = da2::launch_decode(tk, tv, static_cast<const __nv_bfloat16*>(q), seqlens, lambda,
-                         static_cast<__nv_bfloat16*>(out), ws_o, ws_ml, err, B, Smax, Hq, Hkv, nsplit, split_len,
+                         static_cast<__nv_bfloat16*>(out), ws_o, ws_ml, counters, err, B, Smax, Hq, Hkv, nsplit,
+                         split_len,
                          block_table, max_pages, page_shift, 1, reinterpret_cast<cudaStream_t>(stream));
   return status_of(e);
 }
@@ -447,7 +453,8 @@ size_t diffattn_v2_decode_multi_workspace_size(int B, int T, int Smax, int Hq, i
   int split_len = 0, nsplit = 0;
   da2::decode_split_plan(B, Smax, Hkv, &split_len, &nsplit);
   const size_t rows = static_cast<size_t>(B) * T * Hq * nsplit;
-  return rows * static_cast<size_t>(D) * sizeof(float) + rows * 2 * sizeof(float);
+  return rows * static_cast<size_t>(D) * sizeof(float) + rows * 2 * sizeof(float) +
+         (static_cast<size_t>(B) * Hkv * sizeof(int) + 15) / 16 * 16;
 }
 
 int diffattn_v2_decode_multi(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens,
@@ -474,8 +481,10 @@ int diffattn_v2_decode_multi(const void* q, const void* kcache, const void* vcac
   if (encode_bshd(&tv, vcache, D, Hkv, Smax, B, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
   float* ws_o = static_cast<float*>(workspace);
   float* ws_ml = ws_o + static_cast<size_t>(B) * T * Hq * nsplit * D;
+  int* counters = reinterpret_cast<int*>(ws_ml + static_cast<size_t>(B) * T * Hq * nsplit * 2);
   e = da2::launch_decode(tk, tv, static_cast<const __nv_bfloat16*>(q), seqlens, lambda,
-                         static_cast<__nv_bfloat16*>(out), ws_o, ws_ml, err, B, Smax, Hq, Hkv, nsplit, split_len,
+                         static_cast<__nv_bfloat16*>(out), ws_o, ws_ml, counters, err, B, Smax, Hq, Hkv, nsplit,
+                         split_len,
                          nullptr, 0, 0, T, reinterpret_cast<cudaStream_t>(stream));
   return status_of(e);
 }

@@ -1,4 +1,4 @@
-// decode_sm100.cu -- bf16 DiffAttn V2 decode step: split-KV streaming kernel + combine.
+// decode_sm100.cu -- bf16 DiffAttn V2 decode step: split-KV streaming kernel with a fused combine.
 //
 // Operator ("Differential Attention (V2)" lesson, "The differential concept" and "V1 vs V2";
 // pairing per "Differential Transformer V2 soll KI-Training stabiler machen", shared-KV
@@ -23,11 +23,15 @@
 //  * Online softmax per head in the log2 domain. Each warp keeps its own (m, l, O^T); at
 //    the end of the CTA the four warps merge through shared memory and write one partial
 //    (m, l, O unnormalised) per head and split to the workspace.
-//  * The combine kernel (one warp per (b, pair)) merges the splits of both heads with the
-//    log-sum-exp rule and writes O1/L1 - lambda O2/L2, rounded once to bf16.
+//  * Combine, fused: each working split of (b, g) counts itself on a per-(b, g) counter
+//    once its partials are visible device-wide; the split that completes the count merges
+//    all splits of the group's pairs with the log-sum-exp rule (one warp per pair) and
+//    writes O1/L1 - lambda O2/L2, rounded once to bf16. No second kernel, no launch gap.
 //
 // The grid is sized from Smax on the host; CTAs whose split starts past seqlens[b] return
-// at once and the combine reads only the splits that exist, so no host sync is needed.
+// at once (split 0 of an empty sequence writes its zero output) and the merge reads only the
+// splits that exist, so no host sync is needed. The counters are zeroed on the stream
+// before each launch.
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -52,8 +56,11 @@ constexpr uint32_t kSmemBytes = kSmemUsed + 1024;
 struct Params {
   const __nv_bfloat16* q;   // [B,Hq,D]
   const int32_t* seqlens;   // [B]
-  float* ws_o;              // [B,Hq,nsplit,D]
-  float* ws_ml;             // [B,Hq,nsplit,2]
+  float* ws_o;              // [B,T,Hq,nsplit,D]
+  float* ws_ml;             // [B,T,Hq,nsplit,2]
+  int* counters;            // [B,Hkv] working splits done, zero at launch
+  const float* lambda;      // [B,T,Hq/2]
+  __nv_bfloat16* out;       // [B,T,Hq/2,D]
   int* err;
   int B, Smax, Hq, Hkv, nsplit, split_len;
   int T;                    // new tokens per sequence (1: plain decode); T * group <= 16
@@ -63,6 +70,45 @@ struct Params {
   const int32_t* block_table;
   int max_pages, page_shift, box_tok;  // page_size = 1 << page_shift; tokens per TMA box
 };
+
+// One warp merges the splits of both heads of `pair` for row bt = b * T + token and writes
+// O1/L1 - lambda O2/L2. Splits past the token's visible keys hold (m = -inf, l = 0, O = 0) and
+// weigh 0. The partials were written by other CTAs of this grid: they are read through L2.
+__device__ __forceinline__ void combine_pair(const Params& p, int bt, int pair, int ns, int lane) {
+  const int n_pairs = p.Hq >> 1;
+  float res[2][4];
+#pragma unroll
+  for (int br = 0; br < 2; ++br) {
+    const size_t row0 = (static_cast<size_t>(bt) * p.Hq + 2 * pair + br) * p.nsplit;
+    float M = -INFINITY;
+    for (int s = lane; s < ns; s += 32) M = fmaxf(M, __ldcg(p.ws_ml + (row0 + s) * 2));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    const float Mu = (M == -INFINITY) ? 0.f : M;
+    float L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < ns; ++s) {
+      const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.ws_ml) + row0 + s);
+      const float sc = fast_exp2(ml.x - Mu);
+      L += ml.y * sc;
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(p.ws_o + (row0 + s) * HD) + lane);
+      acc.x += v.x * sc;
+      acc.y += v.y * sc;
+      acc.z += v.z * sc;
+      acc.w += v.w * sc;
+    }
+    const float inv = (L > 0.f) ? 1.f / L : 0.f;
+    res[br][0] = __fmul_rn(acc.x, inv);
+    res[br][1] = __fmul_rn(acc.y, inv);
+    res[br][2] = __fmul_rn(acc.z, inv);
+    res[br][3] = __fmul_rn(acc.w, inv);
+  }
+  const float lam = __ldg(p.lambda + static_cast<size_t>(bt) * n_pairs + pair);
+  uint2 packed;
+  packed.x = pack_bf16x2(__fmaf_rn(-lam, res[1][0], res[0][0]), __fmaf_rn(-lam, res[1][1], res[0][1]));
+  packed.y = pack_bf16x2(__fmaf_rn(-lam, res[1][2], res[0][2]), __fmaf_rn(-lam, res[1][3], res[0][3]));
+  reinterpret_cast<uint2*>(p.out + (static_cast<size_t>(bt) * n_pairs + pair) * HD)[lane] = packed;
+}
 
 // NT = number of 8-head column tiles per group (1 for group size <= 8, 2 for 16).
 template <int NT>
@@ -78,15 +124,25 @@ diffattn_decode_split(const __grid_constant__ CUtensorMap tmK, const __grid_cons
   auto empty = [&](int s) -> uint32_t { return sbase + kOffBar + 8u * (kStages + s); };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc);
 
-  // the combine kernel may be scheduled now; it waits for this grid's results before reading
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int split = blockIdx.x;
   const int g = blockIdx.y;
   const int b = blockIdx.z;
   const int group = p.Hq / p.Hkv;
   const int seqlen = min(max(__ldg(p.seqlens + b), 0), p.Smax);
   const int t0 = split * p.split_len;
-  if (t0 >= seqlen) return;  // uniform for the CTA: nothing to read, nothing written
+  if (t0 >= seqlen) {  // uniform for the CTA: nothing to read
+    if (split == 0) {
+      // an empty sequence has no working split to merge it: its outputs are zero
+      const int pairs_g = group >> 1, n_pairs = p.Hq >> 1;
+      for (int i = threadIdx.x; i < p.T * pairs_g * (HD / 8); i += blockDim.x) {
+        const int c = i % (HD / 8), r = i / (HD / 8);
+        const int pair = g * pairs_g + r % pairs_g;
+        reinterpret_cast<uint4*>(p.out + (static_cast<size_t>(b) * p.T + r / pairs_g) * n_pairs * HD +
+                                 static_cast<size_t>(pair) * HD)[c] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    return;
+  }
   const int t1 = min(t0 + p.split_len, seqlen);
   const int n_stages = (t1 - t0 + kTok - 1) / kTok;
 
@@ -334,65 +390,28 @@ diffattn_decode_split(const __grid_constant__ CUtensorMap tmK, const __grid_cons
       }
     }
   }
-}
 
-// One warp per (b, new token, pair): merge the splits of both heads and apply the lambda
-// subtraction. Splits past a token's visible keys hold (m = -inf, l = 0, O = 0) and weigh 0.
-__global__ void __launch_bounds__(128)
-diffattn_decode_combine(const float* __restrict__ ws_o, const float* __restrict__ ws_ml,
-                        const int32_t* __restrict__ seqlens, const float* __restrict__ lambda,
-                        __nv_bfloat16* __restrict__ out, int B, int T, int Smax, int Hq, int nsplit, int split_len) {
-  // launched as a programmatic dependent of the split kernel: wait until its partials are
-  // complete and visible
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int n_pairs = Hq >> 1;
-  const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (wid >= B * T * n_pairs) return;
-  const int bt = wid / n_pairs;  // b * T + token
-  const int b = bt / T;
-  const int pair = wid % n_pairs;
-  const int n = min(max(__ldg(seqlens + b), 0), Smax);
-  const int ns = (n + split_len - 1) / split_len;
-  float res[2][4];
-#pragma unroll
-  for (int br = 0; br < 2; ++br) {
-    const size_t row0 = (static_cast<size_t>(bt) * Hq + 2 * pair + br) * nsplit;
-    float M = -INFINITY;
-    for (int s = lane; s < ns; s += 32) M = fmaxf(M, __ldg(ws_ml + (row0 + s) * 2));
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    const float Mu = (M == -INFINITY) ? 0.f : M;
-    float L = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < ns; ++s) {
-      const float2 ml = __ldg(reinterpret_cast<const float2*>(ws_ml) + row0 + s);
-      const float sc = fast_exp2(ml.x - Mu);
-      L += ml.y * sc;
-      const float4 v = __ldg(reinterpret_cast<const float4*>(ws_o + (row0 + s) * HD) + lane);
-      acc.x += v.x * sc;
-      acc.y += v.y * sc;
-      acc.z += v.z * sc;
-      acc.w += v.w * sc;
-    }
-    const float inv = (L > 0.f) ? 1.f / L : 0.f;
-    res[br][0] = __fmul_rn(acc.x, inv);
-    res[br][1] = __fmul_rn(acc.y, inv);
-    res[br][2] = __fmul_rn(acc.z, inv);
-    res[br][3] = __fmul_rn(acc.w, inv);
-  }
-  const float lam = __ldg(lambda + static_cast<size_t>(bt) * n_pairs + pair);
-  uint2 packed;
-  packed.x = pack_bf16x2(__fmaf_rn(-lam, res[1][0], res[0][0]), __fmaf_rn(-lam, res[1][1], res[0][1]));
-  packed.y = pack_bf16x2(__fmaf_rn(-lam, res[1][2], res[0][2]), __fmaf_rn(-lam, res[1][3], res[0][3]));
-  reinterpret_cast<uint2*>(out + (static_cast<size_t>(bt) * n_pairs + pair) * HD)[lane] = packed;
+  // ---- fused combine: count this split once its partials are visible device-wide; the
+  // split that completes the count for (b, g) merges the group's pairs
+  __threadfence();
+  __syncthreads();
+  volatile int* last_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+  const int ns = (seqlen + p.split_len - 1) / p.split_len;  // working splits of sequence b
+  if (threadIdx.x == 0)
+    *last_flag = (atomicAdd(p.counters + static_cast<size_t>(b) * p.Hkv + g, 1) == ns - 1) ? 1 : 0;
+  __syncthreads();
+  if (!*last_flag) return;
+  __threadfence();  // the other splits' partials, counted before ours, are visible
+  const int pairs_g = group >> 1;
+  for (int item = warp; item < p.T * pairs_g; item += kConsumerWarps + 1)
+    combine_pair(p, b * p.T + item / pairs_g, g * pairs_g + item % pairs_g, ns, lane);
 }
 
 }  // namespace decode
 
 cudaError_t launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const __nv_bfloat16* q,
                           const int32_t* seqlens, const float* lambda, __nv_bfloat16* out, float* ws_o,
-                          float* ws_ml, int* err, int B, int Smax, int Hq, int Hkv, int nsplit,
+                          float* ws_ml, int* counters, int* err, int B, int Smax, int Hq, int Hkv, int nsplit,
                           int split_len, const int32_t* block_table, int max_pages, int page_shift, int T,
                           cudaStream_t stream) {
   using namespace decode;
@@ -401,6 +420,9 @@ cudaError_t launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const 
   p.seqlens = seqlens;
   p.ws_o = ws_o;
   p.ws_ml = ws_ml;
+  p.counters = counters;
+  p.lambda = lambda;
+  p.out = out;
   p.err = err;
   p.B = B;
   p.Smax = Smax;
@@ -416,7 +438,8 @@ cudaError_t launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const 
   p.box_tok = block_table ? min(1 << page_shift, kTok) : kTok;
   const int group = Hq / Hkv;
   dim3 grid(nsplit, Hkv, B);
-  cudaError_t e;
+  cudaError_t e = cudaMemsetAsync(counters, 0, static_cast<size_t>(B) * Hkv * sizeof(int), stream);
+  if (e != cudaSuccess) return e;
   if (T * group > 8) {
     e = cudaFuncSetAttribute(diffattn_decode_split<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -426,22 +449,7 @@ cudaError_t launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const 
     if (e != cudaSuccess) return e;
     diffattn_decode_split<1><<<grid, kThreads, kSmemBytes, stream>>>(tmK, tmV, p);
   }
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  // the combine overlaps its launch with the split kernel's tail (programmatic dependent launch)
-  const int warps = B * T * (Hq / 2);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((warps + 3) / 4);
-  cfg.blockDim = dim3(128);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, diffattn_decode_combine, static_cast<const float*>(ws_o),
-                            static_cast<const float*>(ws_ml), seqlens, lambda, out, B, T, Smax, Hq, nsplit, split_len);
+  return cudaGetLastError();
 }
 
 }  // namespace da2

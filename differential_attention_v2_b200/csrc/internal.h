@@ -41,7 +41,7 @@ cudaError_t launch_backward_sm100(const CUtensorMap& tmQ64, const CUtensorMap& t
 // Smax = max_pages << page_shift. T new tokens per sequence (q [B,T,Hq,D]); T * Hq/Hkv <= 16.
 cudaError_t launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const __nv_bfloat16* q,
                           const int32_t* seqlens, const float* lambda, __nv_bfloat16* out, float* ws_o,
-                          float* ws_ml, int* err, int B, int Smax, int Hq, int Hkv, int nsplit,
+                          float* ws_ml, int* counters, int* err, int B, int Smax, int Hq, int Hkv, int nsplit,
                           int split_len, const int32_t* block_table, int max_pages, int page_shift, int T,
                           cudaStream_t stream);
 

@@ -233,10 +233,12 @@ DA2_API size_t diffattn_v2_decode_workspace_size(int B, int Smax, int Hq, int Hk
  *            16-byte aligned, owned by the caller; calls that share one workspace must not
  *            overlap on the GPU.
  * A sequence with seqlens[b] == 0 gets an all-zero output. Supported: D == 128 and a GQA
- * group size Hq/Hkv in {2, 4, 8, 16}. Kernels: a split-KV streaming kernel (TMA-staged
- * K/V, every visible K/V row read once for all query heads of the group) and a combine
- * kernel merging the per-split (max, sum, output) partials of both branches. The grid is
- * sized from Smax on the host, so the call needs no host synchronisation.
+ * group size Hq/Hkv in {2, 4, 8, 16}. One kernel after a small memset of the workspace's
+ * split counters: split-KV streaming CTAs (TMA-staged K/V, every visible K/V row read once
+ * for all query heads of the group), the last of a (b, KV head)'s splits merging the
+ * per-split (max, sum, output) partials of both branches. The workspace needs no
+ * initialisation. The grid is sized from Smax on the host, so the call needs no host
+ * synchronisation.
  */
 DA2_API int diffattn_v2_decode(const void* q, const void* kcache, const void* vcache,
                        const int32_t* seqlens, const float* lambda, void* out, int B, int Smax,
