@@ -60,7 +60,7 @@ SPEC_HBM_GBS = 8000.0
 NCU_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one launch (B=4 x 4k causal prefill),
     # mean of two captured launches
-    "prefill": {"bytes": 567917696, "source_sha": "ab645937d13ae3b9"},
+    "prefill": {"bytes": 567917696, "source_sha": "1e095f03b271b255"},
     # one B=64 decode step (split kernel with the fused merge), mean of two captured steps
     "decode": {"bytes": 1238145408, "source_sha": "d524185fe62fafcb"},
 }

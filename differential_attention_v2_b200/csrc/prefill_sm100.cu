@@ -357,132 +357,132 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   SortedCursor cur;
 
   if (warp >= 8) {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsSmall));
-  if (warp == 8) {
-    // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      // Counts over all items of this CTA: KV tiles (ring stage and phase) and Q tiles.
-      int k_issued = 0, v_issued = 0, q_issued = 0;
-      bool ok = true;
-      for (int k = 0; ok && work_item<kVarlen, kWindow>(p, k, w, cur, seq_id, seq_nt, n_dense); ++k) {
-        if (w.n_kv == 0) continue;
-        // the single Q buffer is free once the previous item's last score GEMM has read it
-        if (q_issued > 0 && !(ok = mbar_wait(bar(kQEmpty), (q_issued - 1) & 1, abort_flag))) break;
-        mbar_arrive_expect_tx(bar(kQFull), 2 * kTileBytes);
-        for (int h = 0; h < 2; ++h)
-          for (int c = 0; c < 2; ++c)
-            tma_load_4d(sbase + kOffQ + h * kTileBytes + c * kChunkBytes, &tmQ, bar(kQFull), c * 64,
-                        2 * w.pair + h, w.tok0 + w.m0, w.tb);
-        ++q_issued;
-        const int g = (2 * w.pair) / group;
-        for (int it = 0; it < w.n_kv; ++it) {
-          const int j = w.j_first + it;
-          const int n = k_issued;  // this CTA's KV tile count so far
-          const int s = n & 1;
-          const uint32_t ph = (n >> 1) & 1;
-          if (!(ok = mbar_wait(bar(kKEmpty + s), ph ^ 1, abort_flag))) break;
-          mbar_arrive_expect_tx(bar(kKFull + s), kTileBytes);
-          for (int c = 0; c < 2; ++c)
-            tma_load_4d(sbase + kOffK + s * kTileBytes + c * kChunkBytes, &tmK, bar(kKFull + s), c * 64, g,
-                        w.tok0 + j * BN, w.tb);
-          k_issued = n + 1;
-          if (!(ok = mbar_wait(bar(kVEmpty + s), ph ^ 1, abort_flag))) break;
-          mbar_arrive_expect_tx(bar(kVFull + s), kTileBytes);
-          for (int c = 0; c < 2; ++c)
-            tma_load_4d(sbase + kOffV + s * kTileBytes + c * kChunkBytes, &tmV, bar(kVFull + s), c * 64, g,
-                        w.tok0 + j * BN, w.tb);
-          v_issued = n + 1;
-        }
-      }
-      if (*abort_flag) {
-        // let copies still in flight land before the CTA's shared memory is released: at most
-        // one Q tile and one K and one V tile per stage can be outstanding
-        volatile int no_abort = 0;
-        if (q_issued > 0) mbar_wait(bar(kQFull), (q_issued - 1) & 1, &no_abort);
-        for (int n = max(0, k_issued - kStages); n < k_issued; ++n)
-          mbar_wait(bar(kKFull + (n & 1)), (n >> 1) & 1, &no_abort);
-        for (int n = max(0, v_issued - kStages); n < v_issued; ++n)
-          mbar_wait(bar(kVFull + (n & 1)), (n >> 1) & 1, &no_abort);
-      }
-    }
-  } else if (warp == 9) {
-    // -------------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, HD, true);
-      auto desc_q = [&](int h, int kk) {
-        return sdesc_sw128(sbase + kOffQ + h * kTileBytes + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024);
-      };
-      auto desc_k = [&](int s, int kk) {
-        return sdesc_sw128(sbase + kOffK + s * kTileBytes + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024);
-      };
-      // V tile: keys x d with d contiguous (MN-major B operand); 16 keys per K-step.
-      auto desc_v = [&](int s, int kk) {
-        return sdesc_sw128(sbase + kOffV + s * kTileBytes + kk * 2048, kChunkBytes, 1024);
-      };
-      // O_b (+)= P_b V for this CTA's KV tile number n (ring stage n & 1, P barrier phase n & 1):
-      // the first 64 keys as soon as that half of P is in TMEM, the other 64 when the second
-      // half is. acc = false starts the item's sum.
-      auto issue_pv = [&](uint32_t o_tmem, uint32_t p_tmem, int n, bool acc, uint32_t half0, uint32_t half1) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (!mbar_wait(h ? half1 : half0, n & 1, abort_flag)) return false;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
-            mma_bf16_ts(o_tmem, p_tmem + kk * 8, desc_v(n & 1, kk), idesc_pv, (acc || kk > 0) ? 1u : 0u);
-        }
-        return true;
-      };
-      int n0 = 0;       // KV tiles of earlier items
-      int n_items = 0;  // items done
-      bool ok = true;
-      for (int k = 0; ok && work_item<kVarlen, kWindow>(p, k, w, cur, seq_id, seq_nt, n_dense); ++k) {
-        if (w.n_kv == 0) continue;
-        if (!(ok = mbar_wait(bar(kQFull), n_items & 1, abort_flag))) break;
-        for (int j = 0; j < w.n_kv; ++j) {
-          const int n = n0 + j;
-          const int s = n & 1;
-          const uint32_t ph = (n >> 1) & 1;
-          if (!(ok = mbar_wait(bar(kKFull + s), ph, abort_flag))) break;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk)
-            mma_bf16_ss(tmem + kTmS1, desc_q(0, kk), desc_k(s, kk), idesc_qk, kk > 0 ? 1u : 0u);
-          tc_commit(bar(kSFull + 0));
-          if (j > 0) {
-            if (!(ok = issue_pv(tmem + kTmO2, tmem + kTmS2, n - 1, j > 1, bar(kPFull + 2), bar(kPFull + 3)))) break;
-            tc_commit(bar(kVEmpty + ((n - 1) & 1)));
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsSmall));
+    if (warp == 8) {
+      // ------------------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        // Counts over all items of this CTA: KV tiles (ring stage and phase) and Q tiles.
+        int k_issued = 0, v_issued = 0, q_issued = 0;
+        bool ok = true;
+        for (int k = 0; ok && work_item<kVarlen, kWindow>(p, k, w, cur, seq_id, seq_nt, n_dense); ++k) {
+          if (w.n_kv == 0) continue;
+          // the single Q buffer is free once the previous item's last score GEMM has read it
+          if (q_issued > 0 && !(ok = mbar_wait(bar(kQEmpty), (q_issued - 1) & 1, abort_flag))) break;
+          mbar_arrive_expect_tx(bar(kQFull), 2 * kTileBytes);
+          for (int h = 0; h < 2; ++h)
+            for (int c = 0; c < 2; ++c)
+              tma_load_4d(sbase + kOffQ + h * kTileBytes + c * kChunkBytes, &tmQ, bar(kQFull), c * 64,
+                          2 * w.pair + h, w.tok0 + w.m0, w.tb);
+          ++q_issued;
+          const int g = (2 * w.pair) / group;
+          for (int it = 0; it < w.n_kv; ++it) {
+            const int j = w.j_first + it;
+            const int n = k_issued;  // this CTA's KV tile count so far
+            const int s = n & 1;
+            const uint32_t ph = (n >> 1) & 1;
+            if (!(ok = mbar_wait(bar(kKEmpty + s), ph ^ 1, abort_flag))) break;
+            mbar_arrive_expect_tx(bar(kKFull + s), kTileBytes);
+            for (int c = 0; c < 2; ++c)
+              tma_load_4d(sbase + kOffK + s * kTileBytes + c * kChunkBytes, &tmK, bar(kKFull + s), c * 64, g,
+                          w.tok0 + j * BN, w.tb);
+            k_issued = n + 1;
+            if (!(ok = mbar_wait(bar(kVEmpty + s), ph ^ 1, abort_flag))) break;
+            mbar_arrive_expect_tx(bar(kVFull + s), kTileBytes);
+            for (int c = 0; c < 2; ++c)
+              tma_load_4d(sbase + kOffV + s * kTileBytes + c * kChunkBytes, &tmV, bar(kVFull + s), c * 64, g,
+                          w.tok0 + j * BN, w.tb);
+            v_issued = n + 1;
           }
-#pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk)
-            mma_bf16_ss(tmem + kTmS2, desc_q(1, kk), desc_k(s, kk), idesc_qk, kk > 0 ? 1u : 0u);
-          tc_commit(bar(kSFull + 1));
-          tc_commit(bar(kKEmpty + s));
-          if (j == w.n_kv - 1) tc_commit(bar(kQEmpty));
-          if (!(ok = mbar_wait(bar(kVFull + s), ph, abort_flag))) break;
-          if (j == 0 && n_items > 0) {
-            // the first PV of an item overwrites O1 (and O2 after it): the previous item's
-            // epilogue must have read them
-            if (!(ok = mbar_wait(bar(kOEmpty), (n_items - 1) & 1, abort_flag))) break;
+        }
+        if (*abort_flag) {
+          // let copies still in flight land before the CTA's shared memory is released: at most
+          // one Q tile and one K and one V tile per stage can be outstanding
+          volatile int no_abort = 0;
+          if (q_issued > 0) mbar_wait(bar(kQFull), (q_issued - 1) & 1, &no_abort);
+          for (int n = max(0, k_issued - kStages); n < k_issued; ++n)
+            mbar_wait(bar(kKFull + (n & 1)), (n >> 1) & 1, &no_abort);
+          for (int n = max(0, v_issued - kStages); n < v_issued; ++n)
+            mbar_wait(bar(kVFull + (n & 1)), (n >> 1) & 1, &no_abort);
+        }
+      }
+    } else if (warp == 9) {
+      // -------------------------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, HD, true);
+        auto desc_q = [&](int h, int kk) {
+          return sdesc_sw128(sbase + kOffQ + h * kTileBytes + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024);
+        };
+        auto desc_k = [&](int s, int kk) {
+          return sdesc_sw128(sbase + kOffK + s * kTileBytes + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024);
+        };
+        // V tile: keys x d with d contiguous (MN-major B operand); 16 keys per K-step.
+        auto desc_v = [&](int s, int kk) {
+          return sdesc_sw128(sbase + kOffV + s * kTileBytes + kk * 2048, kChunkBytes, 1024);
+        };
+        // O_b (+)= P_b V for this CTA's KV tile number n (ring stage n & 1, P barrier phase n & 1):
+        // the first 64 keys as soon as that half of P is in TMEM, the other 64 when the second
+        // half is. acc = false starts the item's sum.
+        auto issue_pv = [&](uint32_t o_tmem, uint32_t p_tmem, int n, bool acc, uint32_t half0, uint32_t half1) {
+  #pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (!mbar_wait(h ? half1 : half0, n & 1, abort_flag)) return false;
             tc_fence_after();
+  #pragma unroll
+            for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
+              mma_bf16_ts(o_tmem, p_tmem + kk * 8, desc_v(n & 1, kk), idesc_pv, (acc || kk > 0) ? 1u : 0u);
           }
-          if (!(ok = issue_pv(tmem + kTmO1, tmem + kTmS1, n, j > 0, bar(kPFull + 0), bar(kPFull + 1)))) break;
+          return true;
+        };
+        int n0 = 0;       // KV tiles of earlier items
+        int n_items = 0;  // items done
+        bool ok = true;
+        for (int k = 0; ok && work_item<kVarlen, kWindow>(p, k, w, cur, seq_id, seq_nt, n_dense); ++k) {
+          if (w.n_kv == 0) continue;
+          if (!(ok = mbar_wait(bar(kQFull), n_items & 1, abort_flag))) break;
+          for (int j = 0; j < w.n_kv; ++j) {
+            const int n = n0 + j;
+            const int s = n & 1;
+            const uint32_t ph = (n >> 1) & 1;
+            if (!(ok = mbar_wait(bar(kKFull + s), ph, abort_flag))) break;
+            tc_fence_after();
+  #pragma unroll
+            for (int kk = 0; kk < HD / 16; ++kk)
+              mma_bf16_ss(tmem + kTmS1, desc_q(0, kk), desc_k(s, kk), idesc_qk, kk > 0 ? 1u : 0u);
+            tc_commit(bar(kSFull + 0));
+            if (j > 0) {
+              if (!(ok = issue_pv(tmem + kTmO2, tmem + kTmS2, n - 1, j > 1, bar(kPFull + 2), bar(kPFull + 3)))) break;
+              tc_commit(bar(kVEmpty + ((n - 1) & 1)));
+            }
+  #pragma unroll
+            for (int kk = 0; kk < HD / 16; ++kk)
+              mma_bf16_ss(tmem + kTmS2, desc_q(1, kk), desc_k(s, kk), idesc_qk, kk > 0 ? 1u : 0u);
+            tc_commit(bar(kSFull + 1));
+            tc_commit(bar(kKEmpty + s));
+            if (j == w.n_kv - 1) tc_commit(bar(kQEmpty));
+            if (!(ok = mbar_wait(bar(kVFull + s), ph, abort_flag))) break;
+            if (j == 0 && n_items > 0) {
+              // the first PV of an item overwrites O1 (and O2 after it): the previous item's
+              // epilogue must have read them
+              if (!(ok = mbar_wait(bar(kOEmpty), (n_items - 1) & 1, abort_flag))) break;
+              tc_fence_after();
+            }
+            if (!(ok = issue_pv(tmem + kTmO1, tmem + kTmS1, n, j > 0, bar(kPFull + 0), bar(kPFull + 1)))) break;
+          }
+          if (!ok) break;
+          const int nl = n0 + w.n_kv - 1;
+          if (!(ok = issue_pv(tmem + kTmO2, tmem + kTmS2, nl, w.n_kv > 1, bar(kPFull + 2), bar(kPFull + 3)))) break;
+          tc_commit(bar(kVEmpty + (nl & 1)));
+          tc_commit(bar(kOFull));
+          n0 += w.n_kv;
+          ++n_items;
         }
-        if (!ok) break;
-        const int nl = n0 + w.n_kv - 1;
-        if (!(ok = issue_pv(tmem + kTmO2, tmem + kTmS2, nl, w.n_kv > 1, bar(kPFull + 2), bar(kPFull + 3)))) break;
-        tc_commit(bar(kVEmpty + (nl & 1)));
-        tc_commit(bar(kOFull));
-        n0 += w.n_kv;
-        ++n_items;
+        // every MMA of this CTA must be complete before tensor memory is freed
+        tc_commit(bar(kDrain));
+        volatile int no_abort = 0;
+        mbar_wait(bar(kDrain), 0, &no_abort);
       }
-      // every MMA of this CTA must be complete before tensor memory is freed
-      tc_commit(bar(kDrain));
-      volatile int no_abort = 0;
-      mbar_wait(bar(kDrain), 0, &no_abort);
     }
-  }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
