@@ -4,15 +4,17 @@ TEST INFRASTRUCTURE ONLY (see the package docstring): never imported by the prod
 
 Sources (page title, then section / equation):
   [L16]  "Differential Attention (V2)" lesson (AI Engineering from Scratch, phase 10, 16):
+         "The noise floor of softmax" -- the attention weight of key i,
+         w_i = exp(q.k_i / sqrt(d)) / sum_j exp(q.k_j / sqrt(d));
          "The differential concept" -- A1 = softmax(Q1 K1^T / sqrt(d)),
-         A2 = softmax(Q2 K2^T / sqrt(d)), DiffAttn = (A1 - lambda * A2) V;
-         the lambda re-parameterisation lambda = exp(lq1.lk1) - exp(lq2.lk2) + lambda_init;
-         "Build it", Step 1 (numerically stable softmax: subtract the row max, exponentiate,
-         divide by the sum) and Step 3 (two softmax branches, subtract, multiply by V);
+         A2 = softmax(Q2 K2^T / sqrt(d)), DiffAttn = (A1 - lambda * A2) V, and the V1
+         lambda re-parameterisation lambda = exp(lq1.lk1) - exp(lq2.lk2) + lambda_init;
+         key-terms table ("lambda" may be negative; "Signal-to-noise ratio");
          "Exercises" 4 (lambda = 0 is the pure first softmax) and 5 (GQA + V2 cache size).
   [L07]  "Attention variants: sliding window, sparse, differential" lesson (phase 7, 15):
-         "Build it", Step 1 (causal mask: 0 where j <= i, -inf otherwise) and Step 4
-         (diff_attention: causal softmax per branch, then (A1 - lam*A2) @ V).
+         "Sliding window attention" -- keys outside a query's window get -inf in the score
+         matrix; its W = 4 figure and the key-terms table ("each query attends to its last
+         W tokens"); causal attention lets query i see keys j <= i.
   [HF]   "Differential Transformer V2 soll KI-Training stabiler machen" (summary of the
          Hugging Face blog), section "Gemeinsamer KV-Cache statt Spezialkernel": two adjacent
          query heads inside one GQA group share K and V; section "Weniger Ausreisser und
@@ -24,7 +26,7 @@ Readings of points the pages leave open (each also listed in the design notes):
   * the KV head of pair p is g = (2p) // (Hq / Hkv);
   * lambda is one value per token and per output head (= pair): [B, S, Hq/2] for prefill,
     [B, Hq/2] for decode; it arrives already bounded (the model applies the sigmoid);
-  * the score scale is 1/sqrt(D) for both branches (the toy's `scale` read as sqrt(d));
+  * the score scale is 1/sqrt(D) for both branches;
   * causal means key j is visible from query i when j <= i, with Sq == Sk;
   * decode attends to keys [0, seqlen_b), the new token's key already appended.
 """
@@ -57,37 +59,46 @@ __all__ = [
 
 
 def stable_softmax(x: np.ndarray) -> np.ndarray:
-    """Row softmax along the last axis, the two-pass stable form of [L16] Step 1.
+    """Softmax along the last axis: [L16] "The noise floor of softmax", w_i = e^{x_i} / sum_j e^{x_j}.
 
-    m = max(row); e = exp(x - m); return e / sum(e). Entries equal to -inf (masked keys)
-    get weight exactly 0. A row must hold at least one finite entry.
+    Evaluated as w_i = exp(x_i - LSE(x)) with the log-sum-exp LSE(x) = c + log sum_j e^{x_j - c}
+    for c = max_j x_j; the identity holds for every c, and this c keeps every exponent <= 0 so
+    nothing overflows. Entries equal to -inf (masked keys) get weight exactly 0. A row must
+    hold at least one finite entry.
     """
     x = np.asarray(x, dtype=np.float64)
-    m = np.max(x, axis=-1, keepdims=True)
-    e = np.exp(x - m)
-    return e / np.sum(e, axis=-1, keepdims=True)
+    c = np.max(x, axis=-1, keepdims=True)
+    lse = c + np.log(np.sum(np.exp(x - c), axis=-1, keepdims=True))
+    return np.exp(x - lse)
+
+
+def _additive(visible: np.ndarray) -> np.ndarray:
+    """Additive mask of a visibility predicate: 0 where a key is visible, -inf elsewhere
+    ([L07] "Sliding window attention": hidden keys get -inf in the score matrix)."""
+    return np.where(visible, 0.0, -np.inf)
 
 
 def causal_mask(n_q: int, n_k: int, q_offset: int = 0) -> np.ndarray:
-    """Additive causal mask of [L07] Step 1: 0.0 where key j <= query i, else -inf.
+    """Causal visibility: key j is visible from query i exactly when j <= i.
 
     Query rows are numbered q_offset .. q_offset + n_q - 1 (a row block of a longer
     sequence); keys are numbered 0 .. n_k - 1.
     """
     i = np.arange(q_offset, q_offset + n_q)[:, None]
     j = np.arange(n_k)[None, :]
-    return np.where(j <= i, 0.0, -np.inf)
+    return _additive(j <= i)
 
 
 def window_mask(n_q: int, n_k: int, window: int, q_offset: int = 0) -> np.ndarray:
-    """Additive causal sliding-window mask of [L07] Step 2: key j is visible from query i
-    when max(0, i - window + 1) <= j <= i (the window holds the query's own key); 0.0 there,
-    -inf elsewhere. window >= n gives the full causal mask; window = 1 leaves only j = i."""
+    """Causal sliding window of [L07] ("Sliding window attention", its W = 4 figure and the
+    key-terms table): query i sees its last `window` keys, i.e. key j with
+    i - window < j <= i (the window holds the query's own key). window >= n gives the full
+    causal mask; window = 1 leaves only j = i."""
     if window < 1:
         raise ValueError("window must be >= 1")
     i = np.arange(q_offset, q_offset + n_q)[:, None]
     j = np.arange(n_k)[None, :]
-    return np.where((j <= i) & (j >= i - window + 1), 0.0, -np.inf)
+    return _additive((j <= i) & (i - j < window))
 
 
 def pair_layout(Hq: int, Hkv: int):
@@ -110,7 +121,8 @@ def pair_layout(Hq: int, Hkv: int):
 
 
 def diff_attention_block(q1, q2, k, v, lam, mask):
-    """DiffAttn for one pair over a block of query rows: [L16] eq. DiffAttn, [L07] Step 4.
+    """DiffAttn for one pair over a block of query rows: the equations of [L16] "The
+    differential concept", A_b = softmax(Q_b K^T / sqrt(D) + mask), DiffAttn = (A_1 - lambda A_2) V.
 
     q1, q2: [n, D] the two heads of the pair; k, v: [m, D] their shared K/V head;
     lam: [n] one lambda per query row; mask: [n, m] additive (0 or -inf).
@@ -140,7 +152,7 @@ def prefill(q, k, v, lam, causal: bool = True, row_block: int = 512, window=None
     processed in blocks of `row_block` (a memory bound only: every row is computed exactly
     as the definition states, over all its visible keys). `window` (causal only) restricts
     each query to its last `window` keys, the DiffAttn + sliding-window combination that the
-    lesson's "Use it" section names for hybrid layers, with the mask of [L07] Step 2.
+    lesson's "Use it" section names for hybrid layers, with the window of `window_mask`.
     """
     if window is not None and not causal:
         raise ValueError("a sliding window is defined for causal attention")
@@ -377,8 +389,8 @@ def lambda_v2_projection(x, w, bias=None) -> np.ndarray:
 def branch_weights(q1, q2, k, lam, n_visible=None):
     """Attention weights of one query row: (a1, a2, a1 - lam * a2) over its visible keys.
 
-    q1, q2: [D]; k: [m, D]. Keys n_visible.. are masked out (weight 0). Follows [L16]
-    Step 3 (`diff_weights`).
+    q1, q2: [D]; k: [m, D]. Keys n_visible.. are masked out (weight 0). The rows of A_1,
+    A_2 and A_1 - lambda A_2 of [L16] "The differential concept" for one query.
     """
     q1, q2, k = _f64(q1), _f64(q2), _f64(k)
     m = k.shape[0] if n_visible is None else int(n_visible)
@@ -394,8 +406,8 @@ def snr(weights, signal_index: int) -> float:
     """Signal-to-noise ratio of one weight row ([L16] key-terms table, "Signal-to-noise
     ratio"): weight on the signal position over the average weight on the unrelated positions.
 
-    Differential weights can be negative ([L16] Step 3 note), so the average over unrelated
-    positions is taken of the absolute weights.
+    Differential weights can be negative (A_1 - lambda A_2 is a difference of two
+    distributions), so the average over unrelated positions is taken of the absolute weights.
     """
     w = np.asarray(weights, dtype=np.float64)
     others = np.delete(w, signal_index)

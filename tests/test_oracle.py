@@ -227,6 +227,42 @@ def pin_weights_rows_sum():
     return bool(ok)
 
 
+def pin_branch_weights_library():
+    """One query row's weights against the library: torch SDPA with V = I returns the row of
+    softmax(q k^T / sqrt(D)) itself (D = 16, so a dropped or wrong 1/sqrt(D) changes it);
+    keys past n_visible take no weight, which equals SDPA over the visible prefix."""
+    rng = np.random.default_rng(24)
+    D, m, n_vis = 16, 40, 29
+    k = rng.standard_normal((m, D)) * 1.5
+    q1, q2 = rng.standard_normal(D) * 1.5, rng.standard_normal(D) * 1.5
+
+    def sdpa_row(q, n):
+        eye = torch.eye(n, dtype=torch.float64)[None, None]
+        kt = torch.from_numpy(k[:n])[None, None]
+        qt = torch.from_numpy(q)[None, None, None]
+        return torch.nn.functional.scaled_dot_product_attention(qt, kt, eye)[0, 0, 0].numpy()
+
+    ok = True
+    for lam, n in ((0.8, None), (-0.4, n_vis)):
+        a1, a2, w = ora.branch_weights(q1, q2, k, lam, n)
+        nn_ = m if n is None else n
+        r1, r2 = sdpa_row(q1, nn_), sdpa_row(q2, nn_)
+        ok &= len(a1) == nn_ and np.allclose(a1, r1, rtol=1e-12, atol=1e-15)
+        ok &= np.allclose(a2, r2, rtol=1e-12, atol=1e-15)
+        ok &= np.allclose(w, r1 - lam * r2, rtol=1e-12, atol=1e-15)
+    return bool(ok)
+
+
+def pin_snr_hand_values():
+    """Signal-to-noise ratio (lesson key-terms table) on hand-computed rows with negative
+    entries, where the mean of absolute weights differs from the signed mean:
+    [0.5, -0.1, 0.1, -0.2] with the signal at 0 gives 0.5 / (0.4 / 3) = 3.75;
+    [0.1, 0.6, -0.3] with the signal at 1 gives 0.6 / 0.2 = 3.0."""
+    ok = math.isclose(ora.snr([0.5, -0.1, 0.1, -0.2], 0), 3.75, rel_tol=1e-14)
+    ok &= math.isclose(ora.snr(np.array([0.1, 0.6, -0.3]), 1), 3.0, rel_tol=1e-14)
+    return bool(ok)
+
+
 def pin_window_reduces_to_causal_and_self():
     """A window at least S long is the causal mask; window 1 leaves each query only its own
     key, so out[b,i,p] = (1 - lam) v[b,i,g]."""
@@ -471,6 +507,8 @@ ALL_PINS = {
     "noise_mass_golden": pin_noise_mass_golden,
     "uniform_logits": pin_uniform_logits,
     "weights_rows_sum": pin_weights_rows_sum,
+    "branch_weights_library": pin_branch_weights_library,
+    "snr_hand_values": pin_snr_hand_values,
     "window_reduces_to_causal_and_self": pin_window_reduces_to_causal_and_self,
     "window_brute_force": pin_window_brute_force,
     "window_mask_definition": pin_window_mask_definition,

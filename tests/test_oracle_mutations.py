@@ -157,6 +157,19 @@ def _branches_swapped(q, k, v, causal=True):
     return o2, lse2
 
 
+def _branch_weights_no_scale(q1, q2, k, lam, n_visible=None):
+    q1, q2, k = (np.asarray(x, dtype=np.float64) for x in (q1, q2, k))
+    m = k.shape[0] if n_visible is None else int(n_visible)
+    a1 = ora.stable_softmax(k[:m] @ q1)
+    a2 = ora.stable_softmax(k[:m] @ q2)
+    return a1, a2, a1 - float(lam) * a2
+
+
+def _snr_signed_mean(weights, signal_index):
+    w = np.asarray(weights, dtype=np.float64)
+    return float(w[signal_index] / np.mean(np.delete(w, signal_index)))
+
+
 _ORIG_BRANCHES = ora.prefill_branches
 
 MUTANTS = {
@@ -183,6 +196,8 @@ MUTANTS = {
     "backward_dq_unscaled": ("prefill_backward", _backward_variant(dq_unscaled=True)),
     "branches_lse_natural_log": ("prefill_branches", _branches_natural_log),
     "branches_heads_swapped": ("prefill_branches", _branches_swapped),
+    "branch_weights_no_scale": ("branch_weights", _branch_weights_no_scale),
+    "snr_signed_mean": ("snr", _snr_signed_mean),
 }
 
 
