@@ -2,17 +2,24 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
 
-One step is one pass of the whole hot path over one batch of synthetic input:
-  * prefill: causal bf16 DiffAttn V2 over B=4 x S=4096, Hq=64 (32 pairs), Hkv=8, D=128
+One step is one pass of the whole hot path over one batch of synthetic input, on the
+largest single-GPU configurations:
+  * prefill: causal bf16 DiffAttn V2 over B=1 x S=32768, Hq=64 (32 pairs), Hkv=8, D=128
     (one tcgen05 kernel launch), then
-  * decode: one bf16 decode step for 64 sequences with lengths uniform in [1024, 8192]
-    over an [64, 8192, 8, 128] KV cache (one split-KV kernel whose last split per (b, KV head)
-    merges the partials; a memset of its split counters precedes it).
+  * needle decode: one bf16 decode step for 8 sequences of 131072 cached tokens each
+    ([8, 131072, 8, 128] KV cache with one planted needle key per sequence); the V1 lambda
+    is computed on the device from its four re-parameterisation vectors (one small kernel),
+    then one split-KV kernel whose last split per (b, KV head) merges the partials (a memset
+    of its split counters precedes it).
 `value` is the prefill throughput in TFLOP/s (algorithmic FLOPs = 4*D*Hq*B*S(S+1)/2 over
 the prefill kernel's CUDA-event time inside the timed steps); the decode throughput in
-GB/s (every visible K/V row once, plus q, lambda and out) is reported beside it.
-Inputs are resident in HBM before the timed region and are larger than L2 (q alone is
-268 MB and the decode streams 1.2 GB per step), so no extra L2 flush is done.
+GB/s (every visible K/V row once, plus q, lambda and out) is reported beside it. The same
+run then times the second pair of workloads (B=4 x 4096 prefill; B=64 decode with lengths
+uniform in [1024, 8192]) the same way, under `second_workload`.
+Inputs are resident in HBM before the timed region and are larger than L2 (the prefill's
+q alone is 537 MB and the decode streams 4.3 GB per step), so no extra L2 flush is done.
+`e2e` repeats the step through host buffers: pinned uploads of every input and downloads
+of both outputs, on their own streams, overlapped with the kernels across steps.
 
 --impl reference times the float64 CPU oracle (the test oracle, as it stands) on a bounded
 sample of the same workload on the host cores; with N > 1 only rank 0 runs it.
@@ -43,8 +50,13 @@ if ROOT not in sys.path:
 import workloads  # noqa: E402
 
 METRIC = "DiffAttnV2 fwd: prefill TFLOP/s (% bf16 peak); decode GB/s (% HBM)"
-PREFILL_CFG = "prefill_b4_s4096"
-DECODE_CFG = "decode_b64_s8192"
+# The step the headline line times: the largest single-GPU configurations (32k-token causal
+# prefill; needle decode over 8 x 131072 cached tokens with the V1 lambda).
+PREFILL_CFG = "prefill_b1_s32768"
+DECODE_CFG = "needle_decode_b8_s131072"
+# The second prefill and decode workloads, timed the same way in the same run.
+PREFILL_CFG_2 = "prefill_b4_s4096"
+DECODE_CFG_2 = "decode_b64_s8192"
 
 # Measured roofline denominators of this machine's B200s (measured copy bandwidth and
 # cuBLAS bf16 GEMM); used when the peaks file is absent.
@@ -56,6 +68,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the measured peaks
 SPEC_BF16_TFLOPS = 2250.0
 SPEC_HBM_GBS = 8000.0
+
+# workloads the DRAM traffic below was captured on
+TRAFFIC_WORKLOAD = {"prefill": "prefill_b4_s4096", "decode": "decode_b64_s8192"}
 
 NCU_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one launch (B=4 x 4k causal prefill),
@@ -192,12 +207,12 @@ def _max_over_ranks(x, dist):
 
 
 # -------------------------------------------------------------------------- our arm
-def _inputs(rank, do_pre=True, do_dec=True, world=1, strong=False):
+def _inputs(pc_name, dc_name, rank, do_pre=True, do_dec=True, world=1, strong=False):
     """Per-rank inputs. Weak scaling: every rank its own seeded batch of the full size.
     Strong scaling: one seeded problem, each rank its head shard (a whole number of GQA
     groups), so the ranks together compute exactly the single-GPU workload."""
-    pc = workloads.CONFIGS[PREFILL_CFG]
-    dc = workloads.CONFIGS[DECODE_CFG]
+    pc = workloads.CONFIGS[pc_name]
+    dc = workloads.CONFIGS[dc_name]
     if not strong:
         pc = workloads.PrefillCase(**{**pc.__dict__, "seed": pc.seed + 100 * rank})
         dc = workloads.DecodeCase(**{**dc.__dict__, "seed": dc.seed + 100 * rank})
@@ -209,10 +224,218 @@ def _inputs(rank, do_pre=True, do_dec=True, world=1, strong=False):
             pin = shard_prefill_inputs(pin, pc.Hq, pc.Hkv, world, rank)
         if din is not None:
             din = {**din, "q": din["q"][:, q0:q1].contiguous(), "kcache": din["kcache"][:, :, kv0:kv1].contiguous(),
-                   "vcache": din["vcache"][:, :, kv0:kv1].contiguous(), "lam": din["lam"][:, q0 // 2:q1 // 2].contiguous()}
+                   "vcache": din["vcache"][:, :, kv0:kv1].contiguous()}
+            for x in ("lam", "lq1", "lk1", "lq2", "lk2"):
+                if din.get(x) is not None:
+                    t = din[x]
+                    din[x] = (t[:, q0 // 2:q1 // 2] if x == "lam" else t[q0 // 2:q1 // 2]).contiguous()
         pc = workloads.PrefillCase(**{**pc.__dict__, "Hq": q1 - q0, "Hkv": kv1 - kv0})
         dc = workloads.DecodeCase(**{**dc.__dict__, "Hq": q1 - q0, "Hkv": kv1 - kv0})
     return pc, pin, dc, din
+
+
+class Step:
+    """Device-resident inputs and outputs of one step (prefill + decode) and its launches.
+
+    The decode of a V1-lambda workload computes lambda on the device first (one small
+    kernel) from the four re-parameterisation vectors, as a caller of the operator would."""
+
+    def __init__(self, da, pc, pin, dc, din, dev, stream, n_buffers=1):
+        self.da, self.pc, self.dc, self.dev, self.stream = da, pc, dc, dev, stream
+        self.pin, self.din = pin, din
+        self.do_pre, self.do_dec = pin is not None, din is not None
+        self.v1 = self.do_dec and din["lam"] is None
+        self.bufs = []
+        for _ in range(n_buffers):
+            b = {}
+            if self.do_pre:
+                for x in ("q", "k", "v", "lam"):
+                    b[x] = pin[x].to(dev)
+                b["out"] = torch.empty(pc.B, pc.S, pc.Hq // 2, pc.D, dtype=torch.bfloat16, device=dev)
+            if self.do_dec:
+                for x in ("q", "seqlens") + (("lq1", "lk1", "lq2", "lk2") if self.v1 else ("lam",)):
+                    b["d" + x] = din[x].to(dev)
+                if self.v1:
+                    b["dlam"] = torch.empty(dc.B, dc.Hq // 2, dtype=torch.float32, device=dev)
+                b["dout"] = torch.empty(dc.B, dc.Hq // 2, dc.D, dtype=torch.bfloat16, device=dev)
+            self.bufs.append(b)
+        if self.do_dec:
+            # the cache is state that lives on the device; one copy serves every buffer set
+            self.kc = din["kcache"].to(dev)
+            self.vc = din["vcache"].to(dev)
+            self.ws = torch.empty(da.decode_workspace_size(dc.B, dc.Smax, dc.Hq, dc.Hkv, dc.D), dtype=torch.uint8,
+                                  device=dev)
+        self.flops = workloads.prefill_flops(pc.B, pc.S, pc.Hq, pc.D, causal=True) if self.do_pre else 0
+        self.dbytes = workloads.decode_bytes(din["seqlens"].tolist(), dc.Hkv, dc.D, dc.Hq) if self.do_dec else 0
+        # kernels of this library per step: prefill; V1 lambda; decode (the split counters'
+        # memset is a runtime call, not a kernel of this library)
+        self.launches = int(self.do_pre) + (int(self.v1) + 1 if self.do_dec else 0)
+
+    def prefill(self, i=0, stream=None):
+        b = self.bufs[i]
+        self.da.prefill(b["q"], b["k"], b["v"], b["lam"], out=b["out"], stream=stream or self.stream)
+
+    def decode(self, i=0, stream=None):
+        b = self.bufs[i]
+        st = stream or self.stream
+        if self.v1:
+            self.da.lambda_v1(b["dlq1"], b["dlk1"], b["dlq2"], b["dlk2"], self.din["lambda_init"], rows=self.dc.B,
+                              out=b["dlam"], stream=st)
+        self.da.decode(b["dq"], self.kc, self.vc, b["dseqlens"], b["dlam"], out=b["dout"], workspace=self.ws,
+                       stream=st)
+
+    def h2d_names(self):
+        pre = ("q", "k", "v", "lam") if self.do_pre else ()
+        dec = (("q", "seqlens") + (("lq1", "lk1", "lq2", "lk2") if self.v1 else ("lam",))) if self.do_dec else ()
+        return pre, dec
+
+
+def _time_steps(st, steps, dist):
+    """Time `steps` steps on the step's stream: CUDA events around each step's prefill and
+    decode; the whole region bracketed by a barrier and a synchronize on both sides."""
+    stream, dev = st.stream, st.dev
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(dist)
+    torch.cuda.synchronize(dev)
+    t0.record(stream)
+    for i in range(steps):
+        evs[i][0].record(stream)
+        if st.do_pre:
+            st.prefill()
+        evs[i][1].record(stream)
+        if st.do_dec:
+            st.decode()
+        evs[i][2].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    _barrier(dist)
+    total = _max_over_ranks(t0.elapsed_time(t1), dist)
+    pre = _max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in evs), dist)
+    dec = _max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in evs), dist)
+    return total, pre, dec
+
+
+def _e2e(st, steps, dist):
+    """The step end to end through the public API: every step copies its inputs from
+    pinned host memory and its outputs back. Copies run on their own streams, ordered by
+    events against the compute stream, so step i+1's uploads and step i's downloads overlap
+    step i's kernels (two device buffer sets alternate). Returns (ms, h2d_bytes, d2h_bytes)
+    per step, max over ranks."""
+    dev, comp = st.dev, st.stream
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    pre, dec = st.h2d_names()
+    host_in = {x: st.pin[x].pin_memory() for x in pre}
+    host_in.update({"d" + x: st.din[x].pin_memory() for x in dec})
+    outs = (["out"] if st.do_pre else []) + (["dout"] if st.do_dec else [])
+    host_out = [{o: torch.empty(st.bufs[0][o].shape, dtype=st.bufs[0][o].dtype).pin_memory() for o in outs}
+                for _ in range(2)]
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(host_out[0][o].numel() * host_out[0][o].element_size() for o in outs)
+    ev = lambda: torch.cuda.Event()
+
+    def run(n, start_ev):
+        loaded = [None] * n
+        read = [None] * n     # buffer set i % 2 no longer read by step i's kernels
+        fetched = [None] * n  # step i's outputs copied back
+        for i in range(n):
+            b = st.bufs[i % 2]
+            with torch.cuda.stream(up):
+                up.wait_event(start_ev)
+                if i >= 2:
+                    up.wait_event(read[i - 2])  # the buffer set's previous step is done with it
+                for name, t in host_in.items():
+                    b[name].copy_(t, non_blocking=True)
+                loaded[i] = ev()
+                loaded[i].record(up)
+            comp.wait_event(loaded[i])
+            if i >= 2:
+                comp.wait_event(fetched[i - 2])  # outputs of the set's previous step are out
+            if st.do_pre:
+                st.prefill(i % 2, comp)
+            if st.do_dec:
+                st.decode(i % 2, comp)
+            read[i] = ev()
+            read[i].record(comp)
+            with torch.cuda.stream(down):
+                down.wait_event(read[i])
+                for o in outs:
+                    host_out[i % 2][o].copy_(b[o], non_blocking=True)
+                fetched[i] = ev()
+                fetched[i].record(down)
+        comp.wait_event(fetched[n - 1])
+        comp.wait_event(loaded[n - 1])
+
+    s0 = torch.cuda.Event()
+    s0.record(comp)
+    run(2, s0)
+    torch.cuda.synchronize(dev)
+    _barrier(dist)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(comp)
+    run(steps, e0)
+    e1.record(comp)
+    torch.cuda.synchronize(dev)
+    _barrier(dist)
+    ms = _max_over_ranks(e0.elapsed_time(e1), dist) / steps
+    return ms, h2d, d2h
+
+
+def _traffic(kind):
+    tr = NCU_TRAFFIC[kind]
+    src = {"prefill": "prefill_sm100.cu", "decode": "decode_sm100.cu"}[kind]
+    return tr["bytes"] if tr.get("bytes") is not None and tr["source_sha"] == _src_sha(src) else None
+
+
+def _describe(st, world, K, total_ms, pre_ms, dec_ms, peaks, peak_src):
+    """Throughput and roofline objects of one timed step kind."""
+    pre_launch_ms, dec_launch_ms = pre_ms / K, dec_ms / K
+    tflops = st.flops / (pre_launch_ms * 1e-3) / 1e12 if st.do_pre else 0.0
+    gbs = st.dbytes / (dec_launch_ms * 1e-3) / 1e9 if st.do_dec else 0.0
+    peak_t = peaks["bf16_tflops"]
+    pc, dc = st.pc, st.dc
+    res = {
+        "value": round(world * st.flops * K / (pre_ms * 1e-3) / 1e12, 2) if st.do_pre else 0.0,
+        "ms_per_step": round(total_ms / K, 4),
+        "roofline": {
+            "bound": "tensor", "achieved": round(tflops, 2), "peak": peak_t, "unit": "TFLOP/s",
+            "frac": round(tflops / peak_t, 4), "traffic": None,
+            "kernel": "diffattn_prefill_sm100", "flops_per_launch": st.flops,
+            "launch_ms": round(pre_launch_ms, 4), "peak_source": f"{peak_src} bf16_tflops (burst)",
+            "frac_of_spec": round(tflops / SPEC_BF16_TFLOPS, 4), "spec_peak": SPEC_BF16_TFLOPS,
+        },
+        "decode": {
+            "value": round(world * st.dbytes * K / (dec_ms * 1e-3) / 1e9, 1) if st.do_dec else 0.0, "unit": "GB/s",
+            "us_per_step": round(1000 * dec_launch_ms, 2),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                         "kernel": "diffattn_decode_split" + (" (+ lambda_v1_kernel)" if st.v1 else ""),
+                         "bytes_per_launch": st.dbytes, "peak_source": f"{peak_src} hbm_gbs",
+                         "frac_of_spec": round(gbs / SPEC_HBM_GBS, 4), "spec_peak": SPEC_HBM_GBS},
+        },
+        "prefill_cfg": {"B": pc.B, "S": pc.S, "Hq": pc.Hq, "Hkv": pc.Hkv, "D": pc.D, "causal": True,
+                        "flops_per_step": st.flops} if st.do_pre else None,
+        "decode_cfg": {"B": dc.B, "Smax": dc.Smax, "Hq": dc.Hq, "Hkv": dc.Hkv, "D": dc.D,
+                       "sum_seqlens": int(st.din["seqlens"].sum()), "bytes_per_step": st.dbytes,
+                       "lambda": "V1 (computed on the device each step)" if st.v1 else "V2 (given)"}
+        if st.do_dec else None,
+    }
+    return res
+
+
+def _workload_name(pc, dc, do_pre=True, do_dec=True):
+    parts = []
+    if do_pre:
+        parts.append(f"causal bf16 prefill B={pc.B} S={pc.S} Hq={pc.Hq} Hkv={pc.Hkv} D={pc.D}")
+    if do_dec:
+        if dc.needle:
+            parts.append(f"needle bf16 decode B={dc.B} x {dc.Smax} cached tokens Hq={dc.Hq} Hkv={dc.Hkv} D={dc.D}, "
+                         "V1 lambda")
+        else:
+            parts.append(f"bf16 decode B={dc.B} Smax={dc.Smax} len U[{dc.len_lo},{dc.len_hi}] Hq={dc.Hq} "
+                         f"Hkv={dc.Hkv} D={dc.D}")
+    return " + ".join(parts)
 
 
 def run_ours(args, rank, world, local, dist):
@@ -223,171 +446,110 @@ def run_ours(args, rank, world, local, dist):
     do_pre = args.only in (None, "prefill")
     do_dec = args.only in (None, "decode")
     strong = args.scaling == "strong"
-    pc, pin, dc, din = _inputs(rank, do_pre, do_dec, world, strong)
     stream = torch.cuda.current_stream(dev)
+    K = args.steps
+    W = max(args.warmup, 3)
+    peaks, peak_src = _peaks()
 
-    # device-resident inputs and outputs
-    if do_pre:
-        q, k, v, lam = (pin[x].to(dev) for x in ("q", "k", "v", "lam"))
-        out = torch.empty(pc.B, pc.S, pc.Hq // 2, pc.D, dtype=torch.bfloat16, device=dev)
-    if do_dec:
-        dq, kc, vc, sl, dl = (din[x].to(dev) for x in ("q", "kcache", "vcache", "seqlens", "lam"))
-        dout = torch.empty(dc.B, dc.Hq // 2, dc.D, dtype=torch.bfloat16, device=dev)
-        ws = torch.empty(da.decode_workspace_size(dc.B, dc.Smax, dc.Hq, dc.Hkv, dc.D), dtype=torch.uint8,
-                         device=dev)
+    pc, pin, dc, din = _inputs(PREFILL_CFG, DECODE_CFG, rank, do_pre, do_dec, world, strong)
+    st = Step(da, pc, pin if do_pre else None, dc, din if do_dec else None, dev, stream, n_buffers=2)
 
-    flops = workloads.prefill_flops(pc.B, pc.S, pc.Hq, pc.D, causal=True) if do_pre else 0
-    dbytes = workloads.decode_bytes(din["seqlens"].tolist(), dc.Hkv, dc.D, dc.Hq) if do_dec else 0
+    def warm(s):
+        for _ in range(W):
+            if s.do_pre:
+                s.prefill()
+            if s.do_dec:
+                s.decode()
+        torch.cuda.synchronize(dev)
+        if da.device_error(s.stream) != 0:
+            raise RuntimeError("kernel reported a device-side error during warm-up")
 
-    def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
-        if do_pre:
-            da.prefill(q, k, v, lam, out=out, stream=stream)
-        if ev is not None:
-            ev[1].record(stream)
-        if do_dec:
-            da.decode(dq, kc, vc, sl, dl, out=dout, workspace=ws, stream=stream)
-        if ev is not None:
-            ev[2].record(stream)
-
-    for _ in range(max(args.warmup, 3)):
-        step()
-    torch.cuda.synchronize(dev)
-    if da.device_error(stream) != 0:
-        raise RuntimeError("kernel reported a device-side error during warm-up")
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    warm(st)
     clocks = ClockSampler(local) if rank == 0 else None
     if clocks:
         clocks.start()
-    _barrier(dist)
-    torch.cuda.synchronize(dev)
-    t_start.record(stream)
-    for i in range(args.steps):
-        step(evs[i])
-    t_end.record(stream)
-    torch.cuda.synchronize(dev)
-    _barrier(dist)
-    total_ms = t_start.elapsed_time(t_end)
-    pre_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
-    dec_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
-    total_ms = _max_over_ranks(total_ms, dist)
-    pre_ms = _max_over_ranks(pre_ms, dist)
-    dec_ms = _max_over_ranks(dec_ms, dist)
-    err = da.device_error(stream)
-
-    # ------------------------------------------------ end to end through host buffers
-    h = {x: pin[x].pin_memory() for x in ("q", "k", "v", "lam")} if do_pre else {}
-    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory() if do_pre else torch.empty(0)
-    hd = {x: din[x].pin_memory() for x in ("q", "seqlens", "lam")} if do_dec else {}
-    hd_out = torch.empty(dout.shape, dtype=dout.dtype).pin_memory() if do_dec else torch.empty(0)
-    e2e_steps = max(3, min(args.steps, 50))
-
-    def e2e_step():
-        if do_pre:
-            for name, dst in (("q", q), ("k", k), ("v", v), ("lam", lam)):
-                dst.copy_(h[name], non_blocking=True)
-            da.prefill(q, k, v, lam, out=out, stream=stream)
-            h_out.copy_(out, non_blocking=True)
-        if do_dec:
-            for name, dst in (("q", dq), ("seqlens", sl), ("lam", dl)):
-                dst.copy_(hd[name], non_blocking=True)
-            da.decode(dq, kc, vc, sl, dl, out=dout, workspace=ws, stream=stream)
-            hd_out.copy_(dout, non_blocking=True)
-
-    e2e_step()
-    torch.cuda.synchronize(dev)
-    _barrier(dist)
-    torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    _barrier(dist)
-    e2e_ms = _max_over_ranks(e0.elapsed_time(e1), dist)
+    total_ms, pre_ms, dec_ms = _time_steps(st, K, dist)
+    e2e_steps = max(3, min(K, 30))
+    e2e_ms, h2d, d2h = _e2e(st, e2e_steps, dist)
     clk = clocks.stop() if clocks else None
-    err |= da.device_error(stream)
+    err = da.device_error(stream)
     if err:
         raise RuntimeError(f"kernel reported device error {err}")
+    main = _describe(st, world, K, total_ms, pre_ms, dec_ms, peaks, peak_src)
+    main_name = _workload_name(pc, dc, st.do_pre, st.do_dec)
+    main_launches = st.launches
+    main_flops = st.flops
+    main["roofline"]["traffic"] = _traffic("prefill") if TRAFFIC_WORKLOAD["prefill"] == PREFILL_CFG else None
+    main["decode"]["roofline"]["traffic"] = _traffic("decode") if TRAFFIC_WORKLOAD["decode"] == DECODE_CFG else None
 
-    h2d = sum(t.numel() * t.element_size() for t in h.values()) + sum(t.numel() * t.element_size() for t in hd.values())
-    d2h = h_out.numel() * h_out.element_size() + hd_out.numel() * hd_out.element_size()
+    # the second prefill and decode workloads, timed the same way in the same run
+    also = None
+    if not args.no_second and not args.only:
+        pc2, pin2, dc2, din2 = _inputs(PREFILL_CFG_2, DECODE_CFG_2, rank, True, True, world, strong)
+        del st
+        torch.cuda.empty_cache()
+        st2 = Step(da, pc2, pin2, dc2, din2, dev, stream)
+        warm(st2)
+        if clocks:
+            clocks.start()
+        t2, p2, d2 = _time_steps(st2, K, dist)
+        clk2 = clocks.stop() if clocks else None
+        err = da.device_error(stream)
+        if err:
+            raise RuntimeError(f"kernel reported device error {err}")
+        also = _describe(st2, world, K, t2, p2, d2, peaks, peak_src)
+        also["roofline"]["traffic"] = _traffic("prefill") if TRAFFIC_WORKLOAD["prefill"] == PREFILL_CFG_2 else None
+        also["decode"]["roofline"]["traffic"] = (_traffic("decode") if TRAFFIC_WORKLOAD["decode"] == DECODE_CFG_2
+                                                 else None)
+        also["workload"] = _workload_name(pc2, dc2)
+        also["clocks"] = clk2
+        also["gpu_launches"] = st2.launches * K
 
     if rank != 0:
         return None
-    peaks, peak_src = _peaks()
-    K = args.steps
-    pre_launch_ms = pre_ms / K
-    dec_launch_ms = dec_ms / K
-    tflops = flops / (pre_launch_ms * 1e-3) / 1e12 if do_pre else 0.0
-    gbs = dbytes / (dec_launch_ms * 1e-3) / 1e9 if do_dec else 0.0
-    # whole job: every rank's work over the slowest rank's time (each rank's share is equal)
-    value = world * flops * K / (pre_ms * 1e-3) / 1e12 if do_pre else 0.0
-    dec_value = world * dbytes * K / (dec_ms * 1e-3) / 1e9 if do_dec else 0.0
-    peak_t = peaks["bf16_tflops"]
-    tr = NCU_TRAFFIC["prefill"]
-    traffic = tr["bytes"] if tr["source_sha"] == _src_sha("prefill_sm100.cu") else None
-    trd = NCU_TRAFFIC["decode"]
-    traffic_d = trd["bytes"] if trd["source_sha"] == _src_sha("decode_sm100.cu") else None
     line = {
         "metric": METRIC,
-        "value": round(value, 2),
+        "value": main["value"],
         "unit": "TFLOP/s",
         "n_gpus": world,
         "steps": K,
-        "warmup": max(args.warmup, 3),
-        "ms_per_step": round(total_ms / K, 4),
+        "warmup": W,
+        "ms_per_step": main["ms_per_step"],
         "higher_is_better": True,
         "scaling": args.scaling,
         "vs_baseline": None,
         "dtype": "bf16",
-        "data": "synthetic: seeded N(0,1) q/k/v rounded to bf16, lambda = sigmoid(N(0,1)) fp32, "
-                "decode lengths uniform in [1024, 8192]",
+        "data": "synthetic: seeded N(0,1) q/k/v rounded to bf16, lambda = sigmoid(N(0,1)) fp32 for the prefill; "
+                "needle decode: N(0,1) cache with one planted needle key per sequence, V1 lambda from "
+                "N(0, 0.1^2) vectors",
         "config": {
-            "workload": "prefill B=4 S=4096 Hq=64 Hkv=8 D=128 causal bf16 + decode B=64 Smax=8192 "
-                        "len U[1024,8192] Hq=64 Hkv=8 D=128 bf16",
-            "prefill": {"B": pc.B, "S": pc.S, "Hq": pc.Hq, "Hkv": pc.Hkv, "D": pc.D, "causal": True,
-                        "flops_per_step": flops},
-            "decode": {"B": dc.B, "Smax": dc.Smax, "Hq": dc.Hq, "Hkv": dc.Hkv, "D": dc.D,
-                       "sum_seqlens": int(din["seqlens"].sum()) if do_dec else None, "bytes_per_step": dbytes},
+            "workload": main_name,
+            "prefill": main["prefill_cfg"],
+            "decode": main["decode_cfg"],
             "parallelism": (f"head-parallel x{world} (whole GQA groups per rank, no data exchange)" if strong
                             else f"replicas x{world} (independent per-GPU batches)"),
-            "l2": "no flush: inputs larger than L2 (q 268 MB; decode streams 1.2 GB per step)",
+            "l2": "no flush: inputs larger than L2 (prefill q 537 MB; the decode streams 4.3 GB per step)",
         },
-        "decode": {
-            "value": round(dec_value, 1), "unit": "GB/s", "us_per_step": round(1000 * dec_launch_ms, 2),
-            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": traffic_d,
-                         "peak_source": f"{peak_src} hbm_gbs",
-                         "frac_of_spec": round(gbs / SPEC_HBM_GBS, 4), "spec_peak": SPEC_HBM_GBS},
-        },
-        "roofline": {
-            "bound": "tensor", "achieved": round(tflops, 2), "peak": peak_t, "unit": "TFLOP/s",
-            "frac": round(tflops / peak_t, 4), "traffic": traffic,
-            "kernel": "diffattn_prefill_sm100", "flops_per_launch": flops,
-            "launch_ms": round(pre_launch_ms, 4), "peak_source": f"{peak_src} bf16_tflops (burst)",
-            "frac_of_spec": round(tflops / SPEC_BF16_TFLOPS, 4), "spec_peak": SPEC_BF16_TFLOPS,
-        },
+        "decode": main["decode"],
+        "roofline": main["roofline"],
         "e2e": {
-            "value": round(world * flops * e2e_steps / (e2e_ms * 1e-3) / 1e12, 3) if do_pre else None,
+            "value": round(world * main_flops / (e2e_ms * 1e-3) / 1e12, 3) if do_pre else None,
             "unit": "TFLOP/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-            "ms_per_step": round(e2e_ms / e2e_steps, 3),
-            "note": "prefill FLOPs over a step that copies q/k/v/lambda and the decode q/seqlens/lambda "
-                    "from pinned host memory, runs both kernels through the C ABI and copies both "
-                    "outputs back",
+            "ms_per_step": round(e2e_ms, 3),
+            "note": "prefill FLOPs over a step that copies the prefill's q/k/v/lambda and the decode's q, seqlens "
+                    "and lambda inputs from pinned host memory, runs the kernels through the C ABI and copies both "
+                    "outputs back; uploads, kernels and downloads run on three streams ordered by events, so step "
+                    "i+1's uploads and step i's downloads overlap step i's kernels",
         },
-        "gpu_launches": (int(do_pre) + int(do_dec)) * K,
+        "gpu_launches": main_launches * K,
         "clocks": clk,
+        "second_workload": also,
     }
     if args.only:
         line["only"] = args.only
     if world == 1 and not args.no_cpu_baseline and do_pre and do_dec:
-        line["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds, inputs=(pin, din))
     else:
         line["cpu_baseline"] = None
     return line
@@ -438,7 +600,11 @@ def _decode_seqs(inp, case, n_seqs, seed):
         b = int(rng.integers(case.B))
         n = int(inp["seqlens"][b])
         sl = inp["seqlens"][b:b + 1]
-        ora.decode(inp["q"][b:b + 1], inp["kcache"][b:b + 1], inp["vcache"][b:b + 1], sl, inp["lam"][b:b + 1])
+        if inp["lam"] is None:  # V1 lambda: one value per pair from the four vectors
+            lam = ora.lambda_v1(inp["lq1"], inp["lk1"], inp["lq2"], inp["lk2"], inp["lambda_init"])[None, :]
+        else:
+            lam = inp["lam"][b:b + 1]
+        ora.decode(inp["q"][b:b + 1], inp["kcache"][b:b + 1], inp["vcache"][b:b + 1], sl, lam)
         byts += n * case.Hkv * case.D * 2 * 2
     return byts, time.perf_counter() - t0
 
@@ -466,10 +632,10 @@ def cpu_baseline(seconds=15.0, inputs=None):
     f, t = _prefill_units(pin, pc, 4, seed=1)
     n = max(4, int(0.8 * seconds / max(t / 4, 1e-6)))
     f, t = _prefill_units(pin, pc, n, seed=2)
-    b, td = _decode_seqs(din, dc, 2, seed=3)
+    b, td = _decode_seqs(din, dc, 1, seed=3)
     return {"value": round(f / t / 1e12, 6), "unit": "TFLOP/s", "cores": _oracle_threads(), "kind": "oracle",
-            "sample": f"{n} random (batch, pair, 128-row tile) units of the B=4 S=4096 prefill "
-                      f"({t:.1f} s); decode: 2 full sequences of the B=64 decode ({td:.1f} s)",
+            "sample": f"{n} random (batch, pair, 128-row tile) units of the B={pc.B} S={pc.S} prefill "
+                      f"({t:.1f} s); decode: 1 full sequence of the B={dc.B} x {dc.Smax} decode ({td:.1f} s)",
             "decode_gbs": round(b / td / 1e9, 4), "blas": _blas_name()}
 
 
@@ -501,8 +667,8 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1000 * secs / args.steps, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic: the same seeded inputs as the GPU arm",
-        "config": {"workload": "prefill B=4 S=4096 Hq=64 Hkv=8 D=128 causal + decode B=64 Smax=8192 len "
-                               "U[1024,8192]; each step a bounded sample", "prefill_units_per_step": units},
+        "config": {"workload": _workload_name(pc, dc), "sample": "each step a bounded sample",
+                   "prefill_units_per_step": units},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": _oracle_threads(), "kind": "oracle",
                          "sample": f"{units} random (batch, pair, 128-row tile) prefill units per step; "
                                    f"decode: one full sequence on every {max(1, args.steps // 8)}-th step"},
@@ -708,6 +874,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-second", action="store_true",
+                    help="skip the second prefill and decode workloads (B=4 x 4k prefill, B=64 decode)")
     ap.add_argument("--ref-seconds", type=float, default=120.0,
                     help="host-time budget of the whole reference run (warm-up and timed steps)")
     ap.add_argument("--workload", choices=("prefill_long", "decode_needle", "window", "varlen", "paged", "multi",

@@ -29,14 +29,25 @@
  *     a pointer after the call returns.
  *   - Calls are asynchronous on `stream` (NULL = the legacy default stream) and reentrant:
  *     the library holds no per-call state. A return of DA2_OK means the work was enqueued.
+ *     Two pieces of process-wide state exist: the device error word (below), one per device
+ *     and shared by every call on every stream of that device, and the no-allocation decode
+ *     array of diffattn_v2_decode_noalloc.
+ *   - The library caches, per device, the device addresses of its own device variables (the
+ *     error word and the no-allocation array), looked up in the context current at the
+ *     first call on that device. It supports the device's primary context (what the CUDA
+ *     runtime uses by default); the cached addresses do not survive cudaDeviceReset, so a
+ *     process that resets a device must not call the library on it afterwards.
  *   - Argument checks happen on the host before anything is launched; a failed check
  *     returns an error and launches nothing. Null pointers, sizes <= 0 (except the B == 0
  *     or S == 0 no-op), an odd Hq, Hq % (2*Hkv) != 0, pointers not 16-byte aligned and a
  *     too-small workspace give DA2_ERR_INVALID. Valid shapes the kernels do not implement
  *     give DA2_ERR_UNSUPPORTED. A failed CUDA call gives DA2_ERR_CUDA.
  *   - Kernels never trap. Every wait inside a kernel is bounded; on expiry the kernel
- *     records an error word on the device and returns. diffattn_v2_device_error() reads
- *     and clears it.
+ *     records an error word on the device and returns; the outputs of that call are then
+ *     undefined (a decode whose split gave up never writes that (b, KV head)'s output).
+ *     diffattn_v2_device_error() reads and clears the word. There is one word per device,
+ *     not per stream: an error raised by a kernel on any stream is reported to (and
+ *     cleared by) whichever caller reads the word first.
  *   - The score scale is 1/sqrt(D) for both branches. lambda may be any finite fp32
  *     value (the V2 sigmoid-bounded value in (0,1), or a V1 value that may be negative or
  *     above 1).
@@ -353,7 +364,10 @@ DA2_API int diffattn_v2_lambda_v2(const void* x, const void* w_lambda, const flo
  * Synchronise `stream`, then read and clear the device error word that kernels set when a
  * bounded wait expires. *code receives 0 when no kernel reported an error, else the code
  * of the first error recorded (a pipeline wait expired: 1 = in a prefill, 2 = in a decode,
- * 3 = in a backward kernel).
+ * 3 = in a backward kernel). The word belongs to the current device, not to `stream`: it
+ * holds the first error of a kernel on ANY stream of the device since it was last cleared,
+ * and reading it clears it for every caller. Synchronising `stream` only orders the read
+ * after this stream's kernels; kernels of other streams still running may set it later.
  * Returns DA2_ERR_DEVICE when *code != 0, DA2_OK when it is 0, DA2_ERR_CUDA on a CUDA
  * failure. `code` is a HOST pointer and may be NULL.
  */
