@@ -78,6 +78,21 @@ bool heads_ok(int Hq, int Hkv) { return Hq > 0 && Hkv > 0 && (Hq % 2) == 0 && (H
 
 namespace da2 {
 
+size_t decode_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int nsplit) {
+  const size_t rows = static_cast<size_t>(B) * T * Hq * nsplit;
+  return rows * static_cast<size_t>(D) * sizeof(float) + rows * 2 * sizeof(float) +
+         (static_cast<size_t>(B) * Hkv * sizeof(int) + 15) / 16 * 16;
+}
+
+DecodeWorkspace decode_workspace_layout(void* base, int B, int T, int Hq, int D, int nsplit) {
+  const size_t rows = static_cast<size_t>(B) * T * Hq * nsplit;
+  DecodeWorkspace w;
+  w.o = static_cast<float*>(base);
+  w.ml = w.o + rows * static_cast<size_t>(D);
+  w.counters = reinterpret_cast<int*>(w.ml + rows * 2);
+  return w;
+}
+
 void decode_split_plan(int B, int Smax, int Hkv, int* split_len, int* nsplit) {
   // Aim for about 8 waves of 2 CTAs per SM over the (b, g) units, with splits that are a
   // multiple of the 64-token stage and between 512 and 4096 tokens long.
@@ -129,11 +144,12 @@ int diffattn_v2_prefill(const void* q, const void* k, const void* v, const float
   int* err = nullptr;
   cudaError_t e = device_error_ptr(&err);
   if (e != cudaSuccess) return DA2_ERR_CUDA;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, tkh;
   if (encode_bshd(&tq, q, D, Hq, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tk, k, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tv, v, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
-  e = da2::launch_prefill(tq, tk, tv, lambda, static_cast<__nv_bfloat16*>(out), err, B, S, Hq, Hkv, causal, 0,
+  if (encode_bshd(&tkh, k, D, Hkv, S, B, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
+  e = da2::launch_prefill(tq, tk, tv, &tkh, lambda, static_cast<__nv_bfloat16*>(out), err, B, S, Hq, Hkv, causal, 0,
                           nullptr, reinterpret_cast<cudaStream_t>(stream));
   return status_of(e);
 }
@@ -150,12 +166,13 @@ int diffattn_v2_prefill_window(const void* q, const void* k, const void* v, cons
   int* err = nullptr;
   cudaError_t e = device_error_ptr(&err);
   if (e != cudaSuccess) return DA2_ERR_CUDA;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, tkh;
   if (encode_bshd(&tq, q, D, Hq, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tk, k, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tv, v, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  if (encode_bshd(&tkh, k, D, Hkv, S, B, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
   // a window of S or more keys is the plain causal mask
-  e = da2::launch_prefill(tq, tk, tv, lambda, static_cast<__nv_bfloat16*>(out), err, B, S, Hq, Hkv, 1,
+  e = da2::launch_prefill(tq, tk, tv, &tkh, lambda, static_cast<__nv_bfloat16*>(out), err, B, S, Hq, Hkv, 1,
                           window >= S ? 0 : window, nullptr, reinterpret_cast<cudaStream_t>(stream));
   return status_of(e);
 }
@@ -175,11 +192,12 @@ int diffattn_v2_prefill_varlen(const void* q, const void* k, const void* v, cons
   int* err = nullptr;
   cudaError_t e = device_error_ptr(&err);
   if (e != cudaSuccess) return DA2_ERR_CUDA;
-  CUtensorMap tq, tk, tv;  // the packed tokens as one batch of total_tokens rows
+  CUtensorMap tq, tk, tv, tkh;  // the packed tokens as one batch of total_tokens rows
   if (encode_bshd(&tq, q, D, Hq, total_tokens, 1, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tk, k, D, Hkv, total_tokens, 1, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tv, v, D, Hkv, total_tokens, 1, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
-  e = da2::launch_prefill(tq, tk, tv, lambda, static_cast<__nv_bfloat16*>(out), err, B, max_seqlen, Hq, Hkv, causal,
+  if (encode_bshd(&tkh, k, D, Hkv, total_tokens, 1, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
+  e = da2::launch_prefill(tq, tk, tv, &tkh, lambda, static_cast<__nv_bfloat16*>(out), err, B, max_seqlen, Hq, Hkv, causal,
                           0, cu_seqlens, reinterpret_cast<cudaStream_t>(stream));
   return status_of(e);
 }
@@ -213,11 +231,12 @@ int diffattn_v2_prefill_train(const void* q, const void* k, const void* v, const
   int* err = nullptr;
   cudaError_t e = device_error_ptr(&err);
   if (e != cudaSuccess) return DA2_ERR_CUDA;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, tkh;
   if (encode_bshd(&tq, q, D, Hq, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tk, k, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tv, v, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
-  e = da2::launch_prefill(tq, tk, tv, lambda, static_cast<__nv_bfloat16*>(out), err, B, S, Hq, Hkv, causal, 0,
+  if (encode_bshd(&tkh, k, D, Hkv, S, B, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
+  e = da2::launch_prefill(tq, tk, tv, &tkh, lambda, static_cast<__nv_bfloat16*>(out), err, B, S, Hq, Hkv, causal, 0,
                           nullptr, reinterpret_cast<cudaStream_t>(stream), static_cast<__nv_bfloat16*>(o_branch),
                           lse);
   return status_of(e);
@@ -286,12 +305,13 @@ int diffattn_v2_prefill_window_train(const void* q, const void* k, const void* v
   int* err = nullptr;
   cudaError_t e = device_error_ptr(&err);
   if (e != cudaSuccess) return DA2_ERR_CUDA;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, tkh;
   if (encode_bshd(&tq, q, D, Hq, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tk, k, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tv, v, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  if (encode_bshd(&tkh, k, D, Hkv, S, B, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
   // a window of S or more keys is the plain causal mask
-  e = da2::launch_prefill(tq, tk, tv, lambda, static_cast<__nv_bfloat16*>(out), err, B, S, Hq, Hkv, 1,
+  e = da2::launch_prefill(tq, tk, tv, &tkh, lambda, static_cast<__nv_bfloat16*>(out), err, B, S, Hq, Hkv, 1,
                           window >= S ? 0 : window, nullptr, reinterpret_cast<cudaStream_t>(stream),
                           static_cast<__nv_bfloat16*>(o_branch), lse);
   return status_of(e);
@@ -320,11 +340,12 @@ int diffattn_v2_prefill_varlen_train(const void* q, const void* k, const void* v
   int* err = nullptr;
   cudaError_t e = device_error_ptr(&err);
   if (e != cudaSuccess) return DA2_ERR_CUDA;
-  CUtensorMap tq, tk, tv;  // the packed tokens as one batch of total_tokens rows
+  CUtensorMap tq, tk, tv, tkh;  // the packed tokens as one batch of total_tokens rows
   if (encode_bshd(&tq, q, D, Hq, total_tokens, 1, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tk, k, D, Hkv, total_tokens, 1, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tv, v, D, Hkv, total_tokens, 1, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
-  e = da2::launch_prefill(tq, tk, tv, lambda, static_cast<__nv_bfloat16*>(out), err, B, max_seqlen, Hq, Hkv, causal,
+  if (encode_bshd(&tkh, k, D, Hkv, total_tokens, 1, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
+  e = da2::launch_prefill(tq, tk, tv, &tkh, lambda, static_cast<__nv_bfloat16*>(out), err, B, max_seqlen, Hq, Hkv, causal,
                           0, cu_seqlens, reinterpret_cast<cudaStream_t>(stream), static_cast<__nv_bfloat16*>(o_branch),
                           lse);
   return status_of(e);
@@ -373,10 +394,7 @@ size_t diffattn_v2_decode_workspace_size(int B, int Smax, int Hq, int Hkv, int D
   if (B <= 0 || Smax <= 0 || D <= 0 || !heads_ok(Hq, Hkv)) return 0;
   int split_len = 0, nsplit = 0;
   da2::decode_split_plan(B, Smax, Hkv, &split_len, &nsplit);
-  const size_t rows = static_cast<size_t>(B) * Hq * nsplit;
-  // partials O, (m, l), then one split counter per (b, KV head)
-  return rows * static_cast<size_t>(D) * sizeof(float) + rows * 2 * sizeof(float) +
-         (static_cast<size_t>(B) * Hkv * sizeof(int) + 15) / 16 * 16;
+  return da2::decode_workspace_bytes(B, 1, Hq, Hkv, D, nsplit);
 }
 
 int diffattn_v2_decode(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens,
@@ -400,11 +418,9 @@ int diffattn_v2_decode(const void* q, const void* kcache, const void* vcache, co
   CUtensorMap tk, tv;
   if (encode_bshd(&tk, kcache, D, Hkv, Smax, B, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tv, vcache, D, Hkv, Smax, B, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
-  float* ws_o = static_cast<float*>(workspace);
-  float* ws_ml = ws_o + static_cast<size_t>(B) * Hq * nsplit * D;
-  int* counters = reinterpret_cast<int*>(ws_ml + static_cast<size_t>(B) * Hq * nsplit * 2);
+  const da2::DecodeWorkspace ws = da2::decode_workspace_layout(workspace, B, 1, Hq, D, nsplit);
   e = da2::launch_decode(tk, tv, static_cast<const __nv_bfloat16*>(q), seqlens, lambda,
-                         static_cast<__nv_bfloat16*>(out), ws_o, ws_ml, counters, err, B, Smax, Hq, Hkv, nsplit,
+                         static_cast<__nv_bfloat16*>(out), ws.o, ws.ml, ws.counters, err, B, Smax, Hq, Hkv, nsplit,
                          split_len,
                          nullptr, 0, 0, 1, reinterpret_cast<cudaStream_t>(stream));
   return status_of(e);
@@ -438,11 +454,9 @@ int diffattn_v2_decode_paged(const void* q, const void* kpages, const void* vpag
   CUtensorMap tk, tv;  // pages as a [num_pages, page_size] batch of rows
   if (encode_bshd(&tk, kpages, D, Hkv, page_size, num_pages, 64, box) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tv, vpages, D, Hkv, page_size, num_pages, 64, box) != cudaSuccess) return DA2_ERR_CUDA;
-  float* ws_o = static_cast<float*>(workspace);
-  float* ws_ml = ws_o + static_cast<size_t>(B) * Hq * nsplit * D;
-  int* counters = reinterpret_cast<int*>(ws_ml + static_cast<size_t>(B) * Hq * nsplit * 2);
+  const da2::DecodeWorkspace ws = da2::decode_workspace_layout(workspace, B, 1, Hq, D, nsplit);
   e = da2::launch_decode(tk, tv, static_cast<const __nv_bfloat16*>(q), seqlens, lambda,
-                         static_cast<__nv_bfloat16*>(out), ws_o, ws_ml, counters, err, B, Smax, Hq, Hkv, nsplit,
+                         static_cast<__nv_bfloat16*>(out), ws.o, ws.ml, ws.counters, err, B, Smax, Hq, Hkv, nsplit,
                          split_len,
                          block_table, max_pages, page_shift, 1, reinterpret_cast<cudaStream_t>(stream));
   return status_of(e);
@@ -452,9 +466,7 @@ size_t diffattn_v2_decode_multi_workspace_size(int B, int T, int Smax, int Hq, i
   if (B <= 0 || T <= 0 || Smax <= 0 || D <= 0 || !heads_ok(Hq, Hkv)) return 0;
   int split_len = 0, nsplit = 0;
   da2::decode_split_plan(B, Smax, Hkv, &split_len, &nsplit);
-  const size_t rows = static_cast<size_t>(B) * T * Hq * nsplit;
-  return rows * static_cast<size_t>(D) * sizeof(float) + rows * 2 * sizeof(float) +
-         (static_cast<size_t>(B) * Hkv * sizeof(int) + 15) / 16 * 16;
+  return da2::decode_workspace_bytes(B, T, Hq, Hkv, D, nsplit);
 }
 
 int diffattn_v2_decode_multi(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens,
@@ -479,11 +491,9 @@ int diffattn_v2_decode_multi(const void* q, const void* kcache, const void* vcac
   CUtensorMap tk, tv;
   if (encode_bshd(&tk, kcache, D, Hkv, Smax, B, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tv, vcache, D, Hkv, Smax, B, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
-  float* ws_o = static_cast<float*>(workspace);
-  float* ws_ml = ws_o + static_cast<size_t>(B) * T * Hq * nsplit * D;
-  int* counters = reinterpret_cast<int*>(ws_ml + static_cast<size_t>(B) * T * Hq * nsplit * 2);
+  const da2::DecodeWorkspace ws = da2::decode_workspace_layout(workspace, B, T, Hq, D, nsplit);
   e = da2::launch_decode(tk, tv, static_cast<const __nv_bfloat16*>(q), seqlens, lambda,
-                         static_cast<__nv_bfloat16*>(out), ws_o, ws_ml, counters, err, B, Smax, Hq, Hkv, nsplit,
+                         static_cast<__nv_bfloat16*>(out), ws.o, ws.ml, ws.counters, err, B, Smax, Hq, Hkv, nsplit,
                          split_len,
                          nullptr, 0, 0, T, reinterpret_cast<cudaStream_t>(stream));
   return status_of(e);

@@ -12,10 +12,11 @@ namespace da2 {
 // bf16 prefill on tcgen05 (D = 128); window > 0 (causal only) limits query i to keys
 // i-window+1 .. i. With cu_seqlens (device, B+1 entries) the tensors hold B packed sequences
 // as one [1,T] batch and S is the longest sequence. Tensor maps: Q over [B,S,Hq,D], K/V over [B,S,Hkv,D],
-// boxes of 64 (d) x 1 (head) x 128 (rows) x 1, 128-byte swizzle.
+// boxes of 64 (d) x 1 (head) x 128 (rows) x 1, 128-byte swizzle; tmKh (optional) over K with
+// boxes of 64 (d) x 1 x 64 (rows) x 1, for the CTA-pair form (GQA groups of a multiple of 4).
 cudaError_t launch_prefill(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                           const float* lambda, __nv_bfloat16* out, int* err, int B, int S, int Hq, int Hkv,
-                           int causal, int window, const int* cu_seqlens, cudaStream_t stream,
+                           const CUtensorMap* tmKh, const float* lambda, __nv_bfloat16* out, int* err, int B, int S,
+                           int Hq, int Hkv, int causal, int window, const int* cu_seqlens, cudaStream_t stream,
                            __nv_bfloat16* o_branch = nullptr, float* lse = nullptr);
 
 // tcgen05 backward of the bf16 prefill (D = 128): preprocess into the workspace (row terms;
@@ -47,6 +48,18 @@ cudaError_t launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const 
 
 // Tokens per split and number of splits of the bf16 decode for these sizes.
 void decode_split_plan(int B, int Smax, int Hkv, int* split_len, int* nsplit);
+
+// The bf16 decode's workspace, in this order: fp32 partial outputs O [rows, D], fp32 (m, l)
+// [rows, 2], then one int split counter per (b, KV head), padded to 16 bytes; rows =
+// B * T * Hq * nsplit (T new tokens per sequence). Every entry point that hands the split
+// kernel a workspace (caller-provided or the library's own array) lays it out through these.
+struct DecodeWorkspace {
+  float* o;
+  float* ml;
+  int* counters;
+};
+size_t decode_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int nsplit);
+DecodeWorkspace decode_workspace_layout(void* base, int B, int T, int Hq, int D, int nsplit);
 
 // fp32 CUDA-core paths (D in {64, 128}).
 cudaError_t launch_prefill_f32(const float* q, const float* k, const float* v, const float* lambda, float* out,

@@ -36,6 +36,8 @@
 // this is exact up to rounding while skipping most rescales. The epilogue forms
 // O1/l1 - lambda O2/l2 in fp32 and rounds once to bf16.
 
+#include <cstdlib>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -54,15 +56,29 @@ constexpr int kThreads = 384;
 // each role's code to its share: at 200 the softmax path has no spills (at 168 it spilled).
 constexpr int kRegsLaunch = 168, kRegsSmall = 96, kRegsSoftmax = 200;
 static_assert(128 * kRegsSmall + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split exceeds the launch");
-constexpr int kStages = 2;
 
 constexpr uint32_t kChunkBytes = 128 * 64 * 2;     // 128 rows x 64 bf16 (one swizzle-128B half)
 constexpr uint32_t kTileBytes = 2 * kChunkBytes;   // 128 rows x 128 bf16
 
-constexpr uint32_t kOffQ = 0;                                 // Q1, Q2
-constexpr uint32_t kOffK = kOffQ + 2 * kTileBytes;            // K stages
-constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;      // V stages
-constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;    // mbarriers
+// Shared-memory plan of the two kernel forms. One CTA per item: K and V tiles of 128 keys x
+// 128 d in a 2-stage ring. CTA pair (two CTAs of a cluster on an SM pair share every MMA):
+// each CTA holds half of every K tile (64 keys x 128 d) and half of every V tile (128 keys x
+// 64 d), in a 4-stage ring. Both use 192 KB before the barriers.
+template <bool kPair>
+struct Ring {
+  static constexpr int kStages = kPair ? 4 : 2;
+  static constexpr uint32_t kKChunk = kPair ? 64 * 64 * 2 : kChunkBytes;  // one 64-d half of a K stage
+  static constexpr uint32_t kKStage = 2 * kKChunk;
+  static constexpr uint32_t kVStage = kPair ? kChunkBytes : kTileBytes;
+};
+
+constexpr uint32_t kOffQ = 0;                                         // Q1, Q2
+constexpr uint32_t kOffK = kOffQ + 2 * kTileBytes;                    // K stages
+constexpr uint32_t kOffBar = kOffK + 2 * 2 * kTileBytes;              // after the K and V stages
+static_assert(kOffK + Ring<false>::kStages * (Ring<false>::kKStage + Ring<false>::kVStage) == kOffBar, "smem plan");
+static_assert(kOffK + Ring<true>::kStages * (Ring<true>::kKStage + Ring<true>::kVStage) == kOffBar, "smem plan");
+template <bool kPair>
+__host__ __device__ constexpr uint32_t off_v() { return kOffK + Ring<kPair>::kStages * Ring<kPair>::kKStage; }
 constexpr uint32_t kOffMisc = kOffBar + 256;                  // tmem slot, abort flag
 constexpr uint32_t kOffL = kOffMisc + 64;                     // [item parity][branch][row] fp32 row sums
 // packed sequences: sequence ids sorted by row-tile count (longest first), then the counts
@@ -75,18 +91,19 @@ constexpr uint32_t kSmemBytes = kSmemUsed + 1024;             // slack for 1024-
 enum Bar : int {
   kQFull = 0,
   kKFull = 1,    // +stage
-  kKEmpty = 3,   // +stage
-  kVFull = 5,    // +stage
-  kVEmpty = 7,   // +stage
-  kSFull = 9,    // +branch
-  kPFull = 11,   // +2*branch+half: P of keys 64*half .. 64*half+63 is in TMEM
-  kOFull = 15,
-  kDrain = 16,
-  kQEmpty = 17,  // the item's last score GEMM has read Q
-  kOEmpty = 18,  // every softmax thread has read O1, O2 of the item (epilogue done)
-  kLx = 19,      // both branches' row sums of the item are in shared memory
-  kNumBars = 20
+  kKEmpty = 5,   // +stage
+  kVFull = 9,    // +stage
+  kVEmpty = 13,  // +stage
+  kSFull = 17,   // +branch
+  kPFull = 19,   // +2*branch+half: P of keys 64*half .. 64*half+63 is in TMEM
+  kOFull = 23,
+  kDrain = 24,
+  kQEmpty = 25,  // the item's last score GEMM has read Q
+  kOEmpty = 26,  // every softmax thread has read O1, O2 of the item (epilogue done)
+  kLx = 27,      // both branches' row sums of the item are in shared memory
+  kNumBars = 28
 };
+static_assert(kNumBars * 8 <= 256, "barrier slots");
 
 constexpr uint32_t kTmS1 = 0, kTmS2 = 128, kTmO1 = 256, kTmO2 = 384;
 
@@ -127,13 +144,16 @@ struct SortedCursor {
 // packed sequences only non-empty items are listed (seq_id, seq_nt: sorted ids and row-tile
 // counts; n_dense: the list's length); a role's item indices only grow, so its cursor only
 // moves forward.
-template <bool kVarlen, bool kWindow>
+// With kPair the unit of work is a pair of pairs of one KV head: cluster c takes the item and
+// its CTA of rank r computes pair 2u + r (u = the unit's index among the Hq/4 units).
+template <bool kVarlen, bool kWindow, bool kPair>
 __device__ __forceinline__ bool work_item(const Params& p, int k, WorkItem& w, SortedCursor& cur,
-                                          const int* seq_id, const int* seq_nt, int n_dense) {
-  const int n_ctas = static_cast<int>(gridDim.x);
-  const int c = static_cast<int>(blockIdx.x);
+                                          const int* seq_id, const int* seq_nt, int n_dense, uint32_t cta_rank) {
+  constexpr int kCtas = kPair ? 2 : 1;
+  const int n_ctas = static_cast<int>(gridDim.x) / kCtas;   // CTAs, or clusters of two
+  const int c = static_cast<int>(blockIdx.x) / kCtas;
   const int idx = k * n_ctas + ((k & 1) ? n_ctas - 1 - c : c);
-  const int n_pairs = p.Hq >> 1;
+  const int n_pairs = p.Hq >> (kPair ? 2 : 1);   // work units per (sequence, row tile)
   if (kVarlen && p.sorted_seqs) {
     if (idx >= n_dense) return false;
     int t = p.n_row_tiles - 1 - cur.r;
@@ -160,6 +180,7 @@ __device__ __forceinline__ bool work_item(const Params& p, int k, WorkItem& w, S
     w.b = bp / n_pairs;
     w.pair = bp - w.b * n_pairs;
   }
+  if (kPair) w.pair = 2 * w.pair + static_cast<int>(cta_rank);
   w.m0 = w.tile * BM;
   w.S = p.S;
   w.tok0 = 0;
@@ -184,20 +205,22 @@ __device__ __forceinline__ bool work_item(const Params& p, int k, WorkItem& w, S
   return true;
 }
 
-// Set scores of keys outside columns lo..hi of this row to -inf.
-__device__ __forceinline__ void mask_row(uint32_t (&sr)[4][32], int lo, int hi) {
+// Set scores of keys outside columns lo..hi of this thread's NC x 32 columns to -inf.
+template <int NC>
+__device__ __forceinline__ void mask_row(uint32_t (&sr)[NC][32], int lo, int hi) {
 #pragma unroll
-  for (int c = 0; c < 4; ++c)
+  for (int c = 0; c < NC; ++c)
 #pragma unroll
     for (int e = 0; e < 32; ++e)
       if (32 * c + e > hi || 32 * c + e < lo) sr[c][e] = __float_as_uint(-INFINITY);
 }
 
-// Max of the 128 raw scores of a row: 3-input max, four independent chains.
-__device__ __forceinline__ float row_max(const uint32_t (&sr)[4][32]) {
+// Max of this thread's NC x 32 raw scores: 3-input max, four independent chains.
+template <int NC>
+__device__ __forceinline__ float row_max(const uint32_t (&sr)[NC][32]) {
   float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-  for (int c = 0; c < 4; ++c)
+  for (int c = 0; c < NC; ++c)
 #pragma unroll
     for (int e = 0; e < 32; e += 8) {
       m0 = fmax3(m0, __uint_as_float(sr[c][e + 0]), __uint_as_float(sr[c][e + 1]));
@@ -283,12 +306,68 @@ __device__ __forceinline__ float exp_pack_store(const uint32_t (&sr)[4][32], int
   return (s0 + s1) + (s2 + s3);
 }
 
+// Waits on barriers that the other CTA arrives on use the default (CTA-scope acquire) form,
+// as the arrivals do; what they order is tensor memory, through the tcgen05 fences.
+constexpr bool kClusterAcquire = false;
+
+// A bounded wait on one of this CTA's barriers (pwait), or, by the MMA thread, on a barrier
+// that the other CTA's threads arrive on (pwait_x: acquire at cluster scope). With kPair a wait
+// that gives up also raises the other CTA's abort flag (flag_addr: this CTA's flag).
+template <bool kPair>
+__device__ __forceinline__ void raise_peer_abort(uint32_t flag_addr) {
+  if constexpr (kPair) st_cluster_u32(mapa_shared(flag_addr, cluster_ctarank() ^ 1u), 1u);
+}
+template <bool kPair>
+__device__ __forceinline__ bool pwait(uint32_t b, uint32_t parity, volatile int* abort_flag, uint32_t flag_addr) {
+  const bool r = mbar_wait(b, parity, abort_flag);
+  if (kPair && !r) raise_peer_abort<kPair>(flag_addr);
+  return r;
+}
+template <bool kPair>
+__device__ __forceinline__ bool pwait_x(uint32_t b, uint32_t parity, volatile int* abort_flag, uint32_t flag_addr) {
+  const bool r = (kPair && kClusterAcquire) ? mbar_wait_cluster(b, parity, abort_flag) : mbar_wait(b, parity, abort_flag);
+  if (kPair && !r) raise_peer_abort<kPair>(flag_addr);
+  return r;
+}
+
+// A softmax thread's arrival on a barrier the MMA thread waits on, after its tensor-memory
+// stores or loads: every thread on this CTA's barrier, or with kPair once per warp on the even
+// CTA's barrier (bar: this CTA's copy).
+template <bool kPair>
+__device__ __forceinline__ void arrive_for_mma(uint32_t bar, int lane) {
+  tc_fence_before();
+  if constexpr (kPair) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive_cluster(mapa_shared(bar, 0));
+  } else {
+    mbar_arrive(bar);
+  }
+}
+
 // kVarlen: packed sequences (p.cu_seqlens); kWindow: causal sliding window (p.window). The
-// plain [B,S] prefill is the <false, false> instance and carries neither.
-template <bool kVarlen, bool kWindow>
+// plain [B,S] prefill is the <false, false, *> instance and carries neither.
+// kPair: a cluster of two CTAs on an SM pair computes two pairs of the same KV head over the
+// same 128 query rows. The even CTA's MMA thread issues every GEMM once for both
+// (tcgen05.mma.cta_group::2, M = 256: each CTA's own 128 rows of Q or P against a shared K or
+// V tile of which each CTA loaded half), so per unit of work the tensor-core instructions and
+// the shared-memory operand reads per SM are cut (A 4 KB + half of B 2 KB per score
+// instruction and SM instead of 4 + 4 KB) and each SM loads half of every K/V tile.
+// Protocol across the pair (all loads are plain per-CTA TMA copies, none multicast):
+//   * copies of both CTAs count their bytes on the even CTA's full barriers (the even CTA's
+//     producer announces both halves' bytes);
+//   * the MMA thread's commits arrive on the barrier at the same offset in both CTAs
+//     (S ready, O ready, K/V/Q stage free);
+//   * each softmax warp of either CTA arrives once on the even CTA's P and O-read barriers;
+//   * a wait that gives up raises the abort flag of both CTAs; both CTAs leave through one
+//     cluster barrier, after every copy and commit addressed to them has landed.
+template <bool kVarlen, bool kWindow, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
 diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                       const __grid_constant__ CUtensorMap tmV, const Params p) {
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKh,
+                       const Params p) {
+  using R = Ring<kPair>;
+  constexpr int kStages = R::kStages;
+  constexpr uint32_t kOffV = off_v<kPair>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -301,6 +380,12 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   const int lane = threadIdx.x & 31;
   const int n_pairs = p.Hq >> 1;
   const int group = p.Hq / p.Hkv;
+  const uint32_t cta_rank = kPair ? cluster_ctarank() : 0u;
+  const bool leader = cta_rank == 0;
+  // the even CTA's copy of barrier i in the cluster's shared window (this CTA's own without
+  // kPair); computed where used, so that no register holds it across the loops
+  auto bar_lead = [&](int i) -> uint32_t { return kPair ? mapa_shared(bar(i), 0) : bar(i); };
+  const uint32_t flag_addr = sbase + kOffMisc + 8;  // the abort flag's shared address
 
   int* seq_id = reinterpret_cast<int*>(smem + kOffSeq);
   int* seq_nt = seq_id + kMaxSortedSeqs;
@@ -308,8 +393,11 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i) {
       uint32_t count = 1;
-      if (i >= kPFull && i < kPFull + 4) count = 128;  // every softmax thread of the branch
-      if (i == kOEmpty || i == kLx) count = 256;       // every softmax thread
+      // P and O-read barriers: every softmax thread of the branch / CTA, or with kPair one
+      // arrival per softmax warp of both CTAs
+      if (i >= kPFull && i < kPFull + 4) count = kPair ? 8 : 128;
+      if (i == kOEmpty) count = kPair ? 16 : 256;
+      if (i == kLx) count = 256;
       mbar_init(bar(i), count);
     }
     *abort_flag = 0;
@@ -336,20 +424,26 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     if (threadIdx.x == 0) {
       int total = 0;
       for (int b = 0; b < p.B; ++b) total += nt[b];
-      *n_dense_slot = total * (p.Hq >> 1);
+      *n_dense_slot = total * (p.Hq >> (kPair ? 2 : 1));
     }
   }
   if (warp == 8 && lane == 0) {
     tma_prefetch_desc(&tmQ);
-    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(kPair ? &tmKh : &tmK);
     tma_prefetch_desc(&tmV);
   }
   if (warp == 9) {
-    tmem_alloc(smem_u32(tmem_slot), 512);
-    tmem_relinquish();
+    if constexpr (kPair) {
+      tmem_alloc_pair(smem_u32(tmem_slot), 512);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), 512);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (kPair) cluster_sync();  // both CTAs' barriers and tensor memory exist
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int n_dense = (kVarlen && p.sorted_seqs) ? *n_dense_slot : 0;
@@ -364,107 +458,155 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         // Counts over all items of this CTA: KV tiles (ring stage and phase) and Q tiles.
         int k_issued = 0, v_issued = 0, q_issued = 0;
         bool ok = true;
-        for (int k = 0; ok && work_item<kVarlen, kWindow>(p, k, w, cur, seq_id, seq_nt, n_dense); ++k) {
+        // the even CTA announces the bytes of both CTAs' halves
+        const uint32_t pair_mult = kPair ? 2u : 1u;
+        for (int k = 0; ok && work_item<kVarlen, kWindow, kPair>(p, k, w, cur, seq_id, seq_nt, n_dense, cta_rank);
+             ++k) {
           if (w.n_kv == 0) continue;
           // the single Q buffer is free once the previous item's last score GEMM has read it
-          if (q_issued > 0 && !(ok = mbar_wait(bar(kQEmpty), (q_issued - 1) & 1, abort_flag))) break;
-          mbar_arrive_expect_tx(bar(kQFull), 2 * kTileBytes);
+          if (q_issued > 0 && !(ok = pwait<kPair>(bar(kQEmpty), (q_issued - 1) & 1, abort_flag, flag_addr))) break;
+          if (leader) mbar_arrive_expect_tx(bar(kQFull), pair_mult * 2 * kTileBytes);
           for (int h = 0; h < 2; ++h)
-            for (int c = 0; c < 2; ++c)
-              tma_load_4d(sbase + kOffQ + h * kTileBytes + c * kChunkBytes, &tmQ, bar(kQFull), c * 64,
-                          2 * w.pair + h, w.tok0 + w.m0, w.tb);
+            for (int c = 0; c < 2; ++c) {
+              const uint32_t dst = sbase + kOffQ + h * kTileBytes + c * kChunkBytes;
+              if constexpr (kPair)
+                tma_load_4d_pair(dst, &tmQ, bar_lead(kQFull), c * 64, 2 * w.pair + h, w.tok0 + w.m0, w.tb);
+              else
+                tma_load_4d(dst, &tmQ, bar(kQFull), c * 64, 2 * w.pair + h, w.tok0 + w.m0, w.tb);
+            }
           ++q_issued;
           const int g = (2 * w.pair) / group;
           for (int it = 0; it < w.n_kv; ++it) {
             const int j = w.j_first + it;
             const int n = k_issued;  // this CTA's KV tile count so far
-            const int s = n & 1;
-            const uint32_t ph = (n >> 1) & 1;
-            if (!(ok = mbar_wait(bar(kKEmpty + s), ph ^ 1, abort_flag))) break;
-            mbar_arrive_expect_tx(bar(kKFull + s), kTileBytes);
-            for (int c = 0; c < 2; ++c)
-              tma_load_4d(sbase + kOffK + s * kTileBytes + c * kChunkBytes, &tmK, bar(kKFull + s), c * 64, g,
-                          w.tok0 + j * BN, w.tb);
+            const int s = n % kStages;
+            const uint32_t ph = (n / kStages) & 1;
+            if (!(ok = pwait<kPair>(bar(kKEmpty + s), ph ^ 1, abort_flag, flag_addr))) break;
+            if (leader) mbar_arrive_expect_tx(bar(kKFull + s), pair_mult * R::kKStage);
+            for (int c = 0; c < 2; ++c) {
+              const uint32_t dst = sbase + kOffK + s * R::kKStage + c * R::kKChunk;
+              if constexpr (kPair)  // keys 64*rank .. 64*rank+63 of the tile, all 128 d
+                tma_load_4d_pair(dst, &tmKh, bar_lead(kKFull + s), c * 64, g, w.tok0 + j * BN + 64 * cta_rank, w.tb);
+              else
+                tma_load_4d(dst, &tmK, bar(kKFull + s), c * 64, g, w.tok0 + j * BN, w.tb);
+            }
             k_issued = n + 1;
-            if (!(ok = mbar_wait(bar(kVEmpty + s), ph ^ 1, abort_flag))) break;
-            mbar_arrive_expect_tx(bar(kVFull + s), kTileBytes);
-            for (int c = 0; c < 2; ++c)
-              tma_load_4d(sbase + kOffV + s * kTileBytes + c * kChunkBytes, &tmV, bar(kVFull + s), c * 64, g,
-                          w.tok0 + j * BN, w.tb);
+            if (!(ok = pwait<kPair>(bar(kVEmpty + s), ph ^ 1, abort_flag, flag_addr))) break;
+            if (leader) mbar_arrive_expect_tx(bar(kVFull + s), pair_mult * R::kVStage);
+            if constexpr (kPair) {  // all 128 keys, d 64*rank .. 64*rank+63
+              tma_load_4d_pair(sbase + kOffV + s * R::kVStage, &tmV, bar_lead(kVFull + s), 64 * cta_rank, g,
+                               w.tok0 + j * BN, w.tb);
+            } else {
+              for (int c = 0; c < 2; ++c)
+                tma_load_4d(sbase + kOffV + s * R::kVStage + c * kChunkBytes, &tmV, bar(kVFull + s), c * 64, g,
+                            w.tok0 + j * BN, w.tb);
+            }
             v_issued = n + 1;
           }
         }
+        volatile int no_abort = 0;
         if (*abort_flag) {
-          // let copies still in flight land before the CTA's shared memory is released: at most
-          // one Q tile and one K and one V tile per stage can be outstanding
-          volatile int no_abort = 0;
-          if (q_issued > 0) mbar_wait(bar(kQFull), (q_issued - 1) & 1, &no_abort);
+          if constexpr (kPair) {
+            // the copies' completions count on the even CTA's barriers, which this CTA may not
+            // be able to see complete: give any copy still in flight time to land
+            const uint64_t t0 = global_timer_ns();
+            while (global_timer_ns() - t0 < 2000000ull) __nanosleep(1000);
+          } else {
+            // let copies still in flight land before the CTA's shared memory is released: at
+            // most one Q tile and one K and one V tile per stage can be outstanding
+            if (q_issued > 0) mbar_wait(bar(kQFull), (q_issued - 1) & 1, &no_abort);
+            for (int n = max(0, k_issued - kStages); n < k_issued; ++n)
+              mbar_wait(bar(kKFull + n % kStages), (n / kStages) & 1, &no_abort);
+            for (int n = max(0, v_issued - kStages); n < v_issued; ++n)
+              mbar_wait(bar(kVFull + n % kStages), (n / kStages) & 1, &no_abort);
+          }
+        } else if (kPair) {
+          // the even CTA's last commits (stage and Q releases) arrive on this CTA's barriers:
+          // take them before the CTA can leave (an abort raised meanwhile ends the waits; the
+          // even CTA then drains its MMAs, and with them these commits, before both leave)
           for (int n = max(0, k_issued - kStages); n < k_issued; ++n)
-            mbar_wait(bar(kKFull + (n & 1)), (n >> 1) & 1, &no_abort);
+            mbar_wait(bar(kKEmpty + n % kStages), (n / kStages) & 1, abort_flag);
           for (int n = max(0, v_issued - kStages); n < v_issued; ++n)
-            mbar_wait(bar(kVFull + (n & 1)), (n >> 1) & 1, &no_abort);
+            mbar_wait(bar(kVEmpty + n % kStages), (n / kStages) & 1, abort_flag);
+          if (q_issued > 0) mbar_wait(bar(kQEmpty), (q_issued - 1) & 1, abort_flag);
         }
       }
     } else if (warp == 9) {
       // -------------------------------------------------------------------- MMA issuer
-      if (lane == 0) {
-        constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
-        constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, HD, true);
+      // (with kPair only the even CTA's thread issues, for both CTAs)
+      if (lane == 0 && leader) {
+        constexpr int kM = kPair ? 2 * BM : BM;
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(kM, BN, false);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(kM, HD, true);
         auto desc_q = [&](int h, int kk) {
           return sdesc_sw128(sbase + kOffQ + h * kTileBytes + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024);
         };
+        // K stage: keys x d with d contiguous (K-major B operand); with kPair each CTA holds 64 keys
         auto desc_k = [&](int s, int kk) {
-          return sdesc_sw128(sbase + kOffK + s * kTileBytes + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024);
+          return sdesc_sw128(sbase + kOffK + s * R::kKStage + (kk >> 2) * R::kKChunk + (kk & 3) * 32, 16, 1024);
         };
-        // V tile: keys x d with d contiguous (MN-major B operand); 16 keys per K-step.
+        // V stage: keys x d with d contiguous (MN-major B operand); 16 keys per K-step; with
+        // kPair each CTA holds one 64-wide half of d (the leading offset is then unused)
         auto desc_v = [&](int s, int kk) {
-          return sdesc_sw128(sbase + kOffV + s * kTileBytes + kk * 2048, kChunkBytes, 1024);
+          return sdesc_sw128(sbase + kOffV + s * R::kVStage + kk * 2048, kChunkBytes, 1024);
         };
-        // O_b (+)= P_b V for this CTA's KV tile number n (ring stage n & 1, P barrier phase n & 1):
-        // the first 64 keys as soon as that half of P is in TMEM, the other 64 when the second
-        // half is. acc = false starts the item's sum.
+        auto mma_ss = [&](uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+          if constexpr (kPair) mma_bf16_ss_pair(d, a, b, id, acc);
+          else mma_bf16_ss(d, a, b, id, acc);
+        };
+        auto commit = [&](int i) {
+          if constexpr (kPair) tc_commit_pair(bar(i), 0x3);
+          else tc_commit(bar(i));
+        };
+        // O_b (+)= P_b V for this CTA's KV tile number n (ring stage n % kStages, P barrier
+        // phase n & 1): the first 64 keys as soon as that half of P is in TMEM, the other 64
+        // when the second half is. acc = false starts the item's sum.
         auto issue_pv = [&](uint32_t o_tmem, uint32_t p_tmem, int n, bool acc, uint32_t half0, uint32_t half1) {
   #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            if (!mbar_wait(h ? half1 : half0, n & 1, abort_flag)) return false;
+            if (!pwait_x<kPair>(h ? half1 : half0, n & 1, abort_flag, flag_addr)) return false;
             tc_fence_after();
   #pragma unroll
-            for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
-              mma_bf16_ts(o_tmem, p_tmem + kk * 8, desc_v(n & 1, kk), idesc_pv, (acc || kk > 0) ? 1u : 0u);
+            for (int kk = 4 * h; kk < 4 * h + 4; ++kk) {
+              const uint32_t acc_kk = (acc || kk > 0) ? 1u : 0u;
+              if constexpr (kPair) mma_bf16_ts_pair(o_tmem, p_tmem + kk * 8, desc_v(n % kStages, kk), idesc_pv, acc_kk);
+              else mma_bf16_ts(o_tmem, p_tmem + kk * 8, desc_v(n % kStages, kk), idesc_pv, acc_kk);
+            }
           }
           return true;
         };
         int n0 = 0;       // KV tiles of earlier items
         int n_items = 0;  // items done
         bool ok = true;
-        for (int k = 0; ok && work_item<kVarlen, kWindow>(p, k, w, cur, seq_id, seq_nt, n_dense); ++k) {
+        for (int k = 0; ok && work_item<kVarlen, kWindow, kPair>(p, k, w, cur, seq_id, seq_nt, n_dense, cta_rank);
+             ++k) {
           if (w.n_kv == 0) continue;
-          if (!(ok = mbar_wait(bar(kQFull), n_items & 1, abort_flag))) break;
+          if (!(ok = pwait<kPair>(bar(kQFull), n_items & 1, abort_flag, flag_addr))) break;
           for (int j = 0; j < w.n_kv; ++j) {
             const int n = n0 + j;
-            const int s = n & 1;
-            const uint32_t ph = (n >> 1) & 1;
-            if (!(ok = mbar_wait(bar(kKFull + s), ph, abort_flag))) break;
+            const int s = n % kStages;
+            const uint32_t ph = (n / kStages) & 1;
+            if (!(ok = pwait<kPair>(bar(kKFull + s), ph, abort_flag, flag_addr))) break;
             tc_fence_after();
   #pragma unroll
             for (int kk = 0; kk < HD / 16; ++kk)
-              mma_bf16_ss(tmem + kTmS1, desc_q(0, kk), desc_k(s, kk), idesc_qk, kk > 0 ? 1u : 0u);
-            tc_commit(bar(kSFull + 0));
+              mma_ss(tmem + kTmS1, desc_q(0, kk), desc_k(s, kk), idesc_qk, kk > 0 ? 1u : 0u);
+            commit(kSFull + 0);
             if (j > 0) {
               if (!(ok = issue_pv(tmem + kTmO2, tmem + kTmS2, n - 1, j > 1, bar(kPFull + 2), bar(kPFull + 3)))) break;
-              tc_commit(bar(kVEmpty + ((n - 1) & 1)));
+              commit(kVEmpty + (n - 1) % kStages);
             }
   #pragma unroll
             for (int kk = 0; kk < HD / 16; ++kk)
-              mma_bf16_ss(tmem + kTmS2, desc_q(1, kk), desc_k(s, kk), idesc_qk, kk > 0 ? 1u : 0u);
-            tc_commit(bar(kSFull + 1));
-            tc_commit(bar(kKEmpty + s));
-            if (j == w.n_kv - 1) tc_commit(bar(kQEmpty));
-            if (!(ok = mbar_wait(bar(kVFull + s), ph, abort_flag))) break;
+              mma_ss(tmem + kTmS2, desc_q(1, kk), desc_k(s, kk), idesc_qk, kk > 0 ? 1u : 0u);
+            commit(kSFull + 1);
+            commit(kKEmpty + s);
+            if (j == w.n_kv - 1) commit(kQEmpty);
+            if (!(ok = pwait<kPair>(bar(kVFull + s), ph, abort_flag, flag_addr))) break;
             if (j == 0 && n_items > 0) {
               // the first PV of an item overwrites O1 (and O2 after it): the previous item's
               // epilogue must have read them
-              if (!(ok = mbar_wait(bar(kOEmpty), (n_items - 1) & 1, abort_flag))) break;
+              if (!(ok = pwait_x<kPair>(bar(kOEmpty), (n_items - 1) & 1, abort_flag, flag_addr))) break;
               tc_fence_after();
             }
             if (!(ok = issue_pv(tmem + kTmO1, tmem + kTmS1, n, j > 0, bar(kPFull + 0), bar(kPFull + 1)))) break;
@@ -472,13 +614,15 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
           if (!ok) break;
           const int nl = n0 + w.n_kv - 1;
           if (!(ok = issue_pv(tmem + kTmO2, tmem + kTmS2, nl, w.n_kv > 1, bar(kPFull + 2), bar(kPFull + 3)))) break;
-          tc_commit(bar(kVEmpty + (nl & 1)));
-          tc_commit(bar(kOFull));
+          commit(kVEmpty + nl % kStages);
+          commit(kOFull);
           n0 += w.n_kv;
           ++n_items;
         }
-        // every MMA of this CTA must be complete before tensor memory is freed
-        tc_commit(bar(kDrain));
+        // every MMA of this CTA (with kPair: of both CTAs) must be complete before tensor
+        // memory is freed
+        if constexpr (kPair) tc_commit_pair_local(bar(kDrain));
+        else tc_commit(bar(kDrain));
         volatile int no_abort = 0;
         mbar_wait(bar(kDrain), 0, &no_abort);
       }
@@ -495,7 +639,7 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     int n_items = 0;  // items done
     bool ok = true;
 
-    for (int k = 0; ok && work_item<kVarlen, kWindow>(p, k, w, cur, seq_id, seq_nt, n_dense); ++k) {
+    for (int k = 0; ok && work_item<kVarlen, kWindow, kPair>(p, k, w, cur, seq_id, seq_nt, n_dense, cta_rank); ++k) {
       if (w.n_kv == 0) continue;
       const int qi = w.m0 + r;  // query index of this row within its sequence
       const int S = w.S;
@@ -503,7 +647,7 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       float l_run = 0.f;
       for (int it = 0; it < w.n_kv; ++it) {
         const int j = w.j_first + it;  // KV tile index (key position); n0 + it drives the barriers
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(kSFull + br), (n0 + it) & 1, abort_flag));
+        ok = __all_sync(0xffffffffu, pwait<kPair>(bar(kSFull + br), (n0 + it) & 1, abort_flag, flag_addr));
         if (!ok) break;
         tc_fence_after();
         uint32_t sr[4][32];
@@ -526,9 +670,9 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
           if (p.causal && j == w.tile) hi = r;
           hi = min(hi, S - 1 - j * BN);
           const int lo = kWindow ? qi - p.window + 1 - j * BN : 0;
-          mask_row(sr, lo, hi);
+          mask_row<4>(sr, lo, hi);
         }
-        const float mx = row_max(sr) * p.scale_log2;
+        const float mx = row_max<4>(sr) * p.scale_log2;
 
         // raise the running max only when the tile's max exceeds it by more than 2^8
         const bool rescale = mx > m_run + 8.f;
@@ -561,8 +705,7 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
           lsum += tile_masked ? exp_pack_store<false>(sr, half, p.scale_log2, m_use, trow + s_col)
                               : exp_pack_store<true>(sr, half, p.scale_log2, m_use, trow + s_col);
           tmem_st_wait();
-          tc_fence_before();
-          mbar_arrive(bar(kPFull + 2 * br + half));
+          arrive_for_mma<kPair>(bar(kPFull + 2 * br + half), lane);
         }
         l_run += lsum;
       }
@@ -573,14 +716,14 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       // columns 64*br .. 64*br+63 of row r, so the two branches swap row sums through shared
       // memory (one buffer per item parity: a buffer is rewritten two items later, after
       // every thread has passed the kLx and kOEmpty barriers of the item in between)
-      ok = mbar_wait(bar(kOFull), n_items & 1, abort_flag);
+      ok = pwait<kPair>(bar(kOFull), n_items & 1, abort_flag, flag_addr);
       float* lx = l_xchg + (n_items & 1) * 2 * BM;
       lx[br * BM + r] = l_run;
       // training forward: A_b = 2^(s * scale_log2 - lse) recomputes the probabilities later
       if (p.lse != nullptr && qi < S)
         p.lse[(w.row_base + qi) * p.Hq + 2 * w.pair + br] = (m_run == -INFINITY ? 0.f : m_run) + __log2f(l_run);
       mbar_arrive(bar(kLx));
-      ok = mbar_wait(bar(kLx), n_items & 1, abort_flag) && ok;
+      ok = pwait<kPair>(bar(kLx), n_items & 1, abort_flag, flag_addr) && ok;
       ok = __all_sync(0xffffffffu, ok && !*abort_flag);
       if (!ok) break;
       tc_fence_after();
@@ -634,27 +777,32 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         }
       }
       // O1, O2 are read: the next item's first PV may overwrite them
-      tc_fence_before();
-      mbar_arrive(bar(kOEmpty));
+      arrive_for_mma<kPair>(bar(kOEmpty), lane);
       ++n_items;
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  if constexpr (kPair) {
+    // neither CTA leaves (or frees tensor memory) while the other may still address it: the
+    // even CTA has drained every MMA, each producer has taken the commits addressed to it
+    cluster_sync();
+  }
   if (threadIdx.x == 0 && *abort_flag) atomicCAS(p.err, 0, kErrPrefillWait);
   if (warp == 9) {
     __syncwarp();  // lane 0 ran the MMA loop alone; dealloc is warp-collective
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    if constexpr (kPair) tmem_dealloc_pair(tmem, 512);
+    else tmem_dealloc(tmem, 512);
   }
 }
 
 }  // namespace prefill
 
 cudaError_t launch_prefill(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                           const float* lambda, __nv_bfloat16* out, int* err, int B, int S, int Hq, int Hkv,
-                           int causal, int window, const int* cu_seqlens, cudaStream_t stream,
+                           const CUtensorMap* tmKh, const float* lambda, __nv_bfloat16* out, int* err, int B, int S,
+                           int Hq, int Hkv, int causal, int window, const int* cu_seqlens, cudaStream_t stream,
                            __nv_bfloat16* o_branch, float* lse) {
   using namespace prefill;
   Params p;
@@ -671,17 +819,62 @@ cudaError_t launch_prefill(const CUtensorMap& tmQ, const CUtensorMap& tmK, const
   p.window = window;
   p.cu_seqlens = cu_seqlens;  // with packed sequences S is the longest sequence's length
   p.n_row_tiles = (S + BM - 1) / BM;
-  p.n_items = B * (Hq / 2) * p.n_row_tiles;
   p.sorted_seqs = (cu_seqlens != nullptr && B <= kMaxSortedSeqs) ? 1 : 0;
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HD));
-  auto kernel = cu_seqlens ? diffattn_prefill_sm100<true, false>
-                           : (window > 0 ? diffattn_prefill_sm100<false, true> : diffattn_prefill_sm100<false, false>);
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  if (e != cudaSuccess) return e;
   int device = 0, n_sms = 0;
-  e = cudaGetDevice(&device);
+  cudaError_t e = cudaGetDevice(&device);
   if (e != cudaSuccess) return e;
   e = cudaDeviceGetAttribute(&n_sms, cudaDevAttrMultiProcessorCount, device);
+  if (e != cudaSuccess) return e;
+  const bool one_per_item = cu_seqlens != nullptr && !p.sorted_seqs;
+
+  // The CTA-pair form runs when DA2_PREFILL_CTA_PAIR=1 is set in the environment, every KV head
+  // has an even number of pairs (GQA group a multiple of 4), the persistent deal applies and
+  // the caller passed the half-tile K map. It gives bit-identical results; on B200 it measured
+  // about 2% below the one-CTA form (what paces both is each branch's chain of softmax, PV
+  // and next score GEMM, not the number of MMA instructions), so one CTA per item is the
+  // default.
+  const int group = Hq / Hkv;
+  const char* env = getenv("DA2_PREFILL_CTA_PAIR");
+  const bool pair_wanted = env != nullptr && env[0] == '1';
+  const bool use_pair = pair_wanted && tmKh != nullptr && (group % 4) == 0 && !one_per_item;
+  if (use_pair) {
+    p.n_items = B * (Hq / 4) * p.n_row_tiles;
+    if (p.n_items == 0) return cudaSuccess;
+    auto kernel = cu_seqlens ? diffattn_prefill_sm100<true, false, true>
+                             : (window > 0 ? diffattn_prefill_sm100<false, true, true>
+                                           : diffattn_prefill_sm100<false, false, true>);
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(n_sms & ~1), 1, 1);
+    // persistent: as many clusters as can be resident at once (an SM pair each)
+    int n_clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&n_clusters, kernel, &cfg);
+    if (e != cudaSuccess) return e;
+    if (n_clusters <= 0) return cudaErrorInvalidConfiguration;
+    n_clusters = n_clusters < p.n_items ? n_clusters : p.n_items;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * n_clusters), 1, 1);
+    e = cudaLaunchKernelEx(&cfg, kernel, tmQ, tmK, tmV, *tmKh, p);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
+
+  p.n_items = B * (Hq / 2) * p.n_row_tiles;
+  auto kernel = cu_seqlens ? diffattn_prefill_sm100<true, false, false>
+                           : (window > 0 ? diffattn_prefill_sm100<false, true, false>
+                                         : diffattn_prefill_sm100<false, false, false>);
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   if (p.n_items == 0) return cudaSuccess;
   // Persistent: one CTA per SM (the shared memory admits one), each walking its items. Packed
@@ -690,9 +883,8 @@ cudaError_t launch_prefill(const CUtensorMap& tmQ, const CUtensorMap& tmK, const
   // beyond that every item of the full grid gets its own CTA and the hardware's CTA scheduler
   // balances them (a static deal that includes the empty items measured 745 against 800
   // TFLOP/s for 8 sequences of 512-3584 tokens).
-  const bool one_per_item = cu_seqlens != nullptr && !p.sorted_seqs;
   const int n_ctas = (one_per_item || p.n_items < n_sms) ? p.n_items : n_sms;
-  kernel<<<n_ctas, kThreads, kSmemBytes, stream>>>(tmQ, tmK, tmV, p);
+  kernel<<<n_ctas, kThreads, kSmemBytes, stream>>>(tmQ, tmK, tmV, tmK, p);
   return cudaGetLastError();
 }
 
