@@ -81,14 +81,13 @@ extern "C" int diffattn_v2_decode_noalloc(const void* q, const void* kcache, con
   CUtensorMap tk, tv;
   if (da2::encode_bshd_bf16(&tk, kcache, D, Hkv, Smax, B, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
   if (da2::encode_bshd_bf16(&tv, vcache, D, Hkv, Smax, B, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
-  // Same layout as the caller-provided workspace of diffattn_v2_decode. Nothing in it has to
+  // The layout of diffattn_v2_decode's workspace, from the same helper. Nothing in it has to
   // start at zero: the split kernel writes every partial that the merge reads, and the
   // launch zeroes the split counters on the stream first.
-  float* ws_o = static_cast<float*>(scratch);
-  float* ws_ml = ws_o + static_cast<size_t>(B) * Hq * nsplit * D;
-  int* counters = reinterpret_cast<int*>(ws_ml + static_cast<size_t>(B) * Hq * nsplit * 2);
+  const da2::DecodeWorkspace ws = da2::decode_workspace_layout(scratch, B, 1, Hq, D, nsplit);
   cudaError_t e = da2::launch_decode(tk, tv, static_cast<const __nv_bfloat16*>(q), seqlens, lambda,
-                                     static_cast<__nv_bfloat16*>(out), ws_o, ws_ml, counters, err, B, Smax, Hq, Hkv, nsplit,
+                                     static_cast<__nv_bfloat16*>(out), ws.o, ws.ml, ws.counters, err, B, Smax, Hq, Hkv,
+                                     nsplit,
                                      split_len, nullptr, 0, 0, 1, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? DA2_OK : DA2_ERR_CUDA;
 }

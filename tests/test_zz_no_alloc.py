@@ -1,12 +1,13 @@
-"""The no-allocation decode entry point against the regular decode entry point.
+"""The no-allocation decode entry point against the regular decode entry point and the oracle.
 
 diffattn_v2_decode_noalloc serves callers that cannot allocate device memory (a KV-cache
 pool or caching allocator that owns nearly all HBM, plugin interfaces without a workspace):
 its split partials live in the library's fixed 16 MiB device array. Here it is called
-through the C ABI twice in a row, on different inputs, and each output is compared with
-diffattn_v2_decode (caller-provided workspace) within the bf16 tolerance of the other
-tests. The second call reuses the array the first one left behind. This file is named so
-that pytest collects it last.
+through the C ABI on three inputs in a row (GQA groups of 4, 8 and 16; the group of 16 runs
+the kernel form with two 8-column MMA tiles), and each output is compared with
+diffattn_v2_decode (caller-provided workspace) and with the float64 oracle, within the bf16
+tolerance of the other tests. Each call reuses the array the previous one left behind. This
+file is named so that pytest collects it last.
 """
 import ctypes
 
@@ -14,6 +15,7 @@ import pytest
 import torch
 
 import workloads
+from oracle import diffattn_f64 as ora
 from tests.parity import bf16_close
 
 pytestmark = pytest.mark.gpu
@@ -30,10 +32,11 @@ def da():
 
 
 def _inputs(B, Smax, Hq, Hkv, lens, seed):
+    """CPU inputs of one decode step (the oracle reads these; the calls get device copies)."""
     inp = workloads.make_decode(workloads.DecodeCase(B=B, Smax=Smax, Hq=Hq, Hkv=Hkv, D=128, len_lo=1, len_hi=Smax,
                                                      seed=seed))
     inp["seqlens"] = torch.tensor(lens, dtype=torch.int32)
-    return {k: v.cuda() for k, v in inp.items() if k in ("q", "kcache", "vcache", "seqlens", "lam")}
+    return {k: v for k, v in inp.items() if k in ("q", "kcache", "vcache", "seqlens", "lam")}
 
 
 def _noalloc(da, d, out):
@@ -45,12 +48,15 @@ def _noalloc(da, d, out):
                                              Hq, Hkv, D, ctypes.c_void_p(stream))
 
 
-def test_noalloc_decode_matches_decode_on_two_calls(da):
+def test_noalloc_decode_matches_decode_and_oracle_on_three_calls(da):
     cases = [
-        _inputs(4, 3000, 16, 2, [3000, 2000, 1, 0], seed=41),           # several splits, an empty sequence
+        _inputs(4, 3000, 16, 2, [3000, 2000, 1, 0], seed=41),           # group 8, several splits, an empty sequence
         _inputs(8, 6000, 64, 8, [6000, 17, 4096, 1, 5999, 64, 65, 3000], seed=42),
+        _inputs(3, 5000, 64, 4, [5000, 333, 4097], seed=43),            # group 16: two 8-column MMA tiles
+        _inputs(5, 2500, 8, 2, [2500, 1, 1200, 0, 64], seed=44),         # group 4
     ]
-    for n, d in enumerate(cases):
+    for n, h in enumerate(cases):
+        d = {k: v.cuda() for k, v in h.items()}
         need = da.decode_workspace_size(d["q"].shape[0], d["kcache"].shape[1], d["q"].shape[1], d["kcache"].shape[2],
                                         128)
         assert 0 < need <= SCRATCH_BYTES
@@ -59,7 +65,9 @@ def test_noalloc_decode_matches_decode_on_two_calls(da):
         assert _noalloc(da, d, out) == 0
         torch.cuda.synchronize()
         assert da.device_error() == 0
-        bf16_close(out, ref.double().cpu().numpy(), f"no-alloc decode, call {n + 1}")
+        bf16_close(out, ref.double().cpu().numpy(), f"no-alloc decode vs decode, call {n + 1}")
+        oracle = ora.decode(h["q"], h["kcache"], h["vcache"], h["seqlens"], h["lam"])
+        bf16_close(out, oracle, f"no-alloc decode vs oracle, call {n + 1}")
 
 
 def test_noalloc_decode_refuses_sizes_beyond_the_array(da):
