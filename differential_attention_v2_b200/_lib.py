@@ -51,12 +51,15 @@ _SIGNATURES = {
 EXPORTED = tuple(_SIGNATURES)
 
 
-def _load():
-    if not os.path.exists(LIB_PATH):
+def load(path=LIB_PATH):
+    """Load a build of the library (the default, or e.g. its bounds-checking twin
+    libdiffattn_v2_debug.so) with the entry points' argument and result types set. The
+    wrappers below call the module's LIB."""
+    if not os.path.exists(path):
         raise ImportError(
-            f"{LIB_PATH} is missing; build it with `python -m differential_attention_v2_b200.build` "
+            f"{path} is missing; build it with `python -m differential_attention_v2_b200.build` "
             "(nvcc, sm_100a). There is no fallback implementation.")
-    lib = ctypes.CDLL(LIB_PATH)
+    lib = ctypes.CDLL(path)
     for name, (res, args) in _SIGNATURES.items():
         fn = getattr(lib, name)
         fn.restype = res
@@ -64,7 +67,7 @@ def _load():
     return lib
 
 
-LIB = _load()
+LIB = load()
 
 
 class DiffAttnError(RuntimeError):

@@ -26,6 +26,7 @@
 // bf16 operands back over them. A step's scores are produced in two 32-column halves so that
 // the elementwise work on one half overlaps the MMAs of the other.
 
+#include "bounds.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -428,9 +429,15 @@ dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         issued = t + 1;
       }
       if (*abort_flag) {
-        volatile int no_abort = 0;
-        mbar_wait(bar(kFixedFull), 0, &no_abort);
-        for (int t = max(0, issued - kStages); t < issued; ++t) mbar_wait(bar(kXFull + (t & 1)), (t >> 1) & 1, &no_abort);
+        // each wait has its own time limit (a wait that gives up must not end the ones after it)
+        {
+          volatile int na = 0;
+          mbar_wait(bar(kFixedFull), 0, &na);
+        }
+        for (int t = max(0, issued - kStages); t < issued; ++t) {
+          volatile int na = 0;
+          mbar_wait(bar(kXFull + (t & 1)), (t >> 1) & 1, &na);
+        }
       }
     }
   } else if (warp == kMmaWarp) {
@@ -585,9 +592,11 @@ dkdv_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     if (ok) ok = mbar_wait(bar(kDFull), 0, abort_flag);
     if (__all_sync(0xffffffffu, ok && !*abort_flag)) {
       tc_fence_after();
-      const bool valid = key < S;
       const int d0 = (128 / kGroups) * cg;
-      const size_t off = ((row_base + (valid ? key : 0)) * p.Hkv + g) * HD + d0;
+      const size_t off = ((row_base + (key < S ? key : 0)) * p.Hkv + g) * HD + d0;
+      // rows of the whole launch: B x S, or the packed sequences' total
+      const size_t total_rows = kVarlen ? static_cast<size_t>(__ldg(p.cu_seqlens + p.B)) : static_cast<size_t>(p.B) * p.S;
+      const bool valid = key < S && checked(off + 128 / kGroups <= total_rows * p.Hkv * HD, p.err);
       store_row(trow + kTmAcc0 + d0, p.dv + off, 1.f, valid);
       store_row(trow + kTmAcc1 + d0, p.dk + off, p.scale, valid);
     }
@@ -659,9 +668,15 @@ dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         issued = t + 1;
       }
       if (*abort_flag) {
-        volatile int no_abort = 0;
-        mbar_wait(bar(kFixedFull), 0, &no_abort);
-        for (int t = max(0, issued - kStages); t < issued; ++t) mbar_wait(bar(kXFull + (t & 1)), (t >> 1) & 1, &no_abort);
+        // each wait has its own time limit (a wait that gives up must not end the ones after it)
+        {
+          volatile int na = 0;
+          mbar_wait(bar(kFixedFull), 0, &na);
+        }
+        for (int t = max(0, issued - kStages); t < issued; ++t) {
+          volatile int na = 0;
+          mbar_wait(bar(kXFull + (t & 1)), (t >> 1) & 1, &na);
+        }
       }
     }
   } else if (warp == kMmaWarp) {
@@ -798,9 +813,10 @@ dq_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     if (ok) ok = mbar_wait(bar(kDFull), 0, abort_flag);
     if (__all_sync(0xffffffffu, ok && !*abort_flag)) {
       tc_fence_after();
-      const bool valid = qi < S;
       const int d0 = (128 / kGroups) * cg;
-      const size_t off = ((row_base + (valid ? qi : 0)) * p.Hq + 2 * pair) * HD + d0;
+      const size_t off = ((row_base + (qi < S ? qi : 0)) * p.Hq + 2 * pair) * HD + d0;
+      const size_t total_rows = kVarlen ? static_cast<size_t>(__ldg(p.cu_seqlens + p.B)) : static_cast<size_t>(p.B) * p.S;
+      const bool valid = qi < S && checked(off + HD + 128 / kGroups <= total_rows * p.Hq * HD, p.err);
       store_row(trow + kTmAcc0 + d0, p.dq + off, p.scale, valid);
       store_row(trow + kTmAcc1 + d0, p.dq + off + HD, p.scale, valid);
     }

@@ -33,11 +33,19 @@
 // splits that exist, so no host sync is needed. The counters are zeroed on the stream
 // before each launch.
 
+#include "bounds.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
 namespace da2 {
 namespace decode {
+
+#ifdef DA2_DEBUG_BOUNDS
+// Test hook of the debug build: when nonzero, CTA (0, 0, 0) announces but never issues the
+// copies of its ring stage number g_withhold_stage - 1, so that its consumers' bounded waits
+// expire and the kernel leaves through its abort path (set by diffattn_v2_test_withhold_decode_stage).
+__device__ int g_withhold_stage = 0;
+#endif
 
 constexpr int HD = 128;
 constexpr int kTok = 64;                              // tokens per stage
@@ -76,6 +84,10 @@ struct Params {
 // weigh 0. The partials were written by other CTAs of this grid: they are read through L2.
 __device__ __forceinline__ void combine_pair(const Params& p, int bt, int pair, int ns, int lane) {
   const int n_pairs = p.Hq >> 1;
+  const size_t n_rows = static_cast<size_t>(p.B) * p.T * p.Hq * p.nsplit;  // partial rows of the workspace
+  if (!checked(bt < p.B * p.T && pair < n_pairs && ns <= p.nsplit &&
+                   (static_cast<size_t>(bt) * p.Hq + 2 * pair + 1) * p.nsplit + ns <= n_rows, p.err))
+    return;
   float res[2][4];
 #pragma unroll
   for (int br = 0; br < 2; ++br) {
@@ -137,8 +149,9 @@ diffattn_decode_split(const __grid_constant__ CUtensorMap tmK, const __grid_cons
       for (int i = threadIdx.x; i < p.T * pairs_g * (HD / 8); i += blockDim.x) {
         const int c = i % (HD / 8), r = i / (HD / 8);
         const int pair = g * pairs_g + r % pairs_g;
-        reinterpret_cast<uint4*>(p.out + (static_cast<size_t>(b) * p.T + r / pairs_g) * n_pairs * HD +
-                                 static_cast<size_t>(pair) * HD)[c] = make_uint4(0u, 0u, 0u, 0u);
+        if (checked(pair < n_pairs && r / pairs_g < p.T, p.err))
+          reinterpret_cast<uint4*>(p.out + (static_cast<size_t>(b) * p.T + r / pairs_g) * n_pairs * HD +
+                                   static_cast<size_t>(pair) * HD)[c] = make_uint4(0u, 0u, 0u, 0u);
       }
     }
     return;
@@ -168,7 +181,8 @@ diffattn_decode_split(const __grid_constant__ CUtensorMap tmK, const __grid_cons
       // the split's page indices, read once: logical pages first_page .. (t1-1) / page_size
       const int n_pages = ((t1 - 1) >> p.page_shift) - first_page + 1;
       for (int i = lane; i < n_pages; i += 32)
-        pages[i] = __ldg(p.block_table + static_cast<size_t>(b) * p.max_pages + first_page + i);
+        if (checked(i < kMaxSplitPages && first_page + i < p.max_pages, p.err))
+          pages[i] = __ldg(p.block_table + static_cast<size_t>(b) * p.max_pages + first_page + i);
       __syncwarp();
     }
     if (lane == 0) {
@@ -180,6 +194,11 @@ diffattn_decode_split(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         const uint32_t dst = sbase + s * kStageBytes;
         const int tok = t0 + i * kTok;
         mbar_arrive_expect_tx(full(s), kStageBytes);
+        // skipped on a violation: the stage's barrier stays short and the consumers give up
+        if (!checked(within(dst, kStageBytes, sbase, kOffBar) && g < p.Hkv, p.err)) continue;
+#ifdef DA2_DEBUG_BOUNDS
+        if (g_withhold_stage == i + 1 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) continue;
+#endif
         if (!p.block_table) {
           tma_load_4d(dst + 0 * kHalfBytes, &tmK, full(s), 0, g, tok, b);
           tma_load_4d(dst + 1 * kHalfBytes, &tmK, full(s), 64, g, tok, b);
@@ -191,7 +210,8 @@ diffattn_decode_split(const __grid_constant__ CUtensorMap tmK, const __grid_cons
           // Tokens past the sequence read page -1: out of range, filled with zeros.
           for (int sb = 0; sb < kTok; sb += p.box_tok) {
             const int tk = tok + sb;
-            const int page = tk < t1 ? pages[(tk >> p.page_shift) - first_page] : -1;
+            const int pi = (tk >> p.page_shift) - first_page;
+            const int page = (tk < t1 && checked(pi >= 0 && pi < kMaxSplitPages, p.err)) ? pages[pi] : -1;
             const int row = tk & (page_size - 1);
             const uint32_t o = static_cast<uint32_t>(sb) * 128u;
             tma_load_4d(dst + 0 * kHalfBytes + o, &tmK, full(s), 0, g, row, page);
@@ -203,9 +223,12 @@ diffattn_decode_split(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         issued = i + 1;
       }
       if (*abort_flag) {
-        volatile int no_abort = 0;
-        for (int i = max(0, issued - kStages); i < issued; ++i)
+        // let every issued copy land before the CTA's shared memory is released; each wait has
+        // its own time limit (a wait that gives up must not end the ones after it)
+        for (int i = max(0, issued - kStages); i < issued; ++i) {
+          volatile int no_abort = 0;
           mbar_wait(full(i % kStages), (i / kStages) & 1, &no_abort);
+        }
       }
     }
     // the producer warp takes part in the final merge barrier only through __syncthreads
@@ -225,6 +248,7 @@ diffattn_decode_split(const __grid_constant__ CUtensorMap tmK, const __grid_cons
       const int n = nt * 8 + gl;
       const bool hv = n < p.T * group;
       const int tok = hv ? n / group : 0, h = hv ? n % group : 0;
+      checked(hq0 + h < p.Hq && tok < p.T, p.err);  // q row inside [B, T, Hq]
       const uint32_t* qrow =
           reinterpret_cast<const uint32_t*>(p.q + ((static_cast<size_t>(b) * p.T + tok) * p.Hq + hq0 + h) * HD);
 #pragma unroll
@@ -383,6 +407,7 @@ diffattn_decode_split(const __grid_constant__ CUtensorMap tmK, const __grid_cons
       }
       const size_t row =
           ((static_cast<size_t>(b) * p.T + h / group) * p.Hq + g * group + h % group) * p.nsplit + split;
+      if (!checked(row < static_cast<size_t>(p.B) * p.T * p.Hq * p.nsplit, p.err)) continue;
       p.ws_o[row * HD + d] = O;
       if (d == 0) {
         p.ws_ml[row * 2 + 0] = M;
@@ -398,7 +423,8 @@ diffattn_decode_split(const __grid_constant__ CUtensorMap tmK, const __grid_cons
   volatile int* last_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   const int ns = (seqlen + p.split_len - 1) / p.split_len;  // working splits of sequence b
   if (threadIdx.x == 0)
-    *last_flag = (atomicAdd(p.counters + static_cast<size_t>(b) * p.Hkv + g, 1) == ns - 1) ? 1 : 0;
+    *last_flag = (checked(b < p.B && g < p.Hkv && ns <= p.nsplit, p.err) &&
+                  atomicAdd(p.counters + static_cast<size_t>(b) * p.Hkv + g, 1) == ns - 1) ? 1 : 0;
   __syncthreads();
   if (!*last_flag) return;
   __threadfence();  // the other splits' partials, counted before ours, are visible
@@ -408,6 +434,12 @@ diffattn_decode_split(const __grid_constant__ CUtensorMap tmK, const __grid_cons
 }
 
 }  // namespace decode
+
+#ifdef DA2_DEBUG_BOUNDS
+extern "C" __attribute__((visibility("default"))) int diffattn_v2_test_withhold_decode_stage(int stage_plus_one) {
+  return cudaMemcpyToSymbol(decode::g_withhold_stage, &stage_plus_one, sizeof(int)) == cudaSuccess ? 0 : -3;
+}
+#endif
 
 cudaError_t launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const __nv_bfloat16* q,
                           const int32_t* seqlens, const float* lambda, __nv_bfloat16* out, float* ws_o,

@@ -38,6 +38,7 @@
 
 #include <cstdlib>
 
+#include "bounds.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -418,8 +419,10 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       const int nb = nt[b];
       int rank = 0;
       for (int b2 = 0; b2 < p.B; ++b2) rank += (nt[b2] > nb || (nt[b2] == nb && b2 < b)) ? 1 : 0;
-      seq_id[rank] = b;
-      seq_nt[rank] = nb;
+      if (checked(rank < kMaxSortedSeqs, p.err)) {
+        seq_id[rank] = b;
+        seq_nt[rank] = nb;
+      }
     }
     if (threadIdx.x == 0) {
       int total = 0;
@@ -469,6 +472,8 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
           for (int h = 0; h < 2; ++h)
             for (int c = 0; c < 2; ++c) {
               const uint32_t dst = sbase + kOffQ + h * kTileBytes + c * kChunkBytes;
+              if (!checked(within(dst, kChunkBytes, sbase + kOffQ, 2 * kTileBytes) && 2 * w.pair + h < p.Hq, p.err))
+                continue;
               if constexpr (kPair)
                 tma_load_4d_pair(dst, &tmQ, bar_lead(kQFull), c * 64, 2 * w.pair + h, w.tok0 + w.m0, w.tb);
               else
@@ -485,6 +490,7 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             if (leader) mbar_arrive_expect_tx(bar(kKFull + s), pair_mult * R::kKStage);
             for (int c = 0; c < 2; ++c) {
               const uint32_t dst = sbase + kOffK + s * R::kKStage + c * R::kKChunk;
+              if (!checked(within(dst, R::kKChunk, sbase + kOffK, kStages * R::kKStage) && g < p.Hkv, p.err)) continue;
               if constexpr (kPair)  // keys 64*rank .. 64*rank+63 of the tile, all 128 d
                 tma_load_4d_pair(dst, &tmKh, bar_lead(kKFull + s), c * 64, g, w.tok0 + j * BN + 64 * cta_rank, w.tb);
               else
@@ -493,7 +499,10 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             k_issued = n + 1;
             if (!(ok = pwait<kPair>(bar(kVEmpty + s), ph ^ 1, abort_flag, flag_addr))) break;
             if (leader) mbar_arrive_expect_tx(bar(kVFull + s), pair_mult * R::kVStage);
-            if constexpr (kPair) {  // all 128 keys, d 64*rank .. 64*rank+63
+            if (!checked(within(sbase + kOffV + s * R::kVStage, R::kVStage, sbase + kOffV, kStages * R::kVStage) &&
+                             g < p.Hkv, p.err)) {
+              // skipped: the stage's barrier stays short and the MMA thread's wait gives up
+            } else if constexpr (kPair) {  // all 128 keys, d 64*rank .. 64*rank+63
               tma_load_4d_pair(sbase + kOffV + s * R::kVStage, &tmV, bar_lead(kVFull + s), 64 * cta_rank, g,
                                w.tok0 + j * BN, w.tb);
             } else {
@@ -504,7 +513,6 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             v_issued = n + 1;
           }
         }
-        volatile int no_abort = 0;
         if (*abort_flag) {
           if constexpr (kPair) {
             // the copies' completions count on the even CTA's barriers, which this CTA may not
@@ -513,12 +521,20 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             while (global_timer_ns() - t0 < 2000000ull) __nanosleep(1000);
           } else {
             // let copies still in flight land before the CTA's shared memory is released: at
-            // most one Q tile and one K and one V tile per stage can be outstanding
-            if (q_issued > 0) mbar_wait(bar(kQFull), (q_issued - 1) & 1, &no_abort);
-            for (int n = max(0, k_issued - kStages); n < k_issued; ++n)
-              mbar_wait(bar(kKFull + n % kStages), (n / kStages) & 1, &no_abort);
-            for (int n = max(0, v_issued - kStages); n < v_issued; ++n)
-              mbar_wait(bar(kVFull + n % kStages), (n / kStages) & 1, &no_abort);
+            // most one Q tile and one K and one V tile per stage can be outstanding. Each wait
+            // has its own time limit (a wait that gives up must not end the ones after it).
+            if (q_issued > 0) {
+              volatile int na = 0;
+              mbar_wait(bar(kQFull), (q_issued - 1) & 1, &na);
+            }
+            for (int n = max(0, k_issued - kStages); n < k_issued; ++n) {
+              volatile int na = 0;
+              mbar_wait(bar(kKFull + n % kStages), (n / kStages) & 1, &na);
+            }
+            for (int n = max(0, v_issued - kStages); n < v_issued; ++n) {
+              volatile int na = 0;
+              mbar_wait(bar(kVFull + n % kStages), (n / kStages) & 1, &na);
+            }
           }
         } else if (kPair) {
           // the even CTA's last commits (stage and Q releases) arrive on this CTA's barriers:
@@ -577,7 +593,8 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         };
         int n0 = 0;       // KV tiles of earlier items
         int n_items = 0;  // items done
-        bool ok = true;
+        // the four 128-column accumulators fill the 512 allocated columns from column 0
+        bool ok = checked((tmem & 0xFFFFu) == 0u && kTmO2 + HD <= 512u, p.err);
         for (int k = 0; ok && work_item<kVarlen, kWindow, kPair>(p, k, w, cur, seq_id, seq_nt, n_dense, cta_rank);
              ++k) {
           if (w.n_kv == 0) continue;
@@ -720,7 +737,10 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       float* lx = l_xchg + (n_items & 1) * 2 * BM;
       lx[br * BM + r] = l_run;
       // training forward: A_b = 2^(s * scale_log2 - lse) recomputes the probabilities later
-      if (p.lse != nullptr && qi < S)
+      // rows of the whole launch: B x S, or the packed sequences' total
+      const size_t total_rows = kVarlen ? static_cast<size_t>(__ldg(p.cu_seqlens + p.B)) : static_cast<size_t>(p.B) * p.S;
+      if (p.lse != nullptr && qi < S &&
+          checked((w.row_base + qi) * p.Hq + 2 * w.pair + br < total_rows * p.Hq, p.err))
         p.lse[(w.row_base + qi) * p.Hq + 2 * w.pair + br] = (m_run == -INFINITY ? 0.f : m_run) + __log2f(l_run);
       mbar_arrive(bar(kLx));
       ok = pwait<kPair>(bar(kLx), n_items & 1, abort_flag, flag_addr) && ok;
@@ -730,8 +750,8 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       {
         const float inv1 = 1.f / lx[r];
         const float inv2 = 1.f / lx[BM + r];
-        const bool row_valid = qi < S;
-        const size_t row_off = (w.row_base + (row_valid ? qi : 0)) * n_pairs + w.pair;
+        const size_t row_off = (w.row_base + (qi < S ? qi : 0)) * n_pairs + w.pair;
+        const bool row_valid = qi < S && checked(row_off < total_rows * n_pairs, p.err);
         const float lam = row_valid ? __ldg(p.lambda + row_off) : 0.f;
 #pragma unroll 1
         for (int cc = 0; cc < 2; ++cc) {

@@ -15,7 +15,8 @@ namespace da2 {
 // reports through the device error word and then returns without trapping.
 constexpr uint64_t kWaitLimitNs = 250ull * 1000ull * 1000ull;
 
-enum DeviceError : int { kErrNone = 0, kErrPrefillWait = 1, kErrDecodeWait = 2, kErrBackwardWait = 3 };
+// Codes of the device error word. kErrBounds is recorded only by the debug-bounds build.
+enum DeviceError : int { kErrNone = 0, kErrPrefillWait = 1, kErrDecodeWait = 2, kErrBackwardWait = 3, kErrBounds = 4 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -364,7 +364,9 @@ DA2_API int diffattn_v2_lambda_v2(const void* x, const void* w_lambda, const flo
  * Synchronise `stream`, then read and clear the device error word that kernels set when a
  * bounded wait expires. *code receives 0 when no kernel reported an error, else the code
  * of the first error recorded (a pipeline wait expired: 1 = in a prefill, 2 = in a decode,
- * 3 = in a backward kernel). The word belongs to the current device, not to `stream`: it
+ * 3 = in a backward kernel; 4 = an index outside its extent, reported only by the
+ * bounds-checking build libdiffattn_v2_debug.so, whose kernels check their shared-memory,
+ * tensor-memory and global indices and skip an access that would leave its extent). The word belongs to the current device, not to `stream`: it
  * holds the first error of a kernel on ANY stream of the device since it was last cleared,
  * and reading it clears it for every caller. Synchronising `stream` only orders the read
  * after this stream's kernels; kernels of other streams still running may set it later.

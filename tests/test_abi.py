@@ -39,6 +39,19 @@ def test_library_exports_every_declared_symbol(lib):
         assert name in da.EXPORTED, f"binding lacks {name}"
 
 
+def test_bounds_checking_build_exports_every_declared_symbol():
+    """The debug-bounds twin of the library (same sources, -DDA2_DEBUG_BOUNDS) loads and
+    exports the same entry points."""
+    from differential_attention_v2_b200 import _lib
+    from differential_attention_v2_b200.build import DEBUG_LIB_PATH, build
+
+    build(debug_bounds=True)
+    dbg = _lib.load(DEBUG_LIB_PATH)
+    for name in _declared():
+        assert hasattr(dbg, name), name
+    assert dbg.diffattn_v2_version() == 100
+
+
 def test_version_and_status_strings(lib):
     assert lib.diffattn_v2_version() == 100
     for code in (0, -1, -2, -3, -4, 7):
