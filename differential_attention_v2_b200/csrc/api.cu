@@ -109,6 +109,21 @@ void decode_split_plan(int B, int Smax, int Hkv, int* split_len, int* nsplit) {
 // Accessors for other translation units of the library.
 cudaError_t device_error_word(int** out) { return device_error_ptr(out); }
 
+cudaError_t encode_2d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t row_bytes,
+                           uint32_t box_cols, uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  cudaError_t e = get_encoder(&enc);
+  if (e != cudaSuccess) return e;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 cudaError_t encode_bshd_bf16(CUtensorMap* map, const void* base, uint64_t D, uint64_t H, uint64_t S, uint64_t B,
                              uint32_t box0, uint32_t box2) {
   return encode_bshd(map, base, D, H, S, B, box0, box2);
@@ -532,9 +547,15 @@ int diffattn_v2_lambda_v2(const void* x, const void* w_lambda, const float* bias
   if (!aligned16(x) || !aligned16(w_lambda) || !aligned16(lambda_out) || (bias && !aligned16(bias)))
     return DA2_ERR_INVALID;
   if (d_model % 64 != 0 || n_pairs % 8 != 0 || n_pairs > 64) return DA2_ERR_UNSUPPORTED;
-  return status_of(da2::launch_lambda_v2(static_cast<const __nv_bfloat16*>(x),
-                                         static_cast<const __nv_bfloat16*>(w_lambda), bias, T, d_model, n_pairs,
-                                         lambda_out, reinterpret_cast<cudaStream_t>(stream)));
+  int* err = nullptr;
+  if (device_error_ptr(&err) != cudaSuccess) return DA2_ERR_CUDA;
+  CUtensorMap tx, tw;
+  if (da2::encode_2d_bf16(&tx, x, d_model, T, static_cast<uint64_t>(d_model) * 2, 64, 128) != cudaSuccess)
+    return DA2_ERR_CUDA;
+  if (da2::encode_2d_bf16(&tw, w_lambda, n_pairs, d_model, static_cast<uint64_t>(n_pairs) * 2, 64, 64) != cudaSuccess)
+    return DA2_ERR_CUDA;
+  return status_of(da2::launch_lambda_v2(tx, tw, bias, T, d_model, n_pairs, lambda_out, err,
+                                         reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int diffattn_v2_device_error(int* code, da2_stream_t stream) {

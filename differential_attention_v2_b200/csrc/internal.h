@@ -79,9 +79,16 @@ cudaError_t device_error_word(int** out);
 cudaError_t encode_bshd_bf16(CUtensorMap* map, const void* base, uint64_t D, uint64_t H, uint64_t S, uint64_t B,
                              uint32_t box0, uint32_t box2);
 
-// V2 lambda projection sigmoid(x W + bias), x [T, d_model] bf16, W [d_model, n_pairs] bf16,
+// V2 lambda projection sigmoid(x W + bias) on tcgen05: tmX over x [T, d_model] bf16 with
+// boxes of 64 (d_model) x 128 (tokens), tmW over W [d_model, n_pairs] bf16 with boxes of 64
+// (pair columns; those past n_pairs read as zeros) x 64 (d_model), both 128-byte swizzled;
 // bias fp32 [n_pairs] or null; d_model % 64 == 0, n_pairs % 8 == 0 and <= 64.
-cudaError_t launch_lambda_v2(const __nv_bfloat16* x, const __nv_bfloat16* w, const float* bias, int T, int d_model,
-                             int n_pairs, float* out, cudaStream_t stream);
+cudaError_t launch_lambda_v2(const CUtensorMap& tmX, const CUtensorMap& tmW, const float* bias, int T, int d_model,
+                             int n_pairs, float* out, int* err, cudaStream_t stream);
+
+// 2-D bf16 tensor map over a row-major [rows, cols] array with row stride `row_bytes`, box
+// {box_cols, box_rows}, 128-byte swizzle, out-of-range elements read as zero.
+cudaError_t encode_2d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t row_bytes,
+                           uint32_t box_cols, uint32_t box_rows);
 
 }  // namespace da2

@@ -16,7 +16,14 @@ namespace da2 {
 constexpr uint64_t kWaitLimitNs = 250ull * 1000ull * 1000ull;
 
 // Codes of the device error word. kErrBounds is recorded only by the debug-bounds build.
-enum DeviceError : int { kErrNone = 0, kErrPrefillWait = 1, kErrDecodeWait = 2, kErrBackwardWait = 3, kErrBounds = 4 };
+enum DeviceError : int {
+  kErrNone = 0,
+  kErrPrefillWait = 1,
+  kErrDecodeWait = 2,
+  kErrBackwardWait = 3,
+  kErrBounds = 4,
+  kErrLambdaWait = 5
+};
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -86,6 +93,15 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
       "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
+// 2-D tiled tensor load global -> shared, completion counted on `bar` in bytes.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
       : "memory");
 }
 

@@ -354,7 +354,8 @@ DA2_API int diffattn_v2_decode_noalloc(const void* q, const void* kcache, const 
  *   x        bf16 [T, d_model]         w_lambda bf16 [d_model, n_pairs]
  *   bias     fp32 [n_pairs] or NULL    lambda_out fp32 [T, n_pairs] (the prefill/decode
  *                                      lambda layout when T = B*S or T = B)
- * bf16 products accumulated in fp32 on the tensor cores; sigmoid with the accurate expf.
+ * bf16 products accumulated in fp32 on the 5th-generation tensor cores (tcgen05, one CTA per
+ * 128 tokens); sigmoid with the accurate expf.
  * Supported: d_model % 64 == 0, n_pairs % 8 == 0 and n_pairs <= 64 (else DA2_ERR_UNSUPPORTED).
  */
 DA2_API int diffattn_v2_lambda_v2(const void* x, const void* w_lambda, const float* bias, int T, int d_model,
@@ -364,7 +365,7 @@ DA2_API int diffattn_v2_lambda_v2(const void* x, const void* w_lambda, const flo
  * Synchronise `stream`, then read and clear the device error word that kernels set when a
  * bounded wait expires. *code receives 0 when no kernel reported an error, else the code
  * of the first error recorded (a pipeline wait expired: 1 = in a prefill, 2 = in a decode,
- * 3 = in a backward kernel; 4 = an index outside its extent, reported only by the
+ * 3 = in a backward kernel, 5 = in the V2 lambda projection; 4 = an index outside its extent, reported only by the
  * bounds-checking build libdiffattn_v2_debug.so, whose kernels check their shared-memory,
  * tensor-memory and global indices and skip an access that would leave its extent). The word belongs to the current device, not to `stream`: it
  * holds the first error of a kernel on ANY stream of the device since it was last cleared,
