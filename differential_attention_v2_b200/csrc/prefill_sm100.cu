@@ -660,6 +660,15 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       if (w.n_kv == 0) continue;
       const int qi = w.m0 + r;  // query index of this row within its sequence
       const int S = w.S;
+      // this row's lambda, loaded at the start of the item so that its latency hides under
+      // the item's tiles instead of lying on the epilogue's path
+      const size_t lam_off = (w.row_base + (qi < S ? qi : 0)) * n_pairs + w.pair;
+      bool lam_ok = qi < S;
+      if constexpr (kDebugBounds) {
+        const size_t rows = kVarlen ? static_cast<size_t>(__ldg(p.cu_seqlens + p.B)) : static_cast<size_t>(p.B) * p.S;
+        lam_ok = lam_ok && checked(lam_off < rows * n_pairs, p.err);
+      }
+      const float lam_row = lam_ok ? __ldg(p.lambda + lam_off) : 0.f;
       float m_run = -INFINITY;
       float l_run = 0.f;
       for (int it = 0; it < w.n_kv; ++it) {
@@ -752,7 +761,7 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         const float inv2 = 1.f / lx[BM + r];
         const size_t row_off = (w.row_base + (qi < S ? qi : 0)) * n_pairs + w.pair;
         const bool row_valid = qi < S && checked(row_off < total_rows * n_pairs, p.err);
-        const float lam = row_valid ? __ldg(p.lambda + row_off) : 0.f;
+        const float lam = row_valid ? lam_row : 0.f;
 #pragma unroll 1
         for (int cc = 0; cc < 2; ++cc) {
           const uint32_t col = 64 * br + 32 * cc;
