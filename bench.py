@@ -684,16 +684,37 @@ def run_reference(args):
 
 # ------------------------------------------------------------ single-operation lines
 def _time_op(fn, steps, warmup, stream):
+    """Milliseconds per call of `fn` (which launches on the current stream): `warmup` eager
+    calls, then `steps` calls captured in one CUDA graph and replayed once, timed with CUDA
+    events around the replay (the graph removes the host launch gaps that back-to-back eager
+    launches of a short kernel would add). Falls back to eager launches if capture fails.
+    Returns (ms, how)."""
     for _ in range(max(warmup, 3)):
         fn()
     torch.cuda.synchronize()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(steps):
-        fn()
-    t1.record(stream)
+    how = f"one CUDA graph of {steps} launches"
+    try:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for _ in range(steps):
+                fn()
+        run = graph.replay
+        run()  # one untimed replay
+    except Exception:  # capture not possible here: time eager launches
+        how = f"{steps} eager launches"
+        torch.cuda.synchronize()
+
+        def run():
+            for _ in range(steps):
+                fn()
     torch.cuda.synchronize()
-    return t0.elapsed_time(t1) / steps
+    cur = torch.cuda.current_stream()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(cur)
+    run()
+    t1.record(cur)
+    torch.cuda.synchronize()
+    return t0.elapsed_time(t1) / steps, how
 
 
 def run_workload(args):
@@ -718,7 +739,7 @@ def run_workload(args):
             q, k, v, lam = (inp[x][0].to(dev) for x in ("q", "k", "v", "lam"))
             cu = torch.tensor([0] + list(torch.tensor(lens).cumsum(0).tolist()), dtype=torch.int32, device=dev)
             out = torch.empty(T, 32, D, dtype=torch.bfloat16, device=dev)
-            fn = lambda: da.prefill_varlen(q, k, v, lam, cu, max(lens), out=out, stream=stream)
+            fn = lambda: da.prefill_varlen(q, k, v, lam, cu, max(lens), out=out)
             flops = sum(4 * D * 64 * L * (L + 1) // 2 for L in lens)
             cfg = {"workload": f"packed causal prefill of 8 sequences, lengths U[512,3584] (total {T}), Hq=64 Hkv=8 D=128",
                    "lengths": lens}
@@ -729,14 +750,14 @@ def run_workload(args):
             out = torch.empty(case.B, case.S, case.Hq // 2, D, dtype=torch.bfloat16, device=dev)
             if name == "window":
                 W = 1024
-                fn = lambda: da.prefill_window(q, k, v, lam, W, out=out, stream=stream)
+                fn = lambda: da.prefill_window(q, k, v, lam, W, out=out)
                 flops = 4 * D * case.Hq * case.B * sum(min(i + 1, W) for i in range(case.S))
                 cfg = {"workload": f"sliding-window causal prefill, window {W}, B=4 S=4096 Hq=64 Hkv=8 D=128"}
             else:
-                fn = lambda: da.prefill(q, k, v, lam, out=out, stream=stream)
+                fn = lambda: da.prefill(q, k, v, lam, out=out)
                 flops = workloads.prefill_flops(case.B, case.S, case.Hq, D)
                 cfg = {"workload": "causal prefill B=1 S=32768 Hq=64 Hkv=8 D=128"}
-        ms = _time_op(fn, args.steps, args.warmup, stream)
+        ms, how = _time_op(fn, args.steps, args.warmup, stream)
         val = flops / (ms * 1e-3) / 1e12
         unit, peak, bound = "TFLOP/s", peaks["bf16_tflops"], "tensor"
         launches = 1
@@ -763,7 +784,7 @@ def run_workload(args):
             del kc, vc
             out = torch.empty(case.B, case.Hq // 2, D, dtype=torch.bfloat16, device=dev)
             ws = torch.empty(da.decode_workspace_size(case.B, case.Smax, case.Hq, case.Hkv, D), dtype=torch.uint8, device=dev)
-            fn = lambda: da.decode_paged(q, kp, vp, table, sl, lam, out=out, workspace=ws, stream=stream)
+            fn = lambda: da.decode_paged(q, kp, vp, table, sl, lam, out=out, workspace=ws)
             nbytes += case.B * max_pages * 4
             cfg = {"workload": "paged decode (page size 64, shuffled pages) of B=64, lengths U[1024,8192], Hq=64 Hkv=8"}
         elif name == "multi":
@@ -772,15 +793,17 @@ def run_workload(args):
             qm = torch.randn(case.B, Tn, case.Hq, D, generator=g).bfloat16().to(dev)
             lm = torch.sigmoid(torch.randn(case.B, Tn, case.Hq // 2, generator=g)).to(dev)
             out = torch.empty(case.B, Tn, case.Hq // 2, D, dtype=torch.bfloat16, device=dev)
-            fn = lambda: da.decode_multi(qm, kc, vc, sl, lm, out=out, stream=stream)
+            wsm = torch.empty(da.LIB.diffattn_v2_decode_multi_workspace_size(case.B, Tn, case.Smax, case.Hq, case.Hkv, D),
+                              dtype=torch.uint8, device=dev)
+            fn = lambda: da.decode_multi(qm, kc, vc, sl, lm, out=out, workspace=wsm)
             nbytes += (Tn - 1) * case.B * (case.Hq * D * 2 + case.Hq // 2 * (4 + D * 2))
             cfg = {"workload": "2-token (speculative) decode of B=64, lengths U[1024,8192], Hq=64 Hkv=8"}
         else:
             out = torch.empty(case.B, case.Hq // 2, D, dtype=torch.bfloat16, device=dev)
             ws = torch.empty(da.decode_workspace_size(case.B, case.Smax, case.Hq, case.Hkv, D), dtype=torch.uint8, device=dev)
-            fn = lambda: da.decode(q, kc, vc, sl, lam, out=out, workspace=ws, stream=stream)
+            fn = lambda: da.decode(q, kc, vc, sl, lam, out=out, workspace=ws)
             cfg = {"workload": "needle decode B=8, 131072 cached tokens each, V1 lambda, Hq=64 Hkv=8"}
-        ms = _time_op(fn, args.steps, args.warmup, stream)
+        ms, how = _time_op(fn, args.steps, args.warmup, stream)
         val = nbytes / (ms * 1e-3) / 1e9
         unit, peak, bound = "GB/s", peaks["hbm_gbs"], "hbm"
     elif name == "backward":
@@ -788,18 +811,18 @@ def run_workload(args):
         inp = workloads.make_prefill(case)
         q, k, v, lam = (inp[x].to(dev) for x in ("q", "k", "v", "lam"))
         dout = workloads.make_prefill_grad(case).to(dev)
-        out, ob, lse = da.prefill_train(q, k, v, lam, stream=stream)
+        out, ob, lse = da.prefill_train(q, k, v, lam)
         grads = [torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(lam)]
         ws = torch.empty(da.backward_workspace_size(case.B, case.S, case.Hq), dtype=torch.uint8, device=dev)
-        fwd_ms = _time_op(lambda: da.prefill_train(q, k, v, lam, out=out, o_branch=ob, lse=lse, stream=stream),
-                          args.steps, args.warmup, stream)
+        fwd_ms, _ = _time_op(lambda: da.prefill_train(q, k, v, lam, out=out, o_branch=ob, lse=lse),
+                             args.steps, args.warmup, stream)
         fn = lambda: da.backward(q, k, v, lam, ob, lse, dout, dq=grads[0], dk=grads[1], dv=grads[2], dlam=grads[3],
-                                 workspace=ws, stream=stream)
+                                 workspace=ws)
         # chain-rule products per pair and visible (query, key): S_1, S_2 recomputed, dP shared
         # by both branches, dV from the combined weights, dK and dQ of both heads: 8 products
         # of 2*D flops each, twice the forward's 4
         flops = 2 * workloads.prefill_flops(case.B, case.S, case.Hq, D)
-        ms = _time_op(fn, args.steps, args.warmup, stream)
+        ms, how = _time_op(fn, args.steps, args.warmup, stream)
         val = flops / (ms * 1e-3) / 1e12
         unit, peak, bound = "TFLOP/s", peaks["bf16_tflops"], "tensor"
         launches = 3
@@ -812,11 +835,11 @@ def run_workload(args):
         inp = workloads.make_prefill(case)
         q, k, v, lam = (inp[x].to(dev) for x in ("q", "k", "v", "lam"))
         dout = workloads.make_prefill_grad(case).to(dev)
-        out, ob, lse = da.prefill_train(q, k, v, lam, window=W, stream=stream)
+        out, ob, lse = da.prefill_train(q, k, v, lam, window=W)
         ws = torch.empty(da.backward_workspace_size(case.B, case.S, case.Hq), dtype=torch.uint8, device=dev)
-        fn = lambda: da.backward(q, k, v, lam, ob, lse, dout, workspace=ws, window=W, stream=stream)
+        fn = lambda: da.backward(q, k, v, lam, ob, lse, dout, workspace=ws, window=W)
         flops = 2 * 4 * D * case.Hq * case.B * sum(min(i + 1, W) for i in range(case.S))
-        ms = _time_op(fn, args.steps, args.warmup, stream)
+        ms, how = _time_op(fn, args.steps, args.warmup, stream)
         val = flops / (ms * 1e-3) / 1e12
         unit, peak, bound = "TFLOP/s", peaks["bf16_tflops"], "tensor"
         launches = 3
@@ -830,11 +853,11 @@ def run_workload(args):
         q, k, v, lam = (inp[x][0].to(dev) for x in ("q", "k", "v", "lam"))
         dout = workloads.make_prefill_grad(case)[0].to(dev)
         cu = torch.tensor([0] + list(torch.tensor(lens).cumsum(0).tolist()), dtype=torch.int32, device=dev)
-        out, ob, lse = da.prefill_varlen_train(q, k, v, lam, cu, max(lens), stream=stream)
+        out, ob, lse = da.prefill_varlen_train(q, k, v, lam, cu, max(lens))
         ws = torch.empty(da.backward_varlen_workspace_size(len(lens), T, 64), dtype=torch.uint8, device=dev)
-        fn = lambda: da.backward_varlen(q, k, v, lam, ob, lse, dout, cu, max(lens), workspace=ws, stream=stream)
+        fn = lambda: da.backward_varlen(q, k, v, lam, ob, lse, dout, cu, max(lens), workspace=ws)
         flops = 2 * sum(4 * D * 64 * L * (L + 1) // 2 for L in lens)
-        ms = _time_op(fn, args.steps, args.warmup, stream)
+        ms, how = _time_op(fn, args.steps, args.warmup, stream)
         val = flops / (ms * 1e-3) / 1e12
         unit, peak, bound = "TFLOP/s", peaks["bf16_tflops"], "tensor"
         launches = 4
@@ -847,9 +870,9 @@ def run_workload(args):
         w = (torch.randn(dm, npair, generator=g) / dm ** 0.5).bfloat16().to(dev)
         b = torch.randn(npair, generator=g).to(dev)
         out = torch.empty(T, npair, dtype=torch.float32, device=dev)
-        fn = lambda: da.lambda_v2(x, w, b, out=out, stream=stream)
+        fn = lambda: da.lambda_v2(x, w, b, out=out)
         nbytes = T * dm * 2 + dm * npair * 2 + npair * 4 + T * npair * 4
-        ms = _time_op(fn, args.steps, args.warmup, stream)
+        ms, how = _time_op(fn, args.steps, args.warmup, stream)
         val = nbytes / (ms * 1e-3) / 1e9
         unit, peak, bound = "GB/s", peaks["hbm_gbs"], "hbm"
         launches = 1
@@ -866,7 +889,7 @@ def run_workload(args):
                          "frac": round(val / peak, 4), "traffic": None,
                          "frac_of_spec": round(val / (SPEC_BF16_TFLOPS if bound == "tensor" else SPEC_HBM_GBS), 4),
                          "peak_source": f"{peak_src} {'bf16_tflops (burst)' if bound == 'tensor' else 'hbm_gbs'}"},
-            "gpu_launches": launches * args.steps, "workload": name}
+            "gpu_launches": launches * args.steps, "workload": name, "timing": how}
     print(json.dumps(line), flush=True)
 
 
