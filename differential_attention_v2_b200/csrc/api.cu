@@ -124,6 +124,19 @@ cudaError_t encode_2d_bf16(CUtensorMap* map, const void* base, uint64_t cols, ui
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+cudaError_t encode_out_bf16(CUtensorMap* map, void* base, uint64_t D, uint64_t H, uint64_t S, uint64_t B) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  cudaError_t e = get_encoder(&enc);
+  if (e != cudaSuccess) return e;
+  const cuuint64_t dims[4] = {D, H, S, B};
+  const cuuint64_t strides[3] = {D * 2, H * D * 2, S * H * D * 2};
+  const cuuint32_t box[4] = {32, 1, 32, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 cudaError_t encode_bshd_bf16(CUtensorMap* map, const void* base, uint64_t D, uint64_t H, uint64_t S, uint64_t B,
                              uint32_t box0, uint32_t box2) {
   return encode_bshd(map, base, D, H, S, B, box0, box2);
@@ -164,7 +177,9 @@ int diffattn_v2_prefill(const void* q, const void* k, const void* v, const float
   if (encode_bshd(&tk, k, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tv, v, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tkh, k, D, Hkv, S, B, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
-  e = da2::launch_prefill(tq, tk, tv, &tkh, lambda, static_cast<__nv_bfloat16*>(out), err, B, S, Hq, Hkv, causal, 0,
+  CUtensorMap to;
+  if (da2::encode_out_bf16(&to, out, D, Hq / 2, S, B) != cudaSuccess) return DA2_ERR_CUDA;
+  e = da2::launch_prefill(tq, tk, tv, &tkh, to, lambda, static_cast<__nv_bfloat16*>(out), err, B, S, Hq, Hkv, causal, 0,
                           nullptr, reinterpret_cast<cudaStream_t>(stream));
   return status_of(e);
 }
@@ -186,8 +201,10 @@ int diffattn_v2_prefill_window(const void* q, const void* k, const void* v, cons
   if (encode_bshd(&tk, k, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tv, v, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tkh, k, D, Hkv, S, B, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
+  CUtensorMap to;
+  if (da2::encode_out_bf16(&to, out, D, Hq / 2, S, B) != cudaSuccess) return DA2_ERR_CUDA;
   // a window of S or more keys is the plain causal mask
-  e = da2::launch_prefill(tq, tk, tv, &tkh, lambda, static_cast<__nv_bfloat16*>(out), err, B, S, Hq, Hkv, 1,
+  e = da2::launch_prefill(tq, tk, tv, &tkh, to, lambda, static_cast<__nv_bfloat16*>(out), err, B, S, Hq, Hkv, 1,
                           window >= S ? 0 : window, nullptr, reinterpret_cast<cudaStream_t>(stream));
   return status_of(e);
 }
@@ -212,7 +229,9 @@ int diffattn_v2_prefill_varlen(const void* q, const void* k, const void* v, cons
   if (encode_bshd(&tk, k, D, Hkv, total_tokens, 1, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tv, v, D, Hkv, total_tokens, 1, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tkh, k, D, Hkv, total_tokens, 1, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
-  e = da2::launch_prefill(tq, tk, tv, &tkh, lambda, static_cast<__nv_bfloat16*>(out), err, B, max_seqlen, Hq, Hkv, causal,
+  CUtensorMap to;
+  if (da2::encode_out_bf16(&to, out, D, Hq / 2, total_tokens, 1) != cudaSuccess) return DA2_ERR_CUDA;
+  e = da2::launch_prefill(tq, tk, tv, &tkh, to, lambda, static_cast<__nv_bfloat16*>(out), err, B, max_seqlen, Hq, Hkv, causal,
                           0, cu_seqlens, reinterpret_cast<cudaStream_t>(stream));
   return status_of(e);
 }
@@ -251,7 +270,9 @@ int diffattn_v2_prefill_train(const void* q, const void* k, const void* v, const
   if (encode_bshd(&tk, k, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tv, v, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tkh, k, D, Hkv, S, B, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
-  e = da2::launch_prefill(tq, tk, tv, &tkh, lambda, static_cast<__nv_bfloat16*>(out), err, B, S, Hq, Hkv, causal, 0,
+  CUtensorMap to;
+  if (da2::encode_out_bf16(&to, out, D, Hq / 2, S, B) != cudaSuccess) return DA2_ERR_CUDA;
+  e = da2::launch_prefill(tq, tk, tv, &tkh, to, lambda, static_cast<__nv_bfloat16*>(out), err, B, S, Hq, Hkv, causal, 0,
                           nullptr, reinterpret_cast<cudaStream_t>(stream), static_cast<__nv_bfloat16*>(o_branch),
                           lse);
   return status_of(e);
@@ -325,8 +346,10 @@ int diffattn_v2_prefill_window_train(const void* q, const void* k, const void* v
   if (encode_bshd(&tk, k, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tv, v, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tkh, k, D, Hkv, S, B, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
+  CUtensorMap to;
+  if (da2::encode_out_bf16(&to, out, D, Hq / 2, S, B) != cudaSuccess) return DA2_ERR_CUDA;
   // a window of S or more keys is the plain causal mask
-  e = da2::launch_prefill(tq, tk, tv, &tkh, lambda, static_cast<__nv_bfloat16*>(out), err, B, S, Hq, Hkv, 1,
+  e = da2::launch_prefill(tq, tk, tv, &tkh, to, lambda, static_cast<__nv_bfloat16*>(out), err, B, S, Hq, Hkv, 1,
                           window >= S ? 0 : window, nullptr, reinterpret_cast<cudaStream_t>(stream),
                           static_cast<__nv_bfloat16*>(o_branch), lse);
   return status_of(e);
@@ -360,7 +383,9 @@ int diffattn_v2_prefill_varlen_train(const void* q, const void* k, const void* v
   if (encode_bshd(&tk, k, D, Hkv, total_tokens, 1, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tv, v, D, Hkv, total_tokens, 1, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tkh, k, D, Hkv, total_tokens, 1, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
-  e = da2::launch_prefill(tq, tk, tv, &tkh, lambda, static_cast<__nv_bfloat16*>(out), err, B, max_seqlen, Hq, Hkv, causal,
+  CUtensorMap to;
+  if (da2::encode_out_bf16(&to, out, D, Hq / 2, total_tokens, 1) != cudaSuccess) return DA2_ERR_CUDA;
+  e = da2::launch_prefill(tq, tk, tv, &tkh, to, lambda, static_cast<__nv_bfloat16*>(out), err, B, max_seqlen, Hq, Hkv, causal,
                           0, cu_seqlens, reinterpret_cast<cudaStream_t>(stream), static_cast<__nv_bfloat16*>(o_branch),
                           lse);
   return status_of(e);

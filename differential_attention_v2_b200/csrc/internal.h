@@ -13,9 +13,10 @@ namespace da2 {
 // i-window+1 .. i. With cu_seqlens (device, B+1 entries) the tensors hold B packed sequences
 // as one [1,T] batch and S is the longest sequence. Tensor maps: Q over [B,S,Hq,D], K/V over [B,S,Hkv,D],
 // boxes of 64 (d) x 1 (head) x 128 (rows) x 1, 128-byte swizzle; tmKh (optional) over K with
-// boxes of 64 (d) x 1 x 64 (rows) x 1, for the CTA-pair form (GQA groups of a multiple of 4).
+// boxes of 64 (d) x 1 x 64 (rows) x 1, for the CTA-pair form (GQA groups of a multiple of 4);
+// tmO over out [B,S,Hq/2,D] (with cu_seqlens [1,T,Hq/2,D]) from encode_out_bf16.
 cudaError_t launch_prefill(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                           const CUtensorMap* tmKh, const float* lambda, __nv_bfloat16* out, int* err, int B, int S,
+                           const CUtensorMap* tmKh, const CUtensorMap& tmO, const float* lambda, __nv_bfloat16* out, int* err, int B, int S,
                            int Hq, int Hkv, int causal, int window, const int* cu_seqlens, cudaStream_t stream,
                            __nv_bfloat16* o_branch = nullptr, float* lse = nullptr);
 
@@ -78,6 +79,10 @@ cudaError_t device_error_word(int** out);
 // 4-D bf16 tensor map over a row-major [B,S,H,D] array, box {box0, 1, box2, 1}, 128-byte swizzle.
 cudaError_t encode_bshd_bf16(CUtensorMap* map, const void* base, uint64_t D, uint64_t H, uint64_t S, uint64_t B,
                              uint32_t box0, uint32_t box2);
+
+// 4-D bf16 tensor map for the prefill's output stores: [B,S,H,D] (H = Hq/2 pairs), box
+// {32, 1, 32, 1} (32 columns of 32 rows of one pair), 64-byte swizzle.
+cudaError_t encode_out_bf16(CUtensorMap* map, void* base, uint64_t D, uint64_t H, uint64_t S, uint64_t B);
 
 // V2 lambda projection sigmoid(x W + bias) on tcgen05: tmX over x [T, d_model] bf16 with
 // boxes of 64 (d_model) x 128 (tokens), tmW over W [d_model, n_pairs] bf16 with boxes of 64

@@ -85,8 +85,12 @@ constexpr uint32_t kOffL = kOffMisc + 64;                     // [item parity][b
 // packed sequences: sequence ids sorted by row-tile count (longest first), then the counts
 constexpr int kMaxSortedSeqs = 256;
 constexpr uint32_t kOffSeq = kOffL + 2 * 2 * BM * 4;
-constexpr uint32_t kSmemUsed = kOffSeq + 2 * kMaxSortedSeqs * 4;
+// out staging for the tensor stores: 32 rows x 32 columns of bf16 per softmax warp
+constexpr uint32_t kStageBytes = 32 * 32 * 2;
+constexpr uint32_t kOffStage = (kOffSeq + 2 * kMaxSortedSeqs * 4 + 1023) / 1024 * 1024;
+constexpr uint32_t kSmemUsed = kOffStage + 8 * kStageBytes;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;             // slack for 1024-B alignment
+static_assert(kSmemBytes <= 227 * 1024, "shared memory of one CTA");
 
 // mbarrier slots (8 bytes each)
 enum Bar : int {
@@ -100,7 +104,7 @@ enum Bar : int {
   kOFull = 23,
   kDrain = 24,
   kQEmpty = 25,  // the item's last score GEMM has read Q
-  kOEmpty = 26,  // every softmax thread has read O1, O2 of the item (epilogue done)
+  kOEmpty = 26,  // every softmax thread has read O1, O2 of the item into registers
   kLx = 27,      // both branches' row sums of the item are in shared memory
   kNumBars = 28
 };
@@ -307,6 +311,19 @@ __device__ __forceinline__ float exp_pack_store(const uint32_t (&sr)[4][32], int
   return (s0 + s1) + (s2 + s3);
 }
 
+// 32 bf16 values (16 packed pairs) of one row to global memory: two 256-bit stores where dst
+// is 32-byte aligned (the caller's buffers need only 16), else four 128-bit ones.
+__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (&v)[16]) {
+  if ((reinterpret_cast<uintptr_t>(dst) & 31u) == 0) {
+    st_global_v8(dst, v);
+    st_global_v8(dst + 16, v + 8);
+  } else {
+    uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  }
+}
+
 // Waits on barriers that the other CTA arrives on use the default (CTA-scope acquire) form,
 // as the arrivals do; what they order is tensor memory, through the tcgen05 fences.
 constexpr bool kClusterAcquire = false;
@@ -365,7 +382,7 @@ template <bool kVarlen, bool kWindow, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
 diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKh,
-                       const Params p) {
+                       const __grid_constant__ CUtensorMap tmO, const Params p) {
   using R = Ring<kPair>;
   constexpr int kStages = R::kStages;
   constexpr uint32_t kOffV = off_v<kPair>();
@@ -434,6 +451,7 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(kPair ? &tmKh : &tmK);
     tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmO);
   }
   if (warp == 9) {
     if constexpr (kPair) {
@@ -741,8 +759,10 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       // ---- epilogue of the item: out = O1/l1 - lambda O2/l2; thread r of branch br writes
       // columns 64*br .. 64*br+63 of row r, so the two branches swap row sums through shared
       // memory (one buffer per item parity: a buffer is rewritten two items later, after
-      // every thread has passed the kLx and kOEmpty barriers of the item in between)
-      ok = pwait<kPair>(bar(kOFull), n_items & 1, abort_flag, flag_addr);
+      // every thread has passed the kLx and kOEmpty barriers of the item in between). The
+      // row sums go out before the wait for O, and the first 32 of the thread's columns of O1
+      // and O2 are requested from tensor memory before the wait for the other branch's sums,
+      // so that the load's latency passes under that wait.
       float* lx = l_xchg + (n_items & 1) * 2 * BM;
       lx[br * BM + r] = l_run;
       // training forward: A_b = 2^(s * scale_log2 - lse) recomputes the probabilities later
@@ -752,38 +772,51 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
           checked((w.row_base + qi) * p.Hq + 2 * w.pair + br < total_rows * p.Hq, p.err))
         p.lse[(w.row_base + qi) * p.Hq + 2 * w.pair + br] = (m_run == -INFINITY ? 0.f : m_run) + __log2f(l_run);
       mbar_arrive(bar(kLx));
+      ok = __all_sync(0xffffffffu, pwait<kPair>(bar(kOFull), n_items & 1, abort_flag, flag_addr));
+      if (!ok) break;
+      const uint32_t col0 = 64 * br;
+      uint32_t o1[32], o2[32];
+      tc_fence_after();
+      tmem_ld_32x32b_x32(trow + kTmO1 + col0, o1);
+      tmem_ld_32x32b_x32(trow + kTmO2 + col0, o2);
       ok = pwait<kPair>(bar(kLx), n_items & 1, abort_flag, flag_addr) && ok;
+      tmem_ld_wait(o1);
+      reg_fence(o2);
       ok = __all_sync(0xffffffffu, ok && !*abort_flag);
       if (!ok) break;
-      tc_fence_after();
       {
         const float inv1 = 1.f / lx[r];
         const float inv2 = 1.f / lx[BM + r];
         const size_t row_off = (w.row_base + (qi < S ? qi : 0)) * n_pairs + w.pair;
         const bool row_valid = qi < S && checked(row_off < total_rows * n_pairs, p.err);
         const float lam = row_valid ? lam_row : 0.f;
-#pragma unroll 1
+        // out leaves through shared memory and one tensor store per warp and 32 columns
+        // (rows of a [B,S] launch past S are clipped by the store; a packed sequence's rows
+        // past its end belong to the next sequence, so a warp whose 32 rows reach past the
+        // end stores its valid rows itself)
+        const int slab = w.m0 + 32 * (warp & 3);
+        const bool via_tma = kVarlen ? slab + 32 <= S : slab < S;
+        const uint32_t stage = sbase + kOffStage + kStageBytes * static_cast<uint32_t>(warp);
+#pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
-          const uint32_t col = 64 * br + 32 * cc;
-          uint32_t o1[32], o2[32];
-          tmem_ld_32x32b_x32(trow + kTmO1 + col, o1);
-          tmem_ld_32x32b_x32(trow + kTmO2 + col, o2);
-          tmem_ld_wait(o1);
-          reg_fence(o2);
+          const uint32_t col = col0 + 32 * cc;
+          if (cc == 1) {
+            tmem_ld_wait(o1);
+            reg_fence(o2);
+            // O1, O2 are read: the next item's first PV may overwrite them
+            arrive_for_mma<kPair>(bar(kOEmpty), lane);
+          }
           if (p.o_branch != nullptr && row_valid) {
             // per-head normalised O_1, O_2 of the pair, same columns as this thread's out slice
 #pragma unroll
             for (int hb = 0; hb < 2; ++hb) {
               const uint32_t* o = hb ? o2 : o1;
               const float inv = hb ? inv2 : inv1;
-              uint4* dst =
-                  reinterpret_cast<uint4*>(p.o_branch + ((w.row_base + qi) * p.Hq + 2 * w.pair + hb) * HD + col);
+              uint32_t ob[16];
 #pragma unroll
-              for (int v = 0; v < 4; ++v)
-                dst[v] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv),
-                                    pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv),
-                                    pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv),
-                                    pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv));
+              for (int e = 0; e < 16; ++e)
+                ob[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+              store_row32(p.o_branch + ((w.row_base + qi) * p.Hq + 2 * w.pair + hb) * HD + col, ob);
             }
           }
           uint32_t packed[16];
@@ -797,18 +830,35 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                                        __fmul_rn(__uint_as_float(o1[e + 1]), inv1));
             packed[e >> 1] = pack_bf16x2(y0, y1);
           }
-          if (row_valid) {
-            uint4* dst = reinterpret_cast<uint4*>(p.out + row_off * HD + col);
+          if (cc == 0) {
+            tmem_ld_32x32b_x32(trow + kTmO1 + col0 + 32, o1);
+            tmem_ld_32x32b_x32(trow + kTmO2 + col0 + 32, o2);
+          }
+          if (via_tma) {
+            // the warp's buffer is free once its previous store has read it
+            if (lane == 0) bulk_wait_read();
+            __syncwarp();
+            // row `lane` of the 32 x 32 box, 64-byte swizzle: 16-byte chunk c of row l sits
+            // at chunk c ^ ((l >> 1) & 3) (8 consecutive rows then fill all 32 banks)
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+            for (int c = 0; c < 4; ++c)
+              st_shared_v4(stage + 64u * lane + ((static_cast<uint32_t>(c) ^ ((lane >> 1) & 3u)) << 4),
+                           packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+            fence_proxy_async_shared();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_4d(&tmO, stage, static_cast<int>(col), w.pair, w.tok0 + slab, w.tb);
+              bulk_commit();
+            }
+          } else if (row_valid) {
+            store_row32(p.out + row_off * HD + col, packed);
           }
         }
       }
-      // O1, O2 are read: the next item's first PV may overwrite them
-      arrive_for_mma<kPair>(bar(kOEmpty), lane);
       ++n_items;
     }
+    // every tensor store of this thread has completed before the CTA exits
+    if (lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -830,7 +880,7 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 }  // namespace prefill
 
 cudaError_t launch_prefill(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                           const CUtensorMap* tmKh, const float* lambda, __nv_bfloat16* out, int* err, int B, int S,
+                           const CUtensorMap* tmKh, const CUtensorMap& tmO, const float* lambda, __nv_bfloat16* out, int* err, int B, int S,
                            int Hq, int Hkv, int causal, int window, const int* cu_seqlens, cudaStream_t stream,
                            __nv_bfloat16* o_branch, float* lse) {
   using namespace prefill;
@@ -894,7 +944,7 @@ cudaError_t launch_prefill(const CUtensorMap& tmQ, const CUtensorMap& tmK, const
     if (n_clusters <= 0) return cudaErrorInvalidConfiguration;
     n_clusters = n_clusters < p.n_items ? n_clusters : p.n_items;
     cfg.gridDim = dim3(static_cast<unsigned>(2 * n_clusters), 1, 1);
-    e = cudaLaunchKernelEx(&cfg, kernel, tmQ, tmK, tmV, *tmKh, p);
+    e = cudaLaunchKernelEx(&cfg, kernel, tmQ, tmK, tmV, *tmKh, tmO, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
@@ -913,7 +963,7 @@ cudaError_t launch_prefill(const CUtensorMap& tmQ, const CUtensorMap& tmK, const
   // balances them (a static deal that includes the empty items measured 745 against 800
   // TFLOP/s for 8 sequences of 512-3584 tokens).
   const int n_ctas = (one_per_item || p.n_items < n_sms) ? p.n_items : n_sms;
-  kernel<<<n_ctas, kThreads, kSmemBytes, stream>>>(tmQ, tmK, tmV, tmK, p);
+  kernel<<<n_ctas, kThreads, kSmemBytes, stream>>>(tmQ, tmK, tmV, tmK, tmO, p);
   return cudaGetLastError();
 }
 
