@@ -13,16 +13,19 @@
 //
 //   * one CTA per 128-token tile: D[128 tokens x 64] = x_tile[128 x d_model] W[d_model x 64]
 //     on tcgen05.mma (M = 128, N = 64, K = 16), fp32 accumulators in 64 TMEM columns;
-//   * two producer warps stream 64-wide chunks of d_model by TMA, each through its own 6-stage
-//     ring: the x tile (128 rows x 64, K-major, 128-byte swizzle, the A operand) and the W
-//     chunk (64 rows of d_model x 64 pair columns, MN-major, the B operand; the tensor map
-//     covers n_pairs columns, so the columns past n_pairs read as zeros). Measured on B200
-//     (16k tokens x 4096): 6 + 6 stages 4.09 TB/s; deeper x rings with shallower W rings
-//     were slower (10 + 3: 3.82, 12 + 2: 3.19), and so was starting each CTA's walk over
-//     d_model at its own chunk (3.92). What bounds it is the shape of the x stream: 128-byte
-//     pieces of 128 rows 8 KB apart, which a probe of the access pattern alone (no compute)
-//     reads at 5.0 TB/s against 5.8 for contiguous 4 KB pieces;
-//   * an MMA warp issues the four K-steps of each chunk and releases the stage by a commit;
+//   * two producer warps stream 128-wide chunks of d_model by TMA, each through its own
+//     4-stage ring: the x tile (128 rows x 128 as two 64-wide boxes, K-major, 128-byte
+//     swizzle, the A operand) and the W chunk (128 rows of d_model x 64 pair columns as two
+//     64-row boxes, MN-major, the B operand; the tensor map covers n_pairs columns, so the
+//     columns past n_pairs read as zeros). What bounds it is the shape of the x stream: short
+//     pieces of 128 rows 8 KB apart (a probe of the access pattern alone, no compute, read
+//     128-byte pieces at 5.0 TB/s against 5.8 for contiguous 4 KB pieces). Measured on B200
+//     (16k tokens x 4096, 32 pairs, same box, alternating rounds): 256-byte pieces in 4 + 4
+//     stages 4.43 TB/s against 4.16 for 128-byte pieces in 6 + 6 stages; 512-byte pieces fit
+//     only 2 + 2 stages (4.18). Earlier, with 128-byte pieces: deeper x rings with shallower
+//     W rings were slower (10 + 3: 3.82, 12 + 2: 3.19), and so was starting each CTA's walk
+//     over d_model at its own chunk (3.92);
+//   * an MMA warp issues the eight K-steps of each chunk and releases the stage by a commit;
 //   * four epilogue warps (one per TMEM lane quarter) read their rows' accumulators, add the
 //     bias, apply the sigmoid with the accurate expf and write fp32 lambda [T, n_pairs] -- the
 //     layout of the prefill ([B*S, Hq/2]) and decode ([B, Hq/2]) lambda arguments.
@@ -37,13 +40,16 @@ namespace da2 {
 namespace lambda2 {
 
 constexpr int BM = 128;                            // tokens per tile (MMA M)
-constexpr int BK = 64;                             // d_model per stage
+constexpr int kBoxes = 2;                          // 64-wide TMA boxes per stage
+constexpr int BK = 64 * kBoxes;                    // d_model per stage
 constexpr int BN = 64;                             // W columns per stage (MMA N)
-constexpr int kXStages = 6;
-constexpr int kWStages = 6;
+constexpr int kXStages = 4;
+constexpr int kWStages = 4;
 constexpr int kThreads = 224;                      // x producer, MMA issuer, 4 epilogue warps, W producer
-constexpr uint32_t kXBytes = BM * BK * 2;          // 16 KB
-constexpr uint32_t kWBytes = BK * BN * 2;          // 8 KB
+constexpr uint32_t kXBox = BM * 64 * 2;            // 16 KB: 128 rows x 64 of d_model
+constexpr uint32_t kWBox = 64 * BN * 2;            // 8 KB: 64 rows of d_model x 64 columns
+constexpr uint32_t kXBytes = kBoxes * kXBox;
+constexpr uint32_t kWBytes = kBoxes * kWBox;
 constexpr uint32_t kOffW = kXStages * kXBytes;
 constexpr uint32_t kOffBar = kOffW + kWStages * kWBytes;
 constexpr int kNumBars = 2 * kXStages + 2 * kWStages + 1;
@@ -68,7 +74,9 @@ lambda_v2_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int tok0 = blockIdx.x * BM;
-  const int n_chunks = d_model / BK;
+  // d_model is a multiple of 64: a last chunk of 64 reads its second box past the end of x
+  // and W, which the copies fill with zeros (products that add nothing)
+  const int n_chunks = (d_model + BK - 1) / BK;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i) mbar_init(sbase + kOffBar + 8u * i, 1);
@@ -100,11 +108,13 @@ lambda_v2_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         const uint32_t fb = is_x ? xfull(s) : wfull(s);
         if (!mbar_wait(is_x ? xempty(s) : wempty(s), ((kc / stages) & 1) ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(fb, is_x ? kXBytes : kWBytes);
-        if (!checked(c * BK + BK <= d_model, err)) continue;
-        if (is_x)
-          tma_load_2d(sbase + s * kXBytes, &tmX, fb, c * BK, tok0);
-        else
-          tma_load_2d(sbase + kOffW + s * kWBytes, &tmW, fb, 0, c * BK);
+        if (!checked(c * BK < d_model, err)) continue;
+        for (int b = 0; b < kBoxes; ++b) {
+          if (is_x)
+            tma_load_2d(sbase + s * kXBytes + b * kXBox, &tmX, fb, c * BK + 64 * b, tok0);
+          else
+            tma_load_2d(sbase + kOffW + s * kWBytes + b * kWBox, &tmW, fb, 0, c * BK + 64 * b);
+        }
         issued = kc + 1;
       }
       if (*abort_flag) {
@@ -127,10 +137,11 @@ lambda_v2_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
-          // A: x rows, K-major, K-step kk at +32 bytes of the 128-byte swizzled row;
-          // B: W rows of d_model (16 per K-step, 2 KB apart), the 64 columns contiguous
-          const uint64_t adesc = sdesc_sw128(sbase + s * kXBytes + kk * 32, 16, 1024);
-          const uint64_t bdesc = sdesc_sw128(sbase + kOffW + sw * kWBytes + kk * 2048, kWBytes, 1024);
+          // A: x rows, K-major, K-step kk in box kk / 4 at +32 bytes per step of the 128-byte
+          // swizzled row; B: W rows of d_model (16 per K-step, 2 KB apart, the boxes back to
+          // back), the 64 columns contiguous
+          const uint64_t adesc = sdesc_sw128(sbase + s * kXBytes + (kk >> 2) * kXBox + (kk & 3) * 32, 16, 1024);
+          const uint64_t bdesc = sdesc_sw128(sbase + kOffW + sw * kWBytes + kk * 2048, kWBox, 1024);
           mma_bf16_ss(tmem, adesc, bdesc, idesc, (kc > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(xempty(s));

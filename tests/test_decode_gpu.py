@@ -150,7 +150,9 @@ def test_decode_paged_matches_contiguous_and_oracle(da, page_size, lens):
 @pytest.mark.parametrize("T,d_model,n_pairs,with_bias", [
     (1, 64, 8, False), (100, 256, 32, True), (4096, 4096, 32, True), (333, 512, 64, False), (70, 128, 40, True),
     # ragged last 32-token tiles, one 64-wide chunk of d_model, the bench's 16k x 4096 shape
-    (193, 256, 8, False), (20000, 2048, 24, True), (16384, 4096, 32, False)])
+    (193, 256, 8, False), (20000, 2048, 24, True), (16384, 4096, 32, False),
+    # d_model an odd multiple of 64: the kernel's last 128-wide chunk is half past the end
+    (257, 192, 16, True), (130, 320, 8, False)])
 def test_lambda_v2_projection_matches_oracle(da, T, d_model, n_pairs, with_bias):
     g = torch.Generator().manual_seed(T + n_pairs)
     x = torch.randn(T, d_model, generator=g).bfloat16()
