@@ -729,7 +729,7 @@ def run_workload(args):
     peaks, peak_src = _peaks()
     name = args.workload
     D = 128
-    if name in ("prefill_long", "window", "varlen"):
+    if name in ("prefill", "prefill_long", "window", "varlen"):
         if name == "varlen":
             g = torch.Generator().manual_seed(1010)
             lens = torch.randint(512, 3585, (8,), generator=g).tolist()
@@ -756,12 +756,12 @@ def run_workload(args):
             else:
                 fn = lambda: da.prefill(q, k, v, lam, out=out)
                 flops = workloads.prefill_flops(case.B, case.S, case.Hq, D)
-                cfg = {"workload": "causal prefill B=1 S=32768 Hq=64 Hkv=8 D=128"}
+                cfg = {"workload": f"causal prefill B={case.B} S={case.S} Hq=64 Hkv=8 D=128"}
         ms, how = _time_op(fn, args.steps, args.warmup, stream)
         val = flops / (ms * 1e-3) / 1e12
         unit, peak, bound = "TFLOP/s", peaks["bf16_tflops"], "tensor"
         launches = 1
-    elif name in ("decode_needle", "paged", "multi"):
+    elif name in ("decode", "decode_needle", "paged", "multi"):
         case = workloads.CONFIGS["needle_decode_b8_s131072"] if name == "decode_needle" else workloads.CONFIGS["decode_b64_s8192"]
         inp = workloads.make_decode(case)
         kc, vc, sl = (inp[x].to(dev) for x in ("kcache", "vcache", "seqlens"))
@@ -802,7 +802,8 @@ def run_workload(args):
             out = torch.empty(case.B, case.Hq // 2, D, dtype=torch.bfloat16, device=dev)
             ws = torch.empty(da.decode_workspace_size(case.B, case.Smax, case.Hq, case.Hkv, D), dtype=torch.uint8, device=dev)
             fn = lambda: da.decode(q, kc, vc, sl, lam, out=out, workspace=ws)
-            cfg = {"workload": "needle decode B=8, 131072 cached tokens each, V1 lambda, Hq=64 Hkv=8"}
+            cfg = {"workload": "needle decode B=8, 131072 cached tokens each, V1 lambda, Hq=64 Hkv=8" if name == "decode_needle"
+                   else "decode B=64, lengths U[1024,8192], V2 lambda given, Hq=64 Hkv=8"}
         ms, how = _time_op(fn, args.steps, args.warmup, stream)
         val = nbytes / (ms * 1e-3) / 1e9
         unit, peak, bound = "GB/s", peaks["hbm_gbs"], "hbm"
@@ -905,7 +906,8 @@ def main(argv=None):
                     help="skip the second prefill and decode workloads (B=4 x 4k prefill, B=64 decode)")
     ap.add_argument("--ref-seconds", type=float, default=120.0,
                     help="host-time budget of the whole reference run (warm-up and timed steps)")
-    ap.add_argument("--workload", choices=("prefill_long", "decode_needle", "window", "varlen", "paged", "multi",
+    ap.add_argument("--workload", choices=("prefill", "decode", "prefill_long", "decode_needle", "window", "varlen",
+                                           "paged", "multi",
                                            "lambda_v2", "backward", "backward_varlen", "backward_window"),
                     default=None,
                     help="time one other operation alone instead of the default step")
