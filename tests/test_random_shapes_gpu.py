@@ -1,11 +1,14 @@
-"""Seeded random shapes for every bf16 forward entry point against the float64 oracle.
+"""Seeded random shapes for every bf16 forward entry point, and the backward, against the
+float64 oracle.
 
 The fixed cases of the other files pin known edges; these draw sequence lengths, batch sizes,
 GQA groups (2, 4, 8, 16), causal or full attention, window widths, packed-sequence length
 mixes, decode lengths, page sizes and new-token counts from a fixed seed, so that shapes
 nobody picked by hand (ragged tails at every position of a tile, items per CTA of every
 count, partial last splits) run too. The prefill cases with a GQA group of a multiple of 4
-run in both kernel forms (one CTA per item, and CTA pairs) and must agree bit for bit.
+run in both kernel forms (one CTA per item, and CTA pairs) and must agree bit for bit. The
+backward cases draw causal, full or windowed attention and hold the gradients to the same
+bounds as the fixed backward cases.
 """
 import numpy as np
 import pytest
@@ -122,3 +125,35 @@ def test_random_decodes(da, i):
         outm = da.decode_multi(qm.cuda(), d["kcache"], d["vcache"], d["seqlens"], lm.cuda())
         assert da.device_error() == 0
         bf16_close(outm, ora.decode_multi(qm, inp["kcache"], inp["vcache"], lens, lm), f"random multi-token {i}: T={T}")
+
+
+def _backward_cases(n):
+    g = np.random.default_rng(20261204)
+    cases = []
+    for i in range(n):
+        Hq, Hkv = _GROUPS[int(g.integers(len(_GROUPS)))]
+        B = int(g.integers(1, 3))
+        S = int(g.integers(1, 450))
+        mode = ("causal", "full", "window")[int(g.integers(0, 3))]
+        window = int(g.integers(1, max(2, S // 2))) if mode == "window" else 0
+        cases.append((i, B, S, Hq, Hkv, mode, window))
+    return cases
+
+
+@pytest.mark.parametrize("i,B,S,Hq,Hkv,mode,window", _backward_cases(6))
+def test_random_backward(da, i, B, S, Hq, Hkv, mode, window):
+    from tests.parity import grad_close
+
+    case = workloads.PrefillCase(B=B, S=S, Hq=Hq, Hkv=Hkv, D=128, seed=1100 + i)
+    inp = workloads.make_prefill(case)
+    inp["dout"] = workloads.make_prefill_grad(case)
+    d = {k: v.cuda() for k, v in inp.items()}
+    causal = mode != "full"
+    out, ob, lse = da.prefill_train(d["q"], d["k"], d["v"], d["lam"], causal=causal, window=window or None)
+    grads = da.backward(d["q"], d["k"], d["v"], d["lam"], ob, lse, d["dout"], causal=causal, window=window or None)
+    torch.cuda.synchronize()
+    assert da.device_error() == 0
+    ref = ora.prefill_backward(inp["q"], inp["k"], inp["v"], inp["lam"], inp["dout"], causal=causal,
+                               window=window or None)
+    for got, r, name in zip(grads, ref, ("dq", "dk", "dv", "dlam")):
+        grad_close(got, r, f"random backward {i}: B={B} S={S} Hq={Hq} Hkv={Hkv} {mode} window={window} {name}")
