@@ -878,6 +878,36 @@ def run_workload(args):
         unit, peak, bound = "GB/s", peaks["hbm_gbs"], "hbm"
         launches = 1
         cfg = {"workload": "V2 lambda projection sigmoid(x W + b): T=16384 tokens, d_model=4096, 32 pairs"}
+    elif name == "prefill_fused_lambda":
+        # B=4 x 4096 causal prefill whose V2 lambda comes from x [B,S,4096] inside the kernel,
+        # timed against the two-launch path (projection on the tensor cores, then the prefill)
+        case = workloads.CONFIGS["prefill_b4_s4096"]
+        inp = workloads.make_prefill(case)
+        q, k, v = (inp[x].to(dev) for x in ("q", "k", "v"))
+        dm, npair = 4096, case.Hq // 2
+        g = torch.Generator().manual_seed(13)
+        xh = torch.randn(case.B * case.S, dm, generator=g).bfloat16().to(dev)
+        w = (torch.randn(dm, npair, generator=g) / dm ** 0.5).bfloat16().to(dev)
+        wt = w.t().contiguous()
+        b = torch.randn(npair, generator=g).to(dev)
+        out = torch.empty(case.B, case.S, npair, D, dtype=torch.bfloat16, device=dev)
+        lam = torch.empty(case.B * case.S, npair, dtype=torch.float32, device=dev)
+        x3 = xh.view(case.B, case.S, dm)
+        fn = lambda: da.prefill_fused_lambda(q, k, v, x3, wt, b, out=out)
+        flops = workloads.prefill_flops(case.B, case.S, case.Hq, D)
+        ms, how = _time_op(fn, args.steps, args.warmup, stream)
+
+        def two_launch():
+            da.lambda_v2(xh, w, b, out=lam)
+            da.prefill(q, k, v, lam.view(case.B, case.S, npair), out=out)
+
+        ms2, _ = _time_op(two_launch, args.steps, args.warmup, stream)
+        val = flops / (ms * 1e-3) / 1e12
+        unit, peak, bound = "TFLOP/s", peaks["bf16_tflops"], "tensor"
+        launches = 1
+        cfg = {"workload": "causal prefill B=4 S=4096 Hq=64 Hkv=8 D=128 with the V2 lambda computed in the kernel "
+                           "from x [4, 4096, 4096] bf16",
+               "two_launch_ms": round(ms2, 4), "two_launch_tflops": round(flops / (ms2 * 1e-3) / 1e12, 2)}
     else:
         raise SystemExit(f"unknown workload {name}")
     err = da.device_error(stream)
@@ -907,7 +937,7 @@ def main(argv=None):
     ap.add_argument("--ref-seconds", type=float, default=120.0,
                     help="host-time budget of the whole reference run (warm-up and timed steps)")
     ap.add_argument("--workload", choices=("prefill", "decode", "prefill_long", "decode_needle", "window", "varlen",
-                                           "paged", "multi",
+                                           "paged", "multi", "prefill_fused_lambda",
                                            "lambda_v2", "backward", "backward_varlen", "backward_window"),
                     default=None,
                     help="time one other operation alone instead of the default step")

@@ -45,6 +45,7 @@ _SIGNATURES = {
     "diffattn_v2_decode_multi": (_i, [_vp] * 6 + [_i] * 6 + [_vp, _sz, _vp]),
     "diffattn_v2_lambda_v1": (_i, [_vp, _vp, _vp, _vp, _f, _i, _i, _i, _vp, _vp]),
     "diffattn_v2_lambda_v2": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
+    "diffattn_v2_prefill_fused_lambda": (_i, [_vp] * 8 + [_i] * 7 + [_vp]),
     "diffattn_v2_device_error": (_i, [ctypes.POINTER(_i), _vp]),
     "diffattn_v2_decode_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
 }
@@ -414,6 +415,30 @@ def lambda_v2(x, w_lambda, bias=None, out=None, stream=None):
     st = LIB.diffattn_v2_lambda_v2(_ptr(x), _ptr(w_lambda), _ptr(bias), T, d, n_pairs, _ptr(out),
                                    _stream(stream, x.device))
     _check(st, "diffattn_v2_lambda_v2")
+    return out
+
+
+def prefill_fused_lambda(q, k, v, x, w_lambda_t, bias=None, out=None, lambda_out=None, causal=True, stream=None):
+    """bf16 prefill with the V2 lambda sigmoid(x . w_lambda_t[p] + bias[p]) computed inside the
+    kernel: q [B,S,Hq,D], k/v [B,S,Hkv,D], x bf16 [B,S,d_model], w_lambda_t bf16 [Hq/2, d_model]
+    (the projection transposed), bias fp32 [Hq/2] or None; lambda_out fp32 [B,S,Hq/2] receives
+    the lambda when given. Returns out bf16 [B,S,Hq/2,D]."""
+    for t, n, nd in ((q, "q", 4), (k, "k", 4), (v, "v", 4), (x, "x", 3), (w_lambda_t, "w_lambda_t", 2)):
+        _need(t, n, torch.bfloat16, nd)
+    if bias is not None:
+        _need(bias, "bias", torch.float32, 1)
+    if lambda_out is not None:
+        _need(lambda_out, "lambda_out", torch.float32, 3)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    d_model = x.shape[2]
+    if out is None:
+        out = torch.empty((B, S, Hq // 2, D), dtype=torch.bfloat16, device=q.device)
+    _need(out, "out", torch.bfloat16, 4)
+    st = LIB.diffattn_v2_prefill_fused_lambda(_ptr(q), _ptr(k), _ptr(v), _ptr(x), _ptr(w_lambda_t), _ptr(bias),
+                                              _ptr(out), _ptr(lambda_out), B, S, Hq, Hkv, D, d_model,
+                                              1 if causal else 0, _stream(stream, q.device))
+    _check(st, "diffattn_v2_prefill_fused_lambda")
     return out
 
 

@@ -236,6 +236,33 @@ int diffattn_v2_prefill_varlen(const void* q, const void* k, const void* v, cons
   return status_of(e);
 }
 
+int diffattn_v2_prefill_fused_lambda(const void* q, const void* k, const void* v, const void* x,
+                                     const void* w_lambda_t, const float* bias, void* out, float* lambda_out, int B,
+                                     int S, int Hq, int Hkv, int D, int d_model, int causal, da2_stream_t stream) {
+  if (B < 0 || S < 0 || D <= 0 || !heads_ok(Hq, Hkv) || d_model <= 0 || (d_model % 8) != 0) return DA2_ERR_INVALID;
+  if (causal != 0 && causal != 1) return DA2_ERR_INVALID;
+  if (B == 0 || S == 0) return DA2_OK;
+  if (!q || !k || !v || !x || !w_lambda_t || !out) return DA2_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(x) || !aligned16(w_lambda_t) || !aligned16(out) ||
+      (bias && !aligned16(bias)) || (lambda_out && !aligned16(lambda_out)))
+    return DA2_ERR_INVALID;
+  if (D != 128) return DA2_ERR_UNSUPPORTED;
+  if ((S + 127) / 128 > 65535) return DA2_ERR_UNSUPPORTED;
+  int* err = nullptr;
+  cudaError_t e = device_error_ptr(&err);
+  if (e != cudaSuccess) return DA2_ERR_CUDA;
+  CUtensorMap tq, tk, tv, to;
+  if (encode_bshd(&tq, q, D, Hq, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  if (encode_bshd(&tk, k, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  if (encode_bshd(&tv, v, D, Hkv, S, B, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  if (da2::encode_out_bf16(&to, out, D, Hq / 2, S, B) != cudaSuccess) return DA2_ERR_CUDA;
+  e = da2::launch_prefill_lambda_fused(tq, tk, tv, to, static_cast<const __nv_bfloat16*>(x),
+                                       static_cast<const __nv_bfloat16*>(w_lambda_t), bias, lambda_out, d_model,
+                                       static_cast<__nv_bfloat16*>(out), err, B, S, Hq, Hkv, causal,
+                                       reinterpret_cast<cudaStream_t>(stream));
+  return status_of(e);
+}
+
 int diffattn_v2_prefill_f32(const float* q, const float* k, const float* v, const float* lambda, float* out, int B,
                             int S, int Hq, int Hkv, int D, int causal, da2_stream_t stream) {
   if (B < 0 || S < 0 || D <= 0 || !heads_ok(Hq, Hkv)) return DA2_ERR_INVALID;

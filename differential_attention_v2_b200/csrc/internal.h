@@ -20,6 +20,15 @@ cudaError_t launch_prefill(const CUtensorMap& tmQ, const CUtensorMap& tmK, const
                            int Hq, int Hkv, int causal, int window, const int* cu_seqlens, cudaStream_t stream,
                            __nv_bfloat16* o_branch = nullptr, float* lse = nullptr);
 
+// The [B,S] bf16 prefill with the V2 lambda computed in the kernel:
+// lambda[t, p] = sigmoid(x[t] . w_t[p] + bias[p]) with x [B*S, d_model] and w_t [Hq/2, d_model]
+// bf16 (d_model a multiple of 8), bias fp32 [Hq/2] or null; lambda_out (fp32 [B*S, Hq/2]) gets
+// a copy when not null. Tensor maps as for launch_prefill.
+cudaError_t launch_prefill_lambda_fused(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                        const CUtensorMap& tmO, const __nv_bfloat16* x, const __nv_bfloat16* w_t,
+                                        const float* bias, float* lambda_out, int d_model, __nv_bfloat16* out,
+                                        int* err, int B, int S, int Hq, int Hkv, int causal, cudaStream_t stream);
+
 // tcgen05 backward of the bf16 prefill (D = 128): preprocess into the workspace (row terms;
 // backward_stats_bytes, or backward_varlen_workspace_bytes with packed sequences), then the
 // dK/dV and dQ tile kernels. Tensor maps over q [B,S,Hq,D], dout [B,S,Hq/2,D], k and v

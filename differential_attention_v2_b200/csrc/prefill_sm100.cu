@@ -23,7 +23,8 @@
 //   warps 4-7  softmax of branch 2 (head 2p+1)
 //   warp 8     TMA producer (Q per item, K/V tiles through a 2-stage ring across items)
 //   warp 9     tcgen05 MMA issuer; also allocates and frees tensor memory
-//   warps 10-11 idle: they complete warpgroup 2, which hands its registers to warps 0-7
+//   warps 10-11 idle: they complete warpgroup 2, which hands its registers to warps 0-7;
+//              in the fused-lambda form they compute each item's V2 lambda (see below)
 //
 // Issue order on the tensor core for KV tile j: S1_j, PV2_{j-1}, S2_j, PV1_j. Softmax of
 // branch 1 on S1_j overlaps PV2_{j-1} and S2_j; softmax of branch 2 on S2_j overlaps PV1_j
@@ -35,6 +36,14 @@
 // 256); then O and l are rescaled by 2^(m_old - m_new). O/l is the same for any such m, so
 // this is exact up to rounding while skipping most rescales. The epilogue forms
 // O1/l1 - lambda O2/l2 in fp32 and rounds once to bf16.
+//
+// Fused-lambda form (kLamFused, [B,S] inputs): lambda is not read from memory but computed
+// in the kernel from the tokens' hidden states x and the projection of "Differential
+// Transformer V2 soll KI-Training stabiler machen" ("Weniger Ausreisser und
+// Gradientenspitzen": lambda per token and head, bounded by a sigmoid):
+// lambda[t, p] = sigmoid(x[t] . w[p] + bias[p]). Warps 10 and 11 take 64 rows each of every
+// item's tile, dot products over d_model on the CUDA cores, and hand the 128 values to the
+// epilogue through a two-slot ring in shared memory.
 
 #include <cstdlib>
 
@@ -82,9 +91,12 @@ template <bool kPair>
 __host__ __device__ constexpr uint32_t off_v() { return kOffK + Ring<kPair>::kStages * Ring<kPair>::kKStage; }
 constexpr uint32_t kOffMisc = kOffBar + 256;                  // tmem slot, abort flag
 constexpr uint32_t kOffL = kOffMisc + 64;                     // [item parity][branch][row] fp32 row sums
-// packed sequences: sequence ids sorted by row-tile count (longest first), then the counts
+// packed sequences: sequence ids sorted by row-tile count (longest first), then the counts;
+// in the fused-lambda form (never with packed sequences) the same bytes hold the lambda ring
 constexpr int kMaxSortedSeqs = 256;
 constexpr uint32_t kOffSeq = kOffL + 2 * 2 * BM * 4;
+constexpr uint32_t kOffLamRing = kOffSeq;                      // [slot][row] fp32
+static_assert(2 * BM * 4 <= 2 * kMaxSortedSeqs * 4, "lambda ring");
 // out staging for the tensor stores: 32 rows x 32 columns of bf16 per softmax warp
 constexpr uint32_t kStageBytes = 32 * 32 * 2;
 constexpr uint32_t kOffStage = (kOffSeq + 2 * kMaxSortedSeqs * 4 + 1023) / 1024 * 1024;
@@ -106,7 +118,9 @@ enum Bar : int {
   kQEmpty = 25,  // the item's last score GEMM has read Q
   kOEmpty = 26,  // every softmax thread has read O1, O2 of the item into registers
   kLx = 27,      // both branches' row sums of the item are in shared memory
-  kNumBars = 28
+  kLamFull = 28,   // +slot: the fused lambda of the slot's item is in shared memory
+  kLamEmpty = 30,  // +slot: every softmax thread has read it
+  kNumBars = 32
 };
 static_assert(kNumBars * 8 <= 256, "barrier slots");
 
@@ -125,6 +139,12 @@ struct Params {
   int n_items;            // B * (Hq/2) * n_row_tiles
   int sorted_seqs;        // packed sequences dealt as a dense list of non-empty items (B <= kMaxSortedSeqs)
   float scale_log2;       // log2(e)/sqrt(D)
+  // fused lambda (kLamFused): lambda[t, p] = sigmoid(x[t] . wt[p] + bias[p])
+  const __nv_bfloat16* lam_x;   // [B*S, d_model] token hidden states
+  const __nv_bfloat16* lam_wt;  // [Hq/2, d_model] projection, one row per pair
+  const float* lam_bias;        // [Hq/2] or null
+  float* lam_out;               // [B*S, Hq/2] fp32 copy of the computed lambda, or null
+  int d_model;                  // a multiple of 8
 };
 
 // One work item: query rows m0 .. m0+127 of pair `pair` of sequence b, visiting KV tiles
@@ -311,6 +331,28 @@ __device__ __forceinline__ float exp_pack_store(const uint32_t (&sr)[4][32], int
   return (s0 + s1) + (s2 + s3);
 }
 
+// 16 bytes of a stream read once (not kept in L1).
+__device__ __forceinline__ uint4 ld_stream_v4(const void* ptr) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(ptr));
+  return v;
+}
+
+// acc (two fp32 partial sums) += the dot product of 8 bf16 values a and w (bf16 -> fp32 is
+// exact: the 16 bits move to the top of the word).
+__device__ __forceinline__ uint64_t dot8_bf16(uint4 a, uint4 w, uint64_t acc) {
+  const uint32_t av[4] = {a.x, a.y, a.z, a.w}, wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint64_t x2 = f2_pack(__uint_as_float(av[i] << 16), __uint_as_float(av[i] & 0xFFFF0000u));
+    const uint64_t w2 = f2_pack(__uint_as_float(wv[i] << 16), __uint_as_float(wv[i] & 0xFFFF0000u));
+    acc = f2_fma(x2, w2, acc);
+  }
+  return acc;
+}
+
 // 32 bf16 values (16 packed pairs) of one row to global memory: two 256-bit stores where dst
 // is 32-byte aligned (the caller's buffers need only 16), else four 128-bit ones.
 __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (&v)[16]) {
@@ -378,7 +420,7 @@ __device__ __forceinline__ void arrive_for_mma(uint32_t bar, int lane) {
 //   * each softmax warp of either CTA arrives once on the even CTA's P and O-read barriers;
 //   * a wait that gives up raises the abort flag of both CTAs; both CTAs leave through one
 //     cluster barrier, after every copy and commit addressed to them has landed.
-template <bool kVarlen, bool kWindow, bool kPair>
+template <bool kVarlen, bool kWindow, bool kPair, bool kLamFused = false>
 __global__ void __launch_bounds__(kThreads, 1)
 diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKh,
@@ -416,6 +458,8 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       if (i >= kPFull && i < kPFull + 4) count = kPair ? 8 : 128;
       if (i == kOEmpty) count = kPair ? 16 : 256;
       if (i == kLx) count = 256;
+      if (i == kLamFull || i == kLamFull + 1) count = 64;
+      if (i == kLamEmpty || i == kLamEmpty + 1) count = 256;
       mbar_init(bar(i), count);
     }
     *abort_flag = 0;
@@ -661,6 +705,61 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         volatile int no_abort = 0;
         mbar_wait(bar(kDrain), 0, &no_abort);
       }
+    } else if constexpr (kLamFused) {
+      // ------------------------------------------- fused V2 lambda (warps 10 and 11)
+      // Warp 10 takes rows 0-63 of each item's tile, warp 11 rows 64-127, two rows at a time;
+      // lane l sums elements 8l .. 8l+7 of every 256 of d_model, then the warp adds the lanes.
+      float* lam_ring = reinterpret_cast<float*>(smem + kOffLamRing);
+      const int row0 = (warp - 10) * 64;
+      const int n_pairs_l = p.Hq >> 1;
+      int n_li = 0;  // items with KV tiles so far (the ring's count, as the softmax warps')
+      bool ok = true;
+      for (int k = 0; ok && work_item<kVarlen, kWindow, kPair>(p, k, w, cur, seq_id, seq_nt, n_dense, cta_rank);
+           ++k) {
+        if (w.n_kv == 0) continue;
+        const int s = n_li & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(kLamEmpty + s), ((n_li >> 1) & 1) ^ 1, abort_flag));
+        if (!ok) break;
+        const __nv_bfloat16* wrow = p.lam_wt + static_cast<size_t>(w.pair) * p.d_model;
+        const float bias = p.lam_bias != nullptr ? __ldg(p.lam_bias + w.pair) : 0.f;
+#pragma unroll 1
+        for (int rr = 0; rr < 64; rr += 2) {
+          const int qa = w.m0 + row0 + rr;  // rows qa and qa + 1 of the sequence
+          const bool va = qa < w.S, vb = qa + 1 < w.S;
+          const __nv_bfloat16* xa = p.lam_x + (w.row_base + (va ? qa : 0)) * p.d_model;
+          const __nv_bfloat16* xb = p.lam_x + (w.row_base + (vb ? qa + 1 : 0)) * p.d_model;
+          uint64_t acc_a = f2_pack(0.f, 0.f), acc_b = f2_pack(0.f, 0.f);
+#pragma unroll 4
+          for (int d = 8 * lane; d < p.d_model; d += 256) {
+            const uint4 wv = __ldg(reinterpret_cast<const uint4*>(wrow + d));
+            const uint4 av = va ? ld_stream_v4(xa + d) : make_uint4(0u, 0u, 0u, 0u);
+            const uint4 bv = vb ? ld_stream_v4(xb + d) : make_uint4(0u, 0u, 0u, 0u);
+            acc_a = dot8_bf16(av, wv, acc_a);
+            acc_b = dot8_bf16(bv, wv, acc_b);
+          }
+          float a0, a1, b0, b1;
+          f2_unpack(acc_a, a0, a1);
+          f2_unpack(acc_b, b0, b1);
+          float sa = a0 + a1, sb = b0 + b1;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            sa += __shfl_xor_sync(0xffffffffu, sa, o);
+            sb += __shfl_xor_sync(0xffffffffu, sb, o);
+          }
+          if (lane == 0) {
+            const float la = va ? 1.f / (1.f + expf(-(sa + bias))) : 0.f;
+            const float lb = vb ? 1.f / (1.f + expf(-(sb + bias))) : 0.f;
+            lam_ring[s * BM + row0 + rr] = la;
+            lam_ring[s * BM + row0 + rr + 1] = lb;
+            if (p.lam_out != nullptr) {
+              if (va) p.lam_out[(w.row_base + qa) * n_pairs_l + w.pair] = la;
+              if (vb) p.lam_out[(w.row_base + qa + 1) * n_pairs_l + w.pair] = lb;
+            }
+          }
+        }
+        mbar_arrive(bar(kLamFull + s));
+        ++n_li;
+      }
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
@@ -686,7 +785,7 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         const size_t rows = kVarlen ? static_cast<size_t>(__ldg(p.cu_seqlens + p.B)) : static_cast<size_t>(p.B) * p.S;
         lam_ok = lam_ok && checked(lam_off < rows * n_pairs, p.err);
       }
-      const float lam_row = lam_ok ? __ldg(p.lambda + lam_off) : 0.f;
+      float lam_row = (!kLamFused && lam_ok) ? __ldg(p.lambda + lam_off) : 0.f;
       float m_run = -INFINITY;
       float l_run = 0.f;
       for (int it = 0; it < w.n_kv; ++it) {
@@ -755,6 +854,14 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       }
       if (!ok) break;
       n0 += w.n_kv;
+      if constexpr (kLamFused) {
+        // this row's lambda from warps 10 and 11
+        const int ls = n_items & 1;
+        ok = __all_sync(0xffffffffu, pwait<kPair>(bar(kLamFull + ls), (n_items >> 1) & 1, abort_flag, flag_addr));
+        if (!ok) break;
+        lam_row = reinterpret_cast<const float*>(smem + kOffLamRing)[ls * BM + r];
+        mbar_arrive(bar(kLamEmpty + ls));
+      }
 
       // ---- epilogue of the item: out = O1/l1 - lambda O2/l2; thread r of branch br writes
       // columns 64*br .. 64*br+63 of row r, so the two branches swap row sums through shared
@@ -963,6 +1070,45 @@ cudaError_t launch_prefill(const CUtensorMap& tmQ, const CUtensorMap& tmK, const
   // balances them (a static deal that includes the empty items measured 745 against 800
   // TFLOP/s for 8 sequences of 512-3584 tokens).
   const int n_ctas = (one_per_item || p.n_items < n_sms) ? p.n_items : n_sms;
+  kernel<<<n_ctas, kThreads, kSmemBytes, stream>>>(tmQ, tmK, tmV, tmK, tmO, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_lambda_fused(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                        const CUtensorMap& tmO, const __nv_bfloat16* x, const __nv_bfloat16* w_t,
+                                        const float* bias, float* lambda_out, int d_model, __nv_bfloat16* out,
+                                        int* err, int B, int S, int Hq, int Hkv, int causal, cudaStream_t stream) {
+  using namespace prefill;
+  Params p{};
+  p.lambda = nullptr;
+  p.out = out;
+  p.err = err;
+  p.B = B;
+  p.S = S;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.causal = causal;
+  p.window = 0;
+  p.cu_seqlens = nullptr;
+  p.n_row_tiles = (S + BM - 1) / BM;
+  p.sorted_seqs = 0;
+  p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HD));
+  p.lam_x = x;
+  p.lam_wt = w_t;
+  p.lam_bias = bias;
+  p.lam_out = lambda_out;
+  p.d_model = d_model;
+  p.n_items = B * (Hq / 2) * p.n_row_tiles;
+  int device = 0, n_sms = 0;
+  cudaError_t e = cudaGetDevice(&device);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&n_sms, cudaDevAttrMultiProcessorCount, device);
+  if (e != cudaSuccess) return e;
+  auto kernel = diffattn_prefill_sm100<false, false, false, true>;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  if (p.n_items == 0) return cudaSuccess;
+  const int n_ctas = p.n_items < n_sms ? p.n_items : n_sms;
   kernel<<<n_ctas, kThreads, kSmemBytes, stream>>>(tmQ, tmK, tmV, tmK, tmO, p);
   return cudaGetLastError();
 }

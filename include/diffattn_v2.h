@@ -362,6 +362,31 @@ DA2_API int diffattn_v2_lambda_v2(const void* x, const void* w_lambda, const flo
                                   int n_pairs, float* lambda_out, da2_stream_t stream);
 
 /*
+ * bf16 prefill with the V2 lambda fused into the kernel: the same output as
+ * diffattn_v2_prefill with lambda[b,s,p] = sigmoid(x[b,s] . w_lambda_t[p] + bias[p]) (the
+ * projection of diffattn_v2_lambda_v2), computed per work item by two otherwise idle warps of
+ * the prefill kernel instead of by a separate launch. Sources: "Differential Transformer V2
+ * soll KI-Training stabiler machen", section "Weniger Ausreisser und Gradientenspitzen" (the
+ * lambda), and the prefill's sources above.
+ *   q, k, v, out      as diffattn_v2_prefill ([B,S] layouts, D == 128)
+ *   x                 bf16 [B, S, d_model] token hidden states
+ *   w_lambda_t        bf16 [Hq/2, d_model]: the projection TRANSPOSED, one row per pair
+ *                     (w_lambda_t[p][j] = w_lambda[j][p] of diffattn_v2_lambda_v2)
+ *   bias              fp32 [Hq/2] or NULL
+ *   lambda_out        fp32 [B, S, Hq/2] or NULL: a copy of the computed lambda (the layout a
+ *                     training backward reads)
+ * Every pair's work items read their rows of x again (Hq/2 times in all), so this form costs
+ * more memory traffic than diffattn_v2_lambda_v2 followed by diffattn_v2_prefill; it exists
+ * for callers that want one launch. Host checks and errors as diffattn_v2_prefill, plus:
+ * d_model > 0 and a multiple of 8, x and w_lambda_t non-NULL and 16-byte aligned, bias and
+ * lambda_out NULL or 16-byte aligned.
+ */
+DA2_API int diffattn_v2_prefill_fused_lambda(const void* q, const void* k, const void* v, const void* x,
+                                             const void* w_lambda_t, const float* bias, void* out,
+                                             float* lambda_out, int B, int S, int Hq, int Hkv, int D, int d_model,
+                                             int causal, da2_stream_t stream);
+
+/*
  * Synchronise `stream`, then read and clear the device error word that kernels set when a
  * bounded wait expires. *code receives 0 when no kernel reported an error, else the code
  * of the first error recorded (a pipeline wait expired: 1 = in a prefill, 2 = in a decode,

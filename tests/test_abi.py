@@ -179,6 +179,21 @@ def test_lambda_v2_host_checks(lib):
     assert lib.diffattn_v2_lambda_v2(Q, K, None, 0, 128, 32, O, None) == 0
 
 
+def test_prefill_fused_lambda_host_checks(lib):
+    X, W = P + 24576, P + 28672
+    f = lib.diffattn_v2_prefill_fused_lambda
+    assert f(Q, K, V, X, W, None, O, None, 1, 64, 8, 2, 128, 100, 1, None) == -1       # d_model % 8
+    assert f(Q, K, V, X, W, None, O, None, 1, 64, 8, 2, 128, 0, 1, None) == -1         # d_model = 0
+    assert f(Q, K, V, None, W, None, O, None, 1, 64, 8, 2, 128, 256, 1, None) == -1    # null x
+    assert f(Q, K, V, X, None, None, O, None, 1, 64, 8, 2, 128, 256, 1, None) == -1    # null w_lambda_t
+    assert f(Q, K, V, X, W, L + 4, O, None, 1, 64, 8, 2, 128, 256, 1, None) == -1      # misaligned bias
+    assert f(Q, K, V, X, W, None, O, L + 8, 1, 64, 8, 2, 128, 256, 1, None) == -1      # misaligned lambda_out
+    assert f(Q, K, V, X, W, None, O, None, 1, 64, 6, 2, 128, 256, 1, None) == -1       # straddling pair
+    assert f(Q, K, V, X, W, None, O, None, 1, 64, 8, 2, 64, 256, 1, None) == -2        # D = 64
+    assert f(Q, K, V, X, W, None, O, None, 1, 64, 8, 2, 128, 256, 2, None) == -1       # causal flag
+    assert f(Q, K, V, X, W, None, O, None, 0, 64, 8, 2, 128, 256, 1, None) == 0        # B = 0
+
+
 def test_lambda_v1_host_checks(lib):
     assert lib.diffattn_v2_lambda_v1(Q, K, V, L, 0.8, 0, 128, 1, O, None) == -1
     assert lib.diffattn_v2_lambda_v1(Q, K, V, L, 0.8, 4, 0, 1, O, None) == -1
