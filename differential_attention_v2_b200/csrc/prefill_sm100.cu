@@ -749,11 +749,15 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
           if (lane == 0) {
             const float la = va ? 1.f / (1.f + expf(-(sa + bias))) : 0.f;
             const float lb = vb ? 1.f / (1.f + expf(-(sb + bias))) : 0.f;
-            lam_ring[s * BM + row0 + rr] = la;
-            lam_ring[s * BM + row0 + rr + 1] = lb;
+            if (checked(s * BM + row0 + rr + 1 < 2 * BM, p.err)) {
+              lam_ring[s * BM + row0 + rr] = la;
+              lam_ring[s * BM + row0 + rr + 1] = lb;
+            }
             if (p.lam_out != nullptr) {
-              if (va) p.lam_out[(w.row_base + qa) * n_pairs_l + w.pair] = la;
-              if (vb) p.lam_out[(w.row_base + qa + 1) * n_pairs_l + w.pair] = lb;
+              const size_t lam_elems = static_cast<size_t>(p.B) * p.S * n_pairs_l;
+              const size_t ia = (w.row_base + qa) * n_pairs_l + w.pair;
+              if (va && checked(ia < lam_elems, p.err)) p.lam_out[ia] = la;
+              if (vb && checked(ia + n_pairs_l < lam_elems, p.err)) p.lam_out[ia + n_pairs_l] = lb;
             }
           }
         }

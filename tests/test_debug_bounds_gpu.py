@@ -4,7 +4,7 @@ libdiffattn_v2_debug.so is the library compiled with -DDA2_DEBUG_BOUNDS: its ker
 every checked shared-memory offset, tensor-memory column and global index with the extent it
 addresses, and on a violation record code 4 in the device error word and skip the access.
 These tests run the small cases of the prefill (one-CTA and CTA-pair forms, sliding window,
-packed sequences, training outputs), the decode (GQA groups 8 and 16, paged cache,
+packed sequences, training outputs, lambda computed in the kernel), the decode (GQA groups 8 and 16, paged cache,
 multi-token) and the backward through it, and require both a zero error word and the usual
 agreement with the float64 oracle. (No case here is meant to violate a bound.)
 """
@@ -43,6 +43,22 @@ def _clean(da):
     code = da.device_error()
     assert code != ERR_BOUNDS, "a kernel reported an index outside its extent"
     assert code == 0, f"device error {code}"
+
+
+def test_prefill_fused_lambda_in_bounds(dbg):
+    B, S, Hq, Hkv, d_model = 2, 300, 8, 2, 256
+    inp = workloads.make_prefill(workloads.PrefillCase(B=B, S=S, Hq=Hq, Hkv=Hkv, D=128, seed=57))
+    g = torch.Generator().manual_seed(58)
+    x = torch.randn(B, S, d_model, generator=g).bfloat16()
+    w = (torch.randn(d_model, Hq // 2, generator=g) / d_model ** 0.5).bfloat16()
+    d = {k: v.cuda() for k, v in inp.items()}
+    lam = torch.empty(B, S, Hq // 2, device="cuda")
+    out = dbg.prefill_fused_lambda(d["q"], d["k"], d["v"], x.cuda(), w.t().contiguous().cuda(), lambda_out=lam)
+    _clean(dbg)
+    lam_ref = ora.lambda_v2_projection(x.reshape(B * S, d_model), w).reshape(B, S, Hq // 2)
+    np.testing.assert_allclose(lam.cpu().double().numpy(), lam_ref, rtol=0, atol=1e-5)
+    bf16_close(out, ora.prefill(inp["q"], inp["k"], inp["v"], torch.from_numpy(lam_ref).float()),
+               "debug fused-lambda prefill")
 
 
 @pytest.mark.parametrize("pair", ["0", "1"])
