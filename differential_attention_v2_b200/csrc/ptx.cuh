@@ -53,14 +53,21 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// A waiting thread may stay suspended in try_wait for up to this long (it resumes as soon as
+// the phase completes). Under a sustained load the kernels run at the power cap, and fewer
+// wake-ups of waiting warps leave more of it to the tensor cores: against the default limit,
+// 20 us measured +1.0% on the B=4 x 4096 prefill and +0.4% on 1 x 32768 (alternating rounds
+// on one B200), the decode unchanged.
+constexpr uint32_t kWaitSuspendNs = 20000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(done)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "n"(kWaitSuspendNs)
       : "memory");
   return done != 0;
 }
