@@ -812,12 +812,17 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         // some row of the tile has keys of this KV tile below its window
         const bool win_edge = kWindow && j * BN < w.m0 + BM - p.window;
         const bool tile_masked = (p.causal && j == w.tile) || ((j + 1) * BN > S) || win_edge;
+        // dead_h: no row of the warp sees a key of 64-key half h (the diagonal tile's upper
+        // half for rows 0-63, a window's first tile's lower half for rows 64-127)
+        bool dead0 = false, dead1 = false;
         if (tile_masked) {
           int hi = BN - 1;
           if (p.causal && j == w.tile) hi = r;
           hi = min(hi, S - 1 - j * BN);
           const int lo = kWindow ? qi - p.window + 1 - j * BN : 0;
           mask_row<4>(sr, lo, hi);
+          dead0 = __all_sync(0xffffffffu, hi < 0 || lo > 63);
+          dead1 = __all_sync(0xffffffffu, hi < 64 || lo > 127);
         }
         const float mx = row_max<4>(sr) * p.scale_log2;
 
@@ -848,9 +853,18 @@ diffattn_prefill_sm100(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         float lsum = 0.f;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          // masked tiles take every exponential on the MUFU so masked keys stay exactly 0
-          lsum += tile_masked ? exp_pack_store<false>(sr, half, p.scale_log2, m_use, trow + s_col)
-                              : exp_pack_store<true>(sr, half, p.scale_log2, m_use, trow + s_col);
+          // a half no row of the warp sees gets P = 0 without its exponentials (all 2^-inf =
+          // 0); masked tiles take every other exponential on the MUFU so masked keys stay
+          // exactly 0
+          if (half ? dead1 : dead0) {
+            uint32_t zero[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) zero[e] = 0u;
+            tmem_st_32x32b_x32(trow + s_col + 32 * half, zero);
+          } else {
+            lsum += tile_masked ? exp_pack_store<false>(sr, half, p.scale_log2, m_use, trow + s_col)
+                                : exp_pack_store<true>(sr, half, p.scale_log2, m_use, trow + s_col);
+          }
           tmem_st_wait();
           arrive_for_mma<kPair>(bar(kPFull + 2 * br + half), lane);
         }
