@@ -73,8 +73,8 @@ SPEC_HBM_GBS = 8000.0
 # one launch), keyed by workload and by the kernel source it was taken on; reported as null
 # once the source differs from the one captured.
 NCU_TRAFFIC = {
-    # B=1 x 32768 causal prefill: 3489703680 read + 247699968 written
-    ("prefill", "prefill_b1_s32768"): {"bytes": 3737403648, "source_sha": "d4b52fc4971c7b08"},
+    # B=1 x 32768 causal prefill: 3445891328 read + 247948288 written
+    ("prefill", "prefill_b1_s32768"): {"bytes": 3693839616, "source_sha": "7e51d88bae48ec3f"},
     # B=8 x 131072 needle decode (split kernel with the fused merge): 4304263168 + 12806656
     ("decode", "needle_decode_b8_s131072"): {"bytes": 4317069824, "source_sha": "07d184e353942e3c"},
 }

@@ -8,7 +8,7 @@ use raises ImportError (there is no fallback implementation).
 import importlib
 
 _BINDING_NAMES = (
-    "prefill", "prefill_window", "prefill_varlen", "prefill_f32", "prefill_train", "backward",
+    "prefill", "prefill_window", "prefill_varlen", "prefill_varlen_window", "prefill_f32", "prefill_train", "backward",
     "backward_workspace_size", "prefill_varlen_train", "backward_varlen", "backward_varlen_workspace_size", "decode", "decode_f32", "decode_workspace_size", "decode_noalloc", "decode_paged",
     "decode_multi", "lambda_v1", "lambda_v2", "prefill_fused_lambda", "device_error", "version", "load", "DiffAttnError", "EXPORTED", "LIB_PATH",
     "LIB",

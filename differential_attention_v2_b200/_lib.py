@@ -46,6 +46,7 @@ _SIGNATURES = {
     "diffattn_v2_lambda_v1": (_i, [_vp, _vp, _vp, _vp, _f, _i, _i, _i, _vp, _vp]),
     "diffattn_v2_lambda_v2": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
     "diffattn_v2_prefill_fused_lambda": (_i, [_vp] * 8 + [_i] * 7 + [_vp]),
+    "diffattn_v2_prefill_varlen_window": (_i, [_vp] * 6 + [_i] * 7 + [_vp]),
     "diffattn_v2_device_error": (_i, [ctypes.POINTER(_i), _vp]),
     "diffattn_v2_decode_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
 }
@@ -157,6 +158,25 @@ def prefill_varlen(q, k, v, lam, cu_seqlens, max_seqlen, out=None, causal=True, 
     st = LIB.diffattn_v2_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(out), _ptr(cu_seqlens), B,
                                         int(max_seqlen), T, Hq, Hkv, D, 1 if causal else 0, _stream(stream, q.device))
     _check(st, "diffattn_v2_prefill_varlen")
+    return out
+
+
+def prefill_varlen_window(q, k, v, lam, cu_seqlens, max_seqlen, window, out=None, stream=None):
+    """Causal sliding-window prefill of packed sequences (layouts of prefill_varlen): query i
+    of a sequence sees that sequence's keys i-window+1 .. i."""
+    for t, n, nd in ((q, "q", 3), (k, "k", 3), (v, "v", 3)):
+        _need(t, n, torch.bfloat16, nd)
+    _need(lam, "lam", torch.float32, 2)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    T, Hq, D = q.shape
+    Hkv = k.shape[1]
+    B = cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty((T, Hq // 2, D), dtype=torch.bfloat16, device=q.device)
+    _need(out, "out", torch.bfloat16, 3)
+    st = LIB.diffattn_v2_prefill_varlen_window(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(out), _ptr(cu_seqlens), B,
+                                               int(max_seqlen), T, Hq, Hkv, D, int(window), _stream(stream, q.device))
+    _check(st, "diffattn_v2_prefill_varlen_window")
     return out
 
 

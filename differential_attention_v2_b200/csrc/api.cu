@@ -236,6 +236,33 @@ int diffattn_v2_prefill_varlen(const void* q, const void* k, const void* v, cons
   return status_of(e);
 }
 
+int diffattn_v2_prefill_varlen_window(const void* q, const void* k, const void* v, const float* lambda, void* out,
+                                      const int32_t* cu_seqlens, int B, int max_seqlen, int total_tokens, int Hq,
+                                      int Hkv, int D, int window, da2_stream_t stream) {
+  if (B < 0 || max_seqlen < 0 || total_tokens < 0 || D <= 0 || !heads_ok(Hq, Hkv) || window < 1) return DA2_ERR_INVALID;
+  if (B == 0 || max_seqlen == 0 || total_tokens == 0) return DA2_OK;
+  if (!q || !k || !v || !lambda || !out || !cu_seqlens) return DA2_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(lambda) || !aligned16(out) ||
+      !aligned16(cu_seqlens))
+    return DA2_ERR_INVALID;
+  if (D != 128) return DA2_ERR_UNSUPPORTED;
+  if ((max_seqlen + 127) / 128 > 65535) return DA2_ERR_UNSUPPORTED;
+  int* err = nullptr;
+  cudaError_t e = device_error_ptr(&err);
+  if (e != cudaSuccess) return DA2_ERR_CUDA;
+  CUtensorMap tq, tk, tv, tkh;  // the packed tokens as one batch of total_tokens rows
+  if (encode_bshd(&tq, q, D, Hq, total_tokens, 1, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  if (encode_bshd(&tk, k, D, Hkv, total_tokens, 1, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  if (encode_bshd(&tv, v, D, Hkv, total_tokens, 1, 64, 128) != cudaSuccess) return DA2_ERR_CUDA;
+  if (encode_bshd(&tkh, k, D, Hkv, total_tokens, 1, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
+  CUtensorMap to;
+  if (da2::encode_out_bf16(&to, out, D, Hq / 2, total_tokens, 1) != cudaSuccess) return DA2_ERR_CUDA;
+  // a window of max_seqlen or more keys is the plain causal mask for every sequence
+  e = da2::launch_prefill(tq, tk, tv, &tkh, to, lambda, static_cast<__nv_bfloat16*>(out), err, B, max_seqlen, Hq, Hkv,
+                          1, window >= max_seqlen ? 0 : window, cu_seqlens, reinterpret_cast<cudaStream_t>(stream));
+  return status_of(e);
+}
+
 int diffattn_v2_prefill_fused_lambda(const void* q, const void* k, const void* v, const void* x,
                                      const void* w_lambda_t, const float* bias, void* out, float* lambda_out, int B,
                                      int S, int Hq, int Hkv, int D, int d_model, int causal, da2_stream_t stream) {

@@ -1041,7 +1041,8 @@ cudaError_t launch_prefill(const CUtensorMap& tmQ, const CUtensorMap& tmK, const
   const int group = Hq / Hkv;
   const char* env = getenv("DA2_PREFILL_CTA_PAIR");
   const bool pair_wanted = env != nullptr && env[0] == '1';
-  const bool use_pair = pair_wanted && tmKh != nullptr && (group % 4) == 0 && !one_per_item;
+  const bool use_pair = pair_wanted && tmKh != nullptr && (group % 4) == 0 && !one_per_item &&
+                        !(cu_seqlens != nullptr && window > 0);
   if (use_pair) {
     p.n_items = B * (Hq / 4) * p.n_row_tiles;
     if (p.n_items == 0) return cudaSuccess;
@@ -1075,7 +1076,8 @@ cudaError_t launch_prefill(const CUtensorMap& tmQ, const CUtensorMap& tmK, const
   }
 
   p.n_items = B * (Hq / 2) * p.n_row_tiles;
-  auto kernel = cu_seqlens ? diffattn_prefill_sm100<true, false, false>
+  auto kernel = cu_seqlens ? (window > 0 ? diffattn_prefill_sm100<true, true, false>
+                                         : diffattn_prefill_sm100<true, false, false>)
                            : (window > 0 ? diffattn_prefill_sm100<false, true, false>
                                          : diffattn_prefill_sm100<false, false, false>);
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);

@@ -362,6 +362,20 @@ DA2_API int diffattn_v2_lambda_v2(const void* x, const void* w_lambda, const flo
                                   int n_pairs, float* lambda_out, da2_stream_t stream);
 
 /*
+ * Causal sliding-window prefill of packed sequences: diffattn_v2_prefill_varlen's layouts and
+ * sequence rules with diffattn_v2_prefill_window's mask inside every sequence (query i of a
+ * sequence sees that sequence's keys max(0, i-window+1) .. i). Sources: the "Attention
+ * variants" lesson, sliding-window step, and the hybrid layers of the "Differential Attention
+ * (V2)" lesson's "Use it" section, with the packed layout serving engines use. window >= 1;
+ * window >= max_seqlen is the plain causal packed prefill. Host checks and errors as
+ * diffattn_v2_prefill_varlen, plus DA2_ERR_INVALID for window < 1.
+ */
+DA2_API int diffattn_v2_prefill_varlen_window(const void* q, const void* k, const void* v, const float* lambda,
+                                              void* out, const int32_t* cu_seqlens, int B, int max_seqlen,
+                                              int total_tokens, int Hq, int Hkv, int D, int window,
+                                              da2_stream_t stream);
+
+/*
  * bf16 prefill with the V2 lambda fused into the kernel: the same output as
  * diffattn_v2_prefill with lambda[b,s,p] = sigmoid(x[b,s] . w_lambda_t[p] + bias[p]) (the
  * projection of diffattn_v2_lambda_v2), computed per work item by two otherwise idle warps of

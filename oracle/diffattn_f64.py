@@ -175,17 +175,20 @@ def prefill(q, k, v, lam, causal: bool = True, row_block: int = 512, window=None
     return out
 
 
-def prefill_varlen(q, k, v, lam, cu_seqlens, causal: bool = True) -> np.ndarray:
+def prefill_varlen(q, k, v, lam, cu_seqlens, causal: bool = True, window=None) -> np.ndarray:
     """Prefill of sequences packed along the token axis: q [T,Hq,D], k/v [T,Hkv,D],
     lam [T,Hq/2], sequence b = tokens cu_seqlens[b] .. cu_seqlens[b+1]-1. Every sequence is an
-    independent prefill (its queries see only its own keys). Returns out [T,Hq/2,D]."""
+    independent prefill (its queries see only its own keys); with `window` (causal only) the
+    sliding window of the "Attention variants" lesson applies inside each sequence. Returns
+    out [T,Hq/2,D]."""
     cu = [int(x) for x in cu_seqlens]
     T = int(q.shape[0])
     out = np.zeros((T, q.shape[1] // 2, q.shape[2]), dtype=np.float64)
     for b in range(len(cu) - 1):
         s0, s1 = cu[b], cu[b + 1]
         if s1 > s0:
-            out[s0:s1] = prefill(q[None, s0:s1], k[None, s0:s1], v[None, s0:s1], lam[None, s0:s1], causal=causal)[0]
+            out[s0:s1] = prefill(q[None, s0:s1], k[None, s0:s1], v[None, s0:s1], lam[None, s0:s1], causal=causal,
+                                 window=window)[0]
     return out
 
 

@@ -103,6 +103,16 @@ def test_prefill_varlen_host_checks(lib):
     assert lib.diffattn_v2_prefill_varlen(Q, K, V, L, O, C, 2, 64, 100, 8, 2, 128, 3, None) == -1     # causal flag
 
 
+def test_prefill_varlen_window_host_checks(lib):
+    C = P + 28672
+    f = lib.diffattn_v2_prefill_varlen_window
+    assert f(Q, K, V, L, O, C, 2, 64, 100, 8, 2, 128, 0, None) == -1       # window 0
+    assert f(Q, K, V, L, O, None, 2, 64, 100, 8, 2, 128, 16, None) == -1   # no cu_seqlens
+    assert f(Q, K, V, L, O, C, 2, 64, 100, 6, 2, 128, 16, None) == -1      # straddling pair
+    assert f(Q, K, V, L, O, C, 2, 64, 100, 8, 2, 64, 16, None) == -2       # D = 64
+    assert f(Q, K, V, L, O, C, 0, 64, 100, 8, 2, 128, 16, None) == 0       # no sequences
+
+
 def test_prefill_f32_host_checks(lib):
     assert lib.diffattn_v2_prefill_f32(Q, K, V, L, O, 1, 16, 4, 1, 96, 1, None) == -2
     assert lib.diffattn_v2_prefill_f32(Q, K, V, L, O, 1, 16, 4, 3, 64, 1, None) == -1

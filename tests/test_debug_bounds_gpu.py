@@ -4,7 +4,7 @@ libdiffattn_v2_debug.so is the library compiled with -DDA2_DEBUG_BOUNDS: its ker
 every checked shared-memory offset, tensor-memory column and global index with the extent it
 addresses, and on a violation record code 4 in the device error word and skip the access.
 These tests run the small cases of the prefill (one-CTA and CTA-pair forms, sliding window,
-packed sequences, training outputs, lambda computed in the kernel), the decode (GQA groups 8 and 16, paged cache,
+packed sequences with and without a window, training outputs, lambda computed in the kernel), the decode (GQA groups 8 and 16, paged cache,
 multi-token) and the backward through it, and require both a zero error word and the usual
 agreement with the float64 oracle. (No case here is meant to violate a bound.)
 """
@@ -97,6 +97,9 @@ def test_prefill_packed_sequences_in_bounds(dbg):
     out = dbg.prefill_varlen(q.cuda(), k.cuda(), v.cuda(), lam.cuda(), cu.cuda(), max(lens) + 200)
     _clean(dbg)
     bf16_close(out, ora.prefill_varlen(q, k, v, lam, cu.tolist()), "debug packed prefill")
+    out = dbg.prefill_varlen_window(q.cuda(), k.cuda(), v.cuda(), lam.cuda(), cu.cuda(), max(lens), 90)
+    _clean(dbg)
+    bf16_close(out, ora.prefill_varlen(q, k, v, lam, cu.tolist(), window=90), "debug packed window prefill")
 
 
 @pytest.mark.parametrize("B,Smax,Hq,Hkv,lens", [

@@ -312,6 +312,25 @@ def pin_varlen_is_per_sequence_prefill():
     return bool(ok)
 
 
+def pin_varlen_window_is_per_sequence_window():
+    """A sliding window over packed sequences: each sequence equals the brute force's windowed
+    prefill of that sequence alone, and a window longer than every sequence is the causal
+    packed prefill."""
+    q, k, v, lam = _rand_prefill(B=1, S=39, Hq=4, Hkv=1, D=5, seed=17)
+    flat = lambda t: t.reshape(-1, *t.shape[2:])
+    cu = [0, 5, 5, 20, 39]  # lengths 5, 0, 15, 19
+    ok = True
+    for w in (1, 3, 7):
+        out = ora.prefill_varlen(flat(q), flat(k), flat(v), flat(lam), cu, window=w)
+        for a, b_ in zip(cu[:-1], cu[1:]):
+            if b_ > a:
+                ref = np.array(brute.prefill(*(flat(t)[None, a:b_].tolist() for t in (q, k, v, lam)), window=w))[0]
+                ok &= np.allclose(out[a:b_], ref, atol=1e-12)
+    ok &= np.allclose(ora.prefill_varlen(flat(q), flat(k), flat(v), flat(lam), cu, window=19),
+                      ora.prefill_varlen(flat(q), flat(k), flat(v), flat(lam), cu), atol=1e-13)
+    return bool(ok)
+
+
 def pin_paged_decode_gathers_pages():
     """A paged cache with a shuffled block table decodes like the contiguous cache it holds
     (and, through `decode`, like the brute force)."""
@@ -490,6 +509,7 @@ def pin_backward_window():
 
 
 ALL_PINS = {
+    "varlen_window_is_per_sequence_window": pin_varlen_window_is_per_sequence_window,
     "softmax_library": pin_softmax_library,
     "lambda0_is_softmax_attention": pin_lambda0_is_softmax_attention,
     "lambda0_noncausal": lambda: pin_lambda0_is_softmax_attention(causal=False),

@@ -172,7 +172,15 @@ def _snr_signed_mean(weights, signal_index):
 
 _ORIG_BRANCHES = ora.prefill_branches
 
+def _varlen_window_ignored(q, k, v, lam, cu_seqlens, causal=True, window=None):
+    return _VARLEN(q, k, v, lam, cu_seqlens, causal=causal)
+
+
+_VARLEN = ora.prefill_varlen
+
+
 MUTANTS = {
+    "varlen_window_ignored": ("prefill_varlen", _varlen_window_ignored),
     "plus_sign": ("diff_attention_block", _block_plus_sign),
     "no_scale": ("diff_attention_block", _block_no_scale),
     "scale_by_d": ("diff_attention_block", _block_scale_d),

@@ -206,6 +206,41 @@ def test_prefill_varlen_matches_oracle(da, lens, Hq, Hkv, causal, extra):
     bf16_close(out, ref, f"varlen {lens}")
 
 
+@pytest.mark.parametrize("lens,window,Hq,Hkv", [
+    ([300, 1, 0, 200, 129, 700], 64, 8, 2),     # ragged, single token, empty; window inside a tile
+    ([300, 1, 0, 200, 129, 700], 200, 16, 2),   # window wider than a tile
+    ([513, 37, 260], 1, 4, 2),                  # each query sees only itself
+    ([513, 37, 260], 1000, 8, 4),               # window past every sequence: plain causal
+])
+def test_prefill_varlen_window_matches_oracle(da, lens, window, Hq, Hkv):
+    T = sum(lens)
+    g = torch.Generator().manual_seed(T + window)
+    q = torch.randn(T, Hq, 128, generator=g).bfloat16()
+    k = torch.randn(T, Hkv, 128, generator=g).bfloat16()
+    v = torch.randn(T, Hkv, 128, generator=g).bfloat16()
+    lam = torch.sigmoid(torch.randn(T, Hq // 2, generator=g))
+    cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32)
+    out = da.prefill_varlen_window(q.cuda(), k.cuda(), v.cuda(), lam.cuda(), cu.cuda(), max(lens), window)
+    assert da.device_error() == 0
+    ref = ora.prefill_varlen(q, k, v, lam, cu.tolist(), window=window)
+    bf16_close(out, ref, f"varlen window {window} {lens}")
+
+
+@pytest.mark.parametrize("B,S", [(3, 333), (300, 150)])
+def test_prefill_varlen_window_equals_batched_window(da, B, S):
+    """Equal-length packed sequences with a window give the batched window prefill bit for bit
+    (300 sequences: the one-CTA-per-item launch)."""
+    case = workloads.PrefillCase(B=B, S=S, Hq=8, Hkv=2, D=128, seed=10 + B)
+    inp = workloads.make_prefill(case)
+    d = _dev(inp)
+    batched = da.prefill_window(d["q"], d["k"], d["v"], d["lam"], 100)
+    flat = lambda t: t.reshape(-1, *t.shape[2:]).contiguous()
+    cu = torch.arange(0, (B + 1) * S, S, dtype=torch.int32, device="cuda")
+    packed = da.prefill_varlen_window(flat(d["q"]), flat(d["k"]), flat(d["v"]), flat(d["lam"]), cu, S, 100)
+    assert da.device_error() == 0
+    assert torch.equal(packed.view(B, S, 4, 128), batched)
+
+
 def test_prefill_varlen_equals_batched(da):
     """Equal-length packed sequences give the batched prefill's output bit for bit."""
     case = workloads.PrefillCase(B=3, S=333, Hq=16, Hkv=2, D=128, seed=8)
