@@ -37,6 +37,8 @@ _SIGNATURES = {
     "diffattn_v2_prefill_varlen_train": (_i, [_vp] * 8 + [_i] * 7 + [_vp]),
     "diffattn_v2_backward_varlen_workspace_size": (_sz, [_i, _i, _i]),
     "diffattn_v2_backward_varlen": (_i, [_vp] * 12 + [_i] * 7 + [_vp, _sz, _vp]),
+    "diffattn_v2_prefill_varlen_window_train": (_i, [_vp] * 8 + [_i] * 7 + [_vp]),
+    "diffattn_v2_backward_varlen_window": (_i, [_vp] * 12 + [_i] * 7 + [_vp, _sz, _vp]),
     "diffattn_v2_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "diffattn_v2_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "diffattn_v2_decode_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
@@ -264,9 +266,10 @@ def backward(q, k, v, lam, o_branch, lse, dout, causal=True, dq=None, dk=None, d
 
 
 def prefill_varlen_train(q, k, v, lam, cu_seqlens, max_seqlen, out=None, o_branch=None, lse=None, causal=True,
-                         stream=None):
+                         stream=None, window=None):
     """Training forward of packed sequences (layouts of prefill_varlen): returns
-    (out [T,Hq/2,D], o_branch [T,Hq,D], lse [T,Hq])."""
+    (out [T,Hq/2,D], o_branch [T,Hq,D], lse [T,Hq]). With `window` the causal sliding window
+    inside every sequence."""
     for t, n, nd in ((q, "q", 3), (k, "k", 3), (v, "v", 3)):
         _need(t, n, torch.bfloat16, nd)
     _need(lam, "lam", torch.float32, 2)
@@ -280,6 +283,13 @@ def prefill_varlen_train(q, k, v, lam, cu_seqlens, max_seqlen, out=None, o_branc
     _need(out, "out", torch.bfloat16, 3)
     _need(o_branch, "o_branch", torch.bfloat16, 3)
     _need(lse, "lse", torch.float32, 2)
+    if window is not None:
+        st = LIB.diffattn_v2_prefill_varlen_window_train(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(out),
+                                                         _ptr(o_branch), _ptr(lse), _ptr(cu_seqlens), B,
+                                                         int(max_seqlen), T, Hq, Hkv, D, int(window),
+                                                         _stream(stream, q.device))
+        _check(st, "diffattn_v2_prefill_varlen_window_train")
+        return out, o_branch, lse
     st = LIB.diffattn_v2_prefill_varlen_train(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(out), _ptr(o_branch),
                                               _ptr(lse), _ptr(cu_seqlens), B, int(max_seqlen), T, Hq, Hkv, D,
                                               1 if causal else 0, _stream(stream, q.device))
@@ -292,8 +302,9 @@ def backward_varlen_workspace_size(B, total_tokens, Hq) -> int:
 
 
 def backward_varlen(q, k, v, lam, o_branch, lse, dout, cu_seqlens, max_seqlen, causal=True, workspace=None,
-                    stream=None):
-    """Gradients of the packed-sequence prefill: returns (dq, dk, dv, dlam) in the packed layouts."""
+                    stream=None, window=None):
+    """Gradients of the packed-sequence prefill: returns (dq, dk, dv, dlam) in the packed layouts.
+    With `window` the gradients of the causal sliding-window packed prefill."""
     for t, n, nd in ((q, "q", 3), (k, "k", 3), (v, "v", 3), (o_branch, "o_branch", 3), (dout, "dout", 3)):
         _need(t, n, torch.bfloat16, nd)
     _need(lam, "lam", torch.float32, 2)
@@ -306,10 +317,18 @@ def backward_varlen(q, k, v, lam, o_branch, lse, dout, cu_seqlens, max_seqlen, c
     ws_bytes = backward_varlen_workspace_size(B, T, Hq)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+    ws_given = workspace.numel() * workspace.element_size()
+    if window is not None:
+        st = LIB.diffattn_v2_backward_varlen_window(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(o_branch), _ptr(lse),
+                                                    _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlam),
+                                                    _ptr(cu_seqlens), B, int(max_seqlen), T, Hq, Hkv, D, int(window),
+                                                    _ptr(workspace), ws_given, _stream(stream, q.device))
+        _check(st, "diffattn_v2_backward_varlen_window")
+        return dq, dk, dv, dlam
     st = LIB.diffattn_v2_backward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(o_branch), _ptr(lse),
                                          _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlam), _ptr(cu_seqlens), B,
                                          int(max_seqlen), T, Hq, Hkv, D, 1 if causal else 0, _ptr(workspace),
-                                         workspace.numel() * workspace.element_size(), _stream(stream, q.device))
+                                         ws_given, _stream(stream, q.device))
     _check(st, "diffattn_v2_backward_varlen")
     return dq, dk, dv, dlam
 

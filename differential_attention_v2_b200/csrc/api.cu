@@ -418,9 +418,12 @@ int diffattn_v2_backward_window(const void* q, const void* k, const void* v, con
                        window >= S ? 0 : window, workspace, workspace_bytes, stream);
 }
 
-int diffattn_v2_prefill_varlen_train(const void* q, const void* k, const void* v, const float* lambda, void* out,
-                                     void* o_branch, float* lse, const int32_t* cu_seqlens, int B, int max_seqlen,
-                                     int total_tokens, int Hq, int Hkv, int D, int causal, da2_stream_t stream) {
+namespace {
+
+// Training forward of packed sequences; window > 0 (causal only) applies inside each sequence.
+int prefill_varlen_train(const void* q, const void* k, const void* v, const float* lambda, void* out, void* o_branch,
+                         float* lse, const int32_t* cu_seqlens, int B, int max_seqlen, int total_tokens, int Hq,
+                         int Hkv, int D, int causal, int window, da2_stream_t stream) {
   if (B < 0 || max_seqlen < 0 || total_tokens < 0 || D <= 0 || !heads_ok(Hq, Hkv)) return DA2_ERR_INVALID;
   if (causal != 0 && causal != 1) return DA2_ERR_INVALID;
   if (B == 0 || max_seqlen == 0 || total_tokens == 0) return DA2_OK;
@@ -440,9 +443,28 @@ int diffattn_v2_prefill_varlen_train(const void* q, const void* k, const void* v
   CUtensorMap to;
   if (da2::encode_out_bf16(&to, out, D, Hq / 2, total_tokens, 1) != cudaSuccess) return DA2_ERR_CUDA;
   e = da2::launch_prefill(tq, tk, tv, &tkh, to, lambda, static_cast<__nv_bfloat16*>(out), err, B, max_seqlen, Hq, Hkv, causal,
-                          0, cu_seqlens, reinterpret_cast<cudaStream_t>(stream), static_cast<__nv_bfloat16*>(o_branch),
-                          lse);
+                          window, cu_seqlens, reinterpret_cast<cudaStream_t>(stream),
+                          static_cast<__nv_bfloat16*>(o_branch), lse);
   return status_of(e);
+}
+
+}  // namespace
+
+int diffattn_v2_prefill_varlen_train(const void* q, const void* k, const void* v, const float* lambda, void* out,
+                                     void* o_branch, float* lse, const int32_t* cu_seqlens, int B, int max_seqlen,
+                                     int total_tokens, int Hq, int Hkv, int D, int causal, da2_stream_t stream) {
+  return prefill_varlen_train(q, k, v, lambda, out, o_branch, lse, cu_seqlens, B, max_seqlen, total_tokens, Hq, Hkv,
+                              D, causal, 0, stream);
+}
+
+int diffattn_v2_prefill_varlen_window_train(const void* q, const void* k, const void* v, const float* lambda,
+                                            void* out, void* o_branch, float* lse, const int32_t* cu_seqlens, int B,
+                                            int max_seqlen, int total_tokens, int Hq, int Hkv, int D, int window,
+                                            da2_stream_t stream) {
+  if (window < 1) return DA2_ERR_INVALID;
+  // a window of max_seqlen or more keys is the plain causal mask for every sequence
+  return prefill_varlen_train(q, k, v, lambda, out, o_branch, lse, cu_seqlens, B, max_seqlen, total_tokens, Hq, Hkv,
+                              D, 1, window >= max_seqlen ? 0 : window, stream);
 }
 
 size_t diffattn_v2_backward_varlen_workspace_size(int B, int total_tokens, int Hq) {
@@ -450,11 +472,13 @@ size_t diffattn_v2_backward_varlen_workspace_size(int B, int total_tokens, int H
   return da2::backward_varlen_workspace_bytes(B, total_tokens, Hq);
 }
 
-int diffattn_v2_backward_varlen(const void* q, const void* k, const void* v, const float* lambda,
-                                const void* o_branch, const float* lse, const void* dout, void* dq, void* dk,
-                                void* dv, float* dlambda, const int32_t* cu_seqlens, int B, int max_seqlen,
-                                int total_tokens, int Hq, int Hkv, int D, int causal, void* workspace,
-                                size_t workspace_bytes, da2_stream_t stream) {
+namespace {
+
+// Backward of the packed-sequence prefill; window > 0 (causal only) inside each sequence.
+int backward_varlen(const void* q, const void* k, const void* v, const float* lambda, const void* o_branch,
+                    const float* lse, const void* dout, void* dq, void* dk, void* dv, float* dlambda,
+                    const int32_t* cu_seqlens, int B, int max_seqlen, int total_tokens, int Hq, int Hkv, int D,
+                    int causal, int window, void* workspace, size_t workspace_bytes, da2_stream_t stream) {
   if (B < 0 || max_seqlen < 0 || total_tokens < 0 || D <= 0 || !heads_ok(Hq, Hkv)) return DA2_ERR_INVALID;
   if (causal != 0 && causal != 1) return DA2_ERR_INVALID;
   if (B == 0 || max_seqlen == 0 || total_tokens == 0) return DA2_OK;
@@ -481,7 +505,29 @@ int diffattn_v2_backward_varlen(const void* q, const void* k, const void* v, con
       q64, q128, o64, o128, k64, k128, v64, v128, lambda, static_cast<const bf*>(o_branch), lse,
       static_cast<const bf*>(dout), static_cast<bf*>(dq), static_cast<bf*>(dk), static_cast<bf*>(dv), dlambda,
       static_cast<float*>(workspace), err, B, max_seqlen, Hq, Hkv, causal, reinterpret_cast<cudaStream_t>(stream),
-      cu_seqlens, T));
+      cu_seqlens, T, window));
+}
+
+}  // namespace
+
+int diffattn_v2_backward_varlen(const void* q, const void* k, const void* v, const float* lambda,
+                                const void* o_branch, const float* lse, const void* dout, void* dq, void* dk,
+                                void* dv, float* dlambda, const int32_t* cu_seqlens, int B, int max_seqlen,
+                                int total_tokens, int Hq, int Hkv, int D, int causal, void* workspace,
+                                size_t workspace_bytes, da2_stream_t stream) {
+  return backward_varlen(q, k, v, lambda, o_branch, lse, dout, dq, dk, dv, dlambda, cu_seqlens, B, max_seqlen,
+                         total_tokens, Hq, Hkv, D, causal, 0, workspace, workspace_bytes, stream);
+}
+
+int diffattn_v2_backward_varlen_window(const void* q, const void* k, const void* v, const float* lambda,
+                                       const void* o_branch, const float* lse, const void* dout, void* dq, void* dk,
+                                       void* dv, float* dlambda, const int32_t* cu_seqlens, int B, int max_seqlen,
+                                       int total_tokens, int Hq, int Hkv, int D, int window, void* workspace,
+                                       size_t workspace_bytes, da2_stream_t stream) {
+  if (window < 1) return DA2_ERR_INVALID;
+  return backward_varlen(q, k, v, lambda, o_branch, lse, dout, dq, dk, dv, dlambda, cu_seqlens, B, max_seqlen,
+                         total_tokens, Hq, Hkv, D, 1, window >= max_seqlen ? 0 : window, workspace, workspace_bytes,
+                         stream);
 }
 
 size_t diffattn_v2_decode_workspace_size(int B, int Smax, int Hq, int Hkv, int D) {

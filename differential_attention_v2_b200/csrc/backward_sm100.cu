@@ -902,6 +902,7 @@ cudaError_t launch_backward_sm100(const CUtensorMap& tmQ64, const CUtensorMap& t
     kdq<<<dim3(B * n_pairs, p.n_tiles), kThreads, kQSmem, stream>>>(tmQ128, tmO128, tmK64, tmV64, p);
     return cudaGetLastError();
   };
+  if (cu_seqlens && window > 0) return run(dkdv_sm100<true, true>, dq_sm100<true, true>);
   if (cu_seqlens) return run(dkdv_sm100<true, false>, dq_sm100<true, false>);
   if (window > 0) return run(dkdv_sm100<false, true>, dq_sm100<false, true>);
   return run(dkdv_sm100<false, false>, dq_sm100<false, false>);

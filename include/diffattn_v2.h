@@ -226,6 +226,26 @@ DA2_API int diffattn_v2_backward_varlen(const void* q, const void* k, const void
                                         void* workspace, size_t workspace_bytes, da2_stream_t stream);
 
 /*
+ * The same training pair with the causal sliding window inside every packed sequence (the
+ * mask of diffattn_v2_prefill_varlen_window: query i of a sequence sees that sequence's keys
+ * max(0, i-window+1) .. i). Layouts, workspace (diffattn_v2_backward_varlen_workspace_size)
+ * and checks as above; window >= 1 (else DA2_ERR_INVALID), window >= max_seqlen is the plain
+ * causal pair. Sources: the "Attention variants" lesson's sliding-window step with the packed
+ * layout above.
+ */
+DA2_API int diffattn_v2_prefill_varlen_window_train(const void* q, const void* k, const void* v,
+                                                    const float* lambda, void* out, void* o_branch, float* lse,
+                                                    const int32_t* cu_seqlens, int B, int max_seqlen,
+                                                    int total_tokens, int Hq, int Hkv, int D, int window,
+                                                    da2_stream_t stream);
+DA2_API int diffattn_v2_backward_varlen_window(const void* q, const void* k, const void* v, const float* lambda,
+                                               const void* o_branch, const float* lse, const void* dout, void* dq,
+                                               void* dk, void* dv, float* dlambda, const int32_t* cu_seqlens,
+                                               int B, int max_seqlen, int total_tokens, int Hq, int Hkv, int D,
+                                               int window, void* workspace, size_t workspace_bytes,
+                                               da2_stream_t stream);
+
+/*
  * Workspace (bytes) that diffattn_v2_decode needs for these sizes: the per-split partial
  * results (running max, running sum and unnormalised output of each head), fp32. Returns 0
  * for invalid sizes. The workspace holds no state between calls.

@@ -237,11 +237,12 @@ def prefill_backward(q, k, v, lam, dout, causal: bool = True, window=None):
     return dq, dk, dv, dlam
 
 
-def prefill_backward_varlen(q, k, v, lam, dout, cu_seqlens, causal: bool = True):
+def prefill_backward_varlen(q, k, v, lam, dout, cu_seqlens, causal: bool = True, window=None):
     """Gradients of `prefill_varlen` for packed sequences (q [T,Hq,D], k/v [T,Hkv,D],
     lam [T,Hq/2], dout [T,Hq/2,D]): every sequence is an independent prefill, so its
     gradients are those of its own prefill and no token of one sequence has a gradient
-    through another. Returns (dq, dk, dv, dlam) in the packed layouts, float64."""
+    through another; `window` (causal only) as in `prefill_varlen`. Returns (dq, dk, dv, dlam)
+    in the packed layouts, float64."""
     cu = [int(x) for x in cu_seqlens]
     q, k, v, lam, dout = _f64(q), _f64(k), _f64(v), _f64(lam), _f64(dout)
     dq, dk, dv, dlam = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v), np.zeros_like(lam)
@@ -249,7 +250,7 @@ def prefill_backward_varlen(q, k, v, lam, dout, cu_seqlens, causal: bool = True)
         s0, s1 = cu[b], cu[b + 1]
         if s1 > s0:
             g = prefill_backward(q[None, s0:s1], k[None, s0:s1], v[None, s0:s1], lam[None, s0:s1],
-                                 dout[None, s0:s1], causal=causal)
+                                 dout[None, s0:s1], causal=causal, window=window)
             dq[s0:s1], dk[s0:s1], dv[s0:s1], dlam[s0:s1] = (x[0] for x in g)
     return dq, dk, dv, dlam
 

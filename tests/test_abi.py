@@ -113,6 +113,20 @@ def test_prefill_varlen_window_host_checks(lib):
     assert f(Q, K, V, L, O, C, 0, 64, 100, 8, 2, 128, 16, None) == 0       # no sequences
 
 
+def test_varlen_window_training_host_checks(lib):
+    C, W = P + 28672, P + 32768
+    ft = lib.diffattn_v2_prefill_varlen_window_train
+    assert ft(Q, K, V, L, O, O, L, C, 2, 64, 100, 8, 2, 128, 0, None) == -1        # window 0
+    assert ft(Q, K, V, L, O, O, L, None, 2, 64, 100, 8, 2, 128, 16, None) == -1    # no cu_seqlens
+    assert ft(Q, K, V, L, O, O, L, C, 2, 64, 100, 8, 2, 64, 16, None) == -2        # D = 64
+    assert ft(Q, K, V, L, O, O, L, C, 0, 64, 100, 8, 2, 128, 16, None) == 0        # no sequences
+    fb = lib.diffattn_v2_backward_varlen_window
+    args = (Q, K, V, L, O, L, O, Q, K, V, L, C, 2, 64, 100, 8, 2, 128)
+    assert fb(*args, 0, W, 1 << 30, None) == -1                                   # window 0
+    assert fb(*args, 16, W, 0, None) == -1                                        # workspace too small
+    assert fb(Q, K, V, L, O, L, O, Q, K, V, L, C, 2, 64, 100, 8, 2, 64, 16, W, 1 << 30, None) == -2  # D = 64
+
+
 def test_prefill_f32_host_checks(lib):
     assert lib.diffattn_v2_prefill_f32(Q, K, V, L, O, 1, 16, 4, 1, 96, 1, None) == -2
     assert lib.diffattn_v2_prefill_f32(Q, K, V, L, O, 1, 16, 4, 3, 64, 1, None) == -1

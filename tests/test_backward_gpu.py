@@ -155,6 +155,46 @@ def test_backward_varlen_matches_oracle(da, lens, Hq, Hkv, causal):
         grad_close(g, r, f"varlen {lens} causal={causal} {name}")
 
 
+@pytest.mark.parametrize("lens,window,Hq,Hkv", [
+    ([300, 1, 0, 200, 129], 64, 8, 2),     # ragged, single token, empty; window inside a tile
+    ([513, 37, 260], 200, 16, 2),          # window wider than a tile
+    ([300, 90], 1, 4, 2),                  # each query sees only itself
+])
+def test_backward_varlen_window_matches_oracle(da, lens, window, Hq, Hkv):
+    inp, cu = _packed(lens, Hq, Hkv, seed=81 + window)
+    d = {k: v.cuda() for k, v in inp.items()}
+    cu_t = torch.tensor(cu, dtype=torch.int32, device="cuda")
+    mx = max(lens)
+    out, ob, lse = da.prefill_varlen_train(d["q"], d["k"], d["v"], d["lam"], cu_t, mx, window=window)
+    assert torch.equal(out, da.prefill_varlen_window(d["q"], d["k"], d["v"], d["lam"], cu_t, mx, window))
+    grads = da.backward_varlen(d["q"], d["k"], d["v"], d["lam"], ob, lse, d["dout"], cu_t, mx, window=window)
+    torch.cuda.synchronize()
+    assert da.device_error() == 0
+    ref = ora.prefill_backward_varlen(inp["q"], inp["k"], inp["v"], inp["lam"], inp["dout"], cu, window=window)
+    for g, r, name in zip(grads, ref, ("dq", "dk", "dv", "dlam")):
+        grad_close(g, r, f"varlen window={window} {lens} {name}")
+
+
+def test_backward_varlen_window_equal_lengths_equals_batched(da):
+    """Packed sequences of equal length with a window: bit-identical to the batched window backward."""
+    B, S, Hq, Hkv, W = 3, 300, 8, 2, 100
+    case = workloads.PrefillCase(B=B, S=S, Hq=Hq, Hkv=Hkv, D=128, seed=87)
+    inp = workloads.make_prefill(case)
+    inp["dout"] = workloads.make_prefill_grad(case)
+    d = {k: v.cuda() for k, v in inp.items()}
+    out, ob, lse = da.prefill_train(d["q"], d["k"], d["v"], d["lam"], window=W)
+    g_batched = da.backward(d["q"], d["k"], d["v"], d["lam"], ob, lse, d["dout"], window=W)
+    flat = lambda t: t.reshape((B * S,) + t.shape[2:]).contiguous()
+    cu = torch.tensor([0, S, 2 * S, 3 * S], dtype=torch.int32, device="cuda")
+    outp, obp, lsep = da.prefill_varlen_train(flat(d["q"]), flat(d["k"]), flat(d["v"]), flat(d["lam"]), cu, S, window=W)
+    assert torch.equal(outp.view(B, S, Hq // 2, 128), out)
+    g_packed = da.backward_varlen(flat(d["q"]), flat(d["k"]), flat(d["v"]), flat(d["lam"]), obp, lsep, flat(d["dout"]),
+                                  cu, S, window=W)
+    assert da.device_error() == 0
+    for a, b in zip(g_batched, g_packed):
+        assert torch.equal(a.reshape(b.shape), b)
+
+
 def test_backward_varlen_equal_lengths_equals_batched(da):
     """Packed sequences of equal (ragged) length give bit-identical gradients to the batch."""
     B, S, Hq, Hkv = 3, 300, 8, 2

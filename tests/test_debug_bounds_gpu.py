@@ -156,6 +156,23 @@ def test_backward_in_bounds(dbg):
         grad_close(gpu, r, f"debug backward {name}")
 
 
+def test_backward_packed_window_in_bounds(dbg):
+    lens, W, Hq, Hkv = [300, 1, 0, 129], 70, 8, 2
+    T = sum(lens)
+    case = workloads.PrefillCase(B=1, S=T, Hq=Hq, Hkv=Hkv, D=128, seed=59)
+    inp = {k: v[0].contiguous() for k, v in workloads.make_prefill(case).items()}
+    dout = workloads.make_prefill_grad(case)[0].contiguous()
+    d = {k: v.cuda() for k, v in inp.items()}
+    cu = [0] + list(np.cumsum(lens))
+    cu_t = torch.tensor(cu, dtype=torch.int32, device="cuda")
+    out, ob, lse = dbg.prefill_varlen_train(d["q"], d["k"], d["v"], d["lam"], cu_t, max(lens), window=W)
+    grads = dbg.backward_varlen(d["q"], d["k"], d["v"], d["lam"], ob, lse, dout.cuda(), cu_t, max(lens), window=W)
+    _clean(dbg)
+    ref = ora.prefill_backward_varlen(inp["q"], inp["k"], inp["v"], inp["lam"], dout, cu, window=W)
+    for gpu, r, name in zip(grads, ref, ("dq", "dk", "dv", "dlam")):
+        grad_close(gpu, r, f"debug packed window backward {name}")
+
+
 def test_decode_wait_that_expires_reports_and_leaves_the_gpu_usable(dbg):
     """A bounded wait that runs out: the debug build's test hook makes one decode CTA
     announce a ring stage and never copy it. Its consumer warps give up after the wait limit,

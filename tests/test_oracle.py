@@ -508,8 +508,34 @@ def pin_backward_window():
     return bool(ok)
 
 
+def pin_backward_varlen_window():
+    """Sliding-window gradients of packed sequences: central differences of
+    <dout, prefill_varlen(., window=2)> (including a key of the first sequence, which the second
+    never sees), and a window longer than every sequence reduces to the causal packed backward."""
+    q, k, v, lam = _rand_prefill(B=1, S=9, Hq=4, Hkv=2, D=3, seed=29)
+    q, k, v, lam = q[0], k[0], v[0], lam[0]
+    dout = np.random.default_rng(30).standard_normal((9, 2, 3))
+    cu = [0, 4, 9]
+    grads = ora.prefill_backward_varlen(q, k, v, lam, dout, cu, window=2)
+    f = lambda q_, k_, v_, l_: float(np.sum(ora.prefill_varlen(q_, k_, v_, l_, cu, window=2) * dout))
+    eps = 1e-6
+    ok = True
+    for which, idx in ((0, (8, 1, 2)), (1, (2, 1, 0)), (1, (7, 0, 1)), (2, (5, 0, 2)), (3, (3, 1))):
+        args = [q.copy(), k.copy(), v.copy(), lam.copy()]
+        args[which][idx] += eps
+        up = f(*args)
+        args[which][idx] -= 2 * eps
+        dn = f(*args)
+        ok &= abs((up - dn) / (2 * eps) - grads[which][idx]) < 1e-6
+    full = ora.prefill_backward_varlen(q, k, v, lam, dout, cu, window=5)
+    causal = ora.prefill_backward_varlen(q, k, v, lam, dout, cu)
+    ok &= all(np.allclose(a, b, atol=1e-13) for a, b in zip(full, causal))
+    return bool(ok)
+
+
 ALL_PINS = {
     "varlen_window_is_per_sequence_window": pin_varlen_window_is_per_sequence_window,
+    "backward_varlen_window": pin_backward_varlen_window,
     "softmax_library": pin_softmax_library,
     "lambda0_is_softmax_attention": pin_lambda0_is_softmax_attention,
     "lambda0_noncausal": lambda: pin_lambda0_is_softmax_attention(causal=False),

@@ -177,10 +177,16 @@ def _varlen_window_ignored(q, k, v, lam, cu_seqlens, causal=True, window=None):
 
 
 _VARLEN = ora.prefill_varlen
+_BWD_VARLEN = ora.prefill_backward_varlen
+
+
+def _backward_varlen_window_ignored(q, k, v, lam, dout, cu_seqlens, causal=True, window=None):
+    return _BWD_VARLEN(q, k, v, lam, dout, cu_seqlens, causal=causal)
 
 
 MUTANTS = {
     "varlen_window_ignored": ("prefill_varlen", _varlen_window_ignored),
+    "backward_varlen_window_ignored": ("prefill_backward_varlen", _backward_varlen_window_ignored),
     "plus_sign": ("diff_attention_block", _block_plus_sign),
     "no_scale": ("diff_attention_block", _block_no_scale),
     "scale_by_d": ("diff_attention_block", _block_scale_d),
