@@ -75,8 +75,8 @@ SPEC_HBM_GBS = 8000.0
 NCU_TRAFFIC = {
     # B=1 x 32768 causal prefill: 3445891328 read + 247948288 written
     ("prefill", "prefill_b1_s32768"): {"bytes": 3693839616, "source_sha": "7e51d88bae48ec3f"},
-    # B=8 x 131072 needle decode (split kernel with the fused merge): 4304263168 + 12806656
-    ("decode", "needle_decode_b8_s131072"): {"bytes": 4317069824, "source_sha": "07d184e353942e3c"},
+    # B=8 x 131072 needle decode (split kernel with the fused merge): 4304199168 + 12417280
+    ("decode", "needle_decode_b8_s131072"): {"bytes": 4316616448, "source_sha": "34be303ff93304f8"},
 }
 
 

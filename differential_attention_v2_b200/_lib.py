@@ -41,6 +41,7 @@ _SIGNATURES = {
     "diffattn_v2_backward_varlen_window": (_i, [_vp] * 12 + [_i] * 7 + [_vp, _sz, _vp]),
     "diffattn_v2_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "diffattn_v2_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "diffattn_v2_decode_window": (_i, [_vp] * 6 + [_i] * 6 + [_vp, _sz, _vp]),
     "diffattn_v2_decode_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
     "diffattn_v2_decode_paged": (_i, [_vp] * 7 + [_i] * 7 + [_vp, _sz, _vp]),
     "diffattn_v2_decode_multi_workspace_size": (_sz, [_i] * 6),
@@ -337,8 +338,9 @@ def decode_workspace_size(B, Smax, Hq, Hkv, D) -> int:
     return int(LIB.diffattn_v2_decode_workspace_size(B, Smax, Hq, Hkv, D))
 
 
-def decode(q, kcache, vcache, seqlens, lam, out=None, workspace=None, stream=None):
-    """bf16 decode step: q [B,Hq,D], caches [B,Smax,Hkv,D], seqlens int32 [B], lam fp32 [B,Hq/2]."""
+def decode(q, kcache, vcache, seqlens, lam, out=None, workspace=None, stream=None, window=None):
+    """bf16 decode step: q [B,Hq,D], caches [B,Smax,Hkv,D], seqlens int32 [B], lam fp32 [B,Hq/2].
+    With `window` the new token sees only its sequence's last `window` keys."""
     _need(q, "q", torch.bfloat16, 3)
     _need(kcache, "kcache", torch.bfloat16, 4)
     _need(vcache, "vcache", torch.bfloat16, 4)
@@ -352,6 +354,12 @@ def decode(q, kcache, vcache, seqlens, lam, out=None, workspace=None, stream=Non
     need = decode_workspace_size(B, Smax, Hq, Hkv, D)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if window is not None:
+        st = LIB.diffattn_v2_decode_window(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(lam), _ptr(out), B,
+                                           Smax, Hq, Hkv, D, int(window), _ptr(workspace),
+                                           workspace.numel() * workspace.element_size(), _stream(stream, q.device))
+        _check(st, "diffattn_v2_decode_window")
+        return out
     st = LIB.diffattn_v2_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(lam), _ptr(out), B, Smax,
                                 Hq, Hkv, D, _ptr(workspace), workspace.numel() * workspace.element_size(),
                                 _stream(stream, q.device))

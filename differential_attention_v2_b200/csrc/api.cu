@@ -537,10 +537,13 @@ size_t diffattn_v2_decode_workspace_size(int B, int Smax, int Hq, int Hkv, int D
   return da2::decode_workspace_bytes(B, 1, Hq, Hkv, D, nsplit);
 }
 
-int diffattn_v2_decode(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens,
-                       const float* lambda, void* out, int B, int Smax, int Hq, int Hkv, int D, void* workspace,
-                       size_t workspace_bytes, da2_stream_t stream) {
-  if (B < 0 || Smax <= 0 || D <= 0 || !heads_ok(Hq, Hkv)) return DA2_ERR_INVALID;
+namespace {
+
+// The bf16 decode over [B,Smax,Hkv,D] caches; window > 0: only the last `window` keys.
+int decode_bshd(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens, const float* lambda,
+                void* out, int B, int Smax, int Hq, int Hkv, int D, int window, void* workspace,
+                size_t workspace_bytes, da2_stream_t stream) {
+  if (B < 0 || Smax <= 0 || D <= 0 || !heads_ok(Hq, Hkv) || window < 0) return DA2_ERR_INVALID;
   if (B == 0) return DA2_OK;
   if (!q || !kcache || !vcache || !seqlens || !lambda || !out || !workspace) return DA2_ERR_INVALID;
   if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(seqlens) || !aligned16(lambda) ||
@@ -561,9 +564,26 @@ int diffattn_v2_decode(const void* q, const void* kcache, const void* vcache, co
   const da2::DecodeWorkspace ws = da2::decode_workspace_layout(workspace, B, 1, Hq, D, nsplit);
   e = da2::launch_decode(tk, tv, static_cast<const __nv_bfloat16*>(q), seqlens, lambda,
                          static_cast<__nv_bfloat16*>(out), ws.o, ws.ml, ws.counters, err, B, Smax, Hq, Hkv, nsplit,
-                         split_len,
-                         nullptr, 0, 0, 1, reinterpret_cast<cudaStream_t>(stream));
+                         split_len, nullptr, 0, 0, 1, reinterpret_cast<cudaStream_t>(stream), window);
   return status_of(e);
+}
+
+}  // namespace
+
+int diffattn_v2_decode(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens,
+                       const float* lambda, void* out, int B, int Smax, int Hq, int Hkv, int D, void* workspace,
+                       size_t workspace_bytes, da2_stream_t stream) {
+  return decode_bshd(q, kcache, vcache, seqlens, lambda, out, B, Smax, Hq, Hkv, D, 0, workspace, workspace_bytes,
+                     stream);
+}
+
+int diffattn_v2_decode_window(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens,
+                              const float* lambda, void* out, int B, int Smax, int Hq, int Hkv, int D, int window,
+                              void* workspace, size_t workspace_bytes, da2_stream_t stream) {
+  if (window < 1) return DA2_ERR_INVALID;
+  // a window of Smax or more keys sees every cached key
+  return decode_bshd(q, kcache, vcache, seqlens, lambda, out, B, Smax, Hq, Hkv, D, window >= Smax ? 0 : window,
+                     workspace, workspace_bytes, stream);
 }
 
 int diffattn_v2_decode_paged(const void* q, const void* kpages, const void* vpages, const int32_t* block_table,

@@ -72,6 +72,7 @@ struct Params {
   int* err;
   int B, Smax, Hq, Hkv, nsplit, split_len;
   int T;                    // new tokens per sequence (1: plain decode); T * group <= 16
+  int window;               // T == 1: the token sees only keys seqlen-window .. seqlen-1 (0: all)
   float scale_log2;
   // paged caches [num_pages, page_size, Hkv, D]: logical token t of sequence b is row
   // t % page_size of page block_table[b * max_pages + t / page_size]; null = [B, Smax] caches
@@ -141,7 +142,11 @@ diffattn_decode_split(const __grid_constant__ CUtensorMap tmK, const __grid_cons
   const int b = blockIdx.z;
   const int group = p.Hq / p.Hkv;
   const int seqlen = min(max(__ldg(p.seqlens + b), 0), p.Smax);
-  const int t0 = split * p.split_len;
+  // with a sliding window the visible keys start at lo; the splits then start at the stage
+  // boundary below it, so the keys before the window are never read
+  const int lo = p.window > 0 ? max(0, seqlen - p.window) : 0;
+  const int base = lo / kTok * kTok;
+  const int t0 = base + split * p.split_len;
   if (t0 >= seqlen) {  // uniform for the CTA: nothing to read
     if (split == 0) {
       // an empty sequence has no working split to merge it: its outputs are zero
@@ -302,7 +307,7 @@ diffattn_decode_split(const __grid_constant__ CUtensorMap tmK, const __grid_cons
         // seqlen - T + token + 1 (causal among the new tokens)
         const int col_tok = (8 * nt + 2 * tq) / group;
         const int lim = col_tok < p.T ? min(t1, seqlen - p.T + col_tok + 1) : t1;
-        const bool va = tok_a < lim, vb_ = tok_b < lim;
+        const bool va = tok_a < lim && tok_a >= lo, vb_ = tok_b < lim && tok_b >= lo;
         float x[4];
         x[0] = va ? sacc[nt][0] * p.scale_log2 : -INFINITY;
         x[1] = va ? sacc[nt][1] * p.scale_log2 : -INFINITY;
@@ -421,7 +426,7 @@ diffattn_decode_split(const __grid_constant__ CUtensorMap tmK, const __grid_cons
   __threadfence();
   __syncthreads();
   volatile int* last_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
-  const int ns = (seqlen + p.split_len - 1) / p.split_len;  // working splits of sequence b
+  const int ns = (seqlen - base + p.split_len - 1) / p.split_len;  // working splits of sequence b
   if (threadIdx.x == 0)
     *last_flag = (checked(b < p.B && g < p.Hkv && ns <= p.nsplit, p.err) &&
                   atomicAdd(p.counters + static_cast<size_t>(b) * p.Hkv + g, 1) == ns - 1) ? 1 : 0;
@@ -445,7 +450,7 @@ cudaError_t launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const 
                           const int32_t* seqlens, const float* lambda, __nv_bfloat16* out, float* ws_o,
                           float* ws_ml, int* counters, int* err, int B, int Smax, int Hq, int Hkv, int nsplit,
                           int split_len, const int32_t* block_table, int max_pages, int page_shift, int T,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, int window) {
   using namespace decode;
   Params p;
   p.q = q;
@@ -464,6 +469,7 @@ cudaError_t launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const 
   p.split_len = split_len;
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HD));
   p.T = T;
+  p.window = window;
   p.block_table = block_table;
   p.max_pages = max_pages;
   p.page_shift = page_shift;

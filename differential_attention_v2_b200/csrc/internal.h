@@ -54,7 +54,7 @@ cudaError_t launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const 
                           const int32_t* seqlens, const float* lambda, __nv_bfloat16* out, float* ws_o,
                           float* ws_ml, int* counters, int* err, int B, int Smax, int Hq, int Hkv, int nsplit,
                           int split_len, const int32_t* block_table, int max_pages, int page_shift, int T,
-                          cudaStream_t stream);
+                          cudaStream_t stream, int window = 0);
 
 // Tokens per split and number of splits of the bf16 decode for these sizes.
 void decode_split_plan(int B, int Smax, int Hkv, int* split_len, int* nsplit);

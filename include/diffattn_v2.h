@@ -277,6 +277,20 @@ DA2_API int diffattn_v2_decode(const void* q, const void* kcache, const void* vc
                        da2_stream_t stream);
 
 /*
+ * bf16 decode step of a sliding-window layer: as diffattn_v2_decode, but sequence b's new
+ * token sees only its last `window` keys, [max(0, seqlens[b]-window), seqlens[b]) (the mask of
+ * the "Attention variants" lesson's sliding-window step, for the hybrid layers of the
+ * "Differential Attention (V2)" lesson's "Use it" section). The splits start at the 64-token
+ * boundary below the window, so keys before it are not read. Same layouts, workspace size
+ * (diffattn_v2_decode_workspace_size) and checks as diffattn_v2_decode, plus
+ * DA2_ERR_INVALID for window < 1; window >= Smax is the plain decode.
+ */
+DA2_API int diffattn_v2_decode_window(const void* q, const void* kcache, const void* vcache,
+                                      const int32_t* seqlens, const float* lambda, void* out, int B, int Smax,
+                                      int Hq, int Hkv, int D, int window, void* workspace,
+                                      size_t workspace_bytes, da2_stream_t stream);
+
+/*
  * The bf16 decode step over a paged KV cache (the layout serving engines keep): the caches
  * are pages of page_size tokens, and logical token t of sequence b is row t % page_size of
  * page block_table[b * max_pages + t / page_size].

@@ -311,11 +311,13 @@ def prefill_rows(q, k, v, lam, rows, causal: bool = True) -> np.ndarray:
     return np.stack(res) if res else np.zeros((0, q.shape[3]))
 
 
-def decode(q, kcache, vcache, seqlens, lam) -> np.ndarray:
+def decode(q, kcache, vcache, seqlens, lam, window=None) -> np.ndarray:
     """One decode step: out[B, Hq/2, D] in float64.
 
     q [B,Hq,D] is the new token's query; the caches [B,Smax,Hkv,D] already hold its key and
-    value, and sequence b attends to keys [0, seqlens[b]). lam [B,Hq/2]. A sequence with
+    value, and sequence b attends to keys [0, seqlens[b]), or with `window` to its last
+    `window` keys [max(0, seqlens[b]-window), seqlens[b]) (the sliding window of the
+    "Attention variants" lesson for the newest query). lam [B,Hq/2]. A sequence with
     seqlens[b] == 0 has no visible key; its output is defined as 0.
     """
     B, Hq, D = q.shape
@@ -325,16 +327,17 @@ def decode(q, kcache, vcache, seqlens, lam) -> np.ndarray:
         n = int(seqlens[b])
         if n <= 0:
             continue
+        n0 = max(0, n - int(window)) if window is not None else 0
         for g in range(Hkv):
-            kk = _f64(kcache[b, :n, g])
-            vv = _f64(vcache[b, :n, g])
+            kk = _f64(kcache[b, n0:n, g])
+            vv = _f64(vcache[b, n0:n, g])
             for p, h1, h2, gg in pair_layout(Hq, Hkv):
                 if gg != g:
                     continue
                 q1 = _f64(q[b, h1])[None, :]
                 q2 = _f64(q[b, h2])[None, :]
                 lm = np.array([float(lam[b, p])], dtype=np.float64)
-                out[b, p] = diff_attention_block(q1, q2, kk, vv, lm, np.zeros((1, n)))[0]
+                out[b, p] = diff_attention_block(q1, q2, kk, vv, lm, np.zeros((1, n - n0)))[0]
     return out
 
 

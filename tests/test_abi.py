@@ -148,6 +148,15 @@ def test_decode_workspace_size(lib):
     assert da.decode_workspace_size(64, 65536, 64, 8, 128) >= ws
 
 
+def test_decode_window_host_checks(lib):
+    W = P + 32768
+    f = lib.diffattn_v2_decode_window
+    assert f(Q, K, V, L, L, O, 2, 256, 8, 2, 128, 0, W, 1 << 30, None) == -1      # window 0
+    assert f(Q, K, V, L, L, O, 2, 256, 8, 2, 128, 16, W, 0, None) == -1           # workspace too small
+    assert f(Q, K, V, L, L, O, 2, 256, 8, 2, 64, 16, W, 1 << 30, None) == -2      # D = 64
+    assert f(Q, K, V, L, L, O, 0, 256, 8, 2, 128, 16, W, 1 << 30, None) == 0      # B = 0
+
+
 def test_decode_host_checks(lib):
     ws = lib.diffattn_v2_decode_workspace_size(2, 1024, 16, 2, 128)
     S = P + 24576

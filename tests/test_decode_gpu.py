@@ -50,6 +50,25 @@ def test_decode_bf16_matches_oracle(da, B, Smax, Hq, Hkv, lens):
             assert torch.count_nonzero(out[b]).item() == 0
 
 
+@pytest.mark.parametrize("B,Smax,Hq,Hkv,lens,window", [
+    (4, 3000, 64, 8, [3000, 1, 0, 2100], 1),         # only the newest key; an empty sequence
+    (4, 3000, 64, 8, [3000, 130, 64, 2100], 64),     # window of one stage, lengths at stage edges
+    (3, 5000, 32, 2, [5000, 4097, 700], 700),        # group of 16, window starting mid-stage
+    (2, 9000, 16, 4, [9000, 1500], 4096),            # a window spanning several splits
+    (3, 800, 16, 2, [800, 100, 799], 5000),          # window wider than every sequence
+])
+def test_decode_window_matches_oracle(da, B, Smax, Hq, Hkv, lens, window):
+    inp = _decode_case(B, Smax, Hq, Hkv, lens, seed=40 + window)
+    out = da.decode(inp["q"].cuda(), inp["kcache"].cuda(), inp["vcache"].cuda(), inp["seqlens"].cuda(),
+                    inp["lam"].cuda(), window=window)
+    assert da.device_error() == 0
+    ref = ora.decode(inp["q"], inp["kcache"], inp["vcache"], inp["seqlens"], inp["lam"], window=window)
+    bf16_close(out, ref, f"decode window={window} lens={lens}")
+    if window >= max(lens):
+        # the same splits as the plain decode: bit-identical
+        assert torch.equal(out, _run(da, inp))
+
+
 def test_decode_matches_last_prefill_row(da):
     """One decode step over n cached keys equals row n-1 of a prefill of length n."""
     case = workloads.PrefillCase(B=1, S=333, Hq=16, Hkv=2, D=128, seed=21)

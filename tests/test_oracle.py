@@ -165,6 +165,27 @@ def pin_decode_is_last_prefill_row():
     return bool(ok)
 
 
+def pin_decode_window_is_last_window_prefill_row():
+    """A windowed decode step over n cached keys equals row n-1 of a windowed prefill of length
+    n (windows 1, 5 and one longer than the sequence), and brute-force decode over the last
+    `window` keys alone."""
+    B, S, Hq, Hkv, D = 2, 21, 8, 2, 8
+    q, k, v, lam = _rand_prefill(B=B, S=S, Hq=Hq, Hkv=Hkv, D=D, seed=31)
+    seqlens = np.array([S, 13])
+    qd = np.stack([q[0, S - 1], q[1, 12]])
+    lamd = np.stack([lam[0, S - 1], lam[1, 12]])
+    ok = True
+    for w in (1, 5, 40):
+        dec = ora.decode(qd, k, v, seqlens, lamd, window=w)
+        ok &= np.allclose(dec[0], ora.prefill(q, k, v, lam, window=w)[0, S - 1], atol=1e-13)
+        ok &= np.allclose(dec[1], ora.prefill(q[1:, :13], k[1:, :13], v[1:, :13], lam[1:, :13], window=w)[0, 12],
+                          atol=1e-13)
+    n0 = 13 - 5
+    ref = np.array(brute.decode(qd[1:].tolist(), k[1:, n0:13].tolist(), v[1:, n0:13].tolist(), [5], lamd[1:].tolist()))
+    ok &= np.allclose(ora.decode(qd, k, v, seqlens, lamd, window=5)[1], ref[0], atol=1e-12)
+    return bool(ok)
+
+
 def pin_prefill_rows_match_full():
     q, k, v, lam = _rand_prefill(seed=10)
     full = ora.prefill(q, k, v, lam)
@@ -534,6 +555,7 @@ def pin_backward_varlen_window():
 
 
 ALL_PINS = {
+    "decode_window_is_last_window_prefill_row": pin_decode_window_is_last_window_prefill_row,
     "varlen_window_is_per_sequence_window": pin_varlen_window_is_per_sequence_window,
     "backward_varlen_window": pin_backward_varlen_window,
     "softmax_library": pin_softmax_library,

@@ -178,6 +178,11 @@ def _varlen_window_ignored(q, k, v, lam, cu_seqlens, causal=True, window=None):
 
 _VARLEN = ora.prefill_varlen
 _BWD_VARLEN = ora.prefill_backward_varlen
+_DECODE = ora.decode
+
+
+def _decode_window_off_by_one(q, kcache, vcache, seqlens, lam, window=None):
+    return _DECODE(q, kcache, vcache, seqlens, lam, window=None if window is None else window + 1)
 
 
 def _backward_varlen_window_ignored(q, k, v, lam, dout, cu_seqlens, causal=True, window=None):
@@ -186,6 +191,7 @@ def _backward_varlen_window_ignored(q, k, v, lam, dout, cu_seqlens, causal=True,
 
 MUTANTS = {
     "varlen_window_ignored": ("prefill_varlen", _varlen_window_ignored),
+    "decode_window_off_by_one": ("decode", _decode_window_off_by_one),
     "backward_varlen_window_ignored": ("prefill_backward_varlen", _backward_varlen_window_ignored),
     "plus_sign": ("diff_attention_block", _block_plus_sign),
     "no_scale": ("diff_attention_block", _block_no_scale),
