@@ -44,6 +44,7 @@ _SIGNATURES = {
     "diffattn_v2_decode_window": (_i, [_vp] * 6 + [_i] * 6 + [_vp, _sz, _vp]),
     "diffattn_v2_decode_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
     "diffattn_v2_decode_paged": (_i, [_vp] * 7 + [_i] * 7 + [_vp, _sz, _vp]),
+    "diffattn_v2_decode_paged_window": (_i, [_vp] * 7 + [_i] * 8 + [_vp, _sz, _vp]),
     "diffattn_v2_decode_multi_workspace_size": (_sz, [_i] * 6),
     "diffattn_v2_decode_multi": (_i, [_vp] * 6 + [_i] * 6 + [_vp, _sz, _vp]),
     "diffattn_v2_lambda_v1": (_i, [_vp, _vp, _vp, _vp, _f, _i, _i, _i, _vp, _vp]),
@@ -390,9 +391,10 @@ def decode_multi(q, kcache, vcache, seqlens, lam, out=None, workspace=None, stre
     return out
 
 
-def decode_paged(q, kpages, vpages, block_table, seqlens, lam, out=None, workspace=None, stream=None):
+def decode_paged(q, kpages, vpages, block_table, seqlens, lam, out=None, workspace=None, stream=None, window=None):
     """bf16 decode over a paged cache: kpages/vpages [num_pages, page_size, Hkv, D],
-    block_table int32 [B, max_pages], seqlens int32 [B], lam fp32 [B, Hq/2]."""
+    block_table int32 [B, max_pages], seqlens int32 [B], lam fp32 [B, Hq/2]. With `window`
+    the new token sees only its sequence's last `window` keys."""
     _need(q, "q", torch.bfloat16, 3)
     _need(kpages, "kpages", torch.bfloat16, 4)
     _need(vpages, "vpages", torch.bfloat16, 4)
@@ -408,6 +410,13 @@ def decode_paged(q, kpages, vpages, block_table, seqlens, lam, out=None, workspa
     need = decode_workspace_size(B, max_pages * page_size, Hq, Hkv, D)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if window is not None:
+        st = LIB.diffattn_v2_decode_paged_window(_ptr(q), _ptr(kpages), _ptr(vpages), _ptr(block_table), _ptr(seqlens),
+                                                 _ptr(lam), _ptr(out), B, max_pages, page_size, num_pages, Hq, Hkv, D,
+                                                 int(window), _ptr(workspace),
+                                                 workspace.numel() * workspace.element_size(), _stream(stream, q.device))
+        _check(st, "diffattn_v2_decode_paged_window")
+        return out
     st = LIB.diffattn_v2_decode_paged(_ptr(q), _ptr(kpages), _ptr(vpages), _ptr(block_table), _ptr(seqlens), _ptr(lam),
                                       _ptr(out), B, max_pages, page_size, num_pages, Hq, Hkv, D, _ptr(workspace),
                                       workspace.numel() * workspace.element_size(), _stream(stream, q.device))

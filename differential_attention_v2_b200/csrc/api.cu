@@ -586,11 +586,14 @@ int diffattn_v2_decode_window(const void* q, const void* kcache, const void* vca
                      workspace, workspace_bytes, stream);
 }
 
-int diffattn_v2_decode_paged(const void* q, const void* kpages, const void* vpages, const int32_t* block_table,
-                             const int32_t* seqlens, const float* lambda, void* out, int B, int max_pages,
-                             int page_size, int num_pages, int Hq, int Hkv, int D, void* workspace,
-                             size_t workspace_bytes, da2_stream_t stream) {
-  if (B < 0 || max_pages <= 0 || num_pages <= 0 || D <= 0 || !heads_ok(Hq, Hkv)) return DA2_ERR_INVALID;
+namespace {
+
+// The bf16 decode over a paged cache; window > 0: only the last `window` keys.
+int decode_paged(const void* q, const void* kpages, const void* vpages, const int32_t* block_table,
+                 const int32_t* seqlens, const float* lambda, void* out, int B, int max_pages, int page_size,
+                 int num_pages, int Hq, int Hkv, int D, int window, void* workspace, size_t workspace_bytes,
+                 da2_stream_t stream) {
+  if (B < 0 || max_pages <= 0 || num_pages <= 0 || D <= 0 || !heads_ok(Hq, Hkv) || window < 0) return DA2_ERR_INVALID;
   if (page_size < 8 || page_size > 4096 || (page_size & (page_size - 1)) != 0) return DA2_ERR_INVALID;
   if (static_cast<long long>(max_pages) * page_size > (1LL << 30)) return DA2_ERR_INVALID;
   if (B == 0) return DA2_OK;
@@ -617,9 +620,29 @@ int diffattn_v2_decode_paged(const void* q, const void* kpages, const void* vpag
   const da2::DecodeWorkspace ws = da2::decode_workspace_layout(workspace, B, 1, Hq, D, nsplit);
   e = da2::launch_decode(tk, tv, static_cast<const __nv_bfloat16*>(q), seqlens, lambda,
                          static_cast<__nv_bfloat16*>(out), ws.o, ws.ml, ws.counters, err, B, Smax, Hq, Hkv, nsplit,
-                         split_len,
-                         block_table, max_pages, page_shift, 1, reinterpret_cast<cudaStream_t>(stream));
+                         split_len, block_table, max_pages, page_shift, 1, reinterpret_cast<cudaStream_t>(stream),
+                         window >= Smax ? 0 : window);
   return status_of(e);
+}
+
+}  // namespace
+
+int diffattn_v2_decode_paged(const void* q, const void* kpages, const void* vpages, const int32_t* block_table,
+                             const int32_t* seqlens, const float* lambda, void* out, int B, int max_pages,
+                             int page_size, int num_pages, int Hq, int Hkv, int D, void* workspace,
+                             size_t workspace_bytes, da2_stream_t stream) {
+  return decode_paged(q, kpages, vpages, block_table, seqlens, lambda, out, B, max_pages, page_size, num_pages, Hq,
+                      Hkv, D, 0, workspace, workspace_bytes, stream);
+}
+
+int diffattn_v2_decode_paged_window(const void* q, const void* kpages, const void* vpages,
+                                    const int32_t* block_table, const int32_t* seqlens, const float* lambda,
+                                    void* out, int B, int max_pages, int page_size, int num_pages, int Hq, int Hkv,
+                                    int D, int window, void* workspace, size_t workspace_bytes,
+                                    da2_stream_t stream) {
+  if (window < 1) return DA2_ERR_INVALID;
+  return decode_paged(q, kpages, vpages, block_table, seqlens, lambda, out, B, max_pages, page_size, num_pages, Hq,
+                      Hkv, D, window, workspace, workspace_bytes, stream);
 }
 
 size_t diffattn_v2_decode_multi_workspace_size(int B, int T, int Smax, int Hq, int Hkv, int D) {

@@ -291,6 +291,18 @@ DA2_API int diffattn_v2_decode_window(const void* q, const void* kcache, const v
                                       size_t workspace_bytes, da2_stream_t stream);
 
 /*
+ * The sliding-window decode step over a paged cache: diffattn_v2_decode_paged's layouts with
+ * diffattn_v2_decode_window's mask. Block-table entries of pages that hold only keys before
+ * a sequence's window are not read (a serving engine may already have released them).
+ * Checks as diffattn_v2_decode_paged, plus DA2_ERR_INVALID for window < 1.
+ */
+DA2_API int diffattn_v2_decode_paged_window(const void* q, const void* kpages, const void* vpages,
+                                            const int32_t* block_table, const int32_t* seqlens,
+                                            const float* lambda, void* out, int B, int max_pages, int page_size,
+                                            int num_pages, int Hq, int Hkv, int D, int window, void* workspace,
+                                            size_t workspace_bytes, da2_stream_t stream);
+
+/*
  * The bf16 decode step over a paged KV cache (the layout serving engines keep): the caches
  * are pages of page_size tokens, and logical token t of sequence b is row t % page_size of
  * page block_table[b * max_pages + t / page_size].

@@ -341,10 +341,11 @@ def decode(q, kcache, vcache, seqlens, lam, window=None) -> np.ndarray:
     return out
 
 
-def decode_paged(q, kpages, vpages, block_table, seqlens, lam) -> np.ndarray:
+def decode_paged(q, kpages, vpages, block_table, seqlens, lam, window=None) -> np.ndarray:
     """Decode step over a paged cache: kpages/vpages [P, page_size, Hkv, D]; logical token t
     of sequence b lives in page block_table[b][t // page_size] at row t % page_size. The
-    sequence's logical cache is gathered page by page, then `decode` applies as written."""
+    sequence's logical cache is gathered page by page, then `decode` (with `window`) applies
+    as written."""
     page_size = int(kpages.shape[1])
     B = q.shape[0]
     outs = []
@@ -354,7 +355,7 @@ def decode_paged(q, kpages, vpages, block_table, seqlens, lam) -> np.ndarray:
         pages = [int(block_table[b][i]) for i in range(n_pages)]
         kc = np.concatenate([_f64(kpages[pg]) for pg in pages], axis=0)[:n] if n else np.zeros((0,) + tuple(kpages.shape[2:]))
         vc = np.concatenate([_f64(vpages[pg]) for pg in pages], axis=0)[:n] if n else np.zeros((0,) + tuple(vpages.shape[2:]))
-        outs.append(decode(q[b:b + 1], kc[None], vc[None], [n], lam[b:b + 1])[0])
+        outs.append(decode(q[b:b + 1], kc[None], vc[None], [n], lam[b:b + 1], window=window)[0])
     return np.stack(outs)
 
 

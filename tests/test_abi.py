@@ -157,6 +157,15 @@ def test_decode_window_host_checks(lib):
     assert f(Q, K, V, L, L, O, 0, 256, 8, 2, 128, 16, W, 1 << 30, None) == 0      # B = 0
 
 
+def test_decode_paged_window_host_checks(lib):
+    W, T = P + 32768, P + 36864
+    f = lib.diffattn_v2_decode_paged_window
+    assert f(Q, K, V, T, L, L, O, 2, 8, 64, 16, 8, 2, 128, 0, W, 1 << 30, None) == -1      # window 0
+    assert f(Q, K, V, T, L, L, O, 2, 8, 12, 16, 8, 2, 128, 16, W, 1 << 30, None) == -1     # page size not 2^k
+    assert f(Q, K, V, T, L, L, O, 2, 8, 64, 16, 8, 2, 64, 16, W, 1 << 30, None) == -2      # D = 64
+    assert f(Q, K, V, T, L, L, O, 0, 8, 64, 16, 8, 2, 128, 16, W, 1 << 30, None) == 0      # B = 0
+
+
 def test_decode_host_checks(lib):
     ws = lib.diffattn_v2_decode_workspace_size(2, 1024, 16, 2, 128)
     S = P + 24576

@@ -69,6 +69,30 @@ def test_decode_window_matches_oracle(da, B, Smax, Hq, Hkv, lens, window):
         assert torch.equal(out, _run(da, inp))
 
 
+@pytest.mark.parametrize("page_size,window", [(16, 100), (64, 64), (256, 700)])
+def test_decode_paged_window_matches_contiguous(da, page_size, window):
+    """The windowed decode over a shuffled paged copy of the cache: parity with the oracle and
+    bit-identity with the contiguous windowed decode (same Smax, same splits)."""
+    B, Smax, Hq, Hkv = 3, 2048, 32, 4
+    lens = [2048, 700, 90]
+    inp = _decode_case(B, Smax, Hq, Hkv, lens, seed=60 + page_size)
+    n_pg = Smax // page_size
+    g = torch.Generator().manual_seed(61)
+    perm = torch.randperm(B * n_pg, generator=g)
+    kp = torch.empty(B * n_pg, page_size, Hkv, 128, dtype=torch.bfloat16)
+    vp = torch.empty_like(kp)
+    kp[perm] = inp["kcache"].reshape(B * n_pg, page_size, Hkv, 128)
+    vp[perm] = inp["vcache"].reshape(B * n_pg, page_size, Hkv, 128)
+    table = perm.view(B, n_pg).to(torch.int32)
+    d = {k: inp[k].cuda() for k in ("q", "kcache", "vcache", "seqlens", "lam")}
+    out = da.decode_paged(d["q"], kp.cuda(), vp.cuda(), table.cuda(), d["seqlens"], d["lam"], window=window)
+    assert da.device_error() == 0
+    ref = ora.decode_paged(inp["q"], kp, vp, table.tolist(), inp["seqlens"], inp["lam"], window=window)
+    bf16_close(out, ref, f"paged decode window={window} page_size={page_size}")
+    contiguous = da.decode(d["q"], d["kcache"], d["vcache"], d["seqlens"], d["lam"], window=window)
+    assert torch.equal(out, contiguous)
+
+
 def test_decode_matches_last_prefill_row(da):
     """One decode step over n cached keys equals row n-1 of a prefill of length n."""
     case = workloads.PrefillCase(B=1, S=333, Hq=16, Hkv=2, D=128, seed=21)

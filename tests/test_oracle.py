@@ -376,6 +376,32 @@ def pin_paged_decode_gathers_pages():
     return bool(ok)
 
 
+def pin_paged_window_decode_gathers_pages():
+    """The windowed decode over a paged cache equals the brute force over the last `window`
+    keys of the gathered cache."""
+    rng = np.random.default_rng(32)
+    B, Hq, Hkv, D, ps = 2, 8, 2, 6, 4
+    lens = [11, 3]
+    n_pages = 8
+    kp = rng.standard_normal((n_pages, ps, Hkv, D))
+    vp = rng.standard_normal((n_pages, ps, Hkv, D))
+    perm = rng.permutation(n_pages)
+    table = [perm[0:3].tolist(), perm[3:4].tolist() + [0, 0]]
+    q = rng.standard_normal((B, Hq, D))
+    lam = rng.uniform(-1, 2, size=(B, Hq // 2))
+    ok = True
+    for w in (1, 5):
+        out = ora.decode_paged(q, kp, vp, table, lens, lam, window=w)
+        for b in range(B):
+            n = lens[b]
+            n0 = max(0, n - w)
+            kc = np.concatenate([kp[pg] for pg in table[b]], axis=0)[None, n0:n]
+            vc = np.concatenate([vp[pg] for pg in table[b]], axis=0)[None, n0:n]
+            ref = np.array(brute.decode(q[b:b + 1].tolist(), kc.tolist(), vc.tolist(), [n - n0], lam[b:b + 1].tolist()))
+            ok &= np.allclose(out[b], ref[0], atol=1e-12)
+    return bool(ok)
+
+
 def pin_lambda_v2_projection():
     """sigmoid(x W + b): W = 0 gives sigmoid(b) (0.5 without bias, 0.75 for b = ln 3); one
     nonzero weight gives sigmoid(x_k w_k); random inputs match torch.sigmoid(x @ W + b)."""
@@ -555,6 +581,7 @@ def pin_backward_varlen_window():
 
 
 ALL_PINS = {
+    "paged_window_decode_gathers_pages": pin_paged_window_decode_gathers_pages,
     "decode_window_is_last_window_prefill_row": pin_decode_window_is_last_window_prefill_row,
     "varlen_window_is_per_sequence_window": pin_varlen_window_is_per_sequence_window,
     "backward_varlen_window": pin_backward_varlen_window,
