@@ -764,6 +764,23 @@ def run_workload(args):
         val = flops / (ms * 1e-3) / 1e12
         unit, peak, bound = "TFLOP/s", peaks["bf16_tflops"], "tensor"
         launches = 1
+    elif name == "decode_window":
+        # the needle decode's caches (B=8 x 131072) read through a 4096-key window: bytes = the
+        # window's K and V rows, plus q, lambda and out
+        case = workloads.CONFIGS["needle_decode_b8_s131072"]
+        inp = workloads.make_decode(case)
+        kc, vc, sl, q = (inp[x].to(dev) for x in ("kcache", "vcache", "seqlens", "q"))
+        lam = da.lambda_v1(*(inp[x].to(dev) for x in ("lq1", "lk1", "lq2", "lk2")), inp["lambda_init"], rows=case.B)
+        W = 4096
+        out = torch.empty(case.B, case.Hq // 2, D, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(da.decode_workspace_size(case.B, case.Smax, case.Hq, case.Hkv, D), dtype=torch.uint8, device=dev)
+        fn = lambda: da.decode(q, kc, vc, sl, lam, out=out, workspace=ws, window=W)
+        nbytes = workloads.decode_bytes([min(int(n), W) for n in inp["seqlens"].tolist()], case.Hkv, D, case.Hq)
+        ms, how = _time_op(fn, args.steps, args.warmup, stream)
+        val = nbytes / (ms * 1e-3) / 1e9
+        unit, peak, bound = "GB/s", peaks["hbm_gbs"], "hbm"
+        launches = 1
+        cfg = {"workload": "sliding-window decode (window 4096) of B=8 sequences of 131072 cached tokens, Hq=64 Hkv=8"}
     elif name in ("decode", "decode_needle", "paged", "multi"):
         case = workloads.CONFIGS["needle_decode_b8_s131072"] if name == "decode_needle" else workloads.CONFIGS["decode_b64_s8192"]
         inp = workloads.make_decode(case)
@@ -939,7 +956,8 @@ def main(argv=None):
                     help="skip the second prefill and decode workloads (B=4 x 4k prefill, B=64 decode)")
     ap.add_argument("--ref-seconds", type=float, default=120.0,
                     help="host-time budget of the whole reference run (warm-up and timed steps)")
-    ap.add_argument("--workload", choices=("prefill", "decode", "prefill_long", "decode_needle", "window", "varlen",
+    ap.add_argument("--workload", choices=("prefill", "decode", "prefill_long", "decode_needle", "decode_window",
+                                           "window", "varlen",
                                            "paged", "multi", "prefill_fused_lambda",
                                            "lambda_v2", "backward", "backward_varlen", "backward_window"),
                     default=None,
