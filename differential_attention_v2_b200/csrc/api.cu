@@ -93,6 +93,20 @@ DecodeWorkspace decode_workspace_layout(void* base, int B, int T, int Hq, int D,
   return w;
 }
 
+// With a sliding window only the last window (+ up to one stage before it) is read: plan the
+// splits over that span when this gives no more splits than the plan for Smax, for which the
+// caller's workspace is sized.
+void decode_split_plan_window(int B, int Smax, int Hkv, int window, int* split_len, int* nsplit) {
+  decode_split_plan(B, Smax, Hkv, split_len, nsplit);
+  if (window <= 0 || window + 64 >= Smax) return;
+  int L = 0, n = 0;
+  decode_split_plan(B, window + 64, Hkv, &L, &n);
+  if (n <= *nsplit) {
+    *split_len = L;
+    *nsplit = n;
+  }
+}
+
 void decode_split_plan(int B, int Smax, int Hkv, int* split_len, int* nsplit) {
   // Aim for about 8 waves of 2 CTAs per SM over the (b, g) units, with splits that are a
   // multiple of the 64-token stage and between 512 and 4096 tokens long.
@@ -557,7 +571,7 @@ int decode_bshd(const void* q, const void* kcache, const void* vcache, const int
   cudaError_t e = device_error_ptr(&err);
   if (e != cudaSuccess) return DA2_ERR_CUDA;
   int split_len = 0, nsplit = 0;
-  da2::decode_split_plan(B, Smax, Hkv, &split_len, &nsplit);
+  da2::decode_split_plan_window(B, Smax, Hkv, window, &split_len, &nsplit);
   CUtensorMap tk, tv;
   if (encode_bshd(&tk, kcache, D, Hkv, Smax, B, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
   if (encode_bshd(&tv, vcache, D, Hkv, Smax, B, 64, 64) != cudaSuccess) return DA2_ERR_CUDA;
@@ -609,8 +623,9 @@ int decode_paged(const void* q, const void* kpages, const void* vpages, const in
   int* err = nullptr;
   cudaError_t e = device_error_ptr(&err);
   if (e != cudaSuccess) return DA2_ERR_CUDA;
+  if (window >= Smax) window = 0;
   int split_len = 0, nsplit = 0;
-  da2::decode_split_plan(B, Smax, Hkv, &split_len, &nsplit);
+  da2::decode_split_plan_window(B, Smax, Hkv, window, &split_len, &nsplit);
   int page_shift = 0;
   while ((1 << page_shift) < page_size) ++page_shift;
   const uint32_t box = static_cast<uint32_t>(page_size < 64 ? page_size : 64);
@@ -621,7 +636,7 @@ int decode_paged(const void* q, const void* kpages, const void* vpages, const in
   e = da2::launch_decode(tk, tv, static_cast<const __nv_bfloat16*>(q), seqlens, lambda,
                          static_cast<__nv_bfloat16*>(out), ws.o, ws.ml, ws.counters, err, B, Smax, Hq, Hkv, nsplit,
                          split_len, block_table, max_pages, page_shift, 1, reinterpret_cast<cudaStream_t>(stream),
-                         window >= Smax ? 0 : window);
+                         window);
   return status_of(e);
 }
 

@@ -58,6 +58,9 @@ cudaError_t launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const 
 
 // Tokens per split and number of splits of the bf16 decode for these sizes.
 void decode_split_plan(int B, int Smax, int Hkv, int* split_len, int* nsplit);
+// The same for a sliding-window decode (window > 0): splits over the window's span when that
+// needs no more splits than the plan for Smax (the workspace is sized by that plan).
+void decode_split_plan_window(int B, int Smax, int Hkv, int window, int* split_len, int* nsplit);
 
 // The bf16 decode's workspace, in this order: fp32 partial outputs O [rows, D], fp32 (m, l)
 // [rows, 2], then one int split counter per (b, KV head), padded to 16 bytes; rows =

@@ -281,7 +281,8 @@ DA2_API int diffattn_v2_decode(const void* q, const void* kcache, const void* vc
  * token sees only its last `window` keys, [max(0, seqlens[b]-window), seqlens[b]) (the mask of
  * the "Attention variants" lesson's sliding-window step, for the hybrid layers of the
  * "Differential Attention (V2)" lesson's "Use it" section). The splits start at the 64-token
- * boundary below the window, so keys before it are not read. Same layouts, workspace size
+ * boundary below the window, so keys before it are not read, and are planned over the
+ * window's span when that needs no more of them than the plain decode. Same layouts, workspace size
  * (diffattn_v2_decode_workspace_size) and checks as diffattn_v2_decode, plus
  * DA2_ERR_INVALID for window < 1; window >= Smax is the plain decode.
  */

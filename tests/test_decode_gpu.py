@@ -64,8 +64,8 @@ def test_decode_window_matches_oracle(da, B, Smax, Hq, Hkv, lens, window):
     assert da.device_error() == 0
     ref = ora.decode(inp["q"], inp["kcache"], inp["vcache"], inp["seqlens"], inp["lam"], window=window)
     bf16_close(out, ref, f"decode window={window} lens={lens}")
-    if window >= max(lens):
-        # the same splits as the plain decode: bit-identical
+    if window >= Smax:
+        # the plain decode, bit for bit
         assert torch.equal(out, _run(da, inp))
 
 
