@@ -73,10 +73,10 @@ SPEC_HBM_GBS = 8000.0
 # one launch), keyed by workload and by the kernel source it was taken on; reported as null
 # once the source differs from the one captured.
 NCU_TRAFFIC = {
-    # B=1 x 32768 causal prefill: 3445891328 read + 247948288 written
-    ("prefill", "prefill_b1_s32768"): {"bytes": 3693839616, "source_sha": "7e51d88bae48ec3f"},
-    # B=8 x 131072 needle decode (split kernel with the fused merge): 4304199168 + 12417280
-    ("decode", "needle_decode_b8_s131072"): {"bytes": 4316616448, "source_sha": "34be303ff93304f8"},
+    # B=1 x 32768 causal prefill: 3469007104 read + 247027712 written
+    ("prefill", "prefill_b1_s32768"): {"bytes": 3716034816, "source_sha": "9162a0e0f5575922"},
+    # B=8 x 131072 needle decode (split kernel with the fused merge): 4304199936 + 12690688
+    ("decode", "needle_decode_b8_s131072"): {"bytes": 4316890624, "source_sha": "ff96f9e2aabe4153"},
 }
 
 

@@ -4,14 +4,17 @@
 // pairing per "Differential Transformer V2 soll KI-Training stabiler machen", shared-KV
 // section): for the new token of sequence b and pair p (heads 2p, 2p+1, KV head g)
 //   out[b,p] = softmax(q1 K^T/sqrt(D)) V - lambda[b,p] softmax(q2 K^T/sqrt(D)) V
-// over the cached keys [0, seqlens[b]).
+// over the cached keys [0, seqlens[b]), or for a sliding-window layer over the last `window`
+// of them (the window of the "Attention variants" lesson's sliding-window step).
 //
 // Decode is bound by HBM bandwidth: every visible K/V row must be read once, and V2 reads
 // it once for BOTH branches and for every query head of the GQA group (the group's query
 // heads are all pairs that share KV head g). Design:
 //
-//  * Grid (split, g, b). A CTA streams keys [split*L, min((split+1)*L, seqlen)) of KV head
-//    g through a 3-stage shared-memory ring filled by TMA (64 tokens x 128 d of K and of V
+//  * Grid (split, g, b). A CTA streams keys [base + split*L, min(base + (split+1)*L, seqlen))
+//    of KV head g (base = 0, or with a window the 64-token stage boundary at or below its
+//    first key, so keys before the window are not read) through a 3-stage shared-memory
+//    ring filled by TMA (64 tokens x 128 d of K and of V
 //    per stage, 128-byte swizzled so ldmatrix reads are bank-conflict free). Two CTAs fit
 //    on an SM, so up to 6 stages (192 KB) per SM are in flight.
 //  * Four consumer warps each take 16 tokens of every stage and compute, on the legacy

@@ -1035,8 +1035,9 @@ cudaError_t launch_prefill(const CUtensorMap& tmQ, const CUtensorMap& tmK, const
   // The CTA-pair form runs when DA2_PREFILL_CTA_PAIR=1 is set in the environment, every KV head
   // has an even number of pairs (GQA group a multiple of 4), the persistent deal applies and
   // the caller passed the half-tile K map. It gives bit-identical results; on B200 it measured
-  // about 2% below the one-CTA form (what paces both is each branch's chain of softmax, PV
-  // and next score GEMM, not the number of MMA instructions), so one CTA per item is the
+  // about 2% below the one-CTA form in short runs and the same under a sustained load (what
+  // paces both is each branch's chain of softmax, PV and next score GEMM, and then the power
+  // cap, not the number of MMA instructions or operand bytes), so one CTA per item is the
   // default.
   const int group = Hq / Hkv;
   const char* env = getenv("DA2_PREFILL_CTA_PAIR");
